@@ -1,0 +1,243 @@
+"""Plain, slow, fp64 reference for exact attention (the oracle).
+
+TEST INFRASTRUCTURE: only tests, ``__graft_entry__.smoke()`` and the bench's
+CPU-baseline / reference legs may import this module. It shares no code with
+the CUDA path.
+
+What it computes. The pages state that FlashAttention does not change the
+mathematical definition of attention: tiling, online softmax and fusion reach
+exactly the result of the standard computation ("推理加速" interview notes,
+section FlashAttention and "它到底优化了什么"). So the oracle is that standard
+computation written out, with S materialised ("抱infra脚", section "Flash
+Attention 核心技术", the naive workflow S -> P -> O):
+
+    S = scale * Q K^T          (one query head, its key/value head)
+    S[i, j] = -inf             where causal and key j lies after query i
+    m_i = max_j S[i, j];  P = exp(S - m);  l_i = sum_j P[i, j]
+    O = P V / l;          LSE_i = m_i + ln l_i   (natural log)
+
+* Key/value heads are shared by contiguous groups of query heads: query head h
+  reads key/value head h // G with G = Hq / Hkv ("5.2 推理加速的未来趋势",
+  GQA/MQA paragraph).
+* Causal alignment is bottom-right: with Sq queries and Sk keys, query i sits
+  at absolute position i + (Sk - Sq) and sees keys 0 .. i + (Sk - Sq). This
+  is the reading for a prompt chunk appended to cached context ("抱infra脚",
+  Chunked Prefill); it equals the usual top-left mask when Sq == Sk.
+* A row that sees no key has O = 0 and LSE = -inf.
+* Paged KV: token t of sequence b is in physical block table[b, t // 16] at
+  slot t % 16 ("抱infra脚", Paged Attention: fixed-size blocks mapped through
+  a block table). The oracle gathers the logical sequence, then applies the
+  dense definition. It never splits the key range.
+* Split-KV partials are merged with the log-sum-exp weights: with
+  M = max_s LSE_s, LSE = M + ln sum_s exp(LSE_s - M) and
+  O = sum_s exp(LSE_s - LSE) O_s ("GPU Kernel 调度:大模型推理的拐点 2026",
+  Flash Decoding section: partial output / max / sum per chunk merged by the
+  online-softmax formula, each partial carrying a log-sum-exp in FP32).
+
+Pins (tests/test_oracle.py): brute-force ``math.fsum`` loops on tiny inputs,
+closed forms (one key, causal row 0, zero query, constant V, hand-derived
+weights), torch's fp64 CPU ``scaled_dot_product_attention`` with repeated
+K/V, and invariants (key permutation, split-and-combine, paged vs contiguous,
+GQA vs repeated MHA). No function here is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK_SIZE = 16
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Decode bf16 bit patterns (uint16) exactly into float64."""
+    u = np.asarray(bits).astype(np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def _as_f64(x) -> np.ndarray:
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return bf16_bits_to_f64(x)
+    return x.astype(np.float64)
+
+
+def softmax_probs(q, k, scale, q_pos=None):
+    """Materialised P = softmax(scale * q k^T + mask) for one head.
+
+    ``q`` [n, D], ``k`` [Sk, D]; ``q_pos`` (absolute query positions) turns on
+    the causal mask: key j is visible to query i when j <= q_pos[i].
+    Returns ``(P, m, l)`` with ``m`` the row max of the masked scores and ``l``
+    the row sum of exp(S - m). Rows with no visible key get P = 0, m = -inf,
+    l = 0.
+    """
+    q = _as_f64(q)
+    k = _as_f64(k)
+    s = scale * (q @ k.T)
+    if q_pos is not None:
+        j = np.arange(k.shape[0])[None, :]
+        s = np.where(j <= np.asarray(q_pos)[:, None], s, -np.inf)
+    m = s.max(axis=1) if s.shape[1] else np.full(s.shape[0], -np.inf)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    p = np.exp(s - m_safe[:, None])
+    p[empty] = 0.0
+    l = p.sum(axis=1)
+    return p, m, l
+
+
+def attention_rows(q, k, v, scale, q_pos=None):
+    """Attention for a set of query rows against one key/value sequence.
+
+    ``q`` [n, D]; ``k``, ``v`` [Sk, D]; ``q_pos`` as in :func:`softmax_probs`
+    (None = no mask). Returns ``(O [n, D], LSE [n])`` in fp64.
+    """
+    v = _as_f64(v)
+    p, m, l = softmax_probs(q, k, scale, q_pos)
+    empty = l == 0.0
+    l_safe = np.where(empty, 1.0, l)
+    o = (p @ v) / l_safe[:, None]
+    o[empty] = 0.0
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, m + np.log(l_safe))
+    return o, lse
+
+
+def causal_positions(seqlen_q: int, seqlen_k: int) -> np.ndarray:
+    """Absolute positions of the queries under bottom-right alignment."""
+    return np.arange(seqlen_q) + (seqlen_k - seqlen_q)
+
+
+def ref_attention(q, k, v, scale, causal, rows=None):
+    """Dense reference. Q [B,Hq,Sq,D], K/V [B,Hkv,Sk,D] (bf16 bits or floats).
+
+    ``rows`` optionally restricts the computation to a list of
+    ``(b, h, i)`` query rows; then the result is ``(O [n, D], LSE [n])``.
+    Otherwise returns ``(O [B,Hq,Sq,D], LSE [B,Hq,Sq])``.
+    """
+    q = np.asarray(q)
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = np.asarray(k).shape[1], np.asarray(k).shape[2]
+    if Hq % Hkv:
+        raise ValueError("query heads must be a multiple of key/value heads")
+    G = Hq // Hkv
+    pos = causal_positions(Sq, Sk)
+    if rows is not None:
+        out_o = np.zeros((len(rows), D))
+        out_l = np.zeros(len(rows))
+        for n, (b, h, i) in enumerate(rows):
+            o, lse = attention_rows(_as_f64(q[b, h, i:i + 1]), k[b, h // G], v[b, h // G], scale,
+                                    pos[i:i + 1] if causal else None)
+            out_o[n], out_l[n] = o[0], lse[0]
+        return out_o, out_l
+    O = np.zeros((B, Hq, Sq, D))
+    L = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            O[b, h], L[b, h] = attention_rows(q[b, h], k[b, h // G], v[b, h // G], scale,
+                                              pos if causal else None)
+    return O, L
+
+
+def gather_paged(pool, block_table_row, length: int, kv_head: int) -> np.ndarray:
+    """Logical [length, D] keys (or values) of one sequence and KV head.
+
+    Token t comes from ``pool[block_table_row[t // 16], kv_head, t % 16]``.
+    The result keeps the pool's dtype (bf16 bits stay bits).
+    """
+    pool = np.asarray(pool)
+    t = np.arange(length)
+    phys = np.asarray(block_table_row)[t // BLOCK_SIZE]
+    return pool[phys, kv_head, t % BLOCK_SIZE]
+
+
+def ref_decode_paged(q, k_pool, v_pool, block_table, seq_lens, scale, rows=None):
+    """Decode: one query token per sequence; all ``seq_lens[b]`` cached keys visible.
+
+    q [B, Hq, D]; pools [NB, Hkv, 16, D]. Returns O [B, Hq, D], LSE [B, Hq]
+    (or, with ``rows`` = list of (b, h), arrays over those rows).
+    """
+    q = np.asarray(q)
+    B, Hq, D = q.shape
+    Hkv = np.asarray(k_pool).shape[1]
+    G = Hq // Hkv
+    todo = rows if rows is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    O = np.zeros((len(todo), D))
+    L = np.zeros(len(todo))
+    cache = {}
+    for n, (b, h) in enumerate(todo):
+        key = (b, h // G)
+        if key not in cache:
+            cache.clear()
+            kk = gather_paged(k_pool, block_table[b], int(seq_lens[b]), h // G)
+            vv = gather_paged(v_pool, block_table[b], int(seq_lens[b]), h // G)
+            cache[key] = (kk, vv)
+        kk, vv = cache[key]
+        o, lse = attention_rows(_as_f64(q[b, h][None]), kk, vv, scale, None)
+        O[n], L[n] = o[0], lse[0]
+    if rows is None:
+        return O.reshape(B, Hq, D), L.reshape(B, Hq)
+    return O, L
+
+
+def ref_prefill_paged(q, q_lens, k_pool, v_pool, block_table, k_lens, scale, causal, rows=None):
+    """Prefill of query chunks against paged keys/values.
+
+    q [B, Hq, Sq_max, D] with ``q_lens[b]`` valid rows; sequence b has
+    ``k_lens[b]`` cached keys (its own chunk included, so the chunk's queries
+    sit at positions k_lens[b] - q_lens[b] + i under the causal mask).
+    Returns O [B, Hq, Sq_max, D] and LSE [B, Hq, Sq_max] (rows past q_lens are
+    zero / -inf), or arrays over ``rows`` = list of (b, h, i).
+    """
+    q = np.asarray(q)
+    B, Hq, Sqm, D = q.shape
+    Hkv = np.asarray(k_pool).shape[1]
+    G = Hq // Hkv
+    if rows is not None:
+        O = np.zeros((len(rows), D))
+        L = np.zeros(len(rows))
+        for n, (b, h, i) in enumerate(rows):
+            kk = gather_paged(k_pool, block_table[b], int(k_lens[b]), h // G)
+            vv = gather_paged(v_pool, block_table[b], int(k_lens[b]), h // G)
+            pos = causal_positions(int(q_lens[b]), int(k_lens[b]))[i:i + 1]
+            o, lse = attention_rows(_as_f64(q[b, h, i:i + 1]), kk, vv, scale,
+                                    pos if causal else None)
+            O[n], L[n] = o[0], lse[0]
+        return O, L
+    O = np.zeros((B, Hq, Sqm, D))
+    L = np.full((B, Hq, Sqm), -np.inf)
+    for b in range(B):
+        nq, nk = int(q_lens[b]), int(k_lens[b])
+        pos = causal_positions(nq, nk)
+        for kvh in range(Hkv):
+            kk = gather_paged(k_pool, block_table[b], nk, kvh)
+            vv = gather_paged(v_pool, block_table[b], nk, kvh)
+            for h in range(kvh * G, (kvh + 1) * G):
+                O[b, h, :nq], L[b, h, :nq] = attention_rows(
+                    q[b, h, :nq], kk, vv, scale, pos if causal else None)
+    return O, L
+
+
+def combine_partials(part_o, part_lse, splits_per_row=None):
+    """Merge split-KV partials by their log-sum-exp weights.
+
+    ``part_o`` [S, rows, D] holds each split's normalised output, ``part_lse``
+    [S, rows] its log-sum-exp (natural log; -inf for a split with no key).
+    ``splits_per_row`` [rows] limits row r to its first splits. Returns
+    ``(O [rows, D], LSE [rows])``; a row whose splits are all empty gets
+    O = 0, LSE = -inf.
+    """
+    po = _as_f64(part_o)
+    pl = _as_f64(part_lse)
+    S, R, D = po.shape
+    O = np.zeros((R, D))
+    L = np.full(R, -np.inf)
+    for r in range(R):
+        n = S if splits_per_row is None else int(splits_per_row[r])
+        lse = pl[:n, r]
+        if n == 0 or not np.isfinite(lse).any():
+            continue
+        M = lse.max()
+        w = np.exp(lse - M)
+        L[r] = M + np.log(w.sum())
+        wn = np.exp(lse - L[r])
+        O[r] = (wn[:, None] * po[:n, r]).sum(axis=0)
+    return O, L

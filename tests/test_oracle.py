@@ -1,0 +1,321 @@
+"""Pins for the fp64 oracle: things other than the oracle itself that fix its results.
+
+* brute force: pure-Python ``math.fsum`` loops on tiny inputs;
+* closed forms: hand-derived fixtures under tests/golden/, one key, causal
+  row 0, zero query, constant V, one dominant key, rows of P sum to 1;
+* a library special case: torch's fp64 CPU ``scaled_dot_product_attention``
+  with K/V repeated for GQA;
+* invariants: key/value permutation, split-and-combine, paged vs contiguous,
+  GQA vs repeated MHA;
+* planted mistakes: mutated copies of the formula are rejected by the pins.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import attention_ref as ref
+from attention_tiled_exact_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "softmax_closed_form.json")
+
+
+def _nested(x):
+    return np.asarray(x, dtype=np.float64).tolist()
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+# ----------------------------------------------------------------------------
+# brute force
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal", [
+    (1, 1, 1, 4, 4, 8, False),
+    (2, 4, 2, 5, 7, 8, False),
+    (2, 4, 2, 5, 7, 8, True),     # bottom-right offset 2
+    (1, 3, 1, 6, 6, 4, True),     # MQA
+    (1, 2, 2, 7, 5, 4, True),     # Sq > Sk: first two rows see no key
+    (1, 4, 4, 1, 9, 8, False),    # decode-like
+])
+def test_numpy_oracle_matches_brute_force(B, Hq, Hkv, Sq, Sk, D, causal):
+    rng = np.random.default_rng(1234 + Sq * Sk + D)
+    q, k, v = _rand(rng, B, Hq, Sq, D), _rand(rng, B, Hkv, Sk, D), _rand(rng, B, Hkv, Sk, D)
+    scale = 0.37
+    O, L = ref.ref_attention(q, k, v, scale, causal)
+    Ob, Lb = oracle.brute_attention(_nested(q), _nested(k), _nested(v), scale, causal)
+    np.testing.assert_allclose(O, np.array(Ob), rtol=0, atol=1e-12)
+    Lb = np.array(Lb)
+    assert np.array_equal(np.isinf(L), np.isinf(Lb))
+    fin = np.isfinite(Lb)
+    np.testing.assert_allclose(L[fin], Lb[fin], rtol=0, atol=1e-12)
+    if Sq > Sk and causal:
+        assert np.all(O[:, :, : Sq - Sk] == 0) and np.all(np.isneginf(L[:, :, : Sq - Sk]))
+
+
+# ----------------------------------------------------------------------------
+# closed forms
+# ----------------------------------------------------------------------------
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", _golden()["attention"], ids=lambda c: c["name"])
+def test_golden_attention_closed_form(case):
+    O, L = ref.ref_attention(np.array(case["q"]), np.array(case["k"]), np.array(case["v"]),
+                             case["scale"], case["causal"])
+    np.testing.assert_allclose(O, np.array(case["expected_o"]), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(L, np.array(case["expected_lse"]), rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("case", _golden()["combine"], ids=lambda c: c["name"])
+def test_golden_combine_closed_form(case):
+    lse = np.array([[float(x) for x in row] for row in case["part_lse"]])
+    O, L = ref.combine_partials(np.array(case["part_o"]), lse)
+    np.testing.assert_allclose(O, np.array(case["expected_o"]), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(L, np.array(case["expected_lse"]), rtol=0, atol=1e-13)
+
+
+def test_single_key_returns_its_value():
+    rng = np.random.default_rng(0)
+    q, k, v = _rand(rng, 1, 2, 3, 16), _rand(rng, 1, 2, 1, 16), _rand(rng, 1, 2, 1, 16)
+    O, L = ref.ref_attention(q, k, v, 0.25, False)
+    np.testing.assert_array_equal(O, np.broadcast_to(v, O.shape))
+    np.testing.assert_allclose(L[0, :, :], 0.25 * np.einsum("hsd,hd->hs", q[0], k[0, :, 0]),
+                               atol=1e-14)
+
+
+def test_causal_row0_is_first_value_row():
+    rng = np.random.default_rng(1)
+    q, k, v = _rand(rng, 2, 4, 9, 8), _rand(rng, 2, 2, 9, 8), _rand(rng, 2, 2, 9, 8)
+    O, L = ref.ref_attention(q, k, v, 0.5, True)
+    for h in range(4):
+        np.testing.assert_array_equal(O[:, h, 0], v[:, h // 2, 0])
+        np.testing.assert_allclose(L[:, h, 0], 0.5 * np.einsum("bd,bd->b", q[:, h, 0], k[:, h // 2, 0]),
+                                   atol=1e-14)
+
+
+def test_zero_query_gives_mean_of_visible_values():
+    rng = np.random.default_rng(2)
+    Sq, Sk = 5, 8
+    q = np.zeros((1, 2, Sq, 8))
+    k, v = _rand(rng, 1, 1, Sk, 8), _rand(rng, 1, 1, Sk, 8)
+    O, L = ref.ref_attention(q, k, v, 1.0, True)
+    for i in range(Sq):
+        nvis = i + (Sk - Sq) + 1
+        np.testing.assert_allclose(O[0, :, i], np.broadcast_to(v[0, 0, :nvis].mean(0), (2, 8)), atol=1e-14)
+        np.testing.assert_allclose(L[0, :, i], math.log(nvis), atol=1e-14)
+
+
+def test_constant_values_are_returned():
+    rng = np.random.default_rng(3)
+    q, k = _rand(rng, 1, 4, 6, 8), _rand(rng, 1, 2, 10, 8)
+    row = _rand(rng, 8)
+    v = np.broadcast_to(row, (1, 2, 10, 8)).copy()
+    for causal in (False, True):
+        O, _ = ref.ref_attention(q, k, v, 0.3, causal)
+        np.testing.assert_allclose(O, np.broadcast_to(row, O.shape), atol=1e-14)
+
+
+def test_dominant_key_selects_its_value():
+    rng = np.random.default_rng(4)
+    D = 8
+    k = _rand(rng, 1, 1, 12, D) * 0.01
+    q = np.zeros((1, 1, 1, D))
+    q[0, 0, 0, 0] = 1.0
+    k[0, 0, 7, 0] = 2000.0
+    v = _rand(rng, 1, 1, 12, D)
+    O, L = ref.ref_attention(q, k, v, 1.0, False)
+    np.testing.assert_allclose(O[0, 0, 0], v[0, 0, 7], atol=1e-12)
+    assert abs(L[0, 0, 0] - 2000.0) < 1e-9
+
+
+def test_softmax_rows_sum_to_one():
+    rng = np.random.default_rng(5)
+    q, k = _rand(rng, 6, 8), _rand(rng, 11, 8)
+    pos = ref.causal_positions(6, 11)
+    for qp in (None, pos):
+        p, m, l = ref.softmax_probs(q, k, 0.7, qp)
+        np.testing.assert_allclose((p / l[:, None]).sum(axis=1), 1.0, atol=1e-14)
+        assert np.all(p <= 1.0) and np.allclose(p.max(axis=1), 1.0)
+
+
+# ----------------------------------------------------------------------------
+# a library routine as a special case
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("Sq,Sk,causal", [(33, 33, False), (33, 33, True), (17, 40, True), (1, 50, False)])
+def test_matches_torch_sdpa_fp64(Sq, Sk, causal):
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(6 + Sq + Sk)
+    B, Hq, Hkv, D = 2, 8, 2, 16
+    q, k, v = _rand(rng, B, Hq, Sq, D), _rand(rng, B, Hkv, Sk, D), _rand(rng, B, Hkv, Sk, D)
+    scale = 1 / math.sqrt(D)
+    O, L = ref.ref_attention(q, k, v, scale, causal)
+    G = Hq // Hkv
+    tq = torch.from_numpy(q)
+    tk = torch.from_numpy(k).repeat_interleave(G, dim=1)
+    tv = torch.from_numpy(v).repeat_interleave(G, dim=1)
+    mask = None
+    if causal:
+        i = torch.arange(Sq)[:, None] + (Sk - Sq)
+        j = torch.arange(Sk)[None, :]
+        mask = j <= i
+    To = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=scale)
+    np.testing.assert_allclose(O, To.numpy(), rtol=0, atol=1e-12)
+    s = torch.einsum("bhqd,bhkd->bhqk", tq, tk) * scale
+    if mask is not None:
+        s = s.masked_fill(~mask, float("-inf"))
+    np.testing.assert_allclose(L, torch.logsumexp(s, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# invariants
+# ----------------------------------------------------------------------------
+
+
+def test_noncausal_invariant_to_key_permutation():
+    rng = np.random.default_rng(7)
+    q, k, v = _rand(rng, 1, 4, 9, 8), _rand(rng, 1, 2, 13, 8), _rand(rng, 1, 2, 13, 8)
+    perm = rng.permutation(13)
+    O1, L1 = ref.ref_attention(q, k, v, 0.4, False)
+    O2, L2 = ref.ref_attention(q, k[:, :, perm], v[:, :, perm], 0.4, False)
+    np.testing.assert_allclose(O1, O2, atol=1e-13)
+    np.testing.assert_allclose(L1, L2, atol=1e-13)
+
+
+@pytest.mark.parametrize("cuts", [[0, 5, 13], [0, 1, 2, 13], [0, 4, 4, 9, 13], [0, 13]])
+def test_split_combine_equals_single_pass(cuts):
+    rng = np.random.default_rng(8)
+    q, k, v = _rand(rng, 3, 8), _rand(rng, 13, 8), _rand(rng, 13, 8)
+    O, L = ref.attention_rows(q, k, v, 0.6)
+    parts_o, parts_l = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o, l = ref.attention_rows(q, k[a:b], v[a:b], 0.6)
+        parts_o.append(o)
+        parts_l.append(l)
+    Oc, Lc = ref.combine_partials(np.stack(parts_o), np.stack(parts_l))
+    np.testing.assert_allclose(Oc, O, atol=1e-13)
+    np.testing.assert_allclose(Lc, L, atol=1e-13)
+
+
+def test_combine_respects_splits_per_row():
+    rng = np.random.default_rng(9)
+    po, pl = _rand(rng, 4, 3, 8), _rand(rng, 4, 3)
+    pl[2:, 0] = np.nan  # never read for row 0
+    O, L = ref.combine_partials(po, pl, splits_per_row=[2, 4, 1])
+    O0, L0 = ref.combine_partials(po[:2, :1], pl[:2, :1])
+    np.testing.assert_allclose(O[0], O0[0], atol=1e-14)
+    np.testing.assert_allclose(L[2], pl[0, 2], atol=1e-14)
+    np.testing.assert_allclose(O[2], po[0, 2], atol=1e-14)
+
+
+def test_paged_equals_contiguous():
+    lens = np.array([1, 16, 17, 40, 5])
+    d = wl.make_paged_pool(11, lens, kv_heads=2, head_dim=8)
+    rng = np.random.default_rng(10)
+    q = wl.normal_bf16(11, (len(lens), 4, 8), 5)
+    O, L = ref.ref_decode_paged(q, d["k_pool"], d["v_pool"], d["block_table"], lens, 0.35)
+    for b, n in enumerate(lens):
+        for kvh in range(2):
+            kk = np.stack([d["k_pool"][d["block_table"][b, t // 16], kvh, t % 16] for t in range(n)])
+            vv = np.stack([d["v_pool"][d["block_table"][b, t // 16], kvh, t % 16] for t in range(n)])
+            for h in (2 * kvh, 2 * kvh + 1):
+                o, l = ref.attention_rows(ref.bf16_bits_to_f64(q[b, h][None]), kk, vv, 0.35)
+                np.testing.assert_allclose(O[b, h], o[0], atol=1e-13)
+                np.testing.assert_allclose(L[b, h], l[0], atol=1e-13)
+    assert np.isfinite(O).all() and np.isfinite(L).all()  # the NaN sentinels were never read
+    del rng
+
+
+def test_paged_prefill_equals_dense_on_gathered_keys():
+    ctx = np.array([0, 20, 3])
+    qlen = 6
+    lens = ctx + qlen
+    d = wl.make_paged_pool(12, lens, kv_heads=1, head_dim=8)
+    q = wl.normal_bf16(12, (3, 2, qlen, 8), 5)
+    O, L = ref.ref_prefill_paged(q, [qlen] * 3, d["k_pool"], d["v_pool"], d["block_table"], lens, 0.3, True)
+    for b in range(3):
+        kk = ref.gather_paged(d["k_pool"], d["block_table"][b], int(lens[b]), 0)[None, None]
+        vv = ref.gather_paged(d["v_pool"], d["block_table"][b], int(lens[b]), 0)[None, None]
+        Od, Ld = ref.ref_attention(q[b:b + 1], kk, vv, 0.3, True)
+        np.testing.assert_allclose(O[b], Od[0], atol=1e-13)
+        np.testing.assert_allclose(L[b], Ld[0], atol=1e-13)
+
+
+def test_gqa_equals_repeated_mha():
+    rng = np.random.default_rng(13)
+    q, k, v = _rand(rng, 2, 6, 7, 8), _rand(rng, 2, 2, 7, 8), _rand(rng, 2, 2, 7, 8)
+    O1, L1 = ref.ref_attention(q, k, v, 0.5, True)
+    O2, L2 = ref.ref_attention(q, np.repeat(k, 3, axis=1), np.repeat(v, 3, axis=1), 0.5, True)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
+
+
+def test_rows_subset_matches_full():
+    rng = np.random.default_rng(14)
+    q, k, v = _rand(rng, 2, 4, 9, 8), _rand(rng, 2, 2, 12, 8), _rand(rng, 2, 2, 12, 8)
+    O, L = ref.ref_attention(q, k, v, 0.5, True)
+    rows = [(0, 0, 0), (1, 3, 8), (1, 2, 4)]
+    Or, Lr = ref.ref_attention(q, k, v, 0.5, True, rows=rows)
+    for n, (b, h, i) in enumerate(rows):
+        np.testing.assert_allclose(Or[n], O[b, h, i], atol=1e-14)
+        np.testing.assert_allclose(Lr[n], L[b, h, i], atol=1e-14)
+
+
+def test_bf16_decode_is_exact():
+    bits = np.array([0x3F80, 0xC020, 0x0001, 0x7F7F, 0x8000], dtype=np.uint16)
+    vals = ref.bf16_bits_to_f64(bits)
+    assert vals[0] == 1.0 and vals[1] == -2.5 and vals[2] == 2.0 ** -133
+    assert vals[3] == (2 - 2 ** -7) * 2.0 ** 127 and vals[4] == 0.0 and math.copysign(1, vals[4]) < 0
+
+
+# ----------------------------------------------------------------------------
+# planted mistakes: each mutant of the formula must fail a pin
+# ----------------------------------------------------------------------------
+
+
+def _candidate(q, k, v, scale, causal, mutant):
+    """A copy of the definition with one planted mistake (or none)."""
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    O = np.zeros((B, Hq, Sq, D))
+    L = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            kvh = (h % Hkv) if mutant == "gqa_modulo" else h // G
+            s = (1.0 if mutant == "no_scale" else scale) * (q[b, h] @ k[b, kvh].T)
+            if causal:
+                i = np.arange(Sq)[:, None] + (0 if mutant == "top_left" else Sk - Sq)
+                j = np.arange(Sk)[None, :]
+                s = np.where((j < i) if mutant == "strict_mask" else (j <= i), s, -np.inf)
+            m = s.max(1)
+            p = np.exp(s - m[:, None])
+            l = p.sum(1)
+            vv = v[b, kvh].T.T if mutant != "transposed_v" else v[b, kvh][::-1]
+            O[b, h] = (p @ vv) / (l[:, None] if mutant != "no_norm" else 1.0)
+            L[b, h] = (0 if mutant == "lse_no_max" else m) + np.log(l)
+    return O, L
+
+
+@pytest.mark.parametrize("mutant", ["no_scale", "top_left", "strict_mask", "gqa_modulo",
+                                    "transposed_v", "no_norm", "lse_no_max"])
+def test_pins_reject_planted_mistakes(mutant):
+    rng = np.random.default_rng(15)
+    q, k, v = _rand(rng, 1, 4, 5, 4), _rand(rng, 1, 2, 7, 4), _rand(rng, 1, 2, 7, 4)
+    Ob, Lb = oracle.brute_attention(_nested(q), _nested(k), _nested(v), 0.5, True)
+    Oc, Lc = _candidate(q, k, v, 0.5, True, None)
+    assert np.allclose(Oc, Ob, atol=1e-12) and np.allclose(Lc, Lb, atol=1e-12)
+    Om, Lm = _candidate(q, k, v, 0.5, True, mutant)
+    assert not (np.allclose(Om, Ob, atol=1e-6) and np.allclose(Lm, Lb, atol=1e-6))

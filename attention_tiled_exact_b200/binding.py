@@ -1,0 +1,265 @@
+"""ctypes binding of libattn_b200.so.
+
+Argument marshalling only: torch tensors provide device memory and the
+current CUDA stream; every step of the computation runs in the library's
+kernels. The names follow the C ABI declared in include/attn.h.
+
+Importing this module loads the library and fails loudly if it is missing
+(build it with ``python -m attention_tiled_exact_b200.build``). There is no
+CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_FILE = os.path.join(HERE, "libattn_b200.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_WORKSPACE = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_DEVICE_FAULT = 5
+ATTN_ERR_TIMEOUT = 6
+ATTN_ERR_NO_DEVICE = 7
+
+ATTN_DTYPE_BF16 = 0
+ATTN_DTYPE_F32 = 1
+
+ATTN_FAULT_TIMEOUT = 0x1
+ATTN_FAULT_BAD_BLOCK = 0x2
+ATTN_FAULT_BAD_LENGTH = 0x4
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_i64 = ctypes.c_int64
+
+
+class PrefillParams(ctypes.Structure):
+    """Mirror of ``attn_prefill_params``."""
+
+    _fields_ = [
+        ("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp),
+        ("batch", _i32), ("num_q_heads", _i32), ("num_kv_heads", _i32), ("head_dim", _i32),
+        ("seqlen_q", _i32), ("seqlen_k", _i32),
+        ("q_batch_stride", _i64), ("q_head_stride", _i64), ("q_row_stride", _i64),
+        ("k_batch_stride", _i64), ("k_head_stride", _i64), ("k_row_stride", _i64),
+        ("v_batch_stride", _i64), ("v_head_stride", _i64), ("v_row_stride", _i64),
+        ("o_batch_stride", _i64), ("o_head_stride", _i64), ("o_row_stride", _i64),
+        ("scale", ctypes.c_float), ("causal", _i32), ("o_dtype", _i32),
+        ("seqlens_q", _vp), ("seqlens_k", _vp), ("k_cache", _vp), ("v_cache", _vp),
+        ("block_table", _vp), ("max_blocks_per_seq", _i32), ("num_blocks", _i32),
+        ("block_size", _i32), ("error_flags", _vp),
+    ]
+
+
+class DecodeParams(ctypes.Structure):
+    """Mirror of ``attn_decode_params``."""
+
+    _fields_ = [
+        ("q", _vp), ("k_cache", _vp), ("v_cache", _vp), ("block_table", _vp), ("seq_lens", _vp),
+        ("o", _vp), ("lse", _vp),
+        ("batch", _i32), ("num_q_heads", _i32), ("num_kv_heads", _i32), ("head_dim", _i32),
+        ("block_size", _i32), ("max_blocks_per_seq", _i32), ("num_blocks", _i32),
+        ("max_seq_len", _i32), ("num_splits", _i32), ("scale", ctypes.c_float), ("o_dtype", _i32),
+        ("error_flags", _vp),
+    ]
+
+
+def _load():
+    if not os.path.exists(_LIB_FILE):
+        raise ImportError(f"{_LIB_FILE} is missing: build it with "
+                          "`python -m attention_tiled_exact_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(_LIB_FILE)
+    lib.attn_prefill.argtypes = [ctypes.POINTER(PrefillParams), _vp]
+    lib.attn_prefill.restype = ctypes.c_int
+    lib.attn_decode_paged.argtypes = [ctypes.POINTER(DecodeParams), _vp, ctypes.c_size_t,
+                                      ctypes.POINTER(ctypes.c_size_t), _vp]
+    lib.attn_decode_paged.restype = ctypes.c_int
+    lib.splitkv_lse_combine.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp,
+                                        ctypes.c_int, _vp, _vp]
+    lib.splitkv_lse_combine.restype = ctypes.c_int
+    lib.attn_status_string.argtypes = [ctypes.c_int]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_version.argtypes = []
+    lib.attn_version.restype = ctypes.c_int
+    return lib
+
+
+LIB = _load()
+
+
+def library_path() -> str:
+    return _LIB_FILE
+
+
+def status_string(status: int) -> str:
+    return LIB.attn_status_string(int(status)).decode()
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def _check(status: int, where: str):
+    if status != ATTN_OK:
+        raise AttnError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _out_code(dtype) -> int:
+    if dtype == torch.bfloat16:
+        return ATTN_DTYPE_BF16
+    if dtype == torch.float32:
+        return ATTN_DTYPE_F32
+    raise TypeError("output dtype must be bfloat16 or float32")
+
+
+def _need(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+# ----------------------------------------------------------------------------
+# prefill
+# ----------------------------------------------------------------------------
+
+
+def prefill(q, k, v, scale: float | None = None, causal: bool = False, out=None, lse=None,
+            out_dtype=torch.bfloat16, want_lse: bool = True, error_flags=None):
+    """Tiled prefill attention. q [B,Hq,Sq,D], k/v [B,Hkv,Sk,D] bf16 CUDA tensors.
+
+    Returns ``(O [B,Hq,Sq,D], LSE [B,Hq,Sq] fp32 or None)``.
+    """
+    _need(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be 4-D [B, H, S, D]")
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    _need(tuple(v.shape) == tuple(k.shape) and k.shape[0] == B and k.shape[3] == D, "shape mismatch")
+    for t in (q, k, v):
+        _need(t.dtype == torch.bfloat16 and t.is_cuda and t.stride(3) == 1, "bf16 CUDA, last dim contiguous")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Hq, Sq, D), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse.is_contiguous() and lse.dtype == torch.float32 and tuple(lse.shape) == (B, Hq, Sq), "lse")
+    p = PrefillParams()
+    p.q, p.k, p.v, p.o, p.lse = _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse)
+    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.seqlen_q, p.seqlen_k = B, Hq, Hkv, D, Sq, Sk
+    p.q_batch_stride, p.q_head_stride, p.q_row_stride = q.stride(0), q.stride(1), q.stride(2)
+    p.k_batch_stride, p.k_head_stride, p.k_row_stride = k.stride(0), k.stride(1), k.stride(2)
+    p.v_batch_stride, p.v_head_stride, p.v_row_stride = v.stride(0), v.stride(1), v.stride(2)
+    p.o_batch_stride, p.o_head_stride, p.o_row_stride = out.stride(0), out.stride(1), out.stride(2)
+    p.scale, p.causal, p.o_dtype = float(scale), int(bool(causal)), _out_code(out.dtype)
+    p.error_flags = _ptr(error_flags)
+    _check(LIB.attn_prefill(ctypes.byref(p), _stream(q.device)), "attn_prefill")
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------
+
+
+def _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits, out, lse,
+                   error_flags):
+    B, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    p = DecodeParams()
+    p.q, p.k_cache, p.v_cache = _ptr(q), _ptr(k_cache), _ptr(v_cache)
+    p.block_table, p.seq_lens, p.o, p.lse = _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse)
+    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim = B, Hq, Hkv, D
+    p.block_size, p.max_blocks_per_seq, p.num_blocks = BS, block_table.shape[1], NB
+    p.max_seq_len, p.num_splits = int(max_seq_len), int(num_splits)
+    p.scale = float(scale if scale is not None else 1.0 / math.sqrt(D))
+    p.o_dtype = _out_code(out.dtype) if out is not None else ATTN_DTYPE_BF16
+    p.error_flags = _ptr(error_flags)
+    return p
+
+
+def decode_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int = 0,
+                           num_splits: int = 0) -> int:
+    """Bytes of workspace :func:`decode_paged` needs for these shapes."""
+    p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, None, max_seq_len, num_splits, q, None, None)
+    need = ctypes.c_size_t(0)
+    _check(LIB.attn_decode_paged(ctypes.byref(p), None, 0, ctypes.byref(need), None), "attn_decode_paged(size)")
+    return int(need.value)
+
+
+def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None, max_seq_len: int = 0,
+                 num_splits: int = 0, out=None, lse=None, workspace=None, out_dtype=torch.bfloat16,
+                 want_lse: bool = True, error_flags=None):
+    """Flash-Decoding over a paged KV cache.
+
+    q [B,Hq,D] bf16; k_cache/v_cache [NB,Hkv,16,D] bf16; block_table [B,maxblk]
+    int32; seq_lens [B] int32 (all CUDA). ``max_seq_len`` is a host-side
+    upper bound of seq_lens used for the split plan (0 = table capacity).
+    Returns ``(O [B,Hq,D], LSE [B,Hq] or None)``.
+    """
+    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
+    _need(q.dtype == torch.bfloat16 and k_cache.dtype == torch.bfloat16 and v_cache.dtype == torch.bfloat16,
+          "bf16 q and caches")
+    _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
+    _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
+          "int32 block table [B, max_blocks]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "int32 seq_lens [B]")
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits, out, lse,
+                       error_flags)
+    need = ctypes.c_size_t(0)
+    _check(LIB.attn_decode_paged(ctypes.byref(p), None, 0, ctypes.byref(need), None), "attn_decode_paged(size)")
+    if workspace is None and need.value > 0:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(LIB.attn_decode_paged(ctypes.byref(p), ws_ptr, ws_bytes, None, _stream(q.device)),
+           "attn_decode_paged")
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# combine
+# ----------------------------------------------------------------------------
+
+
+def splitkv_lse_combine(part_o, part_lse, splits_per_row=None, out=None, out_lse=None,
+                        out_dtype=torch.float32):
+    """Merge split partials. part_o [S, rows, D] fp32, part_lse [S, rows] fp32.
+
+    Returns ``(O [rows, D], LSE [rows])``.
+    """
+    _need(part_o.dim() == 3 and part_lse.dim() == 2, "part_o [S, rows, D], part_lse [S, rows]")
+    S, R, D = part_o.shape
+    _need(tuple(part_lse.shape) == (S, R), "part_lse shape")
+    _need(part_o.dtype == torch.float32 and part_lse.dtype == torch.float32, "fp32 partials")
+    _need(part_o.is_contiguous() and part_lse.is_contiguous(), "contiguous partials")
+    if splits_per_row is not None:
+        _need(splits_per_row.dtype == torch.int32 and splits_per_row.numel() == R, "int32 splits_per_row [rows]")
+    if out is None:
+        out = torch.empty((R, D), dtype=out_dtype, device=part_o.device)
+    if out_lse is None:
+        out_lse = torch.empty((R,), dtype=torch.float32, device=part_o.device)
+    _check(LIB.splitkv_lse_combine(_ptr(part_o), _ptr(part_lse), S, R, D, _ptr(splits_per_row), _ptr(out),
+                                   _out_code(out.dtype), _ptr(out_lse), _stream(part_o.device)),
+           "splitkv_lse_combine")
+    return out, out_lse

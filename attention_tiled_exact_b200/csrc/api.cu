@@ -1,0 +1,159 @@
+// C ABI of libattn_b200.so: host-side validation and dispatch. Every argument
+// check happens here, before anything is enqueued; the kernels only see
+// arguments that passed. See include/attn.h for the contract.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "attn.h"
+#include "internal.h"
+
+namespace attn {
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool mult8(int64_t s) { return (s % 8) == 0; }
+
+int device_sm_count() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+attn_status_t check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_NO_DEVICE;
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_NO_DEVICE;
+  }
+  return (major == 10 && minor == 0) ? ATTN_OK : ATTN_ERR_NO_DEVICE;
+}
+
+static attn_status_t validate_prefill(const attn_prefill_params* p) {
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->num_q_heads < 0 || p->num_kv_heads < 0 || p->seqlen_q < 0 || p->seqlen_k < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (p->batch > 65535 * 32) return ATTN_ERR_INVALID_ARG;
+  if (p->num_kv_heads == 0 || p->num_q_heads == 0) return ATTN_ERR_INVALID_ARG;
+  if (p->num_q_heads % p->num_kv_heads != 0) return ATTN_ERR_UNSUPPORTED;
+  if (p->head_dim != 64 && p->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!(p->scale > 0.f) || !isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
+  if (p->o_dtype != ATTN_DTYPE_BF16 && p->o_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  const bool paged = p->k_cache != nullptr || p->v_cache != nullptr;
+  if (!p->q || !p->o) return ATTN_ERR_INVALID_ARG;
+  if (paged) {
+    if (!p->k_cache || !p->v_cache || p->k || p->v || !p->block_table || !p->seqlens_k) return ATTN_ERR_INVALID_ARG;
+    if (p->block_size != 16) return ATTN_ERR_UNSUPPORTED;
+    if (p->max_blocks_per_seq <= 0 || p->num_blocks <= 0) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(p->k_cache) || !aligned16(p->v_cache)) return ATTN_ERR_UNSUPPORTED;
+  } else {
+    if ((!p->k || !p->v) && p->seqlen_k > 0) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(p->k) || !aligned16(p->v)) return ATTN_ERR_UNSUPPORTED;
+    if (!mult8(p->k_batch_stride) || !mult8(p->k_head_stride) || !mult8(p->k_row_stride) ||
+        !mult8(p->v_batch_stride) || !mult8(p->v_head_stride) || !mult8(p->v_row_stride))
+      return ATTN_ERR_UNSUPPORTED;
+    if (p->k_row_stride < p->head_dim || p->v_row_stride < p->head_dim) return ATTN_ERR_INVALID_ARG;
+  }
+  if (!aligned16(p->q) || !aligned16(p->o)) return ATTN_ERR_UNSUPPORTED;
+  if (!mult8(p->q_batch_stride) || !mult8(p->q_head_stride) || !mult8(p->q_row_stride) ||
+      !mult8(p->o_batch_stride) || !mult8(p->o_head_stride) || !mult8(p->o_row_stride))
+    return ATTN_ERR_UNSUPPORTED;
+  if (p->q_row_stride < p->head_dim || p->o_row_stride < p->head_dim) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+static attn_status_t validate_decode(const attn_decode_params* p) {
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->batch > 65535) return ATTN_ERR_INVALID_ARG;
+  if (p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->num_kv_heads > 65535) return ATTN_ERR_INVALID_ARG;
+  if (p->num_q_heads % p->num_kv_heads != 0) return ATTN_ERR_UNSUPPORTED;
+  const int g = p->num_q_heads / p->num_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return ATTN_ERR_UNSUPPORTED;
+  if (p->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
+  if (p->block_size != 16) return ATTN_ERR_UNSUPPORTED;
+  if (p->max_blocks_per_seq <= 0 || p->num_blocks <= 0 || p->max_seq_len < 0 || p->num_splits < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if ((int64_t)p->max_blocks_per_seq * 16 > INT32_MAX / 2) return ATTN_ERR_INVALID_ARG;
+  if (!(p->scale > 0.f) || !isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
+  if (p->o_dtype != ATTN_DTYPE_BF16 && p->o_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  if (!p->q || !p->k_cache || !p->v_cache || !p->block_table || !p->seq_lens || !p->o) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
+    return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+}  // namespace attn
+
+extern "C" {
+
+attn_status_t attn_prefill(const attn_prefill_params* p, attn_stream_t stream) {
+  attn_status_t st = attn::validate_prefill(p);
+  if (st != ATTN_OK) return st;
+  if (p->batch == 0 || p->seqlen_q == 0) return ATTN_OK;
+  st = attn::check_device();
+  if (st != ATTN_OK) return st;
+  return attn::launch_prefill(*p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_decode_paged(const attn_decode_params* p, void* workspace, size_t workspace_bytes,
+                                size_t* workspace_needed, attn_stream_t stream) {
+  attn_status_t st = attn::validate_decode(p);
+  if (st != ATTN_OK) return st;
+  const bool have_dev = attn::check_device() == ATTN_OK;
+  attn::DecodePlan plan = attn::plan_decode(*p);
+  if (workspace_needed) *workspace_needed = plan.workspace_bytes;
+  if (workspace == nullptr && workspace_needed != nullptr) return ATTN_OK;  // size query only
+  if (workspace_bytes < plan.workspace_bytes) return ATTN_ERR_WORKSPACE;
+  if (plan.workspace_bytes > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (p->batch == 0) return ATTN_OK;
+  if (!have_dev) return ATTN_ERR_NO_DEVICE;
+  return attn::launch_decode(*p, plan, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status_t splitkv_lse_combine(const float* part_o, const float* part_lse, int num_splits, int rows,
+                                  int head_dim, const int32_t* splits_per_row, void* out_o, attn_dtype_t out_dtype,
+                                  float* out_lse, attn_stream_t stream) {
+  if (num_splits < 0 || rows < 0) return ATTN_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return ATTN_ERR_UNSUPPORTED;
+  if (out_dtype != ATTN_DTYPE_BF16 && out_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  if (rows == 0) return ATTN_OK;
+  if (!out_o || (num_splits > 0 && (!part_o || !part_lse))) return ATTN_ERR_INVALID_ARG;
+  if ((num_splits > 0 && !attn::aligned16(part_o)) || !attn::aligned16(out_o)) return ATTN_ERR_UNSUPPORTED;
+  attn_status_t st = attn::check_device();
+  if (st != ATTN_OK) return st;
+  return attn::launch_combine(part_o, part_lse, num_splits, rows, head_dim, splits_per_row, nullptr, 1, 1, out_o,
+                              out_dtype, out_lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+const char* attn_status_string(attn_status_t status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape, dtype or alignment";
+    case ATTN_ERR_WORKSPACE: return "workspace too small";
+    case ATTN_ERR_CUDA: return "CUDA runtime or launch error";
+    case ATTN_ERR_DEVICE_FAULT: return "device-side fault flagged";
+    case ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    case ATTN_ERR_NO_DEVICE: return "no sm_100 device is current";
+  }
+  return "unknown status";
+}
+
+int attn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,36 @@
+// Internal declarations shared by the C-ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "attn.h"
+
+namespace attn {
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+// Returns ATTN_OK if the current device is sm_100.
+attn_status_t check_device();
+
+// Prefill launcher. Arguments were validated by the caller.
+attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream);
+
+// Decode plan: tokens per split (multiple of 16) and the maximum number of
+// splits a sequence can have.
+struct DecodePlan {
+  int split_tokens;
+  int max_splits;
+  size_t workspace_bytes;
+};
+DecodePlan plan_decode(const attn_decode_params& p);
+
+attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan, void* workspace,
+                            cudaStream_t stream);
+
+attn_status_t launch_combine(const float* part_o, const float* part_lse, int num_splits, int rows,
+                             int head_dim, const int32_t* splits_per_row, const int32_t* seq_lens,
+                             int split_tokens, int rows_per_seq, void* out_o, attn_dtype_t out_dtype,
+                             float* out_lse, cudaStream_t stream);
+
+}  // namespace attn

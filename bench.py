@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+A step is one prefill call over the causal GQA workload (batch 4, 32 query /
+8 key-value heads, 2048 tokens, head_dim 128, bf16, seed 1). The headline
+``value`` is its throughput in TFLOP/s of algorithmic work (4 * head_dim per
+visible query-key pair and query head). The same JSON line also carries the
+paged split-KV decode workload (batch 64, lengths U[1024, 32768], 32/8 heads)
+timed the same way, in GB/s of algorithmic KV traffic.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own full batch (weak scaling, no
+collective on the data path) and rank 0 prints one JSON line with the
+max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_tiled_exact_b200 import workloads as wl  # noqa: E402
+
+METRIC = "attention TFLOP/s (prefill) & KV GB/s (decode), % of B200 roofline"
+PREFILL_CFG = wl.CAUSAL_GQA_2K
+DECODE_CFG = wl.PAGED_DECODE
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {
+    "prefill": ["attention_tiled_exact_b200/csrc/prefill_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
+    "decode": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
+}
+
+
+def kernel_hash(kind: str) -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic(kind: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged since."""
+    path = os.path.join(ROOT, "profiles", f"{kind}_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_sha") != kernel_hash(kind):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.rows.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# workloads on the device
+# ----------------------------------------------------------------------------
+
+
+def _dev_bf16(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def prefill_inputs(rank: int):
+    import dataclasses
+    cfg = dataclasses.replace(PREFILL_CFG, seed=PREFILL_CFG.seed + 1000 * rank)
+    d = wl.make_prefill(cfg)
+    flops = 4.0 * cfg.head_dim * cfg.batch * cfg.q_heads * wl.causal_pairs(cfg.seqlen_q, cfg.seqlen_k, cfg.causal)
+    return cfg, d, flops
+
+
+def decode_inputs(rank: int):
+    import dataclasses
+    cfg = dataclasses.replace(DECODE_CFG, seed=DECODE_CFG.seed + 1000 * rank)
+    d = wl.make_decode(cfg)
+    total_tokens = int(d["kv_lens"].sum())
+    kv_bytes = total_tokens * cfg.kv_heads * cfg.head_dim * 2 * 2
+    io_bytes = cfg.batch * cfg.q_heads * (cfg.head_dim * 2 * 2 + 4)
+    return cfg, d, float(kv_bytes + io_bytes)
+
+
+def time_loop(fn, steps, warmup, world):
+    """CUDA-event time of `steps` back-to-back calls after `warmup` calls (ms per step, max over ranks)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(stop) / steps
+    return max_over_ranks(ms, world)
+
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    from attention_tiled_exact_b200 import binding as attn
+    peaks, peak_src = load_peaks()
+
+    # ---------------- prefill (the headline)
+    cfg, d, flops = prefill_inputs(rank)
+    q, k, v = _dev_bf16(d["q"]), _dev_bf16(d["k"]), _dev_bf16(d["v"])
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+
+    def prefill_step():
+        attn.prefill(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse)
+
+    with ClockSampler(local) as clk:
+        ms = time_loop(prefill_step, args.steps, args.warmup, world)
+    clocks = clk.summary()
+    tflops = flops * world / (ms * 1e-3) / 1e12
+    per_rank_tflops = flops / (ms * 1e-3) / 1e12
+    peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+
+    # e2e through the public call with host buffers: H2D inputs, prefill, D2H output + LSE
+    hq = torch.from_numpy(d["q"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(d["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(d["v"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    ho = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        attn.prefill(q, k, v, cfg.scale, cfg.causal, out=o, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    ms_e2e = time_loop(e2e_step, e2e_steps, 2, world)
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
+    d2h = ho.numel() * 2 + hl.numel() * 4
+    del hq, hk, hv, ho, hl
+
+    # ---------------- decode (secondary), same timing rules
+    dcfg, dd, dbytes = decode_inputs(rank)
+    dq = _dev_bf16(dd["q"])
+    kc, vc = _dev_bf16(dd["k_pool"]), _dev_bf16(dd["v_pool"])
+    bt = torch.from_numpy(dd["block_table"]).cuda()
+    sl = torch.from_numpy(dd["kv_lens"]).cuda()
+    max_len = int(dd["kv_lens"].max())
+    dout = torch.empty_like(dq)
+    dlse = torch.empty(dq.shape[:2], dtype=torch.float32, device="cuda")
+    ws_bytes = attn.decode_workspace_bytes(dq, kc, vc, bt, sl, max_seq_len=max_len)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+
+    def decode_step():
+        attn.decode_paged(dq, kc, vc, bt, sl, dcfg.scale, max_seq_len=max_len, out=dout, lse=dlse, workspace=ws)
+
+    dsteps = max(args.steps, 5)
+    with ClockSampler(local) as dclk:
+        dms = time_loop(decode_step, dsteps, args.warmup, world)
+    peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    dgbs = dbytes * world / (dms * 1e-3) / 1e9
+    per_rank_gbs = dbytes / (dms * 1e-3) / 1e9
+
+    result = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, per-rank seeds)",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "q_heads": cfg.q_heads, "kv_heads": cfg.kv_heads,
+                   "seq_len": cfg.seqlen_q, "head_dim": cfg.head_dim, "causal": cfg.causal,
+                   "parallelism": f"replicas x{world} (no collective)",
+                   "l2": "inputs larger than L2 (Q 64 MiB + K/V 32 MiB + O 64 MiB per step)"},
+        "roofline": {"bound": "tensor", "kernel": "prefill_fwd_kernel<128,4,true>",
+                     "achieved": round(per_rank_tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": round(per_rank_tflops / peak_t, 4),
+                     "peak_source": f"{peak_src} bf16 burst (cuBLAS 8192^3)",
+                     "frac_of_sustained": round(per_rank_tflops / peaks.get("bf16_tflops_sustained", 1400.0), 4),
+                     "traffic": profiled_traffic("prefill"),
+                     "algorithmic_flops_per_launch": flops},
+        "e2e": {"value": round(flops * world / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "decode": {"workload": dcfg.name, "value": round(dgbs, 1), "unit": "GB/s", "ms_per_step": round(dms, 4),
+                   "steps": dsteps, "kv_tokens": int(dd["kv_lens"].sum()),
+                   "roofline": {"bound": "hbm", "achieved": round(per_rank_gbs, 1), "peak": peak_h, "unit": "GB/s",
+                                "frac": round(per_rank_gbs / peak_h, 4), "peak_source": f"{peak_src} copy bandwidth",
+                                "traffic": profiled_traffic("decode"), "algorithmic_bytes_per_launch": dbytes},
+                   "gpu_launches_per_step": 2, "clocks": dclk.summary()},
+    }
+    if rank == 0:
+        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return result
+
+
+# ----------------------------------------------------------------------------
+# the oracle on the host cores
+# ----------------------------------------------------------------------------
+
+
+def cpu_baseline(budget_s: float):
+    """The fp64 oracle as it stands, on whole (batch, head) slices of the prefill workload."""
+    from oracle import attention_ref as ref
+    cfg = PREFILL_CFG
+    d = wl.make_prefill(cfg)
+    G = cfg.q_heads // cfg.kv_heads
+    per_head = 4.0 * cfg.head_dim * wl.causal_pairs(cfg.seqlen_q, cfg.seqlen_k, cfg.causal)
+    done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and done < cfg.batch * cfg.q_heads:
+        b, h = divmod(done, cfg.q_heads)
+        ref.attention_rows(d["q"][b, h], d["k"][b, h // G], d["v"][b, h // G], cfg.scale,
+                           ref.causal_positions(cfg.seqlen_q, cfg.seqlen_k))
+        done += 1
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((x.get("num_threads", 1) for x in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count()
+    return {"value": round(per_head * done / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {cfg.batch * cfg.q_heads} (batch, head) slices of {cfg.name}, fp64, "
+                      f"materialised S, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    per_step_budget = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    from oracle import attention_ref as ref
+    cfg = PREFILL_CFG
+    d = wl.make_prefill(cfg)
+    G = cfg.q_heads // cfg.kv_heads
+    per_head = 4.0 * cfg.head_dim * wl.causal_pairs(cfg.seqlen_q, cfg.seqlen_k, cfg.causal)
+    pos = ref.causal_positions(cfg.seqlen_q, cfg.seqlen_k)
+
+    def step():
+        n, t0 = 0, time.perf_counter()
+        while n == 0 or (time.perf_counter() - t0 < per_step_budget and n < cfg.batch * cfg.q_heads):
+            b, h = divmod(n, cfg.q_heads)
+            ref.attention_rows(d["q"][b, h], d["k"][b, h // G], d["v"][b, h // G], cfg.scale, pos)
+            n += 1
+        return n, time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        step()
+    heads, secs = 0, 0.0
+    for _ in range(args.steps):
+        n, dt = step()
+        heads += n
+        secs += dt
+    value = per_head * heads / secs / 1e12
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((x.get("num_threads", 1) for x in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count()
+    sample = (f"{heads} (batch, head) slices of {cfg.name} over {args.steps} steps "
+              f"(about {per_step_budget:.1f} s each), fp64 oracle")
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "q_heads": cfg.q_heads, "kv_heads": cfg.kv_heads,
+                       "seq_len": cfg.seqlen_q, "head_dim": cfg.head_dim, "causal": cfg.causal},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "kind": "oracle", "cores": threads,
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        res = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

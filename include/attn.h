@@ -1,0 +1,218 @@
+/*
+ * attn.h -- C ABI of libattn_b200.so: exact scaled-dot-product attention on
+ * B200 (sm_100a).
+ *
+ * The operation (all three entry points compute parts of it):
+ *
+ *   O = softmax(Q K^T * scale + causal mask) V,  LSE = ln sum_j exp(scale q.k_j)
+ *
+ * Attention keeps its mathematical definition; tiling, the online softmax and
+ * kernel fusion only change how it is computed ("推理加速" interview notes,
+ * section FlashAttention; "抱infra脚", section Flash Attention 核心技术).
+ * Key/value heads are shared by contiguous groups of G = Hq / Hkv query heads:
+ * query head h reads key/value head h / G ("5.2 推理加速的未来趋势", GQA/MQA).
+ * The causal mask is aligned bottom-right: with Sq queries over Sk keys, query
+ * i sees keys 0 .. i + (Sk - Sq).
+ *
+ * Conventions shared by every call:
+ *  - Element types: Q, K, V and the KV cache are bf16; accumulation is fp32;
+ *    LSE is fp32, natural log; O is bf16 or fp32 (attn_dtype_t).
+ *  - Every pointer is DEVICE memory owned by the caller. The library allocates
+ *    no device memory and keeps no state besides a per-device cache of the SM
+ *    count and of kernel attributes. Host pointers are used only where a
+ *    parameter says "host".
+ *  - Calls are asynchronous and stream-ordered: they validate arguments on the
+ *    host, enqueue kernels on `stream` and return. Nothing synchronises.
+ *  - Errors: a call returns ATTN_OK or an attn_status_t; it never aborts,
+ *    traps or falls back to another implementation. Argument errors are
+ *    detected on the host before anything is enqueued. Faults found on the
+ *    device (a block id outside the pool, a sequence longer than its block
+ *    table, a pipeline wait that ran out of time) skip the affected work and
+ *    OR a bit (ATTN_FAULT_*) into the caller's optional `error_flags` word,
+ *    which the caller reads after synchronising.
+ *  - All entry points are thread-safe; calls on different streams may overlap.
+ */
+#ifndef ATTN_B200_H_
+#define ATTN_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* attn_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent shapes */
+  ATTN_ERR_UNSUPPORTED = 2,   /* head_dim not 64/128, Hq % Hkv != 0, misaligned pointer/stride */
+  ATTN_ERR_WORKSPACE = 3,     /* workspace too small; *workspace_needed says how much */
+  ATTN_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  ATTN_ERR_DEVICE_FAULT = 5,  /* reserved for callers mapping error_flags to a status */
+  ATTN_ERR_TIMEOUT = 6,       /* reserved for callers mapping error_flags to a status */
+  ATTN_ERR_NO_DEVICE = 7      /* no sm_100 device is current */
+} attn_status_t;
+
+typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1 } attn_dtype_t;
+
+/* Bits a kernel ORs into *error_flags. */
+#define ATTN_FAULT_TIMEOUT 0x1      /* a pipeline wait exceeded its bound; the tile was abandoned */
+#define ATTN_FAULT_BAD_BLOCK 0x2    /* a block-table entry was outside [0, num_blocks) */
+#define ATTN_FAULT_BAD_LENGTH 0x4   /* a sequence length exceeded its block table or was negative */
+
+/*
+ * Prefill: tiled attention over a whole query block, one pass over K/V with
+ * the online softmax (running row max and row sum, rescaled as the max grows)
+ * and only O and LSE written back ("推理加速", FlashAttention 的核心思路 flow:
+ * tile Q/K/V, load tiles on chip, attend per tile, online softmax, write the
+ * final output only; "GPU Kernel 调度:大模型推理的拐点 2026", FlashAttention-3
+ * paragraph: Q tiles in parallel, K/V tiles pipelined, producer/consumer roles).
+ *
+ * Layout (element strides; the last dimension, head_dim, is contiguous):
+ *   q [batch, num_q_heads, seqlen_q, head_dim] bf16, strides q_*_stride
+ *   k, v [batch, num_kv_heads, seqlen_k, head_dim] bf16, strides k_*_stride and v_*_stride
+ *   o [batch, num_q_heads, seqlen_q, head_dim] o_dtype, strides o_*_stride
+ *   lse [batch, num_q_heads, seqlen_q] fp32, contiguous; may be NULL
+ * Requirements: head_dim in {64, 128}; num_q_heads % num_kv_heads == 0;
+ * q/k/v base pointers 16-byte aligned and their batch/head/row strides
+ * multiples of 8 elements (16 bytes); o 16-byte aligned with strides that are
+ * multiples of 8 elements; seqlen_q, seqlen_k >= 0 (k and v may be NULL when
+ * seqlen_k == 0: every row then gets O = 0, LSE = -inf); scale > 0 and finite.
+ *
+ * Paged keys/values (chunked prefill over a KV cache, "抱infra脚" Chunked
+ * Prefill and Paged Attention): set k_cache/v_cache non-NULL (then k and v
+ * must be NULL). Sequence b then has seqlens_k[b] keys, token t stored at
+ * k_cache[block_table[b * max_blocks_per_seq + t / block_size], kvh,
+ * t % block_size, :]; the pools are contiguous
+ * [num_blocks, num_kv_heads, block_size, head_dim] with block_size == 16.
+ * seqlens_q (device, [batch], nullable) gives the valid query rows of each
+ * sequence (<= seqlen_q; rows past it are not written); seqlens_k (device,
+ * [batch]) is required in paged mode and each entry must be <=
+ * max_blocks_per_seq * block_size; seqlen_k must then be the maximum of
+ * seqlens_k (an upper bound is fine). The causal alignment uses the
+ * per-sequence lengths.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int batch;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int seqlen_q;
+  int seqlen_k;
+  int64_t q_batch_stride, q_head_stride, q_row_stride;
+  int64_t k_batch_stride, k_head_stride, k_row_stride;
+  int64_t v_batch_stride, v_head_stride, v_row_stride;
+  int64_t o_batch_stride, o_head_stride, o_row_stride;
+  float scale;
+  int causal;
+  attn_dtype_t o_dtype;
+  /* optional per-sequence lengths / paged KV */
+  const int32_t* seqlens_q;
+  const int32_t* seqlens_k;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_table;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int block_size;
+  int32_t* error_flags; /* nullable */
+} attn_prefill_params;
+
+ATTN_API attn_status_t attn_prefill(const attn_prefill_params* p, attn_stream_t stream);
+
+/*
+ * Paged decode (Flash-Decoding): one query token per sequence against its
+ * whole cached context, with the key range cut into splits that run on
+ * different SMs; each split produces a partial output and its log-sum-exp in
+ * fp32, and a small combine kernel merges them ("GPU Kernel 调度:大模型推理的
+ * 拐点 2026", Flash Decoding section; "抱infra脚", Paged Attention: fixed-size
+ * blocks mapped through a block table).
+ *
+ * Layout:
+ *   q [batch, num_q_heads, head_dim] bf16, contiguous
+ *   k_cache, v_cache [num_blocks, num_kv_heads, block_size, head_dim] bf16, contiguous
+ *   block_table [batch, max_blocks_per_seq] int32 (device), row-major
+ *   seq_lens [batch] int32 (device): keys of each sequence, all visible
+ *   o [batch, num_q_heads, head_dim] o_dtype, contiguous
+ *   lse [batch, num_q_heads] fp32, nullable
+ * Requirements: block_size == 16; head_dim == 128; num_q_heads % num_kv_heads
+ * == 0 and num_q_heads / num_kv_heads in {1, 2, 4, 8}; 16-byte aligned
+ * pointers. max_seq_len (host) is an upper bound on seq_lens (0 = use the
+ * table capacity max_blocks_per_seq * block_size); it only sizes the split
+ * plan. num_splits: 0 = automatic, otherwise the number of splits a sequence
+ * of max_seq_len keys is cut into (1 = no split: the partials step is
+ * skipped and the combine is not launched).
+ *
+ * Workspace: device memory of at least *workspace_needed bytes, 256-byte
+ * aligned, owned by the caller, holding the fp32 partials. Pass workspace =
+ * NULL to only query the size (returns ATTN_OK, enqueues nothing). If
+ * workspace_bytes is too small the call returns ATTN_ERR_WORKSPACE and
+ * enqueues nothing. A sequence with 0 keys gets O = 0 and LSE = -inf.
+ */
+typedef struct {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  void* o;
+  float* lse;
+  int batch;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int block_size;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int max_seq_len;
+  int num_splits;
+  float scale;
+  attn_dtype_t o_dtype;
+  int32_t* error_flags; /* nullable */
+} attn_decode_params;
+
+ATTN_API attn_status_t attn_decode_paged(const attn_decode_params* p, void* workspace, size_t workspace_bytes,
+                                size_t* workspace_needed, attn_stream_t stream);
+
+/*
+ * Split-KV log-sum-exp combine ("GPU Kernel 调度:大模型推理的拐点 2026",
+ * Flash Decoding section: partials merged with the online-softmax formula,
+ * each carrying a log-sum-exp accumulated in FP32). For each row r:
+ *   n = splits_per_row ? splits_per_row[r] : num_splits   (0 <= n <= num_splits)
+ *   M = max_{s<n} part_lse[s][r];  LSE = M + ln sum_{s<n} exp(part_lse[s][r] - M)
+ *   O[r] = sum_{s<n} exp(part_lse[s][r] - LSE) * part_o[s][r][:]
+ * A split with LSE = -inf has weight 0 (its part_o is not read); a row with
+ * no finite LSE gets O = 0, LSE = -inf.
+ * Layout: part_o [num_splits, rows, head_dim] fp32, part_lse [num_splits, rows]
+ * fp32, splits_per_row [rows] int32 (device, nullable), out_o [rows, head_dim]
+ * in out_dtype, out_lse [rows] fp32 (nullable). head_dim in {64, 128};
+ * 16-byte aligned pointers.
+ */
+ATTN_API attn_status_t splitkv_lse_combine(const float* part_o, const float* part_lse, int num_splits, int rows,
+                                  int head_dim, const int32_t* splits_per_row, void* out_o,
+                                  attn_dtype_t out_dtype, float* out_lse, attn_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+ATTN_API const char* attn_status_string(attn_status_t status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+ATTN_API int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H_ */

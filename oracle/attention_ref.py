@@ -235,9 +235,10 @@ def combine_partials(part_o, part_lse, splits_per_row=None):
         lse = pl[:n, r]
         if n == 0 or not np.isfinite(lse).any():
             continue
-        M = lse.max()
-        w = np.exp(lse - M)
+        keep = np.isfinite(lse)  # an empty split (LSE = -inf) has weight 0; its output is not read
+        M = lse[keep].max()
+        w = np.exp(lse[keep] - M)
         L[r] = M + np.log(w.sum())
-        wn = np.exp(lse - L[r])
-        O[r] = (wn[:, None] * po[:n, r]).sum(axis=0)
+        wn = np.exp(lse[keep] - L[r])
+        O[r] = (wn[:, None] * po[:n, r][keep]).sum(axis=0)
     return O, L

@@ -1,0 +1,151 @@
+"""Prefill parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Sizes are small enough for the oracle to finish in seconds but span several
+128-row / 128-key tiles with ragged tails; the full-size workloads are checked
+on sampled rows in the launch configuration the bench times.
+"""
+import os
+
+import numpy as np
+import pytest
+
+from attention_tiled_exact_b200 import workloads as wl
+from oracle import attention_ref as ref
+from tests.helpers import assert_lse_close, assert_o_close, to_dev_bf16, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(lib, d, out_dtype=None, p_smem=False, **kw):
+    import torch
+    q, k, v = to_dev_bf16(d["q"]), to_dev_bf16(d["k"]), to_dev_bf16(d["v"])
+    old = os.environ.get("ATTN_PREFILL_P_SMEM")
+    os.environ["ATTN_PREFILL_P_SMEM"] = "1" if p_smem else "0"
+    try:
+        o, lse = lib.prefill(q, k, v, d["scale"], d["causal"], out_dtype=out_dtype or torch.bfloat16, **kw)
+        torch.cuda.synchronize()
+    finally:
+        if old is None:
+            del os.environ["ATTN_PREFILL_P_SMEM"]
+        else:
+            os.environ["ATTN_PREFILL_P_SMEM"] = old
+    return to_f64(o), to_f64(lse)
+
+
+def _case(B, Hq, Hkv, Sq, Sk, D, causal, seed):
+    cfg = wl.PrefillConfig("t", B, Hq, Hkv, Sq, Sk, D, causal, seed)
+    return wl.make_prefill(cfg)
+
+
+def test_tiny_config_with_lse(lib):
+    """1 x 1 x 128 x 64, non-causal, scale 1/8, seed 0; O and the per-row LSE."""
+    import torch
+    d = wl.make_prefill(wl.TINY)
+    O_ref, L_ref = ref.ref_attention(d["q"], d["k"], d["v"], d["scale"], d["causal"])
+    for dt in (torch.bfloat16, torch.float32):
+        o, lse = _run(lib, d, out_dtype=dt)
+        assert_o_close(o, O_ref, dt == torch.bfloat16, "tiny")
+        assert_lse_close(lse, L_ref, "tiny")
+
+
+CASES = [
+    # B, Hq, Hkv, Sq, Sk, D, causal
+    (2, 8, 2, 300, 300, 128, True),     # GQA G=4, ragged third tile
+    (1, 4, 1, 256, 256, 128, True),     # MQA, exact tiles
+    (1, 2, 2, 257, 257, 128, True),     # MHA (G=1: row-block pairs, odd count of row blocks)
+    (1, 6, 2, 200, 333, 64, False),     # G=3 (odd), non-causal, Sk != Sq
+    (1, 16, 2, 130, 400, 128, True),    # G=8, bottom-right causal with Sq < Sk
+    (1, 4, 2, 300, 100, 128, True),     # Sq > Sk: the first 200 rows see no key
+    (2, 4, 4, 1, 700, 128, True),       # a single query row
+    (1, 4, 2, 513, 129, 64, False),     # D=64, ragged keys
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal", CASES)
+def test_prefill_matches_oracle(lib, B, Hq, Hkv, Sq, Sk, D, causal):
+    import torch
+    d = _case(B, Hq, Hkv, Sq, Sk, D, causal, seed=100 + Sq + Sk + D)
+    O_ref, L_ref = ref.ref_attention(d["q"], d["k"], d["v"], d["scale"], causal)
+    o, lse = _run(lib, d, out_dtype=torch.float32)
+    assert_o_close(o, O_ref, False, "fp32 out")
+    assert_lse_close(lse, L_ref, "lse")
+    o16, lse16 = _run(lib, d)
+    assert_o_close(o16, O_ref, True, "bf16 out")
+    assert np.array_equal(lse16, lse)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal", [CASES[0], CASES[3], CASES[5]])
+def test_p_in_shared_memory_variant_agrees(lib, B, Hq, Hkv, Sq, Sk, D, causal):
+    """The variant that stages P in shared memory (a different layout path) matches too."""
+    import torch
+    d = _case(B, Hq, Hkv, Sq, Sk, D, causal, seed=7 + Sq)
+    O_ref, L_ref = ref.ref_attention(d["q"], d["k"], d["v"], d["scale"], causal)
+    o, lse = _run(lib, d, out_dtype=torch.float32, p_smem=True)
+    assert_o_close(o, O_ref, False, "P in smem")
+    assert_lse_close(lse, L_ref, "P in smem")
+
+
+def test_no_keys_gives_zero_and_minus_inf(lib):
+    import torch
+    d = _case(1, 2, 1, 64, 0, 128, False, seed=3)
+    d["k"] = d["k"][:, :, :0]
+    d["v"] = d["v"][:, :, :0]
+    q = to_dev_bf16(d["q"])
+    k = torch.empty((1, 1, 0, 128), dtype=torch.bfloat16, device="cuda")
+    o, lse = lib.prefill(q, k, k, d["scale"], False, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert (to_f64(o) == 0).all() and np.isneginf(to_f64(lse)).all()
+
+
+def test_strided_inputs(lib):
+    """Q/K/V/O as [B, S, H, D] buffers viewed as [B, H, S, D] (non-contiguous strides)."""
+    import torch
+    d = _case(2, 4, 2, 190, 190, 128, True, seed=11)
+    O_ref, L_ref = ref.ref_attention(d["q"], d["k"], d["v"], d["scale"], True)
+    q = to_dev_bf16(np.ascontiguousarray(d["q"].transpose(0, 2, 1, 3))).transpose(1, 2)
+    k = to_dev_bf16(np.ascontiguousarray(d["k"].transpose(0, 2, 1, 3))).transpose(1, 2)
+    v = to_dev_bf16(np.ascontiguousarray(d["v"].transpose(0, 2, 1, 3))).transpose(1, 2)
+    out = torch.empty((2, 190, 4, 128), dtype=torch.float32, device="cuda").transpose(1, 2)
+    o, lse = lib.prefill(q, k, v, d["scale"], True, out=out)
+    torch.cuda.synchronize()
+    assert_o_close(to_f64(o), O_ref, False, "strided")
+    assert_lse_close(to_f64(lse), L_ref, "strided")
+
+
+def test_repeated_calls_are_deterministic(lib):
+    d = _case(1, 8, 2, 384, 384, 128, True, seed=5)
+    o1, l1 = _run(lib, d)
+    o2, l2 = _run(lib, d)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_error_word_stays_clear(lib):
+    import torch
+    d = _case(1, 4, 2, 256, 256, 128, True, seed=6)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, k, v = to_dev_bf16(d["q"]), to_dev_bf16(d["k"]), to_dev_bf16(d["v"])
+    lib.prefill(q, k, v, d["scale"], True, error_flags=flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+
+
+def _sampled_rows(cfg, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = [(0, 0, 0), (cfg.batch - 1, cfg.q_heads - 1, cfg.seqlen_q - 1), (0, 1, 127), (0, 2, 128)]
+    for _ in range(n):
+        rows.append((int(rng.integers(cfg.batch)), int(rng.integers(cfg.q_heads)), int(rng.integers(cfg.seqlen_q))))
+    return rows
+
+
+@pytest.mark.parametrize("cfg", [wl.CAUSAL_GQA_2K, wl.CAUSAL_GQA_16K], ids=lambda c: c.name)
+def test_full_size_sampled_rows(lib, cfg):
+    """Full-size workloads in the bench's launch configuration, checked on sampled rows."""
+    d = wl.make_prefill(cfg)
+    o, lse = _run(lib, d)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    rows = _sampled_rows(cfg, 60, cfg.seed)
+    O_ref, L_ref = ref.ref_attention(d["q"], d["k"], d["v"], d["scale"], cfg.causal, rows=rows)
+    og = np.stack([o[b, h, i] for b, h, i in rows])
+    lg = np.array([lse[b, h, i] for b, h, i in rows])
+    assert_o_close(og, O_ref, True, cfg.name)
+    assert_lse_close(lg, L_ref, cfg.name)

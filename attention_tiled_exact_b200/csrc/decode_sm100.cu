@@ -373,9 +373,10 @@ __global__ void __launch_bounds__(WARPS * 32)
 // ---------------------------------------------------------------------------
 namespace combine {
 
-// One warp per row. Row r's split count comes from splits_per_row, or (decode
-// path) from its sequence length: n = max(1, ceil(L / split_tokens)); rows
-// with n == 1 were written by the decode kernel and are skipped there.
+// One warp per row. Row r's split count is splits_per_row[r] when given,
+// else num_splits when seq_lens is NULL (standalone call), else (decode path)
+// n = max(1, ceil(L / split_tokens)) from its sequence length; on the decode
+// path rows with n == 1 were written by the decode kernel and are skipped.
 template <int HD>
 __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restrict__ part_o,
                                                           const float* __restrict__ part_lse, int num_splits,
@@ -388,9 +389,11 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restric
   const int lane = lane_id();
   if (row >= rows) return;
   int n;
-  if (splits_per_row) {
+  if (splits_per_row) {  // standalone call with per-row counts
     n = min(max(splits_per_row[row], 0), num_splits);
-  } else {
+  } else if (seq_lens == nullptr) {  // standalone call: every row has num_splits partials
+    n = num_splits;
+  } else {  // decode path
     int L = seq_lens[row / rows_per_seq];
     L = min(max(L, 0), max_len);
     n = max(1, (L + split_tokens - 1) / split_tokens);

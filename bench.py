@@ -151,7 +151,8 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -174,9 +175,10 @@ def prefill_inputs(rank: int):
     return cfg, d, flops
 
 
-def decode_inputs(rank: int):
+def decode_inputs(rank: int, batch: int = 0):
     import dataclasses
-    cfg = dataclasses.replace(DECODE_CFG, seed=DECODE_CFG.seed + 1000 * rank)
+    cfg = dataclasses.replace(DECODE_CFG, seed=DECODE_CFG.seed + 1000 * rank,
+                              batch=batch if batch > 0 else DECODE_CFG.batch)
     d = wl.make_decode(cfg)
     total_tokens = int(d["kv_lens"].sum())
     kv_bytes = total_tokens * cfg.kv_heads * cfg.head_dim * 2 * 2
@@ -211,7 +213,20 @@ def run_ours(args, rank, world, local):
     from attention_tiled_exact_b200 import binding as attn
     peaks, peak_src = load_peaks()
 
-    # ---------------- prefill (the headline)
+    result = {}
+    if args.only in (None, "prefill"):
+        result.update(bench_prefill(args, rank, world, local, attn, peaks, peak_src))
+    if args.only in (None, "decode"):
+        result["decode"] = bench_decode(args, rank, world, local, attn, peaks, peak_src)
+    if args.only is not None:
+        result["partial"] = f"--only {args.only}: profiling run, not a bench line"
+    if rank == 0 and args.only is None:
+        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return result
+
+
+def bench_prefill(args, rank, world, local, attn, peaks, peak_src):
+    import torch
     cfg, d, flops = prefill_inputs(rank)
     q, k, v = _dev_bf16(d["q"]), _dev_bf16(d["k"]), _dev_bf16(d["v"])
     o = torch.empty_like(q)
@@ -242,33 +257,14 @@ def run_ours(args, rank, world, local):
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
-    e2e_steps = max(3, min(args.steps, 10))
-    ms_e2e = time_loop(e2e_step, e2e_steps, 2, world)
+    if args.only is None:
+        e2e_steps = max(3, min(args.steps, 10))
+        ms_e2e = time_loop(e2e_step, e2e_steps, 2, world)
+    else:
+        ms_e2e = float("nan")
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
     d2h = ho.numel() * 2 + hl.numel() * 4
     del hq, hk, hv, ho, hl
-
-    # ---------------- decode (secondary), same timing rules
-    dcfg, dd, dbytes = decode_inputs(rank)
-    dq = _dev_bf16(dd["q"])
-    kc, vc = _dev_bf16(dd["k_pool"]), _dev_bf16(dd["v_pool"])
-    bt = torch.from_numpy(dd["block_table"]).cuda()
-    sl = torch.from_numpy(dd["kv_lens"]).cuda()
-    max_len = int(dd["kv_lens"].max())
-    dout = torch.empty_like(dq)
-    dlse = torch.empty(dq.shape[:2], dtype=torch.float32, device="cuda")
-    ws_bytes = attn.decode_workspace_bytes(dq, kc, vc, bt, sl, max_seq_len=max_len)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
-
-    def decode_step():
-        attn.decode_paged(dq, kc, vc, bt, sl, dcfg.scale, max_seq_len=max_len, out=dout, lse=dlse, workspace=ws)
-
-    dsteps = max(args.steps, 5)
-    with ClockSampler(local) as dclk:
-        dms = time_loop(decode_step, dsteps, args.warmup, world)
-    peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    dgbs = dbytes * world / (dms * 1e-3) / 1e9
-    per_rank_gbs = dbytes / (dms * 1e-3) / 1e9
 
     result = {
         "metric": METRIC,
@@ -298,16 +294,40 @@ def run_ours(args, rank, world, local):
                 "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,
         "clocks": clocks,
-        "decode": {"workload": dcfg.name, "value": round(dgbs, 1), "unit": "GB/s", "ms_per_step": round(dms, 4),
-                   "steps": dsteps, "kv_tokens": int(dd["kv_lens"].sum()),
-                   "roofline": {"bound": "hbm", "achieved": round(per_rank_gbs, 1), "peak": peak_h, "unit": "GB/s",
-                                "frac": round(per_rank_gbs / peak_h, 4), "peak_source": f"{peak_src} copy bandwidth",
-                                "traffic": profiled_traffic("decode"), "algorithmic_bytes_per_launch": dbytes},
-                   "gpu_launches_per_step": 2, "clocks": dclk.summary()},
     }
-    if rank == 0:
-        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return result
+
+
+def bench_decode(args, rank, world, local, attn, peaks, peak_src):
+    import torch
+    dcfg, dd, dbytes = decode_inputs(rank, args.decode_batch)
+    dq = _dev_bf16(dd["q"])
+    kc, vc = _dev_bf16(dd["k_pool"]), _dev_bf16(dd["v_pool"])
+    bt = torch.from_numpy(dd["block_table"]).cuda()
+    sl = torch.from_numpy(dd["kv_lens"]).cuda()
+    max_len = int(dd["kv_lens"].max())
+    dout = torch.empty_like(dq)
+    dlse = torch.empty(dq.shape[:2], dtype=torch.float32, device="cuda")
+    ws_bytes = attn.decode_workspace_bytes(dq, kc, vc, bt, sl, max_seq_len=max_len)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+
+    def decode_step():
+        attn.decode_paged(dq, kc, vc, bt, sl, dcfg.scale, max_seq_len=max_len, out=dout, lse=dlse, workspace=ws)
+
+    dsteps = max(args.steps, 5)
+    with ClockSampler(local) as dclk:
+        dms = time_loop(decode_step, dsteps, args.warmup, world)
+    peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    dgbs = dbytes * world / (dms * 1e-3) / 1e9
+    per_rank_gbs = dbytes / (dms * 1e-3) / 1e9
+
+    return {"workload": dcfg.name, "value": round(dgbs, 1), "unit": "GB/s", "ms_per_step": round(dms, 4),
+            "steps": dsteps, "kv_tokens": int(dd["kv_lens"].sum()),
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<4>", "achieved": round(per_rank_gbs, 1),
+                         "peak": peak_h, "unit": "GB/s", "frac": round(per_rank_gbs / peak_h, 4),
+                         "peak_source": f"{peak_src} copy bandwidth", "traffic": profiled_traffic("decode"),
+                         "algorithmic_bytes_per_launch": dbytes},
+            "gpu_launches_per_step": 2, "clocks": dclk.summary()}
 
 
 # ----------------------------------------------------------------------------
@@ -391,6 +411,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="profiling aid: run one workload only (the line is then marked partial)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="profiling aid: fewer decode sequences (default: the full 64)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

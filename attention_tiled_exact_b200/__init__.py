@@ -11,7 +11,7 @@ The library is loaded on first use of one of these names; if it is missing
 the import fails with an error that says how to build it. There is no CPU
 fallback.
 """
-_API = ("prefill", "decode_paged", "splitkv_lse_combine", "decode_workspace_bytes",
+_API = ("prefill", "decode_paged", "decode_paged_noalloc", "splitkv_lse_combine", "decode_workspace_bytes",
         "AttnError", "library_path", "status_string")
 
 

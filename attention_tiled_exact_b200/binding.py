@@ -81,6 +81,8 @@ def _load():
     lib.attn_decode_paged.argtypes = [ctypes.POINTER(DecodeParams), _vp, ctypes.c_size_t,
                                       ctypes.POINTER(ctypes.c_size_t), _vp]
     lib.attn_decode_paged.restype = ctypes.c_int
+    lib.attn_decode_paged_noalloc.argtypes = [ctypes.POINTER(DecodeParams), _vp]
+    lib.attn_decode_paged_noalloc.restype = ctypes.c_int
     lib.splitkv_lse_combine.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp,
                                         ctypes.c_int, _vp, _vp]
     lib.splitkv_lse_combine.restype = ctypes.c_int
@@ -234,6 +236,29 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(LIB.attn_decode_paged(ctypes.byref(p), ws_ptr, ws_bytes, None, _stream(q.device)),
            "attn_decode_paged")
+    return out, lse
+
+
+def decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, out, lse=None, scale: float | None = None,
+                         max_seq_len: int = 0, num_splits: int = 0, error_flags=None):
+    """:func:`decode_paged` for callers that cannot allocate device memory.
+
+    The caller passes every input and the outputs (``out`` [B,Hq,D] bf16 or
+    fp32, ``lse`` [B,Hq] fp32 or None); the split partials go to a fixed 16 MiB
+    array that the library owns on each GPU, so nothing is allocated here or in
+    the library. Calls that overlap on the GPU race on that array.
+    """
+    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
+    _need(q.dtype == torch.bfloat16 and k_cache.dtype == torch.bfloat16 and v_cache.dtype == torch.bfloat16,
+          "bf16 q and caches")
+    _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
+    _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
+          "int32 block table [B, max_blocks]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "int32 seq_lens [B]")
+    _need(out is not None and tuple(out.shape) == tuple(q.shape) and out.is_contiguous(), "out [B, Hq, D]")
+    p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits, out, lse,
+                       error_flags)
+    _check(LIB.attn_decode_paged_noalloc(ctypes.byref(p), _stream(q.device)), "attn_decode_paged_noalloc")
     return out, lse
 
 

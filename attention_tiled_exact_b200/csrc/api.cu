@@ -77,7 +77,7 @@ static attn_status_t validate_prefill(const attn_prefill_params* p) {
   return ATTN_OK;
 }
 
-static attn_status_t validate_decode(const attn_decode_params* p) {
+attn_status_t validate_decode(const attn_decode_params* p) {
   if (!p) return ATTN_ERR_INVALID_ARG;
   if (p->batch < 0 || p->batch > 65535) return ATTN_ERR_INVALID_ARG;
   if (p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->num_kv_heads > 65535) return ATTN_ERR_INVALID_ARG;

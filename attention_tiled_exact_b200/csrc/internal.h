@@ -13,6 +13,9 @@ int device_sm_count();
 // Returns ATTN_OK if the current device is sm_100.
 attn_status_t check_device();
 
+// Host-side argument checks of attn_decode_paged (ATTN_OK when valid).
+attn_status_t validate_decode(const attn_decode_params* p);
+
 // Prefill launcher. Arguments were validated by the caller.
 attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream);
 

@@ -188,6 +188,26 @@ ATTN_API attn_status_t attn_decode_paged(const attn_decode_params* p, void* work
                                 size_t* workspace_needed, attn_stream_t stream);
 
 /*
+ * attn_decode_paged without a workspace argument, for callers that cannot
+ * allocate device memory: a host program that only receives tensor pointers
+ * from another component and has no allocator of its own to pass through this
+ * C ABI, or a latency-critical loop that must not call cudaMalloc (which can
+ * synchronise the device). The pages have no counterpart to this call; it is a
+ * deployment convenience, not part of the method.
+ * Same parameters and results as attn_decode_paged. The split partials live in
+ * a 16 MiB array of device memory owned by the library (held on every GPU that
+ * loads the library until the process exits); nothing is allocated per call.
+ * If the split plan for these shapes needs more than 16 MiB (as
+ * attn_decode_paged would report through workspace_needed), the call returns
+ * ATTN_ERR_WORKSPACE and enqueues nothing; a smaller num_splits lowers the need.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls share the one array: calls whose kernels overlap on the
+ * GPU, e.g. on two streams, race and must be serialised by the caller.
+ */
+ATTN_API attn_status_t attn_decode_paged_noalloc(const attn_decode_params* p, attn_stream_t stream);
+
+/*
  * Split-KV log-sum-exp combine ("GPU Kernel 调度:大模型推理的拐点 2026",
  * Flash Decoding section: partials merged with the online-softmax formula,
  * each carrying a log-sum-exp accumulated in FP32). For each row r:

@@ -11,28 +11,33 @@
 // a producer, with the matrix products and the softmax in different warps
 // ("GPU Kernel 调度:大模型推理的拐点 2026", FlashAttention-2/3 paragraph).
 //
-// B200 design (one CTA per SM, 320 threads):
+// B200 design (one CTA per SM, 384 threads = three warpgroups):
 //   * two Q tiles of 128 rows per CTA. For GQA with an even group size the two
 //     tiles are two query heads of one key/value head on the same rows, so both
-//     tiles need exactly the same K/V range; otherwise they are two row blocks
-//     of one head. K/V tiles are loaded once for both.
-//   * warp 8 (TMA): loads the Q tiles and streams K_j, V_j tiles (128 keys)
-//     into a ring of shared-memory slots with cp.async.bulk.tensor, 128-byte
-//     swizzle, completion on mbarriers.
-//   * warp 9 (MMA): one thread issues tcgen05.mma. S_t = Q_t K_j^T (M=128,
-//     N=128, K=head_dim) lands in tensor memory; O_t += P_t V_j reads P_t from
-//     tensor memory (or shared memory in the reference variant) and V_j from
-//     shared memory. The issue order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1) lets
-//     one tile's softmax overlap the other tile's matrix products.
+//     tiles need exactly the same key range; otherwise they are two row blocks
+//     of one head. Every K/V block is loaded once for both tiles.
+//   * keys advance in blocks of 64. Each tile owns 128 TMEM columns for S,
+//     used as two 64-column halves: S of block i lands in half i % 2, so the
+//     scores of block i+1 are computed while the softmax works on block i and
+//     the softmax does not wait for the tensor core. P (bf16 pairs) overwrites
+//     the first 32 columns of its half and feeds the P V product from TMEM.
+//   * warp 8 (TMA): loads the Q tiles and streams K and V blocks into two
+//     shared-memory rings (128-byte swizzle), K two blocks ahead of V.
+//   * warps 9 and 10 (MMA): one thread per tile issues that tile's
+//     tcgen05.mma instructions. Per block i: O_t += P_t(i) V_i (A from TMEM),
+//     then S_t(i+2) = Q_t K_{i+2}^T into the half P_t(i) just vacated (MMAs
+//     from one thread execute in issue order; the two tiles share nothing in
+//     TMEM). Two issuers on different SM sub-partitions keep MMA issue from
+//     being starved by the busy softmax warps that share each sub-partition.
 //   * warps 0-3 / 4-7 (softmax, one warpgroup per tile, one thread per row):
-//     read S from tensor memory, mask (diagonal and tail tiles only), update the
-//     running max, p = 2^(s*scale*log2e - m), running sum, write P (bf16) back
-//     to tensor memory, and rescale O in tensor memory when the max grew by
-//     more than 2^8 (otherwise the stale max is kept, which leaves O and the
-//     row sum consistent). The same warps run the epilogue: O / l -> global,
+//     read S, mask (diagonal and tail blocks only), update the running max,
+//     p = 2^(s*scale*log2e - m), running sum, write P to TMEM. The running max
+//     is only moved when it grows by more than 2^8 (which keeps O and the row
+//     sum consistent); then O is rescaled in TMEM after the previous P V has
+//     completed. The same warps run the epilogue: O / l -> global,
 //     LSE = (m + log2 l) * ln 2.
-//   * tensor memory: S_0 cols [0,128), S_1 [128,256), O_0 [256,256+D),
-//     O_1 [384,384+D); P_t (bf16 pairs) overwrites the first 64 columns of S_t.
+//   * TMEM: S_0 / P_0 cols [0,128), S_1 / P_1 [128,256), O_0 [256,256+D),
+//     O_1 [384,384+D).
 //   * every mbarrier wait is bounded; on a timeout the CTA raises a flag in
 //     shared memory, all roles stop, in-flight copies and MMAs are drained
 //     (again bounded), tensor memory is freed, and ATTN_FAULT_TIMEOUT is ORed
@@ -41,6 +46,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "internal.h"
@@ -50,10 +56,23 @@ namespace attn {
 namespace prefill {
 
 constexpr int BM = 128;            // query rows per Q tile
-constexpr int BN = 128;            // keys per K/V tile
-constexpr int NUM_THREADS = 320;   // 8 softmax warps + TMA warp + MMA warp
+constexpr int BK = 64;             // keys per block
+constexpr int NUM_THREADS = 384;   // warpgroups: softmax tile 0, softmax tile 1, {TMA, MMA 0, MMA 1, idle}
+constexpr int SOFTMAX_WARPS = 8;
 constexpr int TMA_WARP = 8;
-constexpr int MMA_WARP = 9;
+constexpr int MMA_WARP = 9;        // issues tile 0's MMAs (and owns the TMEM allocation)
+constexpr int MMA1_WARP = 10;      // issues tile 1's MMAs
+constexpr int KSTAGES = 4;         // K blocks in flight
+constexpr int VSTAGES = 4;         // V blocks in flight
+// Register split. The block is launched with REG_LAUNCH registers per thread
+// (384 threads x 168 = 64512 registers); the third warpgroup gives registers
+// back and the two softmax warpgroups take them: 2*128*216 + 128*72 = 64512.
+// The host refuses to launch unless the compiled kernel uses exactly
+// REG_LAUNCH registers, so the split can never ask for more than the block has.
+constexpr int REG_LAUNCH = 168;
+constexpr int REG_SOFTMAX = 216;
+constexpr int REG_OTHER = 72;
+static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER == NUM_THREADS * REG_LAUNCH, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_LIMIT = 2000000000LL;  // cycles (~1 s)
 constexpr float RESCALE_THRESHOLD = 8.0f;        // log2 units: rescale only when the max grows by > 2^8
@@ -70,26 +89,21 @@ struct Args {
   float* lse;
   int o_f32;
   long long o_bs, o_hs, o_rs;
-  // paged keys/values
-  int paged;
-  const int32_t* block_table;
-  int max_blocks_per_seq;
-  int num_blocks;
   int32_t* error_flags;
 };
 
-template <int D, int NSTAGE, bool P_TMEM>
+template <int D>
 struct Layout {
-  static constexpr int CHUNKS = D / 64;               // 64-column (128-byte) boxes per row
-  static constexpr int Q_TILE = BM * D * 2;           // bytes
-  static constexpr int KV_TILE = BN * D * 2;
-  static constexpr int P_TILE = BM * BN * 2;
+  static constexpr int CHUNKS = D / 64;           // 64-column (128-byte) boxes per row
+  static constexpr int Q_TILE = BM * D * 2;       // bytes
+  static constexpr int KV_TILE = BK * D * 2;
   static constexpr int Q_OFF = 0;
-  static constexpr int KV_OFF = Q_OFF + 2 * Q_TILE;
-  static constexpr int P_OFF = KV_OFF + NSTAGE * KV_TILE;
-  static constexpr int BAR_OFF = P_OFF + (P_TMEM ? 0 : 2 * P_TILE);
-  // barriers: q_full, kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2], p_full[2], o_full[2], mma_done
-  static constexpr int NUM_BARS = 1 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+  static constexpr int K_OFF = Q_OFF + 2 * Q_TILE;
+  static constexpr int V_OFF = K_OFF + KSTAGES * KV_TILE;
+  static constexpr int BAR_OFF = V_OFF + VSTAGES * KV_TILE;
+  // q_full, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2][2], p_full[2][2], o_ready[2], o_full[2],
+  // mma_done
+  static constexpr int NUM_BARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 4 + 4 + 2 + 2 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM_BYTES = BYTES + 1024;  // slack for 1024-byte alignment
@@ -100,7 +114,7 @@ struct Work {
   int head[2];
   int row0[2];
   int active[2];
-  int n_kv[2];
+  int n_kv[2];  // key blocks of BK each
   int sq, sk;
 };
 
@@ -143,25 +157,111 @@ __device__ __forceinline__ Work decode_work(const Args& a, int item) {
       const int lim = last_row + (w.sk - w.sq) + 1;  // keys [0, lim) visible to the tile's last row
       kend = max(0, min(w.sk, lim));
     }
-    w.n_kv[t] = w.active[t] ? (kend + BN - 1) / BN : 0;
+    w.n_kv[t] = w.active[t] ? (kend + BK - 1) / BK : 0;
   }
   return w;
 }
 
-template <int D, int NSTAGE, bool P_TMEM>
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of inputs on the FMA pipe (the MUFU unit is the scarce
+// resource of this kernel). Range reduction rounds x to the nearest integer n
+// by adding 1.5 * 2^23 (the integer lands in the low mantissa bits), so
+// x = n + f with |f| <= 1/2; 2^f comes from a degree-3 polynomial fitted for
+// this kernel (minimax in relative error on [-1/2, 1/2] by Lawson's
+// iteratively reweighted least squares; max relative error 7.5e-5, far below
+// the 2^-9 rounding of the bf16 P it feeds); n is then added to the exponent
+// field. Inputs are clamped at -126, so tiny results come out as ~2^-126
+// instead of 0, and must stay below 128.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float C0 = 0.9999280571937561f, C1 = 0.6932609677314758f, C2 = 0.2426111251115799f,
+                  C3 = 0.0551716648042202f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(C3, C3), f, make_float2(C2, C2));
+  p = __ffma2_rn(p, f, make_float2(C1, C1));
+  p = __ffma2_rn(p, f, make_float2(C0, C0));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Exponentials of one 64-score row block (s[]), their sum, and the packed bf16
+// P stored to TMEM 16 columns at a time. EMU8: in every 8 consecutive pairs, a
+// spread-out EMU8 of them take exp2 on the FMA pipe (exp2_poly2), the rest on
+// MUFU.
+template <int EMU8>
+__device__ __forceinline__ void exp_pack_store(const float (&s)[BK], float sl2, float m_off, uint32_t tP,
+                                               float2& acc) {
+  const float2 sc2 = make_float2(sl2, sl2);
+  const float2 mo2 = make_float2(-m_off, -m_off);
+  float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+#pragma unroll
+  for (int ch = 0; ch < BK / 32; ++ch) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = ch * 32 + 2 * i;
+      const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, mo2);
+      float2 pr;
+      if (((i * EMU8) & 7) < EMU8) {
+        pr = exp2_poly2(x);
+      } else {
+        pr.x = ex2_approx(x.x);
+        pr.y = ex2_approx(x.y);
+      }
+      if ((i & 3) == 0) a0 = __fadd2_rn(a0, pr);
+      if ((i & 3) == 1) a1 = __fadd2_rn(a1, pr);
+      if ((i & 3) == 2) a2 = __fadd2_rn(a2, pr);
+      if ((i & 3) == 3) a3 = __fadd2_rn(a3, pr);
+      pk[i] = pack_bf16x2(pr.x, pr.y);
+    }
+    tmem_st16(tP + ch * 16, pk);
+  }
+  acc = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// All lanes of the warp get the same answer (a timeout seen by one lane is
+// seen by all), so warp-collective instructions after it stay converged.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, WAIT_LIMIT));
+}
+
+template <int D, int EMU8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const Args args) {
-  using L = Layout<D, NSTAGE, P_TMEM>;
+  using L = Layout<D>;
+  static_assert(EMU8 >= 0 && EMU8 <= 8, "EMU8");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 1 + NSTAGE;
-  uint64_t* s_full = bars + 1 + 2 * NSTAGE;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
+  uint64_t* k_full = q_full + 1;
+  uint64_t* k_empty = k_full + KSTAGES;
+  uint64_t* v_full = k_empty + KSTAGES;
+  uint64_t* v_empty = v_full + VSTAGES;
+  uint64_t* s_full = v_empty + VSTAGES;  // [tile][half]
+  // One P barrier per S half: the softmax can run at most one block ahead of
+  // the MMA warp's wait on a given half, so a parity wait never aliases.
+  uint64_t* p_full = s_full + 4;  // [tile][half]
+  uint64_t* o_ready = p_full + 4;
+  uint64_t* o_full = o_ready + 2;
   uint64_t* mma_done = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
@@ -171,16 +271,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    // A K/V slot is free again once both MMA issuers have released it.
+    for (int s = 0; s < KSTAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 2);
+    }
+    for (int s = 0; s < VSTAGES; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 2);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&o_ready[t], 1);
       mbar_init(&o_full[t], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -196,117 +304,125 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const Work w = decode_work(args, blockIdx.x);
   const int n_kv = max(w.n_kv[0], w.n_kv[1]);
 
-  if (warp == TMA_WARP) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
+  if (warp >= SOFTMAX_WARPS) {
+    regs_dec<REG_OTHER>();
+    if (warp == TMA_WARP && lane == 0) {
+      // ---------------------------------------------------------------- producer
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       const uint32_t q_bytes = (w.active[0] + w.active[1]) * L::Q_TILE;
-      mbar_arrive_expect_tx(q_full, q_bytes);
+      if (q_bytes) mbar_arrive_expect_tx(q_full, q_bytes);
       for (int t = 0; t < 2; ++t) {
         if (!w.active[t]) continue;
         for (int c = 0; c < L::CHUNKS; ++c)
           tma_load_4d(smem + L::Q_OFF + t * L::Q_TILE + c * (BM * 128), &tm_q, q_full, c * 64, w.row0[t],
                       w.head[t], w.b);
       }
-      int issued = 0;
+      // Consumption order: K0, K1, then (V_i, K_{i+2}) for i = 0, 1, ...
+      int nk = 0, nv = 0;  // blocks issued so far into each ring
       bool ok = true;
-      for (int i = 0; i < 2 * n_kv && ok; ++i) {
-        const int j = i >> 1;
-        const int s = i % NSTAGE;
-        if (i >= NSTAGE) ok = mbar_wait_bounded(&kv_empty[s], ((i / NSTAGE) - 1) & 1, abort_flag, WAIT_LIMIT);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&kv_full[s], L::KV_TILE);
-        const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
+      auto load = [&](bool is_v, int blk) -> bool {
+        int& cnt = is_v ? nv : nk;
+        const int stages = is_v ? VSTAGES : KSTAGES;
+        uint64_t* full = is_v ? v_full : k_full;
+        uint64_t* empty = is_v ? v_empty : k_empty;
+        const int s = cnt % stages;
+        if (cnt >= stages && !mbar_wait_bounded(&empty[s], ((cnt / stages) - 1) & 1, abort_flag, WAIT_LIMIT))
+          return false;
+        mbar_arrive_expect_tx(&full[s], L::KV_TILE);
+        uint8_t* dst = smem + (is_v ? L::V_OFF : L::K_OFF) + s * L::KV_TILE;
         for (int c = 0; c < L::CHUNKS; ++c)
-          tma_load_4d(smem + L::KV_OFF + s * L::KV_TILE + c * (BN * 128), tm, &kv_full[s], c * 64, j * BN,
-                      w.kvh, w.b);
-        issued = i + 1;
+          tma_load_4d(dst + c * (BK * 128), is_v ? &tm_v : &tm_k, &full[s], c * 64, blk * BK, w.kvh, w.b);
+        ++cnt;
+        return true;
+      };
+      for (int i = 0; i < min(n_kv, 2) && ok; ++i) ok = load(false, i);
+      for (int i = 0; i < n_kv && ok; ++i) {
+        ok = load(true, i);
+        if (ok && i + 2 < n_kv) ok = load(false, i + 2);
       }
       // Drain: wait for the last copy issued into each slot, so no copy is in
       // flight when the CTA exits (matters only on the abort path).
-      for (int i = max(0, issued - NSTAGE); i < issued; ++i)
-        mbar_wait_bounded(&kv_full[i % NSTAGE], (i / NSTAGE) & 1, abort_flag, WAIT_LIMIT);
-      if (w.active[0] || w.active[1]) mbar_wait_bounded(q_full, 0, abort_flag, WAIT_LIMIT);
-    }
-  } else if (warp == MMA_WARP) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t ID_S = instr_desc_bf16(BM, BN, 0);
+      for (int i = max(0, nk - KSTAGES); i < nk; ++i)
+        mbar_wait_bounded(&k_full[i % KSTAGES], (i / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+      for (int i = max(0, nv - VSTAGES); i < nv; ++i)
+        mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
+      if (q_bytes) mbar_wait_bounded(q_full, 0, abort_flag, WAIT_LIMIT);
+    } else if ((warp == MMA_WARP || warp == MMA1_WARP) && lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer of tile t
+      const int t = warp - MMA_WARP;
+      const int nt = w.n_kv[t];
+      const int nu = w.n_kv[t ^ 1];
+      constexpr uint32_t ID_S = instr_desc_bf16(BM, BK, 0);
       constexpr uint32_t ID_PV = instr_desc_bf16(BM, D, 1);
-      const uint32_t q_smem = smem_addr(smem + L::Q_OFF);
-      const uint32_t kv_smem = smem_addr(smem + L::KV_OFF);
-      auto issue_s = [&](int t, int j) {
-        const uint32_t qa = q_smem + t * L::Q_TILE;
-        const uint32_t ka = kv_smem + ((2 * j) % NSTAGE) * L::KV_TILE;
+      // Descriptors are computed once; advancing one by a byte offset adds
+      // (offset >> 4) to its start-address field (no carry: shared memory
+      // addresses stay below 256 KB).
+      const uint64_t q_desc = smem_desc_sw128(smem_addr(smem + L::Q_OFF + t * L::Q_TILE), 16, 1024);
+      const uint64_t k_desc = smem_desc_sw128(smem_addr(smem + L::K_OFF), 16, 1024);       // K-major
+      const uint64_t v_desc = smem_desc_sw128(smem_addr(smem + L::V_OFF), BK * 128, 1024);  // MN-major
+      const uint32_t d_s = tmem_base + t * 128;
+      const uint32_t d_o = tmem_base + 256 + t * 128;
+      // S_t(i) = Q_t K_i^T into half i % 2 of this tile's S columns.
+      auto issue_s = [&](int i) {
+        const uint64_t ka = k_desc + (uint64_t)(((i % KSTAGES) * L::KV_TILE) >> 4);
+        const uint32_t d = d_s + (i & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          mma_ss(tmem_base + t * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                 ID_S, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(d, q_desc + (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4),
+                 ka + (uint64_t)(((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4), ID_S, kk > 0);
       };
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t va = kv_smem + ((2 * j + 1) % NSTAGE) * L::KV_TILE;
+      // O_t += P_t(i) V_i, P from TMEM (bf16 pairs in half i % 2).
+      auto issue_pv = [&](int i) {
+        const uint64_t va = v_desc + (uint64_t)(((i % VSTAGES) * L::KV_TILE) >> 4);
+        const uint32_t pa = d_s + (i & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(va + kk * 16 * 128, BN * 128, 1024);
-          if constexpr (P_TMEM) {
-            mma_ts(tmem_base + 256 + t * 128, tmem_base + t * 128 + kk * 8, bdesc, ID_PV, (j > 0) || (kk > 0));
-          } else {
-            const uint32_t pa = smem_addr(smem + L::P_OFF + t * L::P_TILE) + (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-            mma_ss(tmem_base + 256 + t * 128, smem_desc_sw128(pa, 16, 1024), bdesc, ID_PV, (j > 0) || (kk > 0));
-          }
-        }
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_ts(d_o, pa + kk * 8, va + (uint64_t)((kk * 16 * 128) >> 4), ID_PV, (i > 0) || (kk > 0));
+      };
+      // Release a K/V slot; when the other tile has no work for this block,
+      // also arrive on its behalf.
+      auto release = [&](uint64_t* bar, int blk) {
+        mma_commit(bar);
+        if (blk >= nu) mbar_arrive(bar);
       };
       bool ok = true;
-      if (n_kv > 0) {
-        ok = mbar_wait_bounded(q_full, 0, abort_flag, WAIT_LIMIT) &&
-             mbar_wait_bounded(&kv_full[0], 0, abort_flag, WAIT_LIMIT);
-        if (ok) {
-          tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if (w.n_kv[t] > 0) {
-              issue_s(t, 0);
-              mma_commit(&s_full[t]);
-            }
-          mma_commit(&kv_empty[0]);
-        }
+      if (nt > 0) ok = mbar_wait_bounded(q_full, 0, abort_flag, WAIT_LIMIT);
+      for (int i = 0; i < min(nt, 2) && ok; ++i) {
+        ok = mbar_wait_bounded(&k_full[i % KSTAGES], (i / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(i);
+        mma_commit(&s_full[t * 2 + (i & 1)]);
+        release(&k_empty[i % KSTAGES], i);
       }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int iv = 2 * j + 1, ik = 2 * j + 2;
-        ok = mbar_wait_bounded(&kv_full[iv % NSTAGE], (iv / NSTAGE) & 1, abort_flag, WAIT_LIMIT);
-        bool k_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= w.n_kv[t]) continue;
-          ok = mbar_wait_bounded(&p_full[t], j & 1, abort_flag, WAIT_LIMIT);
+      for (int i = 0; i < nt && ok; ++i) {
+        ok = mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT) &&
+             mbar_wait_bounded(&p_full[t * 2 + (i & 1)], (i >> 1) & 1, abort_flag, WAIT_LIMIT);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(i);
+        mma_commit(&o_ready[t]);
+        if (i == nt - 1) mma_commit(&o_full[t]);
+        release(&v_empty[i % VSTAGES], i);
+        const int ik = i + 2;
+        if (ik < nt) {
+          ok = mbar_wait_bounded(&k_full[ik % KSTAGES], (ik / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(t, j);
-          if (j == w.n_kv[t] - 1) {
-            mma_commit(&o_full[t]);
-          } else {
-            if (!k_ready) {
-              ok = mbar_wait_bounded(&kv_full[ik % NSTAGE], (ik / NSTAGE) & 1, abort_flag, WAIT_LIMIT);
-              if (!ok) break;
-              tc_fence_after();
-              k_ready = true;
-            }
-            issue_s(t, j + 1);
-            mma_commit(&s_full[t]);
-          }
+          issue_s(ik);
+          mma_commit(&s_full[t * 2 + (ik & 1)]);
+          release(&k_empty[ik % KSTAGES], ik);
         }
-        if (!ok) break;
-        mma_commit(&kv_empty[iv % NSTAGE]);
-        if (k_ready) mma_commit(&kv_empty[ik % NSTAGE]);
       }
-      // Wait until every MMA issued above has completed before tensor memory
-      // can be released (bounded; matters on the abort path).
+      // Wait until every MMA issued by both issuers has completed before
+      // tensor memory can be released (bounded; matters on the abort path).
       mma_commit(mma_done);
       mbar_wait_bounded(mma_done, 0, abort_flag, WAIT_LIMIT);
     }
   } else {
+    regs_inc<REG_SOFTMAX>();
     // ---------------------------------------------------------------- softmax + epilogue
     const int t = warp >> 2;
     const int sub = warp & 3;
@@ -321,84 +437,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float m2 = -INFINITY;  // running max of s * scale * log2(e)
       float l = 0.f;         // running sum of 2^(s*scale*log2e - m2)
       bool ok = true;
-      for (int j = 0; j < w.n_kv[t]; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[t], j & 1, abort_flag, WAIT_LIMIT));
+      for (int i = 0; i < w.n_kv[t]; ++i) {
+        ok = warp_wait(&s_full[t * 2 + (i & 1)], (i >> 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        uint32_t sb[BN];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, &sb[c * 32]);
+        const uint32_t tSi = tS + (i & 1) * 64;
+        uint32_t sb[BK];
+        tmem_ld32(tSi, &sb[0]);
+        tmem_ld32(tSi + 32, &sb[32]);
         tmem_ld_wait();
-        float s[BN];
+        float s[BK];
 #pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sb[c]);
-        const int k0 = j * BN;
-        const bool need_mask = (k0 + BN > w.sk) || (args.causal && (k0 + BN - 1 > w.row0[t] + (w.sk - w.sq)));
+        for (int c = 0; c < BK; ++c) s[c] = __uint_as_float(sb[c]);
+        const int k0 = i * BK;
+        const bool need_mask = (k0 + BK > w.sk) || (args.causal && (k0 + BK - 1 > w.row0[t] + (w.sk - w.sq)));
         if (need_mask) {
           const int lim = args.causal ? min(w.sk, qpos + 1) : w.sk;  // keys [0, lim) visible
 #pragma unroll
-          for (int c = 0; c < BN; ++c)
+          for (int c = 0; c < BK; ++c)
             if (k0 + c >= lim) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // Row max: eight independent max3 chains.
+        float am[8];
 #pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int k = 0; k < 8; ++k) am[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+        for (int c = 16; c < BK; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) am[k] = max3f(am[k], s[c + k], s[c + k + 8]);
+        const float mx = max3f(max3f(am[0], am[1], am[2]), max3f(am[3], am[4], am[5]), fmaxf(am[6], am[7]));
         const float m_new = fmaxf(m2, mx * sl2);
         const bool upd = (m_new - m2) > RESCALE_THRESHOLD;  // false when both are -inf (NaN compare)
         const float alpha = upd ? ex2_approx(m2 - m_new) : 1.f;
         if (upd) m2 = m_new;
         const float m_off = (m2 == -INFINITY) ? 0.f : m2;
-        float rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          s[c] = ex2_approx(fmaf(s[c], sl2, -m_off));
-          rs += s[c];
-        }
-        l = l * alpha + rs;
-        if (j > 0 && __any_sync(0xffffffffu, upd)) {
-          // O_t is stable here: PV(j-1) completed before S(j) was signalled.
+        if (i > 0 && __any_sync(0xffffffffu, upd)) {
+          // Rescale O once the previous P V (block i-1) has landed.
+          ok = warp_wait(&o_ready[t], (i - 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
             tmem_ld32(tO + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
             tmem_st32(tO + c * 32, o);
           }
-          tmem_st_wait();
         }
-        if constexpr (P_TMEM) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]);
-            tmem_st32(tS + h * 32, pk);
-          }
-          tmem_st_wait();
-        } else {
-          // P row r into the 128-byte-swizzled K-major tile: 16-byte unit u of a
-          // 128-byte row sits at unit (u ^ (r % 8)).
-          uint8_t* prow = smem + L::P_OFF + t * L::P_TILE + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-          for (int u = 0; u < BN / 8; ++u) {
-            const int chunk = u >> 3, uu = u & 7;
-            uint4 v;
-            v.x = pack_bf16x2(s[u * 8 + 0], s[u * 8 + 1]);
-            v.y = pack_bf16x2(s[u * 8 + 2], s[u * 8 + 3]);
-            v.z = pack_bf16x2(s[u * 8 + 4], s[u * 8 + 5]);
-            v.w = pack_bf16x2(s[u * 8 + 6], s[u * 8 + 7]);
-            *reinterpret_cast<uint4*>(prow + chunk * (BM * 128) + ((uu ^ (r & 7)) * 16)) = v;
-          }
-          fence_proxy_async_smem();
-        }
+        float2 acc;
+        if (need_mask)
+          exp_pack_store<0>(s, sl2, m_off, tSi, acc);
+        else
+          exp_pack_store<EMU8>(s, sl2, m_off, tSi, acc);
+        l = l * alpha + (acc.x + acc.y);
+        tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[t]);
+        mbar_arrive(&p_full[t * 2 + (i & 1)]);
       }
       // ------------------------------------------------------------ epilogue
       const bool has_keys = w.n_kv[t] > 0;
-      if (ok && has_keys) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_full[t], 0, abort_flag, WAIT_LIMIT));
+      if (ok && has_keys) ok = warp_wait(&o_full[t], 0, abort_flag);
       if (ok) {
         const bool store = qrow < w.sq;
         const bool empty = !(l > 0.f);
@@ -418,27 +518,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_ld_wait();
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = 0u;
+            for (int k = 0; k < 32; ++k) o[k] = 0u;
           }
           if (!store) continue;
           if (args.o_f32) {
             float* dst = reinterpret_cast<float*>(args.o) + obase + c * 32;
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              float4 v = make_float4(__uint_as_float(o[i]) * inv_l, __uint_as_float(o[i + 1]) * inv_l,
-                                     __uint_as_float(o[i + 2]) * inv_l, __uint_as_float(o[i + 3]) * inv_l);
-              *reinterpret_cast<float4*>(dst + i) = v;
+            for (int k = 0; k < 32; k += 4) {
+              float4 v = make_float4(__uint_as_float(o[k]) * inv_l, __uint_as_float(o[k + 1]) * inv_l,
+                                     __uint_as_float(o[k + 2]) * inv_l, __uint_as_float(o[k + 3]) * inv_l);
+              *reinterpret_cast<float4*>(dst + k) = v;
             }
           } else {
             __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.o) + obase + c * 32;
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
+            for (int k = 0; k < 32; k += 8) {
               uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(o[i + 0]) * inv_l, __uint_as_float(o[i + 1]) * inv_l);
-              v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv_l, __uint_as_float(o[i + 3]) * inv_l);
-              v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv_l, __uint_as_float(o[i + 5]) * inv_l);
-              v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv_l, __uint_as_float(o[i + 7]) * inv_l);
-              *reinterpret_cast<uint4*>(dst + i) = v;
+              v.x = pack_bf16x2(__uint_as_float(o[k + 0]) * inv_l, __uint_as_float(o[k + 1]) * inv_l);
+              v.y = pack_bf16x2(__uint_as_float(o[k + 2]) * inv_l, __uint_as_float(o[k + 3]) * inv_l);
+              v.z = pack_bf16x2(__uint_as_float(o[k + 4]) * inv_l, __uint_as_float(o[k + 5]) * inv_l);
+              v.w = pack_bf16x2(__uint_as_float(o[k + 6]) * inv_l, __uint_as_float(o[k + 7]) * inv_l);
+              *reinterpret_cast<uint4*>(dst + k) = v;
             }
           }
         }
@@ -490,30 +590,37 @@ static bool encode_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int NSTAGE, bool P_TMEM>
+template <int D, int EMU8>
 static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                     const Args& a, int items, cudaStream_t stream) {
-  using L = Layout<D, NSTAGE, P_TMEM>;
+  using L = Layout<D>;
   static_assert(L::SMEM_BYTES <= 232448, "shared memory budget");
-  auto kern = prefill_fwd_kernel<D, NSTAGE, P_TMEM>;
-  static bool configured = false;  // per process; the attribute is per function
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES) != cudaSuccess)
+  auto kern = prefill_fwd_kernel<D, EMU8>;
+  static int state = 0;  // 0 = unchecked, 1 = ready, -1 = unusable
+  if (state == 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+      cudaGetLastError();
       return ATTN_ERR_CUDA;
-    configured = true;
+    }
+    // The in-kernel register split assumes exactly REG_LAUNCH registers per
+    // thread at launch; anything else could make setmaxnreg.inc wait forever.
+    if (fa.numRegs != REG_LAUNCH) {
+      state = -1;
+    } else if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES) !=
+               cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    } else {
+      state = 1;
+    }
   }
+  if (state != 1) return ATTN_ERR_UNSUPPORTED;
   kern<<<items, NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // namespace prefill
-
-// Debug knob: ATTN_PREFILL_P_SMEM=1 selects the variant that stages P in
-// shared memory (a second, independently laid out path for cross-checking).
-static int prefill_p_in_smem() {
-  const char* e = getenv("ATTN_PREFILL_P_SMEM");
-  return (e && e[0] == '1') ? 1 : 0;
-}
 
 attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) {
   using namespace prefill;
@@ -526,9 +633,9 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
     return ATTN_ERR_CUDA;
   if (p.seqlen_k > 0) {
     if (!encode_4d(&tk, p.k, D, p.seqlen_k, p.num_kv_heads, p.batch, p.k_row_stride * 2, p.k_head_stride * 2,
-                   p.k_batch_stride * 2, BN) ||
+                   p.k_batch_stride * 2, BK) ||
         !encode_4d(&tv, p.v, D, p.seqlen_k, p.num_kv_heads, p.batch, p.v_row_stride * 2, p.v_head_stride * 2,
-                   p.v_batch_stride * 2, BN))
+                   p.v_batch_stride * 2, BK))
       return ATTN_ERR_CUDA;
   } else {
     tk = tq;  // no keys: nothing is loaded through these maps
@@ -564,13 +671,10 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
   if (items <= 0) return ATTN_OK;
   if (items > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
 
-  const bool p_smem = prefill_p_in_smem() != 0;
-  if (D == 128) {
-    if (p_smem) return launch_variant<128, 2, false>(tq, tk, tv, a, (int)items, stream);
-    return launch_variant<128, 4, true>(tq, tk, tv, a, (int)items, stream);
-  }
-  if (p_smem) return launch_variant<64, 4, false>(tq, tk, tv, a, (int)items, stream);
-  return launch_variant<64, 6, true>(tq, tk, tv, a, (int)items, stream);
+  // A quarter of the exponentials go to the FMA-pipe polynomial (measured best
+  // on B200 for head_dim 128: the MUFU pipe is the scarcer resource).
+  if (D == 128) return launch_variant<128, 2>(tq, tk, tv, a, (int)items, stream);
+  return launch_variant<64, 2>(tq, tk, tv, a, (int)items, stream);
 }
 
 }  // namespace attn

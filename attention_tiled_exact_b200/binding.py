@@ -174,6 +174,48 @@ def prefill(q, k, v, scale: float | None = None, causal: bool = False, out=None,
     return out, lse
 
 
+def prefill_paged(q, k_cache, v_cache, block_table, seqlens_k, seqlens_q=None, scale: float | None = None,
+                  causal: bool = True, out=None, lse=None, out_dtype=torch.bfloat16, want_lse: bool = True,
+                  error_flags=None):
+    """Prefill of query chunks against a paged KV cache (chunked prefill).
+
+    q [B,Hq,Sq,D] bf16 (rows past seqlens_q[b] are not written);
+    k_cache/v_cache [NB,Hkv,16,D] bf16; block_table [B,max_blocks] int32;
+    seqlens_k [B] int32: cached keys of each sequence, the chunk's own keys
+    included (bottom-right causal alignment). Returns ``(O, LSE)``.
+    """
+    _need(q.dim() == 4 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
+    B, Hq, Sq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    _need(D2 == D and q.dtype == torch.bfloat16 and k_cache.dtype == torch.bfloat16 and
+          v_cache.dtype == torch.bfloat16 and q.stride(3) == 1, "bf16 q and caches, last dim contiguous")
+    _need(k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous caches")
+    _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.shape[0] == B,
+          "int32 block table [B, max_blocks]")
+    _need(seqlens_k.dtype == torch.int32 and seqlens_k.numel() == B, "int32 seqlens_k [B]")
+    if seqlens_q is not None:
+        _need(seqlens_q.dtype == torch.int32 and seqlens_q.numel() == B, "int32 seqlens_q [B]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Hq, Sq, D), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    p = PrefillParams()
+    p.q, p.o, p.lse = _ptr(q), _ptr(out), _ptr(lse)
+    p.k_cache, p.v_cache, p.block_table = _ptr(k_cache), _ptr(v_cache), _ptr(block_table)
+    p.seqlens_k, p.seqlens_q = _ptr(seqlens_k), _ptr(seqlens_q)
+    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.seqlen_q = B, Hq, Hkv, D, Sq
+    p.seqlen_k = block_table.shape[1] * BS  # upper bound of seqlens_k
+    p.max_blocks_per_seq, p.num_blocks, p.block_size = block_table.shape[1], NB, BS
+    p.q_batch_stride, p.q_head_stride, p.q_row_stride = q.stride(0), q.stride(1), q.stride(2)
+    p.o_batch_stride, p.o_head_stride, p.o_row_stride = out.stride(0), out.stride(1), out.stride(2)
+    p.scale, p.causal, p.o_dtype = float(scale), int(bool(causal)), _out_code(out.dtype)
+    p.error_flags = _ptr(error_flags)
+    _check(LIB.attn_prefill(ctypes.byref(p), _stream(q.device)), "attn_prefill(paged)")
+    return out, lse
+
+
 # ----------------------------------------------------------------------------
 # decode
 # ----------------------------------------------------------------------------

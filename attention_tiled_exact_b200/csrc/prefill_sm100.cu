@@ -90,6 +90,10 @@ struct Args {
   int o_f32;
   long long o_bs, o_hs, o_rs;
   int32_t* error_flags;
+  // paged keys/values (PAGED kernels only)
+  const int32_t* block_table;
+  int max_blocks;
+  int num_blocks;
 };
 
 template <int D>
@@ -103,7 +107,7 @@ struct Layout {
   static constexpr int BAR_OFF = V_OFF + VSTAGES * KV_TILE;
   // q_full, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2][2], p_full[2][2], o_ready[2], o_full[2],
   // mma_done
-  static constexpr int NUM_BARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 4 + 4 + 2 + 2 + 1;
+  static constexpr int NUM_BARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 4 + 4 + 2 + 2 + 1 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM_BYTES = BYTES + 1024;  // slack for 1024-byte alignment
@@ -149,6 +153,7 @@ __device__ __forceinline__ Work decode_work(const Args& a, int item) {
   if (w.sq > a.seqlen_q) w.sq = a.seqlen_q;
   if (w.sq < 0) w.sq = 0;
   if (w.sk < 0) w.sk = 0;
+  if (a.block_table && w.sk > a.max_blocks * 16) w.sk = a.max_blocks * 16;  // flagged by the producer
   for (int t = 0; t < 2; ++t) {
     w.active[t] = w.row0[t] < w.sq;
     int kend = w.sk;
@@ -242,7 +247,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, WAIT_LIMIT));
 }
 
-template <int D, int EMU8>
+// PAGED: K and V come from a pool of 16-token blocks [num_blocks, Hkv, 16, D]
+// addressed through the block table; the K/V tensor maps then cover the pool.
+template <int D, int EMU8, bool PAGED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const Args args) {
@@ -263,6 +270,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* o_ready = p_full + 4;
   uint64_t* o_full = o_ready + 2;
   uint64_t* mma_done = o_full + 2;
+  uint64_t* v_clean = mma_done + 1;  // paged: the last V block's rows past the sequence end are zeroed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
@@ -289,6 +297,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&o_full[t], 1);
     }
     mbar_init(mma_done, 2);
+    mbar_init(v_clean, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -304,51 +313,103 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const Work w = decode_work(args, blockIdx.x);
   const int n_kv = max(w.n_kv[0], w.n_kv[1]);
 
+  // Paged: the last V block holds rows past the sequence end (tail slots of a
+  // partly filled cache block) that must read as zero before P V uses them.
+  const bool v_fix = PAGED && n_kv > 0 && (w.sk & 15) != 0 && n_kv * BK > w.sk;
+
   if (warp >= SOFTMAX_WARPS) {
     regs_dec<REG_OTHER>();
-    if (warp == TMA_WARP && lane == 0) {
+    if (warp == TMA_WARP) {
       // ---------------------------------------------------------------- producer
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      const uint32_t q_bytes = (w.active[0] + w.active[1]) * L::Q_TILE;
-      if (q_bytes) mbar_arrive_expect_tx(q_full, q_bytes);
-      for (int t = 0; t < 2; ++t) {
-        if (!w.active[t]) continue;
-        for (int c = 0; c < L::CHUNKS; ++c)
-          tma_load_4d(smem + L::Q_OFF + t * L::Q_TILE + c * (BM * 128), &tm_q, q_full, c * 64, w.row0[t],
-                      w.head[t], w.b);
-      }
-      // Consumption order: K0, K1, then (V_i, K_{i+2}) for i = 0, 1, ...
       int nk = 0, nv = 0;  // blocks issued so far into each ring
-      bool ok = true;
-      auto load = [&](bool is_v, int blk) -> bool {
-        int& cnt = is_v ? nv : nk;
-        const int stages = is_v ? VSTAGES : KSTAGES;
-        uint64_t* full = is_v ? v_full : k_full;
-        uint64_t* empty = is_v ? v_empty : k_empty;
-        const int s = cnt % stages;
-        if (cnt >= stages && !mbar_wait_bounded(&empty[s], ((cnt / stages) - 1) & 1, abort_flag, WAIT_LIMIT))
-          return false;
-        mbar_arrive_expect_tx(&full[s], L::KV_TILE);
-        uint8_t* dst = smem + (is_v ? L::V_OFF : L::K_OFF) + s * L::KV_TILE;
-        for (int c = 0; c < L::CHUNKS; ++c)
-          tma_load_4d(dst + c * (BK * 128), is_v ? &tm_v : &tm_k, &full[s], c * 64, blk * BK, w.kvh, w.b);
-        ++cnt;
-        return true;
-      };
-      for (int i = 0; i < min(n_kv, 2) && ok; ++i) ok = load(false, i);
-      for (int i = 0; i < n_kv && ok; ++i) {
-        ok = load(true, i);
-        if (ok && i + 2 < n_kv) ok = load(false, i + 2);
+      const uint32_t q_bytes = (w.active[0] + w.active[1]) * L::Q_TILE;
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        if (PAGED && args.seqlens_k[w.b] > args.max_blocks * 16 && args.error_flags)
+          atomicOr(args.error_flags, ATTN_FAULT_BAD_LENGTH);
+        if (q_bytes) mbar_arrive_expect_tx(q_full, q_bytes);
+        for (int t = 0; t < 2; ++t) {
+          if (!w.active[t]) continue;
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_4d(smem + L::Q_OFF + t * L::Q_TILE + c * (BM * 128), &tm_q, q_full, c * 64, w.row0[t],
+                        w.head[t], w.b);
+        }
+        const int32_t* table = PAGED ? args.block_table + (long long)w.b * args.max_blocks : nullptr;
+        // Consumption order: K0, K1, then (V_i, K_{i+2}) for i = 0, 1, ...
+        bool ok = true;
+        auto load = [&](bool is_v, int blk) -> bool {
+          int& cnt = is_v ? nv : nk;
+          const int stages = is_v ? VSTAGES : KSTAGES;
+          uint64_t* full = is_v ? v_full : k_full;
+          uint64_t* empty = is_v ? v_empty : k_empty;
+          const int s = cnt % stages;
+          if (cnt >= stages && !mbar_wait_bounded(&empty[s], ((cnt / stages) - 1) & 1, abort_flag, WAIT_LIMIT))
+            return false;
+          mbar_arrive_expect_tx(&full[s], L::KV_TILE);
+          uint8_t* dst = smem + (is_v ? L::V_OFF : L::K_OFF) + s * L::KV_TILE;
+          const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+          if constexpr (!PAGED) {
+            for (int c = 0; c < L::CHUNKS; ++c) tma_load_4d(dst + c * (BK * 128), tm, &full[s], c * 64, blk * BK, w.kvh, w.b);
+          } else {
+            // Four 16-token cache blocks; a block past the sequence end (or a
+            // table entry outside the pool) is read from one past the pool's
+            // last block, which TMA fills with zeros.
+            for (int j = 0; j < BK / 16; ++j) {
+              const int tok = blk * BK + j * 16;
+              int phys = args.num_blocks;
+              if (tok < w.sk) {
+                const int e = table[tok >> 4];
+                if (e >= 0 && e < args.num_blocks)
+                  phys = e;
+                else if (args.error_flags)
+                  atomicOr(args.error_flags, ATTN_FAULT_BAD_BLOCK);
+              }
+              for (int c = 0; c < L::CHUNKS; ++c)
+                tma_load_4d(dst + c * (BK * 128) + j * (16 * 128), tm, &full[s], c * 64, 0, w.kvh, phys);
+            }
+          }
+          ++cnt;
+          return true;
+        };
+        for (int i = 0; i < min(n_kv, 2) && ok; ++i) ok = load(false, i);
+        for (int i = 0; i < n_kv && ok; ++i) {
+          ok = load(true, i);
+          if (ok && i + 2 < n_kv) ok = load(false, i + 2);
+        }
       }
-      // Drain: wait for the last copy issued into each slot, so no copy is in
-      // flight when the CTA exits (matters only on the abort path).
-      for (int i = max(0, nk - KSTAGES); i < nk; ++i)
-        mbar_wait_bounded(&k_full[i % KSTAGES], (i / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
-      for (int i = max(0, nv - VSTAGES); i < nv; ++i)
-        mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
-      if (q_bytes) mbar_wait_bounded(q_full, 0, abort_flag, WAIT_LIMIT);
+      nv = __shfl_sync(0xffffffffu, nv, 0);
+      nk = __shfl_sync(0xffffffffu, nk, 0);
+      if (v_fix && nv == n_kv) {
+        // Zero the rows of the last V block at or past the sequence end, then
+        // hand the block to the MMA issuers through v_clean.
+        const int i = n_kv - 1, s = i % VSTAGES;
+        if (warp_wait(&v_full[s], (i / VSTAGES) & 1, abort_flag)) {
+          uint8_t* blkp = smem + L::V_OFF + s * L::KV_TILE;
+          const int r0 = w.sk - i * BK;  // first row to clear
+          const int nbytes_row = 128;
+          for (int idx = lane; idx < (BK - r0) * L::CHUNKS * (nbytes_row / 16); idx += 32) {
+            const int u = idx % (nbytes_row / 16);
+            const int rc = idx / (nbytes_row / 16);
+            const int row = r0 + rc % (BK - r0);
+            const int c = rc / (BK - r0);
+            *reinterpret_cast<uint4*>(blkp + c * (BK * 128) + row * 128 + u * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(v_clean);
+        }
+      }
+      if (lane == 0) {
+        // Drain: wait for the last copy issued into each slot, so no copy is in
+        // flight when the CTA exits (matters only on the abort path).
+        for (int i = max(0, nk - KSTAGES); i < nk; ++i)
+          mbar_wait_bounded(&k_full[i % KSTAGES], (i / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+        for (int i = max(0, nv - VSTAGES); i < nv; ++i)
+          mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
+        if (q_bytes) mbar_wait_bounded(q_full, 0, abort_flag, WAIT_LIMIT);
+      }
     } else if ((warp == MMA_WARP || warp == MMA1_WARP) && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer of tile t
       const int t = warp - MMA_WARP;
@@ -399,6 +460,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int i = 0; i < nt && ok; ++i) {
         ok = mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT) &&
+             (!(v_fix && i == n_kv - 1) || mbar_wait_bounded(v_clean, 0, abort_flag, WAIT_LIMIT)) &&
              mbar_wait_bounded(&p_full[t * 2 + (i & 1)], (i >> 1) & 1, abort_flag, WAIT_LIMIT);
         if (!ok) break;
         tc_fence_after();
@@ -590,12 +652,12 @@ static bool encode_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int EMU8>
+template <int D, int EMU8, bool PAGED>
 static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                     const Args& a, int items, cudaStream_t stream) {
   using L = Layout<D>;
   static_assert(L::SMEM_BYTES <= 232448, "shared memory budget");
-  auto kern = prefill_fwd_kernel<D, EMU8>;
+  auto kern = prefill_fwd_kernel<D, EMU8, PAGED>;
   static int state = 0;  // 0 = unchecked, 1 = ready, -1 = unusable
   if (state == 0) {
     cudaFuncAttributes fa;
@@ -625,13 +687,19 @@ static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk
 attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) {
   using namespace prefill;
   if (p.batch == 0 || p.seqlen_q == 0 || p.num_q_heads == 0) return ATTN_OK;
-  if (p.k_cache != nullptr) return ATTN_ERR_UNSUPPORTED;  // paged prefill: not in this build yet
+  const bool paged = p.k_cache != nullptr;
   const int D = p.head_dim;
   CUtensorMap tq, tk, tv;
   if (!encode_4d(&tq, p.q, D, p.seqlen_q, p.num_q_heads, p.batch, p.q_row_stride * 2, p.q_head_stride * 2,
                  p.q_batch_stride * 2, BM))
     return ATTN_ERR_CUDA;
-  if (p.seqlen_k > 0) {
+  if (paged) {
+    // Pools [num_blocks, Hkv, 16, D]: one 16-row box per cache block and D chunk.
+    const uint64_t row = (uint64_t)D * 2, blk = 16 * row, nb = blk * p.num_kv_heads;
+    if (!encode_4d(&tk, p.k_cache, D, 16, p.num_kv_heads, p.num_blocks, row, blk, nb, 16) ||
+        !encode_4d(&tv, p.v_cache, D, 16, p.num_kv_heads, p.num_blocks, row, blk, nb, 16))
+      return ATTN_ERR_CUDA;
+  } else if (p.seqlen_k > 0) {
     if (!encode_4d(&tk, p.k, D, p.seqlen_k, p.num_kv_heads, p.batch, p.k_row_stride * 2, p.k_head_stride * 2,
                    p.k_batch_stride * 2, BK) ||
         !encode_4d(&tv, p.v, D, p.seqlen_k, p.num_kv_heads, p.batch, p.v_row_stride * 2, p.v_head_stride * 2,
@@ -663,6 +731,11 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
   a.o_hs = p.o_head_stride;
   a.o_rs = p.o_row_stride;
   a.error_flags = p.error_flags;
+  if (paged) {
+    a.block_table = p.block_table;
+    a.max_blocks = p.max_blocks_per_seq;
+    a.num_blocks = p.num_blocks;
+  }
   long long items;
   if (a.pair_heads)
     items = (long long)a.n_row_blocks * p.batch * p.num_kv_heads * (a.group / 2);
@@ -673,8 +746,12 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
 
   // A quarter of the exponentials go to the FMA-pipe polynomial (measured best
   // on B200 for head_dim 128: the MUFU pipe is the scarcer resource).
-  if (D == 128) return launch_variant<128, 2>(tq, tk, tv, a, (int)items, stream);
-  return launch_variant<64, 2>(tq, tk, tv, a, (int)items, stream);
+  if (paged) {
+    if (D == 128) return launch_variant<128, 2, true>(tq, tk, tv, a, (int)items, stream);
+    return launch_variant<64, 2, true>(tq, tk, tv, a, (int)items, stream);
+  }
+  if (D == 128) return launch_variant<128, 2, false>(tq, tk, tv, a, (int)items, stream);
+  return launch_variant<64, 2, false>(tq, tk, tv, a, (int)items, stream);
 }
 
 }  // namespace attn

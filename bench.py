@@ -6,7 +6,9 @@ A step is one prefill call over the causal GQA workload (batch 4, 32 query /
 ``value`` is its throughput in TFLOP/s of algorithmic work (4 * head_dim per
 visible query-key pair and query head). The same JSON line also carries the
 paged split-KV decode workload (batch 64, lengths U[1024, 32768], 32/8 heads)
-timed the same way, in GB/s of algorithmic KV traffic.
+timed the same way, in GB/s of algorithmic KV traffic, and the mixed batch
+(8 prefill chunks of 512 queries on cached context plus 128 decode rows over
+one paged cache) as a fraction of the combined tensor + HBM roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -218,6 +220,8 @@ def run_ours(args, rank, world, local):
         result.update(bench_prefill(args, rank, world, local, attn, peaks, peak_src))
     if args.only in (None, "decode"):
         result["decode"] = bench_decode(args, rank, world, local, attn, peaks, peak_src)
+    if args.only in (None, "mixed"):
+        result["mixed"] = bench_mixed(args, rank, world, local, attn, peaks, peak_src)
     if args.only is not None:
         result["partial"] = f"--only {args.only}: profiling run, not a bench line"
     if rank == 0 and args.only is None:
@@ -330,6 +334,49 @@ def bench_decode(args, rank, world, local, attn, peaks, peak_src):
             "gpu_launches_per_step": 2, "clocks": dclk.summary()}
 
 
+def bench_mixed(args, rank, world, local, attn, peaks, peak_src):
+    """Chunked prefill of 8 x 512 queries on cached context + 128 decode rows, one pass."""
+    import dataclasses
+
+    import torch
+    cfg = dataclasses.replace(wl.MIXED, seed=wl.MIXED.seed + 1000 * rank)
+    d = wl.make_mixed(cfg)
+    nc = cfg.chunks
+    kc, vc = _dev_bf16(d["k_pool"]), _dev_bf16(d["v_pool"])
+    table = torch.from_numpy(d["block_table"]).cuda()
+    lens = torch.from_numpy(d["kv_lens"]).cuda()
+    tp, lp = table[:nc].contiguous(), lens[:nc].contiguous()
+    td, ld = table[nc:].contiguous(), lens[nc:].contiguous()
+    qc, qd = _dev_bf16(d["q_chunk"]), _dev_bf16(d["q_dec"])
+    oc = torch.empty_like(qc)
+    lsec = torch.empty(qc.shape[:3], dtype=torch.float32, device="cuda")
+    od = torch.empty_like(qd)
+    lsed = torch.empty(qd.shape[:2], dtype=torch.float32, device="cuda")
+    max_dec = int(d["kv_lens"][nc:].max())
+    ws = torch.empty(max(1, attn.decode_workspace_bytes(qd, kc, vc, td, ld, max_seq_len=max_dec)),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        attn.prefill_paged(qc, kc, vc, tp, lp, None, cfg.scale, True, out=oc, lse=lsec)
+        attn.decode_paged(qd, kc, vc, td, ld, cfg.scale, max_seq_len=max_dec, out=od, lse=lsed, workspace=ws)
+
+    steps = max(args.steps, 5)
+    with ClockSampler(local) as clk:
+        ms = time_loop(step, steps, args.warmup, world)
+    flops = 4.0 * cfg.head_dim * cfg.q_heads * sum(
+        wl.causal_pairs(cfg.chunk_len, int(k), True) for k in d["kv_lens"][:nc])
+    dec_bytes = float(int(d["kv_lens"][nc:].sum()) * cfg.kv_heads * cfg.head_dim * 2 * 2 +
+                      cfg.decodes * cfg.q_heads * (cfg.head_dim * 4 + 4))
+    peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    ideal_ms = (flops / (peak_t * 1e12) + dec_bytes / (peak_h * 1e9)) * 1e3
+    return {"workload": cfg.name, "ms_per_step": round(ms, 4), "steps": steps,
+            "prefill_tflop": round(flops / 1e12, 4), "decode_gb": round(dec_bytes / 1e9, 3),
+            "roofline": {"bound": "tensor+hbm", "ideal_ms": round(ideal_ms, 4), "frac": round(ideal_ms / ms, 4),
+                         "peak_source": f"{peak_src}: {peak_t} TFLOP/s bf16, {peak_h} GB/s"},
+            "gpu_launches_per_step": 3, "clocks": clk.summary()}
+
+
 # ----------------------------------------------------------------------------
 # the oracle on the host cores
 # ----------------------------------------------------------------------------
@@ -411,7 +458,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "mixed"], default=None,
                     help="profiling aid: run one workload only (the line is then marked partial)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="profiling aid: fewer decode sequences (default: the full 64)")

@@ -105,9 +105,9 @@ struct Layout {
   static constexpr int K_OFF = Q_OFF + 2 * Q_TILE;
   static constexpr int V_OFF = K_OFF + KSTAGES * KV_TILE;
   static constexpr int BAR_OFF = V_OFF + VSTAGES * KV_TILE;
-  // q_full, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2][2], p_full[2][2], o_ready[2], o_full[2],
-  // mma_done
-  static constexpr int NUM_BARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 4 + 4 + 2 + 2 + 1 + 1;
+  // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2][2], p_full[2][2], o_ready[2],
+  // o_full[2], mma_done
+  static constexpr int NUM_BARS = 2 + 2 * KSTAGES + 2 * VSTAGES + 4 + 4 + 2 + 2 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM_BYTES = BYTES + 1024;  // slack for 1024-byte alignment
@@ -165,6 +165,15 @@ __device__ __forceinline__ Work decode_work(const Args& a, int item) {
     w.n_kv[t] = w.active[t] ? (kend + BK - 1) / BK : 0;
   }
   return w;
+}
+
+// The k-th work item of CTA c in boustrophedon order over heaviest-first
+// items: c, 2G-1-c, 2G+c, 4G-1-c, ... (G = gridDim.x), which pairs heavy and
+// light causal items on every CTA. Returns -1 past the end.
+__device__ __forceinline__ int snake_item(int k, int n_items) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const int item = k * G + ((k & 1) ? (G - 1 - c) : c);
+  return item < n_items ? item : -1;
 }
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -247,30 +256,33 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, WAIT_LIMIT));
 }
 
+// Persistent: CTA c processes work items in the snake order of snake_item
+// (items are numbered heaviest first). All barrier phases run on per-CTA counters that continue across
+// items, so the next item's Q load and first S MMAs overlap this item's tail.
 // PAGED: K and V come from a pool of 16-token blocks [num_blocks, Hkv, 16, D]
 // addressed through the block table; the K/V tensor maps then cover the pool.
 template <int D, int EMU8, bool PAGED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const Args args) {
+                       const __grid_constant__ CUtensorMap tm_v, const Args args, int n_items) {
   using L = Layout<D>;
   static_assert(EMU8 >= 0 && EMU8 <= 8, "EMU8");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* q_full = bars;
-  uint64_t* k_full = q_full + 1;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* k_full = q_empty + 1;
   uint64_t* k_empty = k_full + KSTAGES;
   uint64_t* v_full = k_empty + KSTAGES;
   uint64_t* v_empty = v_full + VSTAGES;
   uint64_t* s_full = v_empty + VSTAGES;  // [tile][half]
   // One P barrier per S half: the softmax can run at most one block ahead of
-  // the MMA warp's wait on a given half, so a parity wait never aliases.
+  // its issuer's wait on a given half, so a parity wait never aliases.
   uint64_t* p_full = s_full + 4;  // [tile][half]
   uint64_t* o_ready = p_full + 4;
   uint64_t* o_full = o_ready + 2;
   uint64_t* mma_done = o_full + 2;
-  uint64_t* v_clean = mma_done + 1;  // paged: the last V block's rows past the sequence end are zeroed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
@@ -279,6 +291,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 2);  // both issuers' last S MMA of an item has read Q
     // A K/V slot is free again once both MMA issuers have released it.
     for (int s = 0; s < KSTAGES; ++s) {
       mbar_init(&k_full[s], 1);
@@ -297,7 +310,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&o_full[t], 1);
     }
     mbar_init(mma_done, 2);
-    mbar_init(v_clean, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -310,35 +322,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const Work w = decode_work(args, blockIdx.x);
-  const int n_kv = max(w.n_kv[0], w.n_kv[1]);
-
-  // Paged: the last V block holds rows past the sequence end (tail slots of a
-  // partly filled cache block) that must read as zero before P V uses them.
-  const bool v_fix = PAGED && n_kv > 0 && (w.sk & 15) != 0 && n_kv * BK > w.sk;
-
   if (warp >= SOFTMAX_WARPS) {
     regs_dec<REG_OTHER>();
-    if (warp == TMA_WARP) {
+    if (warp == TMA_WARP && lane == 0) {
       // ---------------------------------------------------------------- producer
-      int nk = 0, nv = 0;  // blocks issued so far into each ring
-      const uint32_t q_bytes = (w.active[0] + w.active[1]) * L::Q_TILE;
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int nk = 0, nv = 0;  // K / V blocks issued so far (all items)
+      int nq = 0;          // items whose Q was loaded
+      bool ok = true;
+      for (int kk_item = 0, item; ok && (item = snake_item(kk_item, n_items)) >= 0; ++kk_item) {
+        const Work w = decode_work(args, item);
+        const int n_kv = max(w.n_kv[0], w.n_kv[1]);
+        if (!w.active[0] && !w.active[1]) continue;
         if (PAGED && args.seqlens_k[w.b] > args.max_blocks * 16 && args.error_flags)
           atomicOr(args.error_flags, ATTN_FAULT_BAD_LENGTH);
-        if (q_bytes) mbar_arrive_expect_tx(q_full, q_bytes);
+        // Q tiles: wait until both issuers' last S MMA of the previous item has read them.
+        if (nq > 0 && !mbar_wait_bounded(q_empty, (nq - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        mbar_arrive_expect_tx(q_full, (w.active[0] + w.active[1]) * L::Q_TILE);
         for (int t = 0; t < 2; ++t) {
           if (!w.active[t]) continue;
           for (int c = 0; c < L::CHUNKS; ++c)
             tma_load_4d(smem + L::Q_OFF + t * L::Q_TILE + c * (BM * 128), &tm_q, q_full, c * 64, w.row0[t],
                         w.head[t], w.b);
         }
+        ++nq;
         const int32_t* table = PAGED ? args.block_table + (long long)w.b * args.max_blocks : nullptr;
-        // Consumption order: K0, K1, then (V_i, K_{i+2}) for i = 0, 1, ...
-        bool ok = true;
         auto load = [&](bool is_v, int blk) -> bool {
           int& cnt = is_v ? nv : nk;
           const int stages = is_v ? VSTAGES : KSTAGES;
@@ -351,7 +361,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* dst = smem + (is_v ? L::V_OFF : L::K_OFF) + s * L::KV_TILE;
           const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
           if constexpr (!PAGED) {
-            for (int c = 0; c < L::CHUNKS; ++c) tma_load_4d(dst + c * (BK * 128), tm, &full[s], c * 64, blk * BK, w.kvh, w.b);
+            for (int c = 0; c < L::CHUNKS; ++c)
+              tma_load_4d(dst + c * (BK * 128), tm, &full[s], c * 64, blk * BK, w.kvh, w.b);
           } else {
             // Four 16-token cache blocks; a block past the sequence end (or a
             // table entry outside the pool) is read from one past the pool's
@@ -373,48 +384,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ++cnt;
           return true;
         };
+        // Consumption order within an item: K0, K1, then (V_i, K_{i+2}).
         for (int i = 0; i < min(n_kv, 2) && ok; ++i) ok = load(false, i);
         for (int i = 0; i < n_kv && ok; ++i) {
           ok = load(true, i);
           if (ok && i + 2 < n_kv) ok = load(false, i + 2);
         }
       }
-      nv = __shfl_sync(0xffffffffu, nv, 0);
-      nk = __shfl_sync(0xffffffffu, nk, 0);
-      if (v_fix && nv == n_kv) {
-        // Zero the rows of the last V block at or past the sequence end, then
-        // hand the block to the MMA issuers through v_clean.
-        const int i = n_kv - 1, s = i % VSTAGES;
-        if (warp_wait(&v_full[s], (i / VSTAGES) & 1, abort_flag)) {
-          uint8_t* blkp = smem + L::V_OFF + s * L::KV_TILE;
-          const int r0 = w.sk - i * BK;  // first row to clear
-          const int nbytes_row = 128;
-          for (int idx = lane; idx < (BK - r0) * L::CHUNKS * (nbytes_row / 16); idx += 32) {
-            const int u = idx % (nbytes_row / 16);
-            const int rc = idx / (nbytes_row / 16);
-            const int row = r0 + rc % (BK - r0);
-            const int c = rc / (BK - r0);
-            *reinterpret_cast<uint4*>(blkp + c * (BK * 128) + row * 128 + u * 16) = make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(v_clean);
-        }
-      }
-      if (lane == 0) {
-        // Drain: wait for the last copy issued into each slot, so no copy is in
-        // flight when the CTA exits (matters only on the abort path).
-        for (int i = max(0, nk - KSTAGES); i < nk; ++i)
-          mbar_wait_bounded(&k_full[i % KSTAGES], (i / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
-        for (int i = max(0, nv - VSTAGES); i < nv; ++i)
-          mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
-        if (q_bytes) mbar_wait_bounded(q_full, 0, abort_flag, WAIT_LIMIT);
-      }
+      // Drain: wait for the last copy issued into each slot, so no copy is in
+      // flight when the CTA exits (matters only on the abort path).
+      for (int i = max(0, nk - KSTAGES); i < nk; ++i)
+        mbar_wait_bounded(&k_full[i % KSTAGES], (i / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+      for (int i = max(0, nv - VSTAGES); i < nv; ++i)
+        mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
+      if (nq > 0) mbar_wait_bounded(q_full, (nq - 1) & 1, abort_flag, WAIT_LIMIT);
     } else if ((warp == MMA_WARP || warp == MMA1_WARP) && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer of tile t
       const int t = warp - MMA_WARP;
-      const int nt = w.n_kv[t];
-      const int nu = w.n_kv[t ^ 1];
       constexpr uint32_t ID_S = instr_desc_bf16(BM, BK, 0);
       constexpr uint32_t ID_PV = instr_desc_bf16(BM, D, 1);
       // Descriptors are computed once; advancing one by a byte offset adds
@@ -425,58 +411,80 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t v_desc = smem_desc_sw128(smem_addr(smem + L::V_OFF), BK * 128, 1024);  // MN-major
       const uint32_t d_s = tmem_base + t * 128;
       const uint32_t d_o = tmem_base + 256 + t * 128;
-      // S_t(i) = Q_t K_i^T into half i % 2 of this tile's S columns.
-      auto issue_s = [&](int i) {
-        const uint64_t ka = k_desc + (uint64_t)(((i % KSTAGES) * L::KV_TILE) >> 4);
-        const uint32_t d = d_s + (i & 1) * 64;
+      // S_t = Q_t K^T of global block g into half g % 2 (K block in ring slot ks).
+      auto issue_s = [&](int g, int ks) {
+        const uint64_t ka = k_desc + (uint64_t)(((ks % KSTAGES) * L::KV_TILE) >> 4);
+        const uint32_t d = d_s + (g & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(d, q_desc + (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4),
                  ka + (uint64_t)(((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4), ID_S, kk > 0);
       };
-      // O_t += P_t(i) V_i, P from TMEM (bf16 pairs in half i % 2).
-      auto issue_pv = [&](int i) {
-        const uint64_t va = v_desc + (uint64_t)(((i % VSTAGES) * L::KV_TILE) >> 4);
-        const uint32_t pa = d_s + (i & 1) * 64;
+      // O_t (+)= P_t V, P from TMEM (bf16 pairs in half g % 2), V in ring slot vs.
+      auto issue_pv = [&](int g, int vs, bool first) {
+        const uint64_t va = v_desc + (uint64_t)(((vs % VSTAGES) * L::KV_TILE) >> 4);
+        const uint32_t pa = d_s + (g & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
-          mma_ts(d_o, pa + kk * 8, va + (uint64_t)((kk * 16 * 128) >> 4), ID_PV, (i > 0) || (kk > 0));
+          mma_ts(d_o, pa + kk * 8, va + (uint64_t)((kk * 16 * 128) >> 4), ID_PV, !first || (kk > 0));
       };
-      // Release a K/V slot; when the other tile has no work for this block,
-      // also arrive on its behalf.
-      auto release = [&](uint64_t* bar, int blk) {
-        mma_commit(bar);
-        if (blk >= nu) mbar_arrive(bar);
-      };
+      int gb = 0;   // this tile's blocks so far (all items): S half / P barrier phases
+      int kb = 0;   // K / V blocks loaded before the current item (both rings advance alike)
+      int nq = 0;   // active items so far (Q phases)
       bool ok = true;
-      if (nt > 0) ok = mbar_wait_bounded(q_full, 0, abort_flag, WAIT_LIMIT);
-      for (int i = 0; i < min(nt, 2) && ok; ++i) {
-        ok = mbar_wait_bounded(&k_full[i % KSTAGES], (i / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(i);
-        mma_commit(&s_full[t * 2 + (i & 1)]);
-        release(&k_empty[i % KSTAGES], i);
-      }
-      for (int i = 0; i < nt && ok; ++i) {
-        ok = mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT) &&
-             (!(v_fix && i == n_kv - 1) || mbar_wait_bounded(v_clean, 0, abort_flag, WAIT_LIMIT)) &&
-             mbar_wait_bounded(&p_full[t * 2 + (i & 1)], (i >> 1) & 1, abort_flag, WAIT_LIMIT);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(i);
-        mma_commit(&o_ready[t]);
-        if (i == nt - 1) mma_commit(&o_full[t]);
-        release(&v_empty[i % VSTAGES], i);
-        const int ik = i + 2;
-        if (ik < nt) {
-          ok = mbar_wait_bounded(&k_full[ik % KSTAGES], (ik / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+      for (int kk_item = 0, item; ok && (item = snake_item(kk_item, n_items)) >= 0; ++kk_item) {
+        const Work w = decode_work(args, item);
+        if (!w.active[0] && !w.active[1]) continue;
+        const int nt = w.n_kv[t], nu = w.n_kv[t ^ 1];
+        const int n_kv = max(nt, nu);
+        // Release a K/V slot; when the other tile has no work for this block,
+        // also arrive on its behalf.
+        auto release = [&](uint64_t* bar, int blk) {
+          mma_commit(bar);
+          if (blk >= nu) mbar_arrive(bar);
+        };
+        // Even with no block of its own, wait for this item's Q: its arrival on
+        // q_empty below must count toward this item's phase, not the previous one.
+        ok = mbar_wait_bounded(q_full, nq & 1, abort_flag, WAIT_LIMIT);
+        for (int i = 0; i < min(nt, 2) && ok; ++i) {
+          const int kg = kb + i;  // K_i is the (kb + i)-th K block: K0, K1 lead each item
+          ok = mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
           if (!ok) break;
           tc_fence_after();
-          issue_s(ik);
-          mma_commit(&s_full[t * 2 + (ik & 1)]);
-          release(&k_empty[ik % KSTAGES], ik);
+          issue_s(gb + i, kg);
+          mma_commit(&s_full[t * 2 + ((gb + i) & 1)]);
+          release(&k_empty[kg % KSTAGES], i);
         }
+        if (ok && nt <= 2) {
+          // This tile's last S MMA of the item has been issued.
+          if (nt > 0) mma_commit(q_empty); else mbar_arrive(q_empty);
+        }
+        for (int i = 0; i < nt && ok; ++i) {
+          const int g = gb + i;
+          const int vg = kb + i;  // V_i is the (kb + i)-th V block
+          ok = mbar_wait_bounded(&v_full[vg % VSTAGES], (vg / VSTAGES) & 1, abort_flag, WAIT_LIMIT) &&
+               mbar_wait_bounded(&p_full[t * 2 + (g & 1)], (g >> 1) & 1, abort_flag, WAIT_LIMIT);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(g, vg, i == 0);
+          mma_commit(&o_ready[t]);
+          if (i == nt - 1) mma_commit(&o_full[t]);
+          release(&v_empty[vg % VSTAGES], i);
+          const int ik = i + 2;
+          if (ik < nt) {
+            const int kg = kb + ik;
+            ok = mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(g + 2, kg);
+            mma_commit(&s_full[t * 2 + (g & 1)]);
+            release(&k_empty[kg % KSTAGES], ik);
+            if (ik == nt - 1) mma_commit(q_empty);
+          }
+        }
+        gb += nt;
+        kb += n_kv;
+        ++nq;
       }
       // Wait until every MMA issued by both issuers has completed before
       // tensor memory can be released (bounded; matters on the abort path).
@@ -489,21 +497,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int t = warp >> 2;
     const int sub = warp & 3;
     const int r = sub * 32 + lane;  // row within the tile == TMEM lane
-    if (w.active[t]) {
-      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(sub * 32) << 16);
-      const uint32_t tS = lane_base + t * 128;
-      const uint32_t tO = lane_base + 256 + t * 128;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(sub * 32) << 16);
+    const uint32_t tS = lane_base + t * 128;
+    const uint32_t tO = lane_base + 256 + t * 128;
+    const float sl2 = args.scale_log2;
+    int gb = 0;  // this tile's blocks so far (all items)
+    int kb = 0;  // K / V blocks loaded before the current item
+    int nf = 0;  // items this tile finished (o_full phases)
+    bool ok = true;
+    for (int kk_item = 0, item; ok && (item = snake_item(kk_item, n_items)) >= 0; ++kk_item) {
+      const Work w = decode_work(args, item);
+      if (!w.active[0] && !w.active[1]) continue;
+      const int n_kv = max(w.n_kv[0], w.n_kv[1]);
+      const int nt = w.n_kv[t];
+      if (!w.active[t]) {
+        kb += n_kv;
+        continue;
+      }
+      // Paged: the item's last V block may hold rows past the sequence end
+      // (tail slots of a partly filled cache block); they are zeroed in shared
+      // memory before this tile's last P V, because 0 * NaN would poison O.
+      const bool v_fix = PAGED && nt == n_kv && nt > 0 && (w.sk & 15) != 0 && nt * BK > w.sk;
       const int qrow = w.row0[t] + r;
       const int qpos = qrow + (w.sk - w.sq);  // absolute position (bottom-right causal)
-      const float sl2 = args.scale_log2;
       float m2 = -INFINITY;  // running max of s * scale * log2(e)
       float l = 0.f;         // running sum of 2^(s*scale*log2e - m2)
-      bool ok = true;
-      for (int i = 0; i < w.n_kv[t]; ++i) {
-        ok = warp_wait(&s_full[t * 2 + (i & 1)], (i >> 1) & 1, abort_flag);
+      for (int i = 0; i < nt; ++i) {
+        const int g = gb + i;
+        ok = warp_wait(&s_full[t * 2 + (g & 1)], (g >> 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tSi = tS + (i & 1) * 64;
+        const uint32_t tSi = tS + (g & 1) * 64;
         uint32_t sb[BK];
         tmem_ld32(tSi, &sb[0]);
         tmem_ld32(tSi + 32, &sb[32]);
@@ -534,8 +558,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (upd) m2 = m_new;
         const float m_off = (m2 == -INFINITY) ? 0.f : m2;
         if (i > 0 && __any_sync(0xffffffffu, upd)) {
-          // Rescale O once the previous P V (block i-1) has landed.
-          ok = warp_wait(&o_ready[t], (i - 1) & 1, abort_flag);
+          // Rescale O once the previous P V (block g-1) has landed.
+          ok = warp_wait(&o_ready[t], (g - 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -554,57 +578,78 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         else
           exp_pack_store<EMU8>(s, sl2, m_off, tSi, acc);
         l = l * alpha + (acc.x + acc.y);
+        if (v_fix && i == nt - 1) {
+          const int vg = kb + i, vs = vg % VSTAGES;
+          ok = warp_wait(&v_full[vs], (vg / VSTAGES) & 1, abort_flag);
+          if (!ok) break;
+          uint8_t* vblk = smem + L::V_OFF + vs * L::KV_TILE;
+          const int r0 = w.sk - k0;  // first row past the sequence end
+          const int units = (BK - r0) * L::CHUNKS * 8;  // 16-byte units to clear
+          for (int u = r; u < units; u += 128) {
+            const int unit = u & 7, rc = u >> 3;
+            const int row = r0 + rc % (BK - r0), c = rc / (BK - r0);
+            *reinterpret_cast<uint4*>(vblk + c * (BK * 128) + row * 128 + unit * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[t * 2 + (i & 1)]);
+        mbar_arrive(&p_full[t * 2 + (g & 1)]);
       }
+      gb += nt;
+      kb += n_kv;
+      if (!ok) break;
       // ------------------------------------------------------------ epilogue
-      const bool has_keys = w.n_kv[t] > 0;
-      if (ok && has_keys) ok = warp_wait(&o_full[t], 0, abort_flag);
-      if (ok) {
-        const bool store = qrow < w.sq;
-        const bool empty = !(l > 0.f);
-        const float inv_l = empty ? 0.f : 1.f / l;
-        const long long obase =
-            (long long)w.b * args.o_bs + (long long)w.head[t] * args.o_hs + (long long)qrow * args.o_rs;
-        if (args.lse && store) {
-          const float lse = empty ? -INFINITY : (m2 + log2f(l)) * 0.69314718055994530942f;
-          args.lse[((long long)w.b * args.hq + w.head[t]) * args.seqlen_q + qrow] = lse;
+      const bool has_keys = nt > 0;
+      if (has_keys) {
+        ok = warp_wait(&o_full[t], nf & 1, abort_flag);
+        ++nf;
+        if (!ok) break;
+      }
+      const bool store = qrow < w.sq;
+      const bool empty = !(l > 0.f);
+      const float inv_l = empty ? 0.f : 1.f / l;
+      const long long obase =
+          (long long)w.b * args.o_bs + (long long)w.head[t] * args.o_hs + (long long)qrow * args.o_rs;
+      if (args.lse && store) {
+        const float lse = empty ? -INFINITY : (m2 + log2f(l)) * 0.69314718055994530942f;
+        args.lse[((long long)w.b * args.hq + w.head[t]) * args.seqlen_q + qrow] = lse;
+      }
+      if (has_keys) tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (has_keys) {  // warp-uniform: every lane issues the collective load
+          tmem_ld32(tO + c * 32, o);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
-        if (has_keys) tc_fence_after();
+        if (!store) continue;
+        if (args.o_f32) {
+          float* dst = reinterpret_cast<float*>(args.o) + obase + c * 32;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          if (has_keys) {  // warp-uniform: every lane issues the collective load
-            tmem_ld32(tO + c * 32, o);
-            tmem_ld_wait();
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = 0u;
+          for (int k = 0; k < 32; k += 4) {
+            float4 v = make_float4(__uint_as_float(o[k]) * inv_l, __uint_as_float(o[k + 1]) * inv_l,
+                                   __uint_as_float(o[k + 2]) * inv_l, __uint_as_float(o[k + 3]) * inv_l);
+            *reinterpret_cast<float4*>(dst + k) = v;
           }
-          if (!store) continue;
-          if (args.o_f32) {
-            float* dst = reinterpret_cast<float*>(args.o) + obase + c * 32;
+        } else {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.o) + obase + c * 32;
 #pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-              float4 v = make_float4(__uint_as_float(o[k]) * inv_l, __uint_as_float(o[k + 1]) * inv_l,
-                                     __uint_as_float(o[k + 2]) * inv_l, __uint_as_float(o[k + 3]) * inv_l);
-              *reinterpret_cast<float4*>(dst + k) = v;
-            }
-          } else {
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.o) + obase + c * 32;
-#pragma unroll
-            for (int k = 0; k < 32; k += 8) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(o[k + 0]) * inv_l, __uint_as_float(o[k + 1]) * inv_l);
-              v.y = pack_bf16x2(__uint_as_float(o[k + 2]) * inv_l, __uint_as_float(o[k + 3]) * inv_l);
-              v.z = pack_bf16x2(__uint_as_float(o[k + 4]) * inv_l, __uint_as_float(o[k + 5]) * inv_l);
-              v.w = pack_bf16x2(__uint_as_float(o[k + 6]) * inv_l, __uint_as_float(o[k + 7]) * inv_l);
-              *reinterpret_cast<uint4*>(dst + k) = v;
-            }
+          for (int k = 0; k < 32; k += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[k + 0]) * inv_l, __uint_as_float(o[k + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[k + 2]) * inv_l, __uint_as_float(o[k + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[k + 4]) * inv_l, __uint_as_float(o[k + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[k + 6]) * inv_l, __uint_as_float(o[k + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(dst + k) = v;
           }
         }
       }
+      // The next item's first P V overwrites O_t only after this thread's
+      // next p_full arrival, which follows these loads (tcgen05.wait::ld).
     }
   }
 
@@ -678,7 +723,8 @@ static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk
     }
   }
   if (state != 1) return ATTN_ERR_UNSUPPORTED;
-  kern<<<items, NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  const int grid = items < device_sm_count() ? items : device_sm_count();
+  kern<<<grid, NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, a, items);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -222,6 +222,8 @@ def run_ours(args, rank, world, local):
         result["decode"] = bench_decode(args, rank, world, local, attn, peaks, peak_src)
     if args.only in (None, "mixed"):
         result["mixed"] = bench_mixed(args, rank, world, local, attn, peaks, peak_src)
+    if args.only in (None, "prefill16k"):
+        result["prefill_16k"] = bench_prefill_16k(args, rank, world, local, attn, peaks, peak_src)
     if args.only is not None:
         result["partial"] = f"--only {args.only}: profiling run, not a bench line"
     if rank == 0 and args.only is None:
@@ -332,6 +334,28 @@ def bench_decode(args, rank, world, local, attn, peaks, peak_src):
                          "peak_source": f"{peak_src} copy bandwidth", "traffic": profiled_traffic("decode"),
                          "algorithmic_bytes_per_launch": dbytes},
             "gpu_launches_per_step": 2, "clocks": dclk.summary()}
+
+
+def bench_prefill_16k(args, rank, world, local, attn, peaks, peak_src):
+    """Long-context causal GQA prefill: batch 1, 32/8 heads, 16384 tokens, head_dim 128."""
+    import dataclasses
+
+    import torch
+    cfg = dataclasses.replace(wl.CAUSAL_GQA_16K, seed=wl.CAUSAL_GQA_16K.seed + 1000 * rank)
+    d = wl.make_prefill(cfg)
+    flops = 4.0 * cfg.head_dim * cfg.batch * cfg.q_heads * wl.causal_pairs(cfg.seqlen_q, cfg.seqlen_k, cfg.causal)
+    q, k, v = _dev_bf16(d["q"]), _dev_bf16(d["k"]), _dev_bf16(d["v"])
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    steps = max(5, min(args.steps, 20))
+    with ClockSampler(local) as clk:
+        ms = time_loop(lambda: attn.prefill(q, k, v, cfg.scale, True, out=o, lse=lse), steps, args.warmup, world)
+    tf = flops / (ms * 1e-3) / 1e12
+    peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    return {"workload": cfg.name, "value": round(tf * world, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "steps": steps, "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peak_t,
+                                         "frac": round(tf / peak_t, 4), "algorithmic_flops_per_launch": flops},
+            "gpu_launches_per_step": 1, "clocks": clk.summary()}
 
 
 def bench_mixed(args, rank, world, local, attn, peaks, peak_src):
@@ -458,7 +482,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--only", choices=["prefill", "decode", "mixed"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "mixed", "prefill16k"], default=None,
                     help="profiling aid: run one workload only (the line is then marked partial)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="profiling aid: fewer decode sequences (default: the full 64)")

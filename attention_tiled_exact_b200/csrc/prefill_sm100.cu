@@ -62,8 +62,8 @@ constexpr int SOFTMAX_WARPS = 8;
 constexpr int TMA_WARP = 8;
 constexpr int MMA_WARP = 9;        // issues tile 0's MMAs (and owns the TMEM allocation)
 constexpr int MMA1_WARP = 10;      // issues tile 1's MMAs
-constexpr int KSTAGES = 4;         // K blocks in flight
-constexpr int VSTAGES = 4;         // V blocks in flight
+constexpr int KSTAGES = 3;         // K blocks in flight
+constexpr int VSTAGES = 3;         // V blocks in flight
 // Register split. The block is launched with REG_LAUNCH registers per thread
 // (384 threads x 168 = 64512 registers); the third warpgroup gives registers
 // back and the two softmax warpgroups take them: 2*128*216 + 128*72 = 64512.
@@ -88,6 +88,7 @@ struct Args {
   void* o;
   float* lse;
   int o_f32;
+  int o_tma;  // O rows of a full 32-row warp slice go out through the tm_o tile store
   long long o_bs, o_hs, o_rs;
   int32_t* error_flags;
   // paged keys/values (PAGED kernels only)
@@ -104,7 +105,11 @@ struct Layout {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + 2 * Q_TILE;
   static constexpr int V_OFF = K_OFF + KSTAGES * KV_TILE;
-  static constexpr int BAR_OFF = V_OFF + VSTAGES * KV_TILE;
+  // Output staging: 32 rows x D bf16 per softmax warp (half the row for fp32
+  // output), written in 128-byte-swizzled boxes of 32 rows x 128 bytes.
+  static constexpr int W_STAGE = 32 * D * 2;
+  static constexpr int O_OFF = V_OFF + VSTAGES * KV_TILE;
+  static constexpr int BAR_OFF = O_OFF + SOFTMAX_WARPS * W_STAGE;
   // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2][2], p_full[2][2], o_ready[2],
   // o_full[2], mma_done
   static constexpr int NUM_BARS = 2 + 2 * KSTAGES + 2 * VSTAGES + 4 + 4 + 2 + 2 + 1;
@@ -250,6 +255,73 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Epilogue of one warp's 32 rows through shared memory and tile stores.
+// Lane l owns row l: its O row (TMEM lane) is scaled by inv_l, converted and
+// written into a 128-byte-swizzled box (16-byte unit u of row l lands at unit
+// u ^ (l & 7), so the 32 lanes' stores hit all banks), then lane 0 issues one
+// tile store per 32-row x 128-byte box. A staging area holds 32 x D bf16
+// values: bf16 output goes out in one round, fp32 in two. Before a staging
+// area is rewritten, lane 0 waits until the previous stores have read it.
+template <int D, bool F32>
+__device__ __forceinline__ void store_rows_tma(const CUtensorMap* tm_o, uint8_t* stage, uint32_t tO, bool has_keys,
+                                               float inv_l, int row0, int head, int b) {
+  constexpr int COLS = F32 ? 32 : 64;  // columns per 128-byte box
+  constexpr int BOXES = D / COLS;
+  constexpr int PER_ROUND = (32 * D * 2) / 4096;
+  const int lane = lane_id();
+  const int sw = lane & 7;
+#pragma unroll
+  for (int b0 = 0; b0 < BOXES; b0 += PER_ROUND) {
+    if (lane == 0) bulk_wait_group_read0();
+    __syncwarp();
+#pragma unroll
+    for (int bb = 0; bb < PER_ROUND; ++bb) {
+      uint8_t* row = stage + bb * 4096 + lane * 128;
+#pragma unroll
+      for (int h = 0; h < COLS / 32; ++h) {
+        const int c = (b0 + bb) * (COLS / 32) + h;  // 32-column TMEM chunk
+        uint32_t o[32];
+        if (has_keys) {  // warp-uniform: every lane issues the collective load
+          tmem_ld32(tO + c * 32, o);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        }
+        if constexpr (F32) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            uint4 v;
+            v.x = __float_as_uint(__uint_as_float(o[4 * u + 0]) * inv_l);
+            v.y = __float_as_uint(__uint_as_float(o[4 * u + 1]) * inv_l);
+            v.z = __float_as_uint(__uint_as_float(o[4 * u + 2]) * inv_l);
+            v.w = __float_as_uint(__uint_as_float(o[4 * u + 3]) * inv_l);
+            *reinterpret_cast<uint4*>(row + ((u ^ sw) << 4)) = v;
+          }
+        } else {
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            const int u = h * 4 + u4;
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * u4 + 0]) * inv_l, __uint_as_float(o[8 * u4 + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * u4 + 2]) * inv_l, __uint_as_float(o[8 * u4 + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * u4 + 4]) * inv_l, __uint_as_float(o[8 * u4 + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * u4 + 6]) * inv_l, __uint_as_float(o[8 * u4 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(row + ((u ^ sw) << 4)) = v;
+          }
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int bb = 0; bb < PER_ROUND; ++bb) tma_store_4d(tm_o, stage + bb * 4096, (b0 + bb) * COLS, row0, head, b);
+      bulk_commit_group();
+    }
+  }
+}
+
 // All lanes of the warp get the same answer (a timeout seen by one lane is
 // seen by all), so warp-collective instructions after it stay converged.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -264,7 +336,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 template <int D, int EMU8, bool PAGED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const Args args, int n_items) {
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const Args args, int n_items) {
   using L = Layout<D>;
   static_assert(EMU8 >= 0 && EMU8 <= 8, "EMU8");
   extern __shared__ uint8_t smem_raw[];
@@ -348,6 +421,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         w.head[t], w.b);
         }
         ++nq;
+        // Bring the next item's Q tiles into L2 now, so that its shared-memory
+        // load at the end of this item does not wait on HBM.
+        {
+          const int nxt = snake_item(kk_item + 1, n_items);
+          if (nxt >= 0) {
+            const Work wn = decode_work(args, nxt);
+            for (int t = 0; t < 2; ++t) {
+              if (!wn.active[t]) continue;
+              for (int c = 0; c < L::CHUNKS; ++c) tma_prefetch_l2_4d(&tm_q, c * 64, wn.row0[t], wn.head[t], wn.b);
+            }
+          }
+        }
         const int32_t* table = PAGED ? args.block_table + (long long)w.b * args.max_blocks : nullptr;
         auto load = [&](bool is_v, int blk) -> bool {
           int& cnt = is_v ? nv : nk;
@@ -616,6 +701,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         args.lse[((long long)w.b * args.hq + w.head[t]) * args.seqlen_q + qrow] = lse;
       }
       if (has_keys) tc_fence_after();
+      if (args.o_tma && w.row0[t] + sub * 32 + 32 <= w.sq) {  // warp-uniform
+        // This warp's 32 rows: stage them in shared memory (128-byte swizzle,
+        // conflict-free) and write them with tile stores issued by lane 0.
+        uint8_t* stage = smem + L::O_OFF + warp * L::W_STAGE;
+        const int r0 = w.row0[t] + sub * 32;
+        if (args.o_f32)
+          store_rows_tma<D, true>(&tm_o, stage, tO, has_keys, inv_l, r0, w.head[t], w.b);
+        else
+          store_rows_tma<D, false>(&tm_o, stage, tO, has_keys, inv_l, r0, w.head[t], w.b);
+        continue;
+      }
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -651,6 +747,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // The next item's first P V overwrites O_t only after this thread's
       // next p_full arrival, which follows these loads (tcgen05.wait::ld).
     }
+    // Tile stores still in flight must finish before the CTA exits.
+    if (lane == 0) bulk_wait_group0();
   }
 
   tc_fence_before();
@@ -681,17 +779,18 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 4-D bf16 map over [d3][d2][d1][d0 = head_dim] with byte strides s1..s3, box
-// (64, box_rows, 1, 1), 128-byte swizzle, zero fill out of bounds.
+// 4-D map over [d3][d2][d1][d0 = head_dim] with byte strides s1..s3, box
+// (128 bytes of d0, box_rows, 1, 1), 128-byte swizzle, zero fill out of bounds.
 static bool encode_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
-                      uint64_t s1, uint64_t s2, uint64_t s3, uint32_t box_rows) {
+                      uint64_t s1, uint64_t s2, uint64_t s3, uint32_t box_rows, bool f32 = false) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {d0, d1, d2, d3};
   cuuint64_t strides[3] = {s1, s2, s3};
-  cuuint32_t box[4] = {64, box_rows, 1, 1};
+  cuuint32_t box[4] = {f32 ? 32u : 64u, box_rows, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -699,7 +798,7 @@ static bool encode_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t 
 
 template <int D, int EMU8, bool PAGED>
 static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                    const Args& a, int items, cudaStream_t stream) {
+                                    const CUtensorMap& to, const Args& a, int items, cudaStream_t stream) {
   using L = Layout<D>;
   static_assert(L::SMEM_BYTES <= 232448, "shared memory budget");
   auto kern = prefill_fwd_kernel<D, EMU8, PAGED>;
@@ -724,7 +823,7 @@ static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk
   }
   if (state != 1) return ATTN_ERR_UNSUPPORTED;
   const int grid = items < device_sm_count() ? items : device_sm_count();
-  kern<<<grid, NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, a, items);
+  kern<<<grid, NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, to, a, items);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -776,6 +875,15 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
   a.o_bs = p.o_batch_stride;
   a.o_hs = p.o_head_stride;
   a.o_rs = p.o_row_stride;
+  // O goes out through tile stores when its map encodes (the API's alignment
+  // rules make that the normal case); otherwise every row is stored directly.
+  const int esz = a.o_f32 ? 4 : 2;
+  CUtensorMap to;
+  a.o_tma = encode_4d(&to, p.o, D, p.seqlen_q, p.num_q_heads, p.batch, p.o_row_stride * esz,
+                      p.o_head_stride * esz, p.o_batch_stride * esz, 32, a.o_f32 != 0)
+                ? 1
+                : 0;
+  if (!a.o_tma) to = tq;  // never read
   a.error_flags = p.error_flags;
   if (paged) {
     a.block_table = p.block_table;
@@ -793,11 +901,11 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
   // A quarter of the exponentials go to the FMA-pipe polynomial (measured best
   // on B200 for head_dim 128: the MUFU pipe is the scarcer resource).
   if (paged) {
-    if (D == 128) return launch_variant<128, 2, true>(tq, tk, tv, a, (int)items, stream);
-    return launch_variant<64, 2, true>(tq, tk, tv, a, (int)items, stream);
+    if (D == 128) return launch_variant<128, 2, true>(tq, tk, tv, to, a, (int)items, stream);
+    return launch_variant<64, 2, true>(tq, tk, tv, to, a, (int)items, stream);
   }
-  if (D == 128) return launch_variant<128, 2, false>(tq, tk, tv, a, (int)items, stream);
-  return launch_variant<64, 2, false>(tq, tk, tv, a, (int)items, stream);
+  if (D == 128) return launch_variant<128, 2, false>(tq, tk, tv, to, a, (int)items, stream);
+  return launch_variant<64, 2, false>(tq, tk, tv, to, a, (int)items, stream);
 }
 
 }  // namespace attn

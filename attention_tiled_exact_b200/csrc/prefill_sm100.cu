@@ -11,31 +11,28 @@
 // a producer, with the matrix products and the softmax in different warps
 // ("GPU Kernel 调度:大模型推理的拐点 2026", FlashAttention-2/3 paragraph).
 //
-// B200 design (one CTA per SM, 384 threads = three warpgroups):
+// B200 design (one persistent CTA per SM, 384 threads = three warpgroups):
 //   * two Q tiles of 128 rows per CTA. For GQA with an even group size the two
 //     tiles are two query heads of one key/value head on the same rows, so both
 //     tiles need exactly the same key range; otherwise they are two row blocks
 //     of one head. Every K/V block is loaded once for both tiles.
-//   * keys advance in blocks of 64. Each tile owns 128 TMEM columns for S,
-//     used as two 64-column halves: S of block i lands in half i % 2, so the
-//     scores of block i+1 are computed while the softmax works on block i and
-//     the softmax does not wait for the tensor core. P (bf16 pairs) overwrites
-//     the first 32 columns of its half and feeds the P V product from TMEM.
-//   * warp 8 (TMA): loads the Q tiles and streams K and V blocks into two
-//     shared-memory rings (128-byte swizzle), K two blocks ahead of V.
-//   * warps 9 and 10 (MMA): one thread per tile issues that tile's
-//     tcgen05.mma instructions. Per block i: O_t += P_t(i) V_i (A from TMEM),
-//     then S_t(i+2) = Q_t K_{i+2}^T into the half P_t(i) just vacated (MMAs
-//     from one thread execute in issue order; the two tiles share nothing in
-//     TMEM). Two issuers on different SM sub-partitions keep MMA issue from
-//     being starved by the busy softmax warps that share each sub-partition.
+//   * keys advance in blocks of 128, so every S MMA is a full-rate
+//     M=128 x N=128 instruction. Each tile owns 128 TMEM columns for S; P
+//     (bf16 pairs) overwrites their first 64 columns and feeds P V from TMEM.
+//   * the two tiles ping-pong: one thread (warp 9) issues every MMA in the
+//     order P_0 V_i, S_0(i+1), P_1 V_i, S_1(i+1), so the tensor core works on
+//     one tile's products while the other tile's softmax runs.
+//   * warp 8 (TMA): loads the Q tiles (the next work item's Q is prefetched
+//     into L2 one item ahead) and streams K and V blocks through two-stage
+//     shared-memory rings (128-byte swizzle) in the order the MMAs use them.
 //   * warps 0-3 / 4-7 (softmax, one warpgroup per tile, one thread per row):
 //     read S, mask (diagonal and tail blocks only), update the running max,
 //     p = 2^(s*scale*log2e - m), running sum, write P to TMEM. The running max
 //     is only moved when it grows by more than 2^8 (which keeps O and the row
-//     sum consistent); then O is rescaled in TMEM after the previous P V has
-//     completed. The same warps run the epilogue: O / l -> global,
-//     LSE = (m + log2 l) * ln 2.
+//     sum consistent); then O is rescaled in TMEM (the previous P V has
+//     completed by the time S of the next block is signalled). The same warps
+//     run the epilogue: O / l staged in swizzled shared memory and written by
+//     TMA tile stores, LSE = (m + log2 l) * ln 2.
 //   * TMEM: S_0 / P_0 cols [0,128), S_1 / P_1 [128,256), O_0 [256,256+D),
 //     O_1 [384,384+D).
 //   * every mbarrier wait is bounded; on a timeout the CTA raises a flag in
@@ -56,14 +53,13 @@ namespace attn {
 namespace prefill {
 
 constexpr int BM = 128;            // query rows per Q tile
-constexpr int BK = 64;             // keys per block
-constexpr int NUM_THREADS = 384;   // warpgroups: softmax tile 0, softmax tile 1, {TMA, MMA 0, MMA 1, idle}
+constexpr int BK = 128;            // keys per block
+constexpr int NUM_THREADS = 384;   // warpgroups: softmax tile 0, softmax tile 1, {TMA, MMA, idle, idle}
 constexpr int SOFTMAX_WARPS = 8;
 constexpr int TMA_WARP = 8;
-constexpr int MMA_WARP = 9;        // issues tile 0's MMAs (and owns the TMEM allocation)
-constexpr int MMA1_WARP = 10;      // issues tile 1's MMAs
-constexpr int KSTAGES = 3;         // K blocks in flight
-constexpr int VSTAGES = 3;         // V blocks in flight
+constexpr int MMA_WARP = 9;        // issues every MMA (and owns the TMEM allocation)
+constexpr int KSTAGES = 2;         // K blocks in flight
+constexpr int VSTAGES = 2;         // V blocks in flight
 // Register split. The block is launched with REG_LAUNCH registers per thread
 // (384 threads x 168 = 64512 registers); the third warpgroup gives registers
 // back and the two softmax warpgroups take them: 2*128*216 + 128*72 = 64512.
@@ -105,14 +101,13 @@ struct Layout {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + 2 * Q_TILE;
   static constexpr int V_OFF = K_OFF + KSTAGES * KV_TILE;
-  // Output staging: 32 rows x D bf16 per softmax warp (half the row for fp32
-  // output), written in 128-byte-swizzled boxes of 32 rows x 128 bytes.
-  static constexpr int W_STAGE = 32 * D * 2;
+  // Output staging: one 128-byte-swizzled box of 32 rows x 128 bytes per
+  // softmax warp.
+  static constexpr int W_STAGE = 32 * 128;
   static constexpr int O_OFF = V_OFF + VSTAGES * KV_TILE;
   static constexpr int BAR_OFF = O_OFF + SOFTMAX_WARPS * W_STAGE;
-  // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2][2], p_full[2][2], o_ready[2],
-  // o_full[2], mma_done
-  static constexpr int NUM_BARS = 2 + 2 * KSTAGES + 2 * VSTAGES + 4 + 4 + 2 + 2 + 1;
+  // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2], p_full[2], o_full[2], mma_done
+  static constexpr int NUM_BARS = 2 + 2 * KSTAGES + 2 * VSTAGES + 2 + 2 + 2 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM_BYTES = BYTES + 1024;  // slack for 1024-byte alignment
@@ -259,15 +254,15 @@ __device__ __forceinline__ void regs_dec() {
 // Lane l owns row l: its O row (TMEM lane) is scaled by inv_l, converted and
 // written into a 128-byte-swizzled box (16-byte unit u of row l lands at unit
 // u ^ (l & 7), so the 32 lanes' stores hit all banks), then lane 0 issues one
-// tile store per 32-row x 128-byte box. A staging area holds 32 x D bf16
-// values: bf16 output goes out in one round, fp32 in two. Before a staging
-// area is rewritten, lane 0 waits until the previous stores have read it.
+// tile store per 32-row x 128-byte box. A staging area holds one box, so a
+// row goes out in D / 64 (bf16) or D / 32 (fp32) rounds; before a staging
+// area is rewritten, lane 0 waits until the previous store has read it.
 template <int D, bool F32>
 __device__ __forceinline__ void store_rows_tma(const CUtensorMap* tm_o, uint8_t* stage, uint32_t tO, bool has_keys,
                                                float inv_l, int row0, int head, int b) {
   constexpr int COLS = F32 ? 32 : 64;  // columns per 128-byte box
   constexpr int BOXES = D / COLS;
-  constexpr int PER_ROUND = (32 * D * 2) / 4096;
+  constexpr int PER_ROUND = 1;
   const int lane = lane_id();
   const int sw = lane & 7;
 #pragma unroll
@@ -329,8 +324,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Persistent: CTA c processes work items in the snake order of snake_item
-// (items are numbered heaviest first). All barrier phases run on per-CTA counters that continue across
-// items, so the next item's Q load and first S MMAs overlap this item's tail.
+// (items are numbered heaviest first). All barrier phases run on per-CTA
+// counters that continue across items, so the next item's Q load and first S
+// MMA overlap this item's tail.
 // PAGED: K and V come from a pool of 16-token blocks [num_blocks, Hkv, 16, D]
 // addressed through the block table; the K/V tensor maps then cover the pool.
 template <int D, int EMU8, bool PAGED>
@@ -349,12 +345,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* k_empty = k_full + KSTAGES;
   uint64_t* v_full = k_empty + KSTAGES;
   uint64_t* v_empty = v_full + VSTAGES;
-  uint64_t* s_full = v_empty + VSTAGES;  // [tile][half]
-  // One P barrier per S half: the softmax can run at most one block ahead of
-  // its issuer's wait on a given half, so a parity wait never aliases.
-  uint64_t* p_full = s_full + 4;  // [tile][half]
-  uint64_t* o_ready = p_full + 4;
-  uint64_t* o_full = o_ready + 2;
+  // Per tile. S of block i+1 is issued only after P of block i has arrived,
+  // so neither side can run a phase ahead and a parity wait never aliases.
+  uint64_t* s_full = v_empty + VSTAGES;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
   uint64_t* mma_done = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
@@ -364,25 +359,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 2);  // both issuers' last S MMA of an item has read Q
-    // A K/V slot is free again once both MMA issuers have released it.
+    mbar_init(q_empty, 1);  // the item's last S MMA has read Q
     for (int s = 0; s < KSTAGES; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 2);
+      mbar_init(&k_empty[s], 1);
     }
     for (int s = 0; s < VSTAGES; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 2);
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&o_ready[t], 1);
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
       mbar_init(&o_full[t], 1);
     }
-    mbar_init(mma_done, 2);
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -411,7 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!w.active[0] && !w.active[1]) continue;
         if (PAGED && args.seqlens_k[w.b] > args.max_blocks * 16 && args.error_flags)
           atomicOr(args.error_flags, ATTN_FAULT_BAD_LENGTH);
-        // Q tiles: wait until both issuers' last S MMA of the previous item has read them.
+        // Q tiles: wait until the last S MMA of the previous item has read them.
         if (nq > 0 && !mbar_wait_bounded(q_empty, (nq - 1) & 1, abort_flag, WAIT_LIMIT)) break;
         mbar_arrive_expect_tx(q_full, (w.active[0] + w.active[1]) * L::Q_TILE);
         for (int t = 0; t < 2; ++t) {
@@ -449,9 +440,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = 0; c < L::CHUNKS; ++c)
               tma_load_4d(dst + c * (BK * 128), tm, &full[s], c * 64, blk * BK, w.kvh, w.b);
           } else {
-            // Four 16-token cache blocks; a block past the sequence end (or a
-            // table entry outside the pool) is read from one past the pool's
-            // last block, which TMA fills with zeros.
+            // BK / 16 cache blocks; a block past the sequence end (or a table
+            // entry outside the pool) is read from one past the pool's last
+            // block, which TMA fills with zeros.
             for (int j = 0; j < BK / 16; ++j) {
               const int tok = blk * BK + j * 16;
               int phys = args.num_blocks;
@@ -469,11 +460,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ++cnt;
           return true;
         };
-        // Consumption order within an item: K0, K1, then (V_i, K_{i+2}).
-        for (int i = 0; i < min(n_kv, 2) && ok; ++i) ok = load(false, i);
+        // The tensor core consumes K_0, V_0, K_1, V_1, ...; each load first
+        // waits for the block two back in its ring to be released.
         for (int i = 0; i < n_kv && ok; ++i) {
-          ok = load(true, i);
-          if (ok && i + 2 < n_kv) ok = load(false, i + 2);
+          ok = load(false, i);
+          if (ok) ok = load(true, i);
         }
       }
       // Drain: wait for the last copy issued into each slot, so no copy is in
@@ -483,96 +474,103 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int i = max(0, nv - VSTAGES); i < nv; ++i)
         mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
       if (nq > 0) mbar_wait_bounded(q_full, (nq - 1) & 1, abort_flag, WAIT_LIMIT);
-    } else if ((warp == MMA_WARP || warp == MMA1_WARP) && lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer of tile t
-      const int t = warp - MMA_WARP;
+    } else if (warp == MMA_WARP && lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer (both tiles)
+      // One thread issues every MMA in the fixed order S_0(0), S_1(0), then per
+      // block i: P_0 V_i, S_0(i+1), P_1 V_i, S_1(i+1). The tensor core runs them
+      // in that order, so tile 1's products fill the pipe while tile 0's
+      // softmax works and the other way round.
       constexpr uint32_t ID_S = instr_desc_bf16(BM, BK, 0);
       constexpr uint32_t ID_PV = instr_desc_bf16(BM, D, 1);
-      // Descriptors are computed once; advancing one by a byte offset adds
-      // (offset >> 4) to its start-address field (no carry: shared memory
-      // addresses stay below 256 KB).
-      const uint64_t q_desc = smem_desc_sw128(smem_addr(smem + L::Q_OFF + t * L::Q_TILE), 16, 1024);
-      const uint64_t k_desc = smem_desc_sw128(smem_addr(smem + L::K_OFF), 16, 1024);       // K-major
-      const uint64_t v_desc = smem_desc_sw128(smem_addr(smem + L::V_OFF), BK * 128, 1024);  // MN-major
-      const uint32_t d_s = tmem_base + t * 128;
-      const uint32_t d_o = tmem_base + 256 + t * 128;
-      // S_t = Q_t K^T of global block g into half g % 2 (K block in ring slot ks).
-      auto issue_s = [&](int g, int ks) {
-        const uint64_t ka = k_desc + (uint64_t)(((ks % KSTAGES) * L::KV_TILE) >> 4);
-        const uint32_t d = d_s + (g & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(d, q_desc + (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4),
-                 ka + (uint64_t)(((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4), ID_S, kk > 0);
+      // Shared-memory descriptors as low words (start address, leading byte
+      // offset) over one common high word (stride 1024 bytes, 128-byte
+      // swizzle); each MMA adds its k-step offset as an immediate.
+      const uint32_t hi = sw128_desc_hi(1024);
+      const uint32_t q_lo = sw128_desc_lo(smem_addr(smem + L::Q_OFF), 16);       // K-major
+      const uint32_t k_lo = sw128_desc_lo(smem_addr(smem + L::K_OFF), 16);       // K-major
+      const uint32_t v_lo = sw128_desc_lo(smem_addr(smem + L::V_OFF), BK * 128);  // MN-major
+      const uint32_t id_s = ID_S, id_pv = ID_PV;
+      // S_t = Q_t K^T for the K block in ring position kg.
+      auto issue_s = [&](int t, int kg) {
+        const uint32_t qa = q_lo + (uint32_t)((t * L::Q_TILE) >> 4);
+        const uint32_t ka = k_lo + (uint32_t)(((kg % KSTAGES) * L::KV_TILE) >> 4);
+        const uint32_t d = tmem_base + t * 128;
+        static_for<0, D / 16>([&](auto c) {
+          constexpr int kk = decltype(c)::value;
+          constexpr uint32_t a_off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+          constexpr uint32_t b_off = ((kk >> 2) * (BK * 128) + (kk & 3) * 32) >> 4;
+          mma_ss_lo<a_off, b_off>(d, qa, ka, hi, id_s, kk > 0 ? 1u : 0u);
+        });
       };
-      // O_t (+)= P_t V, P from TMEM (bf16 pairs in half g % 2), V in ring slot vs.
-      auto issue_pv = [&](int g, int vs, bool first) {
-        const uint64_t va = v_desc + (uint64_t)(((vs % VSTAGES) * L::KV_TILE) >> 4);
-        const uint32_t pa = d_s + (g & 1) * 64;
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          mma_ts(d_o, pa + kk * 8, va + (uint64_t)((kk * 16 * 128) >> 4), ID_PV, !first || (kk > 0));
+      // O_t (+)= P_t V, P from TMEM (bf16 pairs over S_t's first BK / 2
+      // columns), V in ring position vg.
+      auto issue_pv = [&](int t, int vg, bool first) {
+        const uint32_t va = v_lo + (uint32_t)(((vg % VSTAGES) * L::KV_TILE) >> 4);
+        const uint32_t d = tmem_base + 256 + t * 128, a = tmem_base + t * 128;
+        static_for<0, BK / 16>([&](auto c) {
+          constexpr int kk = decltype(c)::value;
+          constexpr uint32_t b_off = (kk * 16 * 128) >> 4;
+          mma_ts_lo<kk * 8, b_off>(d, a, va, hi, id_pv, (!first || kk > 0) ? 1u : 0u);
+        });
       };
-      int gb = 0;   // this tile's blocks so far (all items): S half / P barrier phases
-      int kb = 0;   // K / V blocks loaded before the current item (both rings advance alike)
-      int nq = 0;   // active items so far (Q phases)
+      int gb[2] = {0, 0};  // each tile's blocks so far (all items): S / P barrier phases
+      int kb = 0;          // K / V blocks loaded before the current item (both rings advance alike)
+      int nq = 0;          // active items so far (Q phases)
       bool ok = true;
       for (int kk_item = 0, item; ok && (item = snake_item(kk_item, n_items)) >= 0; ++kk_item) {
         const Work w = decode_work(args, item);
         if (!w.active[0] && !w.active[1]) continue;
-        const int nt = w.n_kv[t], nu = w.n_kv[t ^ 1];
-        const int n_kv = max(nt, nu);
-        // Release a K/V slot; when the other tile has no work for this block,
-        // also arrive on its behalf.
-        auto release = [&](uint64_t* bar, int blk) {
-          mma_commit(bar);
-          if (blk >= nu) mbar_arrive(bar);
+        const int n_kv = max(w.n_kv[0], w.n_kv[1]);
+        // S of block i for every tile that has it; then K_i can be released.
+        auto s_blocks = [&](int i) -> bool {
+          const int kg = kb + i;
+          if (!mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, WAIT_LIMIT)) return false;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (i >= w.n_kv[t]) continue;
+            issue_s(t, kg);
+            mma_commit(&s_full[t]);
+          }
+          mma_commit(&k_empty[kg % KSTAGES]);
+          if (i == n_kv - 1) mma_commit(q_empty);  // the item's last S MMA has been issued
+          return true;
         };
-        // Even with no block of its own, wait for this item's Q: its arrival on
-        // q_empty below must count toward this item's phase, not the previous one.
         ok = mbar_wait_bounded(q_full, nq & 1, abort_flag, WAIT_LIMIT);
-        for (int i = 0; i < min(nt, 2) && ok; ++i) {
-          const int kg = kb + i;  // K_i is the (kb + i)-th K block: K0, K1 lead each item
-          ok = mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(gb + i, kg);
-          mma_commit(&s_full[t * 2 + ((gb + i) & 1)]);
-          release(&k_empty[kg % KSTAGES], i);
-        }
-        if (ok && nt <= 2) {
-          // This tile's last S MMA of the item has been issued.
-          if (nt > 0) mma_commit(q_empty); else mbar_arrive(q_empty);
-        }
-        for (int i = 0; i < nt && ok; ++i) {
-          const int g = gb + i;
+        if (ok) ok = s_blocks(0);
+        for (int i = 0; i < n_kv && ok; ++i) {
           const int vg = kb + i;  // V_i is the (kb + i)-th V block
-          ok = mbar_wait_bounded(&v_full[vg % VSTAGES], (vg / VSTAGES) & 1, abort_flag, WAIT_LIMIT) &&
-               mbar_wait_bounded(&p_full[t * 2 + (g & 1)], (g >> 1) & 1, abort_flag, WAIT_LIMIT);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(g, vg, i == 0);
-          mma_commit(&o_ready[t]);
-          if (i == nt - 1) mma_commit(&o_full[t]);
-          release(&v_empty[vg % VSTAGES], i);
-          const int ik = i + 2;
-          if (ik < nt) {
-            const int kg = kb + ik;
-            ok = mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+          ok = mbar_wait_bounded(&v_full[vg % VSTAGES], (vg / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
+          const bool next = i + 1 < n_kv;
+          const int kg = kb + i + 1;
+          if (ok && next) ok = mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (i >= w.n_kv[t]) continue;
+            ok = mbar_wait_bounded(&p_full[t], (gb[t] + i) & 1, abort_flag, WAIT_LIMIT);
             if (!ok) break;
             tc_fence_after();
-            issue_s(g + 2, kg);
-            mma_commit(&s_full[t * 2 + (g & 1)]);
-            release(&k_empty[kg % KSTAGES], ik);
-            if (ik == nt - 1) mma_commit(q_empty);
+            issue_pv(t, vg, i == 0);
+            if (i == w.n_kv[t] - 1) mma_commit(&o_full[t]);
+            // S_t(i+1) overwrites the P just read: MMAs from one thread run
+            // in issue order.
+            if (i + 1 < w.n_kv[t]) {
+              issue_s(t, kg);
+              mma_commit(&s_full[t]);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&v_empty[vg % VSTAGES]);
+          if (next) {
+            mma_commit(&k_empty[kg % KSTAGES]);
+            if (i + 1 == n_kv - 1) mma_commit(q_empty);
           }
         }
-        gb += nt;
+        gb[0] += w.n_kv[0];
+        gb[1] += w.n_kv[1];
         kb += n_kv;
         ++nq;
       }
-      // Wait until every MMA issued by both issuers has completed before
-      // tensor memory can be released (bounded; matters on the abort path).
+      // Wait until every MMA has completed before tensor memory can be
+      // released (bounded; matters on the abort path).
       mma_commit(mma_done);
       mbar_wait_bounded(mma_done, 0, abort_flag, WAIT_LIMIT);
     }
@@ -609,13 +607,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float l = 0.f;         // running sum of 2^(s*scale*log2e - m2)
       for (int i = 0; i < nt; ++i) {
         const int g = gb + i;
-        ok = warp_wait(&s_full[t * 2 + (g & 1)], (g >> 1) & 1, abort_flag);
+        ok = warp_wait(&s_full[t], g & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tSi = tS + (g & 1) * 64;
         uint32_t sb[BK];
-        tmem_ld32(tSi, &sb[0]);
-        tmem_ld32(tSi + 32, &sb[32]);
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) tmem_ld32(tS + c * 32, &sb[c * 32]);
         tmem_ld_wait();
         float s[BK];
 #pragma unroll
@@ -643,10 +640,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (upd) m2 = m_new;
         const float m_off = (m2 == -INFINITY) ? 0.f : m2;
         if (i > 0 && __any_sync(0xffffffffu, upd)) {
-          // Rescale O once the previous P V (block g-1) has landed.
-          ok = warp_wait(&o_ready[t], (g - 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
+          // Rescale O in place. Its last writer, P V of the previous block,
+          // has completed: the commit that signalled this S tracks every
+          // earlier MMA of the issuer.
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -659,9 +655,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         float2 acc;
         if (need_mask)
-          exp_pack_store<0>(s, sl2, m_off, tSi, acc);
+          exp_pack_store<0>(s, sl2, m_off, tS, acc);
         else
-          exp_pack_store<EMU8>(s, sl2, m_off, tSi, acc);
+          exp_pack_store<EMU8>(s, sl2, m_off, tS, acc);
         l = l * alpha + (acc.x + acc.y);
         if (v_fix && i == nt - 1) {
           const int vg = kb + i, vs = vg % VSTAGES;
@@ -679,7 +675,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[t * 2 + (g & 1)]);
+        mbar_arrive(&p_full[t]);
       }
       gb += nt;
       kb += n_kv;
@@ -702,8 +698,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (has_keys) tc_fence_after();
       if (args.o_tma && w.row0[t] + sub * 32 + 32 <= w.sq) {  // warp-uniform
-        // This warp's 32 rows: stage them in shared memory (128-byte swizzle,
-        // conflict-free) and write them with tile stores issued by lane 0.
         uint8_t* stage = smem + L::O_OFF + warp * L::W_STAGE;
         const int r0 = w.row0[t] + sub * 32;
         if (args.o_f32)

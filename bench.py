@@ -289,7 +289,7 @@ def bench_prefill(args, rank, world, local, attn, peaks, peak_src):
                    "seq_len": cfg.seqlen_q, "head_dim": cfg.head_dim, "causal": cfg.causal,
                    "parallelism": f"replicas x{world} (no collective)",
                    "l2": "inputs larger than L2 (Q 64 MiB + K/V 32 MiB + O 64 MiB per step)"},
-        "roofline": {"bound": "tensor", "kernel": "prefill_fwd_kernel<128,4,true>",
+        "roofline": {"bound": "tensor", "kernel": "prefill_fwd_kernel<128,2,false>",
                      "achieved": round(per_rank_tflops, 2), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(per_rank_tflops / peak_t, 4),
                      "peak_source": f"{peak_src} bf16 burst (cuBLAS 8192^3)",

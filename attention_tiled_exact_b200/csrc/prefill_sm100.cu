@@ -73,8 +73,26 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_LIMIT = 2000000000LL;  // cycles (~1 s)
 constexpr float RESCALE_THRESHOLD = 8.0f;        // log2 units: rescale only when the max grows by > 2^8
 
+// Division by a runtime constant d for dividends in [0, 2^31): with
+// l = ceil(log2 d), p = 31 + l and m = ceil(2^p / d), n / d = (n * m) >> p
+// exactly (m * d - 2^p < d <= 2^l, so n * (m * d - 2^p) < 2^p). Set up on the
+// host; one 64-bit multiply and a shift on the device.
+struct FastDiv {
+  unsigned long long m;
+  int p, d;
+  __host__ void init(int divisor) {
+    d = divisor;
+    int l = 0;
+    while ((1ll << l) < (long long)divisor) ++l;
+    p = 31 + l;
+    m = ((1ull << p) + (unsigned long long)divisor - 1) / (unsigned long long)divisor;
+  }
+  __device__ __forceinline__ int div(int n) const { return (int)(((unsigned long long)(unsigned)n * m) >> p); }
+};
+
 struct Args {
   int batch, hq, hkv, group, seqlen_q, seqlen_k;
+  FastDiv fd_outer, fd_mid, fd_inner;  // item decode: per-row-block count, then the two inner factors
   float scale_log2;
   int causal;
   int pair_heads;
@@ -125,25 +143,28 @@ struct Work {
 __device__ __forceinline__ Work decode_work(const Args& a, int item) {
   Work w;
   if (a.pair_heads) {
-    const int pairs = a.group / 2;
-    const int per_rb = a.batch * a.hkv * pairs;
-    const int rb = a.n_row_blocks - 1 - item / per_rb;  // heaviest (causal) row blocks first
-    int r = item % per_rb;
-    const int pair = r % pairs;
-    r /= pairs;
-    w.kvh = r % a.hkv;
-    w.b = r / a.hkv;
+    // fd_outer: batch * hkv * pairs, fd_mid: pairs, fd_inner: hkv
+    const int pairs = a.fd_mid.d;
+    const int q0 = a.fd_outer.div(item);
+    const int rb = a.n_row_blocks - 1 - q0;  // heaviest (causal) row blocks first
+    int r = item - q0 * a.fd_outer.d;
+    const int q1 = a.fd_mid.div(r);
+    const int pair = r - q1 * pairs;
+    r = q1;
+    w.b = a.fd_inner.div(r);
+    w.kvh = r - w.b * a.hkv;
     w.head[0] = w.kvh * a.group + 2 * pair;
     w.head[1] = w.head[0] + 1;
     w.row0[0] = w.row0[1] = rb * BM;
   } else {
+    // fd_outer: batch * hq, fd_mid: hq, fd_inner: group
     const int npairs = (a.n_row_blocks + 1) / 2;
-    const int per = a.batch * a.hq;
-    const int p = npairs - 1 - item / per;
-    const int r = item % per;
-    const int h = r % a.hq;
-    w.b = r / a.hq;
-    w.kvh = h / a.group;
+    const int q0 = a.fd_outer.div(item);
+    const int p = npairs - 1 - q0;
+    const int r = item - q0 * a.fd_outer.d;
+    w.b = a.fd_mid.div(r);
+    const int h = r - w.b * a.hq;
+    w.kvh = a.fd_inner.div(h);
     w.head[0] = w.head[1] = h;
     w.row0[0] = 2 * p * BM;
     w.row0[1] = (2 * p + 1) * BM;
@@ -681,21 +702,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       kb += n_kv;
       if (!ok) break;
       // ------------------------------------------------------------ epilogue
+      // 1 / l and the LSE need no TMEM: done while the last P V runs.
+      const bool store = qrow < w.sq;
+      const bool empty = !(l > 0.f);
+      const float inv_l = empty ? 0.f : 1.f / l;
+      if (args.lse && store) {
+        const float lse = empty ? -INFINITY : (m2 + log2f(l)) * 0.69314718055994530942f;
+        args.lse[((long long)w.b * args.hq + w.head[t]) * args.seqlen_q + qrow] = lse;
+      }
       const bool has_keys = nt > 0;
       if (has_keys) {
         ok = warp_wait(&o_full[t], nf & 1, abort_flag);
         ++nf;
         if (!ok) break;
       }
-      const bool store = qrow < w.sq;
-      const bool empty = !(l > 0.f);
-      const float inv_l = empty ? 0.f : 1.f / l;
       const long long obase =
           (long long)w.b * args.o_bs + (long long)w.head[t] * args.o_hs + (long long)qrow * args.o_rs;
-      if (args.lse && store) {
-        const float lse = empty ? -INFINITY : (m2 + log2f(l)) * 0.69314718055994530942f;
-        args.lse[((long long)w.b * args.hq + w.head[t]) * args.seqlen_q + qrow] = lse;
-      }
       if (has_keys) tc_fence_after();
       if (args.o_tma && w.row0[t] + sub * 32 + 32 <= w.sq) {  // warp-uniform
         uint8_t* stage = smem + L::O_OFF + warp * L::W_STAGE;
@@ -860,6 +882,15 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.causal = p.causal ? 1 : 0;
   a.pair_heads = (a.group % 2 == 0) ? 1 : 0;
+  if (a.pair_heads) {
+    a.fd_outer.init(p.batch * p.num_kv_heads * (a.group / 2));
+    a.fd_mid.init(a.group / 2);
+    a.fd_inner.init(p.num_kv_heads);
+  } else {
+    a.fd_outer.init(p.batch * p.num_q_heads);
+    a.fd_mid.init(p.num_q_heads);
+    a.fd_inner.init(a.group);
+  }
   a.n_row_blocks = (p.seqlen_q + BM - 1) / BM;
   a.seqlens_q = p.seqlens_q;
   a.seqlens_k = p.seqlens_k;

@@ -227,11 +227,12 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Exponentials of one 64-score row block (s[]), their sum, and the packed bf16
-// P stored to TMEM 16 columns at a time. EMU8: in every 8 consecutive pairs, a
-// spread-out EMU8 of them take exp2 on the FMA pipe (exp2_poly2), the rest on
-// MUFU.
-template <int EMU8>
+// Exponentials of one row block of scores (s[]), their sum, and the packed
+// bf16 P stored to TMEM 16 columns at a time. EMU8: in every 8 consecutive
+// pairs, a spread-out EMU8 of them take exp2 on the FMA pipe (exp2_poly2), the
+// rest on MUFU. MASKED: masked scores are -inf; the polynomial clamps its
+// input, so its results are then replaced by an exact 0 (MUFU gives 0 itself).
+template <int EMU8, bool MASKED = false>
 __device__ __forceinline__ void exp_pack_store(const float (&s)[BK], float sl2, float m_off, uint32_t tP,
                                                float2& acc) {
   const float2 sc2 = make_float2(sl2, sl2);
@@ -247,6 +248,10 @@ __device__ __forceinline__ void exp_pack_store(const float (&s)[BK], float sl2, 
       float2 pr;
       if (((i * EMU8) & 7) < EMU8) {
         pr = exp2_poly2(x);
+        if (MASKED) {
+          pr.x = x.x == -INFINITY ? 0.f : pr.x;
+          pr.y = x.y == -INFINITY ? 0.f : pr.y;
+        }
       } else {
         pr.x = ex2_approx(x.x);
         pr.y = ex2_approx(x.y);
@@ -676,7 +681,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         float2 acc;
         if (need_mask)
-          exp_pack_store<0>(s, sl2, m_off, tS, acc);
+          exp_pack_store<EMU8, true>(s, sl2, m_off, tS, acc);
         else
           exp_pack_store<EMU8>(s, sl2, m_off, tS, acc);
         l = l * alpha + (acc.x + acc.y);

@@ -72,6 +72,10 @@ static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER == NUM_THREADS * REG_LAUNC
 constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_LIMIT = 2000000000LL;  // cycles (~1 s)
 constexpr float RESCALE_THRESHOLD = 8.0f;        // log2 units: rescale only when the max grows by > 2^8
+// Variable-length launches with at most SORT_MAX_ITEMS items sort the items by
+// cost before the snake assignment; a CTA then keeps at most LIST_MAX of them.
+constexpr int SORT_MAX_ITEMS = 4096;
+constexpr int LIST_MAX = 64;
 
 // Division by a runtime constant d for dividends in [0, 2^31): with
 // l = ceil(log2 d), p = 31 + l and m = ceil(2^p / d), n / d = (n * m) >> p
@@ -103,6 +107,7 @@ struct Args {
   float* lse;
   int o_f32;
   int o_tma;  // O rows of a full 32-row warp slice go out through the tm_o tile store
+  int sort_items;  // order items by cost (variable lengths) instead of row block
   long long o_bs, o_hs, o_rs;
   int32_t* error_flags;
   // paged keys/values (PAGED kernels only)
@@ -126,8 +131,10 @@ struct Layout {
   static constexpr int BAR_OFF = O_OFF + SOFTMAX_WARPS * W_STAGE;
   // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2], p_full[2], o_full[2], mma_done
   static constexpr int NUM_BARS = 2 + 2 * KSTAGES + 2 * VSTAGES + 2 + 2 + 2 + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr int BYTES = MISC_OFF + 16;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem address, abort flag, item count
+  static constexpr int LIST_OFF = MISC_OFF + 16;            // this CTA's items when they are sorted
+  static constexpr int BYTES = LIST_OFF + LIST_MAX * 4;
+  static_assert(SORT_MAX_ITEMS * 8 <= KSTAGES * KV_TILE, "item sort scratch lives in the K ring");
   static constexpr int SMEM_BYTES = BYTES + 1024;  // slack for 1024-byte alignment
 };
 
@@ -195,6 +202,51 @@ __device__ __forceinline__ int snake_item(int k, int n_items) {
   const int G = gridDim.x, c = blockIdx.x;
   const int item = k * G + ((k & 1) ? (G - 1 - c) : c);
   return item < n_items ? item : -1;
+}
+
+// Variable-length work: every CTA sorts all items by cost, largest first
+// (bitonic sort of (cost, ~item) keys in shared scratch, all threads), and
+// keeps the ones at its snake positions in the sorted list. Cost is the
+// item's key-block count plus a fixed per-item overhead of about 1.4 blocks
+// (epilogue and pipeline refill, measured). The scratch is the K ring, which
+// no copy has touched yet; a proxy fence orders these writes before the
+// first TMA writes there.
+__device__ void order_items(const Args& a, int n_items, unsigned long long* keys, int* list, int* n_mine) {
+  int np2 = 1;
+  while (np2 < n_items) np2 <<= 1;
+  for (int i = threadIdx.x; i < np2; i += blockDim.x) {
+    unsigned long long key = 0;  // padding sorts last
+    if (i < n_items) {
+      const Work w = decode_work(a, i);
+      const int n = (w.active[0] || w.active[1]) ? max(w.n_kv[0], w.n_kv[1]) : 0;
+      const unsigned cost = (unsigned)n * 8u + 11u;
+      key = ((unsigned long long)cost << 32) | (unsigned long long)(~(unsigned)i);  // ties: lower item first
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  for (int k = 2; k <= np2; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < np2; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long x = keys[i], y = keys[ixj];
+          if (((i & k) == 0) ? (x < y) : (x > y)) {  // descending overall
+            keys[i] = y;
+            keys[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int k = 0, pos; (pos = snake_item(k, n_items)) >= 0 && n < LIST_MAX; ++k)
+      list[n++] = (int)(~(unsigned)(keys[pos] & 0xffffffffull));
+    *n_mine = n;
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
 }
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -411,6 +463,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  int* item_list = reinterpret_cast<int*>(smem + L::LIST_OFF);
+  int* n_mine = reinterpret_cast<int*>(smem + L::MISC_OFF + 8);
+  if (args.sort_items)
+    order_items(args, n_items, reinterpret_cast<unsigned long long*>(smem + L::K_OFF), item_list, n_mine);
+  // The k-th item of this CTA (-1 past its last).
+  auto cta_item = [&](int k) -> int {
+    if (args.sort_items) return k < *n_mine ? item_list[k] : -1;
+    return snake_item(k, n_items);
+  };
 
   if (warp >= SOFTMAX_WARPS) {
     regs_dec<REG_OTHER>();
@@ -422,7 +483,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int nk = 0, nv = 0;  // K / V blocks issued so far (all items)
       int nq = 0;          // items whose Q was loaded
       bool ok = true;
-      for (int kk_item = 0, item; ok && (item = snake_item(kk_item, n_items)) >= 0; ++kk_item) {
+      for (int kk_item = 0, item; ok && (item = cta_item(kk_item)) >= 0; ++kk_item) {
         const Work w = decode_work(args, item);
         const int n_kv = max(w.n_kv[0], w.n_kv[1]);
         if (!w.active[0] && !w.active[1]) continue;
@@ -441,7 +502,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Bring the next item's Q tiles into L2 now, so that its shared-memory
         // load at the end of this item does not wait on HBM.
         {
-          const int nxt = snake_item(kk_item + 1, n_items);
+          const int nxt = cta_item(kk_item + 1);
           if (nxt >= 0) {
             const Work wn = decode_work(args, nxt);
             for (int t = 0; t < 2; ++t) {
@@ -543,7 +604,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int kb = 0;          // K / V blocks loaded before the current item (both rings advance alike)
       int nq = 0;          // active items so far (Q phases)
       bool ok = true;
-      for (int kk_item = 0, item; ok && (item = snake_item(kk_item, n_items)) >= 0; ++kk_item) {
+      for (int kk_item = 0, item; ok && (item = cta_item(kk_item)) >= 0; ++kk_item) {
         const Work w = decode_work(args, item);
         if (!w.active[0] && !w.active[1]) continue;
         const int n_kv = max(w.n_kv[0], w.n_kv[1]);
@@ -614,7 +675,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int kb = 0;  // K / V blocks loaded before the current item
     int nf = 0;  // items this tile finished (o_full phases)
     bool ok = true;
-    for (int kk_item = 0, item; ok && (item = snake_item(kk_item, n_items)) >= 0; ++kk_item) {
+    for (int kk_item = 0, item; ok && (item = cta_item(kk_item)) >= 0; ++kk_item) {
       const Work w = decode_work(args, item);
       if (!w.active[0] && !w.active[1]) continue;
       const int n_kv = max(w.n_kv[0], w.n_kv[1]);
@@ -844,7 +905,10 @@ static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk
   }
   if (state != 1) return ATTN_ERR_UNSUPPORTED;
   const int grid = items < device_sm_count() ? items : device_sm_count();
-  kern<<<grid, NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, to, a, items);
+  Args ak = a;
+  // Sort only when lengths vary per sequence and every CTA's share fits its list.
+  ak.sort_items = (a.seqlens_q || a.seqlens_k) && items <= SORT_MAX_ITEMS && (items + grid - 1) / grid <= LIST_MAX;
+  kern<<<grid, NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, to, ak, items);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

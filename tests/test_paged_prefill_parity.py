@@ -53,6 +53,37 @@ def test_paged_prefill_matches_oracle(lib, ctx, q_len, Hq, Hkv, D):
     assert_o_close(o16, O_ref, True, "paged prefill bf16")
 
 
+@pytest.mark.parametrize("n_seq,q_len,Hq,Hkv,D", [
+    (12, 256, 8, 2, 128),   # 96 work items: sorted by cost before they are dealt to the SMs
+    (260, 128, 32, 4, 64),  # 4160 work items: more than the sort takes, plain snake order
+])
+def test_paged_prefill_many_items(lib, n_seq, q_len, Hq, Hkv, D):
+    """Variable lengths with either item order: every valid row is written once
+    and matches the oracle (sampled rows), rows past q_lens[b] stay untouched."""
+    import torch
+    rng = np.random.default_rng(n_seq)
+    d = _chunks(rng.integers(0, 300, n_seq), q_len, Hq, Hkv, D, seed=90 + n_seq)
+    d["q_lens"] = rng.integers(1, q_len + 1, n_seq).astype(np.int32)
+    q = to_dev_bf16(d["q"])
+    out = torch.full(q.shape, 7.0, dtype=torch.float32, device="cuda")
+    lse = torch.full(q.shape[:3], 7.0, dtype=torch.float32, device="cuda")
+    lib.prefill_paged(q, to_dev_bf16(d["k_pool"]), to_dev_bf16(d["v_pool"]), to_dev_i32(d["block_table"]),
+                      to_dev_i32(d["kv_lens"]), to_dev_i32(d["q_lens"]), d["scale"], True, out=out, lse=lse)
+    torch.cuda.synchronize()
+    o, l = to_f64(out), to_f64(lse)
+    valid = np.arange(q_len)[None, None, :] < d["q_lens"][:, None, None]
+    assert np.isfinite(l[np.broadcast_to(valid, l.shape)]).all()
+    assert (l[~np.broadcast_to(valid, l.shape)] == 7.0).all() and (o[~np.broadcast_to(valid, l.shape)] == 7.0).all()
+    rows = [(0, 0, 0), (n_seq - 1, Hq - 1, int(d["q_lens"][-1]) - 1)]
+    for _ in range(60):
+        b = int(rng.integers(n_seq))
+        rows.append((b, int(rng.integers(Hq)), int(rng.integers(d["q_lens"][b]))))
+    O_ref, L_ref = ref.ref_prefill_paged(d["q"], d["q_lens"], d["k_pool"], d["v_pool"], d["block_table"],
+                                         d["kv_lens"], d["scale"], True, rows=rows)
+    assert_o_close(np.stack([o[b, h, i] for b, h, i in rows]), O_ref, False, "many items")
+    assert_lse_close(np.array([l[b, h, i] for b, h, i in rows]), L_ref, "many items lse")
+
+
 def test_paged_equals_dense_bitwise(lib):
     """Same tokens, dense [B,H,S,D] layout vs identity-ordered pages: identical bits."""
     import torch

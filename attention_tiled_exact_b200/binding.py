@@ -142,9 +142,12 @@ def _need(cond, msg):
 
 
 def prefill(q, k, v, scale: float | None = None, causal: bool = False, out=None, lse=None,
-            out_dtype=torch.bfloat16, want_lse: bool = True, error_flags=None):
+            out_dtype=torch.bfloat16, want_lse: bool = True, error_flags=None, seqlens_q=None, seqlens_k=None):
     """Tiled prefill attention. q [B,Hq,Sq,D], k/v [B,Hkv,Sk,D] bf16 CUDA tensors.
 
+    seqlens_q / seqlens_k (int32 [B] CUDA tensors, optional): valid query rows
+    and keys of each sequence of a padded batch (rows past seqlens_q[b] are
+    not written).
     Returns ``(O [B,Hq,Sq,D], LSE [B,Hq,Sq] fp32 or None)``.
     """
     _need(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be 4-D [B, H, S, D]")
@@ -170,6 +173,10 @@ def prefill(q, k, v, scale: float | None = None, causal: bool = False, out=None,
     p.o_batch_stride, p.o_head_stride, p.o_row_stride = out.stride(0), out.stride(1), out.stride(2)
     p.scale, p.causal, p.o_dtype = float(scale), int(bool(causal)), _out_code(out.dtype)
     p.error_flags = _ptr(error_flags)
+    for name, t in (("seqlens_q", seqlens_q), ("seqlens_k", seqlens_k)):
+        if t is not None:
+            _need(t.dtype == torch.int32 and t.is_cuda and t.is_contiguous() and t.numel() == B, f"int32 {name} [B]")
+    p.seqlens_q, p.seqlens_k = _ptr(seqlens_q), _ptr(seqlens_k)
     _check(LIB.attn_prefill(ctypes.byref(p), _stream(q.device)), "attn_prefill")
     return out, lse
 

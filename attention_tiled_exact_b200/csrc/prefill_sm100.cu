@@ -182,6 +182,7 @@ __device__ __forceinline__ Work decode_work(const Args& a, int item) {
   if (w.sq < 0) w.sq = 0;
   if (w.sk < 0) w.sk = 0;
   if (a.block_table && w.sk > a.max_blocks * 16) w.sk = a.max_blocks * 16;  // flagged by the producer
+  if (!a.block_table && w.sk > a.seqlen_k) w.sk = a.seqlen_k;  // dense keys end at the tensor's length
   for (int t = 0; t < 2; ++t) {
     w.active[t] = w.row0[t] < w.sq;
     int kend = w.sk;

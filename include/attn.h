@@ -86,6 +86,10 @@ typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1 } attn_dtype_t;
  * multiples of 8 elements (16 bytes); o 16-byte aligned with strides that are
  * multiples of 8 elements; seqlen_q, seqlen_k >= 0 (k and v may be NULL when
  * seqlen_k == 0: every row then gets O = 0, LSE = -inf); scale > 0 and finite.
+ * Variable lengths in a padded dense batch: seqlens_q and seqlens_k (device,
+ * [batch], each nullable) give sequence b's valid query rows (<= seqlen_q;
+ * rows past it are not written) and keys (larger values are clamped to
+ * seqlen_k); the causal alignment then uses the per-sequence lengths.
  *
  * Paged keys/values (chunked prefill over a KV cache, "抱infra脚" Chunked
  * Prefill and Paged Attention): set k_cache/v_cache non-NULL (then k and v

@@ -9,7 +9,7 @@ import pytest
 
 from attention_tiled_exact_b200 import workloads as wl
 from oracle import attention_ref as ref
-from tests.helpers import assert_lse_close, assert_o_close, to_dev_bf16, to_f64
+from tests.helpers import assert_lse_close, assert_o_close, to_dev_bf16, to_dev_i32, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -89,6 +89,34 @@ def test_strided_inputs(lib):
     torch.cuda.synchronize()
     assert_o_close(to_f64(o), O_ref, False, "strided")
     assert_lse_close(to_f64(lse), L_ref, "strided")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_dense_varlen_padded_batch(lib, causal):
+    """A padded dense batch with per-sequence query and key lengths: every sequence
+    matches the oracle on its own slice (bottom-right causal alignment per
+    sequence), rows past seqlens_q[b] are left untouched, a key length past the
+    tensor is clamped to it, and a sequence without keys gets O = 0, LSE = -inf."""
+    import torch
+    B, Hq, Hkv, Sq, Sk, D = 6, 8, 2, 300, 420, 128
+    d = _case(B, Hq, Hkv, Sq, Sk, D, causal, seed=77)
+    rng = np.random.default_rng(7)
+    lq = rng.integers(1, Sq + 1, B).astype(np.int32)
+    lk = rng.integers(1, Sk + 1, B).astype(np.int32)
+    lq[0], lk[1], lk[2], lk[3] = Sq, Sk, 0, Sk + 50  # full rows, full keys, no keys, clamped keys
+    q, k, v = to_dev_bf16(d["q"]), to_dev_bf16(d["k"]), to_dev_bf16(d["v"])
+    out = torch.full((B, Hq, Sq, D), 7.0, dtype=torch.float32, device="cuda")
+    lse = torch.full((B, Hq, Sq), 7.0, dtype=torch.float32, device="cuda")
+    lib.prefill(q, k, v, d["scale"], causal, out=out, lse=lse, seqlens_q=to_dev_i32(lq), seqlens_k=to_dev_i32(lk))
+    torch.cuda.synchronize()
+    o, l = to_f64(out), to_f64(lse)
+    for b in range(B):
+        nq, nk = int(lq[b]), min(int(lk[b]), Sk)
+        O_ref, L_ref = ref.ref_attention(d["q"][b:b + 1, :, :nq], d["k"][b:b + 1, :, :nk], d["v"][b:b + 1, :, :nk],
+                                         d["scale"], causal)
+        assert_o_close(o[b:b + 1, :, :nq], O_ref, False, f"seq {b}")
+        assert_lse_close(l[b:b + 1, :, :nq], L_ref, f"seq {b} lse")
+        assert (o[b, :, nq:] == 7.0).all() and (l[b, :, nq:] == 7.0).all(), f"seq {b}: rows past seqlens_q written"
 
 
 def test_repeated_calls_are_deterministic(lib):

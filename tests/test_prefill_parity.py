@@ -91,15 +91,19 @@ def test_strided_inputs(lib):
     assert_lse_close(to_f64(lse), L_ref, "strided")
 
 
-@pytest.mark.parametrize("causal", [True, False])
-def test_dense_varlen_padded_batch(lib, causal):
+@pytest.mark.parametrize("Hq,Hkv,D,causal", [
+    (8, 2, 128, True),   # GQA G=4: two query heads per item
+    (8, 2, 128, False),
+    (6, 2, 64, True),    # G=3 (odd): two row blocks of one head per item, D=64
+])
+def test_dense_varlen_padded_batch(lib, Hq, Hkv, D, causal):
     """A padded dense batch with per-sequence query and key lengths: every sequence
     matches the oracle on its own slice (bottom-right causal alignment per
     sequence), rows past seqlens_q[b] are left untouched, a key length past the
     tensor is clamped to it, and a sequence without keys gets O = 0, LSE = -inf."""
     import torch
-    B, Hq, Hkv, Sq, Sk, D = 6, 8, 2, 300, 420, 128
-    d = _case(B, Hq, Hkv, Sq, Sk, D, causal, seed=77)
+    B, Sq, Sk = 6, 300, 420
+    d = _case(B, Hq, Hkv, Sq, Sk, D, causal, seed=77 + D + Hq)
     rng = np.random.default_rng(7)
     lq = rng.integers(1, Sq + 1, B).astype(np.int32)
     lk = rng.integers(1, Sk + 1, B).astype(np.int32)

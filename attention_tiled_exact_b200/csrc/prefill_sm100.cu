@@ -513,6 +513,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         const int32_t* table = PAGED ? args.block_table + (long long)w.b * args.max_blocks : nullptr;
+        // Paged: the physical cache blocks of key block blk, read from the
+        // table once for K and V and all before any copy is issued (the copies
+        // are ordered memory operations, so reading the table between them
+        // would expose one global-load latency per cache block). A block past
+        // the sequence end, or a table entry outside the pool (flagged), is
+        // read from one past the pool's last block, which TMA fills with zeros.
+        int phys[BK / 16];
+        auto fetch_table = [&](int blk) {
+          if constexpr (PAGED) {
+            int e[BK / 16];
+#pragma unroll
+            for (int j = 0; j < BK / 16; ++j) {
+              const int tok = blk * BK + j * 16;
+              e[j] = tok < w.sk ? table[tok >> 4] : args.num_blocks;
+            }
+#pragma unroll
+            for (int j = 0; j < BK / 16; ++j) {
+              const int tok = blk * BK + j * 16;
+              const bool good = e[j] >= 0 && e[j] < args.num_blocks;
+              if (tok < w.sk && !good && args.error_flags) atomicOr(args.error_flags, ATTN_FAULT_BAD_BLOCK);
+              phys[j] = good ? e[j] : args.num_blocks;
+            }
+          }
+        };
         auto load = [&](bool is_v, int blk) -> bool {
           int& cnt = is_v ? nv : nk;
           const int stages = is_v ? VSTAGES : KSTAGES;
@@ -528,22 +552,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = 0; c < L::CHUNKS; ++c)
               tma_load_4d(dst + c * (BK * 128), tm, &full[s], c * 64, blk * BK, w.kvh, w.b);
           } else {
-            // BK / 16 cache blocks; a block past the sequence end (or a table
-            // entry outside the pool) is read from one past the pool's last
-            // block, which TMA fills with zeros.
-            for (int j = 0; j < BK / 16; ++j) {
-              const int tok = blk * BK + j * 16;
-              int phys = args.num_blocks;
-              if (tok < w.sk) {
-                const int e = table[tok >> 4];
-                if (e >= 0 && e < args.num_blocks)
-                  phys = e;
-                else if (args.error_flags)
-                  atomicOr(args.error_flags, ATTN_FAULT_BAD_BLOCK);
-              }
+            for (int j = 0; j < BK / 16; ++j)
               for (int c = 0; c < L::CHUNKS; ++c)
-                tma_load_4d(dst + c * (BK * 128) + j * (16 * 128), tm, &full[s], c * 64, 0, w.kvh, phys);
-            }
+                tma_load_4d(dst + c * (BK * 128) + j * (16 * 128), tm, &full[s], c * 64, 0, w.kvh, phys[j]);
           }
           ++cnt;
           return true;
@@ -551,6 +562,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // The tensor core consumes K_0, V_0, K_1, V_1, ...; each load first
         // waits for the block two back in its ring to be released.
         for (int i = 0; i < n_kv && ok; ++i) {
+          fetch_table(i);
           ok = load(false, i);
           if (ok) ok = load(true, i);
         }

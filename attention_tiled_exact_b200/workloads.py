@@ -230,6 +230,50 @@ def make_paged_pool(seed: int, kv_lens, kv_heads: int, head_dim: int, spare_bloc
                 kv_lens=kv_lens, spare_ids=spare)
 
 
+# FP8 E4M3 (OCP, no infinities): sign bit 7, exponent bits 6..3 with bias 7,
+# mantissa bits 2..0; exponent 0 is subnormal (m / 8 * 2^-6); code 0x7F is NaN.
+# The non-negative finite codes 0x00..0x7E in increasing order of value:
+def _e4m3_table() -> np.ndarray:
+    c = np.arange(0x7F)
+    e, m = c >> 3, (c & 7).astype(np.float64)
+    return np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+
+
+_E4M3_VALUES = _e4m3_table()
+FP8_NAN = np.uint8(0x7F)
+
+
+def e4m3_codes(x) -> np.ndarray:
+    """Round values to the nearest FP8 E4M3 code (ties to the even code),
+    saturating at +-448; NaN maps to the NaN code."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.clip(np.searchsorted(_E4M3_VALUES, a, side="left"), 0, len(_E4M3_VALUES) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - _E4M3_VALUES[lo], _E4M3_VALUES[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = code | (np.signbit(x).astype(np.uint8) << 7)
+    return np.where(np.isnan(x), FP8_NAN, code).astype(np.uint8)
+
+
+def make_decode_fp8(cfg: DecodeConfig, kv_lens=None, identity: bool = False) -> dict:
+    """Paged decode inputs with an FP8 E4M3 cache and one scale per tensor.
+
+    The N(0,1) bf16 pools of :func:`make_decode` are quantised to codes with
+    scale = max|x| / 448 over the valid entries (NaN sentinels in spare blocks
+    and tail slots become the NaN code). Returns the make_decode dict with
+    ``k_pool`` / ``v_pool`` as uint8 codes and ``k_scale`` / ``v_scale``.
+    """
+    d = make_decode(cfg, kv_lens=kv_lens, identity=identity)
+    for name in ("k", "v"):
+        f = (d[name + "_pool"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        scale = float(np.nanmax(np.abs(f))) / 448.0 if np.isfinite(f).any() else 1.0
+        d[name + "_pool"] = e4m3_codes(f / scale)
+        d[name + "_scale"] = scale
+    return d
+
+
 def make_decode(cfg: DecodeConfig, kv_lens=None, identity: bool = False) -> dict:
     """Paged decode inputs: q [B, Hq, D] and a paged pool for the lengths."""
     if kv_lens is None:

@@ -39,6 +39,15 @@ closed forms (one key, causal row 0, zero query, constant V, hand-derived
 weights), torch's fp64 CPU ``scaled_dot_product_attention`` with repeated
 K/V, and invariants (key permutation, split-and-combine, paged vs contiguous,
 GQA vs repeated MHA). No function here is "parity unpinned".
+
+FP8 KV cache ("5.2 推理加速的未来趋势：新算法、新硬件、新协同", 协同层 section:
+an FP8 KV cache halves its memory at almost no accuracy cost). The pages give
+no format details or scale convention; the reading taken here is the OCP
+E4M3 format without infinities (sign, 4 exponent bits with bias 7, 3 mantissa
+bits; S.1111.111 is NaN) and one scale per tensor: a cached code c stands for
+decode(c) * k_scale (keys) or decode(c) * v_scale (values). Pins: decoded
+values of hand-checked codes, every code against torch's float8_e4m3fn, and
+FP8 decode equal to the bf16-style definition on the dequantised values.
 """
 from __future__ import annotations
 
@@ -51,6 +60,21 @@ def bf16_bits_to_f64(bits) -> np.ndarray:
     """Decode bf16 bit patterns (uint16) exactly into float64."""
     u = np.asarray(bits).astype(np.uint16).astype(np.uint32) << np.uint32(16)
     return u.view(np.float32).astype(np.float64)
+
+
+def e4m3_bits_to_f64(bits) -> np.ndarray:
+    """Decode FP8 E4M3 codes (uint8) exactly into float64.
+
+    Bit 7 is the sign, bits 6..3 the exponent e (bias 7), bits 2..0 the
+    mantissa m: e == 0 gives the subnormal m / 8 * 2^-6, otherwise the value
+    is (1 + m / 8) * 2^(e - 7); e == 15 with m == 7 is NaN (no infinities).
+    """
+    b = np.asarray(bits).astype(np.int64)
+    sign = np.where((b & 0x80) != 0, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    return np.where((e == 15) & (b & 0x7 == 7), np.nan, sign * mag)
 
 
 def _as_f64(x) -> np.ndarray:
@@ -176,6 +200,18 @@ def ref_decode_paged(q, k_pool, v_pool, block_table, seq_lens, scale, rows=None)
     if rows is None:
         return O.reshape(B, Hq, D), L.reshape(B, Hq)
     return O, L
+
+
+def ref_decode_paged_fp8(q, k_pool, v_pool, k_scale, v_scale, block_table, seq_lens, scale, rows=None):
+    """Decode over an FP8 E4M3 cache with one scale per tensor.
+
+    Pools hold uint8 codes [NB, Hkv, 16, D]; the cached key (value) is
+    decode(code) * k_scale (v_scale). The decode definition above then applies
+    unchanged to those values.
+    """
+    kf = e4m3_bits_to_f64(k_pool) * float(k_scale)
+    vf = e4m3_bits_to_f64(v_pool) * float(v_scale)
+    return ref_decode_paged(q, kf, vf, block_table, seq_lens, scale, rows)
 
 
 def ref_prefill_paged(q, q_lens, k_pool, v_pool, block_table, k_lens, scale, causal, rows=None):

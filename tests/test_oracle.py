@@ -319,3 +319,53 @@ def test_pins_reject_planted_mistakes(mutant):
     assert np.allclose(Oc, Ob, atol=1e-12) and np.allclose(Lc, Lb, atol=1e-12)
     Om, Lm = _candidate(q, k, v, 0.5, True, mutant)
     assert not (np.allclose(Om, Ob, atol=1e-6) and np.allclose(Lm, Lb, atol=1e-6))
+
+
+# ----------------------------------------------------------------------------
+# FP8 E4M3 cache: the format decode and the decode oracle over it
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x38, 1.0), (0x40, 2.0), (0x3C, 1.5), (0x3F, 1.875), (0x7E, 448.0), (0xFE, -448.0),
+    (0x77, 240.0), (0x08, 2.0 ** -6), (0x07, 7 * 2.0 ** -9), (0x01, 2.0 ** -9), (0xB8, -1.0), (0x30, 0.5),
+])
+def test_e4m3_decode_hand_codes(code, value):
+    """Values worked out by hand from the format: exponent bias 7, 3 mantissa bits, subnormals at e = 0."""
+    assert ref.e4m3_bits_to_f64(np.array([code], dtype=np.uint8))[0] == value
+
+
+def test_e4m3_decode_matches_torch_on_every_code():
+    torch = pytest.importorskip("torch")
+    codes = np.arange(256, dtype=np.uint8)
+    t = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    o = ref.e4m3_bits_to_f64(codes)
+    assert np.array_equal(np.isnan(t), np.isnan(o)) and np.isnan(o).sum() == 2  # 0x7F and 0xFF
+    assert np.array_equal(t[~np.isnan(t)], o[~np.isnan(o)])
+    assert np.array_equal(np.signbit(t[~np.isnan(t)]), np.signbit(o[~np.isnan(o)]))
+
+
+def test_fp8_decode_oracle_matches_brute_force():
+    """Tiny FP8 cache: the paged FP8 decode oracle against math.fsum loops on the
+    hand-gathered, hand-dequantised keys and values of every sequence."""
+    cfg = wl.DecodeConfig("t", 3, 4, 2, 8, 1, 1, 21)
+    lens = np.array([5, 17, 1], dtype=np.int32)
+    d = wl.make_decode_fp8(cfg, kv_lens=lens)
+    O, L = ref.ref_decode_paged_fp8(d["q"], d["k_pool"], d["v_pool"], d["k_scale"], d["v_scale"],
+                                    d["block_table"], lens, d["scale"])
+    qf = ref.bf16_bits_to_f64(d["q"])
+
+    def dequant(code, s):  # sign, exponent bias 7, 3 mantissa bits
+        c = int(code)
+        sign = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 15, c & 7
+        return sign * s * ((m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7))
+
+    for b, Lb in enumerate(lens):
+        toks = [(d["block_table"][b][t // 16], t % 16) for t in range(Lb)]
+        for h in range(4):
+            kvh = h // 2
+            kk = [[[dequant(d["k_pool"][p, kvh, s, j], d["k_scale"]) for j in range(8)] for p, s in toks]]
+            vv = [[[dequant(d["v_pool"][p, kvh, s, j], d["v_scale"]) for j in range(8)] for p, s in toks]]
+            Ob, Lbr = oracle.brute_attention([[[list(qf[b, h])]]], [kk], [vv], d["scale"], False)
+            assert np.allclose(O[b, h], Ob[0][0][0], atol=1e-12) and abs(L[b, h] - Lbr[0][0][0]) < 1e-12

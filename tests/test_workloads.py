@@ -70,3 +70,17 @@ def test_pair_counts():
     assert wl.causal_pairs(4, 6, True) == 3 + 4 + 5 + 6
     assert wl.causal_pairs(6, 4, True) == 0 + 0 + 1 + 2 + 3 + 4
     assert wl.causal_pairs(5, 7, False) == 35
+
+
+def test_e4m3_encoder_round_trips_every_finite_code():
+    """Every finite E4M3 value encodes back to its own code (+0 / -0 kept apart)."""
+    from oracle import attention_ref as ref
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = ref.e4m3_bits_to_f64(codes)
+    assert np.array_equal(wl.e4m3_codes(vals), codes)
+
+
+def test_e4m3_encoder_rounding():
+    """Ties go to the even code, values past 448 saturate, NaN stays NaN."""
+    x = np.array([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 500.0, -1e9, np.nan])
+    assert [int(c) for c in wl.e4m3_codes(x)] == [0x38, 0x3A, 0x00, 0x02, 0x7E, 0xFE, 0x7F]

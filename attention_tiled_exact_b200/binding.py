@@ -30,6 +30,7 @@ ATTN_ERR_NO_DEVICE = 7
 
 ATTN_DTYPE_BF16 = 0
 ATTN_DTYPE_F32 = 1
+ATTN_DTYPE_FP8_E4M3 = 2
 
 ATTN_FAULT_TIMEOUT = 0x1
 ATTN_FAULT_BAD_BLOCK = 0x2
@@ -67,7 +68,7 @@ class DecodeParams(ctypes.Structure):
         ("batch", _i32), ("num_q_heads", _i32), ("num_kv_heads", _i32), ("head_dim", _i32),
         ("block_size", _i32), ("max_blocks_per_seq", _i32), ("num_blocks", _i32),
         ("max_seq_len", _i32), ("num_splits", _i32), ("scale", ctypes.c_float), ("o_dtype", _i32),
-        ("error_flags", _vp),
+        ("error_flags", _vp), ("kv_dtype", _i32), ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
     ]
 
 
@@ -228,8 +229,12 @@ def prefill_paged(q, k_cache, v_cache, block_table, seqlens_k, seqlens_q=None, s
 # ----------------------------------------------------------------------------
 
 
+def _is_fp8(t) -> bool:
+    return t.dtype in (torch.uint8, torch.float8_e4m3fn)
+
+
 def _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits, out, lse,
-                   error_flags):
+                   error_flags, k_scale=None, v_scale=None):
     B, Hq, D = q.shape
     NB, Hkv, BS, D2 = k_cache.shape
     p = DecodeParams()
@@ -241,6 +246,9 @@ def _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_le
     p.scale = float(scale if scale is not None else 1.0 / math.sqrt(D))
     p.o_dtype = _out_code(out.dtype) if out is not None else ATTN_DTYPE_BF16
     p.error_flags = _ptr(error_flags)
+    if _is_fp8(k_cache):
+        p.kv_dtype = ATTN_DTYPE_FP8_E4M3
+        p.k_scale, p.v_scale = float(k_scale if k_scale is not None else 1.0), float(v_scale if v_scale is not None else 1.0)
     return p
 
 
@@ -255,17 +263,18 @@ def decode_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, max_seq_l
 
 def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None, max_seq_len: int = 0,
                  num_splits: int = 0, out=None, lse=None, workspace=None, out_dtype=torch.bfloat16,
-                 want_lse: bool = True, error_flags=None):
+                 want_lse: bool = True, error_flags=None, k_scale=None, v_scale=None):
     """Flash-Decoding over a paged KV cache.
 
-    q [B,Hq,D] bf16; k_cache/v_cache [NB,Hkv,16,D] bf16; block_table [B,maxblk]
-    int32; seq_lens [B] int32 (all CUDA). ``max_seq_len`` is a host-side
-    upper bound of seq_lens used for the split plan (0 = table capacity).
-    Returns ``(O [B,Hq,D], LSE [B,Hq] or None)``.
+    q [B,Hq,D] bf16; k_cache/v_cache [NB,Hkv,16,D] bf16, or FP8 E4M3 codes
+    (torch.uint8 or torch.float8_e4m3fn) standing for code * k_scale and
+    code * v_scale; block_table [B,maxblk] int32; seq_lens [B] int32 (all
+    CUDA). ``max_seq_len`` is a host-side upper bound of seq_lens used for the
+    split plan (0 = table capacity). Returns ``(O [B,Hq,D], LSE [B,Hq] or None)``.
     """
     _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
-    _need(q.dtype == torch.bfloat16 and k_cache.dtype == torch.bfloat16 and v_cache.dtype == torch.bfloat16,
-          "bf16 q and caches")
+    _need(q.dtype == torch.bfloat16 and k_cache.dtype == v_cache.dtype and
+          (k_cache.dtype == torch.bfloat16 or _is_fp8(k_cache)), "bf16 q; bf16 or FP8 E4M3 caches")
     _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
     _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
           "int32 block table [B, max_blocks]")
@@ -276,7 +285,7 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None
     if lse is None and want_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits, out, lse,
-                       error_flags)
+                       error_flags, k_scale, v_scale)
     need = ctypes.c_size_t(0)
     _check(LIB.attn_decode_paged(ctypes.byref(p), None, 0, ctypes.byref(need), None), "attn_decode_paged(size)")
     if workspace is None and need.value > 0:
@@ -289,7 +298,7 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None
 
 
 def decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, out, lse=None, scale: float | None = None,
-                         max_seq_len: int = 0, num_splits: int = 0, error_flags=None):
+                         max_seq_len: int = 0, num_splits: int = 0, error_flags=None, k_scale=None, v_scale=None):
     """:func:`decode_paged` for callers that cannot allocate device memory.
 
     The caller passes every input and the outputs (``out`` [B,Hq,D] bf16 or
@@ -298,15 +307,15 @@ def decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, out, lse=No
     the library. Calls that overlap on the GPU race on that array.
     """
     _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
-    _need(q.dtype == torch.bfloat16 and k_cache.dtype == torch.bfloat16 and v_cache.dtype == torch.bfloat16,
-          "bf16 q and caches")
+    _need(q.dtype == torch.bfloat16 and k_cache.dtype == v_cache.dtype and
+          (k_cache.dtype == torch.bfloat16 or _is_fp8(k_cache)), "bf16 q; bf16 or FP8 E4M3 caches")
     _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
     _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
           "int32 block table [B, max_blocks]")
     _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "int32 seq_lens [B]")
     _need(out is not None and tuple(out.shape) == tuple(q.shape) and out.is_contiguous(), "out [B, Hq, D]")
     p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits, out, lse,
-                       error_flags)
+                       error_flags, k_scale, v_scale)
     _check(LIB.attn_decode_paged_noalloc(ctypes.byref(p), _stream(q.device)), "attn_decode_paged_noalloc")
     return out, lse
 

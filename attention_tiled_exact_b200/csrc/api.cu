@@ -91,6 +91,10 @@ attn_status_t validate_decode(const attn_decode_params* p) {
   if ((int64_t)p->max_blocks_per_seq * 16 > INT32_MAX / 2) return ATTN_ERR_INVALID_ARG;
   if (!(p->scale > 0.f) || !isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
   if (p->o_dtype != ATTN_DTYPE_BF16 && p->o_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  if (p->kv_dtype != ATTN_DTYPE_BF16 && p->kv_dtype != ATTN_DTYPE_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  if (p->kv_dtype == ATTN_DTYPE_FP8_E4M3 &&
+      (!(p->k_scale > 0.f) || !isfinite(p->k_scale) || !(p->v_scale > 0.f) || !isfinite(p->v_scale)))
+    return ATTN_ERR_INVALID_ARG;
   if (!p->q || !p->k_cache || !p->v_cache || !p->block_table || !p->seq_lens || !p->o) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
     return ATTN_ERR_UNSUPPORTED;

@@ -15,21 +15,32 @@
 //     the block table with coalesced 16-byte cp.async copies (a warp moves a
 //     4 KB K block and a 4 KB V block per step, 512 contiguous bytes per
 //     instruction) into a 3-stage per-warp shared-memory ring;
-//   * q.k: lane (half h, chunk c) holds 8 head_dim elements of 8 tokens; partial
-//     dot products for all G heads use packed fp32 FMAs, then a transposing
-//     butterfly over the 16 lanes of a half-warp finishes them with 8G/16
-//     values per lane;
-//   * online softmax per head with the running max kept stale until it grows by
-//     more than 2^8 (O and the row sum stay consistent); p is exchanged through
-//     shared memory; O accumulates p * v with packed fp32 FMAs;
+//   * q.k on the warp-level tensor cores (mma.sync m16n8k16, fp32 accumulate):
+//     the G query heads are the rows of A (zero-padded to 16), the block's 16
+//     tokens the columns of B, with head_dim permuted identically on both
+//     sides so that each thread reads its K row slice as contiguous 16-byte
+//     loads; the online softmax of a head then runs on its 4 lanes with
+//     shuffles, the running max kept stale until it grows by more than 2^8 (O
+//     and the row sum stay consistent);
+//   * O += p * v: for bf16 caches on the CUDA cores in fp32 (p goes through
+//     shared memory to lanes holding 8 head_dim elements of 8 tokens, packed
+//     fp32 FMAs); for FP8 caches also on the tensor cores with P kept in
+//     registers as fp16 (the score fragments of the two 8-token tiles form
+//     the A fragment of one k = 16 step), which keeps the FP8 kernel on the
+//     memory bound instead of the instruction bound;
 //   * masked tokens (past the sequence end, or a block whose table entry is out
 //     of range) get p = 0 and their values are never multiplied in, so stale or
 //     NaN cache contents cannot leak into the result;
 //   * the 4 warps' states are merged in shared memory; a sequence with a single
 //     split writes O and LSE directly, otherwise the split writes its partial.
+//   * FP8 cache (E4M3 codes, one scale per tensor): blocks are 2 KB, pairs of
+//     codes are widened exactly to fp16 with cvt.rn.f16x2.e4m3x2, the key
+//     scale multiplies the scores and the value scale O once at the end.
 // Combine kernel: one warp per (sequence, query head) row, 16-byte loads.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
+#include <string.h>
 #include <stdint.h>
 
 #include "internal.h"
@@ -48,8 +59,9 @@ constexpr float LN2 = 0.69314718055994530942f;
 
 struct Args {
   const __nv_bfloat16* q;
-  const __nv_bfloat16* k_cache;
-  const __nv_bfloat16* v_cache;
+  const uint8_t* k_cache;  // bf16 elements, or E4M3 codes for the FP8 kernels
+  const uint8_t* v_cache;
+  float k_scale, v_scale;  // FP8 only
   const int32_t* block_table;
   const int32_t* seq_lens;
   void* o;
@@ -62,11 +74,10 @@ struct Args {
   int32_t* error_flags;
 };
 
-template <int G>
+template <int G, bool FP8 = false>
 struct Smem {
-  uint8_t kv[WARPS][NST][2][BLOCK_BYTES];  // 96 KB
-  float sc[WARPS][G][BS];                  // scores (log2 units)
-  float p[WARPS][2][BS / 2][G];            // probabilities, [token parity][token / 2][head]
+  uint8_t kv[WARPS][NST][2][FP8 ? BLOCK_BYTES / 2 : BLOCK_BYTES];  // 96 KB (bf16) / 48 KB (FP8)
+  float p[WARPS][2][BS / 2][G];  // bf16 caches: probabilities, [token parity][token / 2][head]
   float alpha[WARPS][G];
 };
 
@@ -90,6 +101,67 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
+// Two E4M3 codes (low byte = first element) widened exactly to fp32: every
+// E4M3 value, subnormals included, is a normal fp16 value.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t w) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(w));
+  __half2 h;
+  memcpy(&h, &h2, 4);
+  return __half22float2(h);
+}
+
+// D(16x8, fp32) += A(16x16) * B(16x8), warp-level tensor-core MMA with bf16 or
+// fp16 operands (two packed elements per register).
+template <bool F16>
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  if constexpr (F16)
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(w));
+  return h2;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const float2 f = bf16x2_to_float2(w);
+  __half2 h = __floats2half2_rn(f.x, f.y);
+  uint32_t r;
+  memcpy(&r, &h, 4);
+  return r;
+}
+
+// Eight cache elements of one row (this lane's head_dim chunk) as fp32 pairs.
+template <bool FP8>
+__device__ __forceinline__ void load_row8(const uint8_t* row, int c, bool zero, float2 (&x)[4]) {
+  if constexpr (FP8) {
+    uint2 r = *reinterpret_cast<const uint2*>(row + c * 8);
+    if (zero) r = make_uint2(0u, 0u);
+    x[0] = e4m3x2_to_float2(r.x & 0xffffu);
+    x[1] = e4m3x2_to_float2(r.x >> 16);
+    x[2] = e4m3x2_to_float2(r.y & 0xffffu);
+    x[3] = e4m3x2_to_float2(r.y >> 16);
+  } else {
+    uint4 r = *reinterpret_cast<const uint4*>(row + c * 16);
+    if (zero) r = make_uint4(0u, 0u, 0u, 0u);
+    x[0] = bf16x2_to_float2(r.x);
+    x[1] = bf16x2_to_float2(r.y);
+    x[2] = bf16x2_to_float2(r.z);
+    x[3] = bf16x2_to_float2(r.w);
+  }
+}
+
 // Sequence length clamped to the block table's capacity (flagging a fault).
 __device__ __forceinline__ int checked_len(const Args& a, int b) {
   int L = a.seq_lens[b];
@@ -100,13 +172,30 @@ __device__ __forceinline__ int checked_len(const Args& a, int b) {
   return L;
 }
 
-template <int G>
+// q.k on the warp-level tensor cores. The G query heads are the rows
+// of A (padded to 16 with zeros), the block's 16 tokens the columns of B (two
+// n = 8 tiles), head_dim the reduction in 8 steps of 16. Inside a step, the
+// reduction index that thread t holds (2t, 2t+1, 2t+8, 2t+9) is mapped to the
+// physical elements 32 t + 4 step + (0, 1, 2, 3) in both A and B (a dot
+// product does not depend on the order of its terms), so each thread reads
+// its K row as 32 contiguous elements. Scores land with head = lane / 4 and
+// tokens 8 n + 2 (lane % 4) + (0, 1): the softmax of a head runs on its 4
+// lanes with shuffles.
+// MMA_PV: O += P V on the tensor cores as well. P stays in
+// registers (the score fragments of the two 8-token tiles form the A fragment
+// of one k = 16 step), V is the B operand with head_dim permuted so that n-tile
+// j, column n reads element 16 n + j: each thread then gathers its 4 token rows
+// (2t, 2t+1, 2t+8, 2t+9) as 16 contiguous elements and holds the output of
+// head lane / 4 for the 32 contiguous elements 32 (lane % 4) + 0..31.
+template <int G, bool FP8, bool MMA_PV>
 __global__ void __launch_bounds__(WARPS * 32)
     decode_split_kernel(const Args a) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
-  constexpr int NF = (G >= 2) ? G / 2 : 1;  // scores per lane after the reduction
+  constexpr int ELEM = FP8 ? 1 : 2;              // bytes per cache element
+  constexpr int ROW = D * ELEM;                  // bytes per cached token row
+  constexpr int CHUNKS16 = BS * ROW / (16 * 32);  // 16-byte copies per lane per block
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  Smem<G>& sm = *reinterpret_cast<Smem<G>*>(smem_raw);
+  Smem<G, FP8>& sm = *reinterpret_cast<Smem<G, FP8>*>(smem_raw);
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
@@ -126,16 +215,22 @@ __global__ void __launch_bounds__(WARPS * 32)
   const int blk_end = (t_end + BS - 1) / BS;
   const int32_t* table = a.block_table + (long long)b * a.max_blocks;
 
-  // q for the G heads: this lane's 8 elements (chunk c), as 4 pairs per head.
-  float2 q2[G][4];
+  // A fragments of q (head lane / 4, elements 32 (lane % 4) + 4 step + (0, 1)
+  // and (2, 3)); rows past G and rows 8..15 are zero. fp16 operands for FP8
+  // caches (every E4M3 value is exact in fp16), bf16 otherwise.
+  uint32_t qa[8][2];
+  {
+    const int gq = lane >> 2, tq = lane & 3;
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const uint4 raw =
-        *reinterpret_cast<const uint4*>(a.q + ((long long)b * a.hq + kvh * G + g) * D + c * 8);
-    q2[g][0] = bf16x2_to_float2(raw.x);
-    q2[g][1] = bf16x2_to_float2(raw.y);
-    q2[g][2] = bf16x2_to_float2(raw.z);
-    q2[g][3] = bf16x2_to_float2(raw.w);
+    for (int w = 0; w < 4; ++w) {
+      uint4 r = make_uint4(0u, 0u, 0u, 0u);
+      if (gq < G)
+        r = *reinterpret_cast<const uint4*>(a.q + ((long long)b * a.hq + kvh * G + gq) * D + 32 * tq + 8 * w);
+      qa[2 * w][0] = FP8 ? bf16x2_to_f16x2(r.x) : r.x;
+      qa[2 * w][1] = FP8 ? bf16x2_to_f16x2(r.y) : r.y;
+      qa[2 * w + 1][0] = FP8 ? bf16x2_to_f16x2(r.z) : r.z;
+      qa[2 * w + 1][1] = FP8 ? bf16x2_to_f16x2(r.w) : r.w;
+    }
   }
 
   float2 o2[G][4];
@@ -143,7 +238,12 @@ __global__ void __launch_bounds__(WARPS * 32)
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int m = 0; m < 4; ++m) o2[g][m] = make_float2(0.f, 0.f);
-  float m_run = -INFINITY, l_run = 0.f;  // meaningful in lanes g < G (head g)
+  float ot[16][2];  // MMA_PV: O of head lane / 4, element 32 (lane % 4) + 16 j + nt in ot[nt][j]
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) ot[nt][0] = ot[nt][1] = 0.f;
+  float zpad[2] = {0.f, 0.f};  // rows 8..15 of the MMA accumulator: padding, always zero
+  // Running max / sum of head g, replicated in its lanes 4g .. 4g+3.
+  float m_run = -INFINITY, l_run = 0.f;
 
   // This warp's blocks: blk_begin + warp, + WARPS, ...
   const int n_mine = (blk_end - blk_begin - warp + WARPS - 1) / WARPS;
@@ -158,15 +258,15 @@ __global__ void __launch_bounds__(WARPS * 32)
       bool valid;
       const int ph = phys_of(block_of(n), valid);
       if (valid) {
-        const long long off = ((long long)ph * a.hkv + kvh) * (BS * D);
-        const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(a.k_cache + off);
-        const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(a.v_cache + off);
+        const long long off = ((long long)ph * a.hkv + kvh) * (BS * ROW);  // bytes
+        const uint8_t* ksrc = a.k_cache + off;
+        const uint8_t* vsrc = a.v_cache + off;
         uint8_t* kdst = sm.kv[warp][n % NST][0];
         uint8_t* vdst = sm.kv[warp][n % NST][1];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cp_async16(kdst + (i * 32 + lane) * 16, ksrc + (i * 32 + lane) * 16);
+        for (int i = 0; i < CHUNKS16; ++i) cp_async16(kdst + (i * 32 + lane) * 16, ksrc + (i * 32 + lane) * 16);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cp_async16(vdst + (i * 32 + lane) * 16, vsrc + (i * 32 + lane) * 16);
+        for (int i = 0; i < CHUNKS16; ++i) cp_async16(vdst + (i * 32 + lane) * 16, vsrc + (i * 32 + lane) * 16);
       }
     }
     cp_async_commit();
@@ -188,87 +288,134 @@ __global__ void __launch_bounds__(WARPS * 32)
     const uint8_t* kblk = sm.kv[warp][n % NST][0];
     const uint8_t* vblk = sm.kv[warp][n % NST][1];
 
-    // ---- partial q.k for 8 tokens (2i + hw) x G heads over this lane's 8 elements
-    float v[8 * G];
+    // ---- S = q K^T on the tensor cores, then the online softmax per head on its 4 lanes
+    const int gq = lane >> 2, tq = lane & 3;
+    float cacc[2][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint4 kr = *reinterpret_cast<const uint4*>(kblk + (2 * i + hw) * (D * 2) + c * 16);
-      const float2 k0 = bf16x2_to_float2(kr.x), k1 = bf16x2_to_float2(kr.y), k2 = bf16x2_to_float2(kr.z),
-                   k3 = bf16x2_to_float2(kr.w);
+    for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float2 acc = __fmul2_rn(q2[g][0], k0);
-        acc = __ffma2_rn(q2[g][1], k1, acc);
-        acc = __ffma2_rn(q2[g][2], k2, acc);
-        acc = __ffma2_rn(q2[g][3], k3, acc);
-        v[i * G + g] = acc.x + acc.y;
+      for (int j = 0; j < 4; ++j) cacc[nt][j] = 0.f;
+      const uint8_t* krow = kblk + (8 * nt + gq) * ROW + 32 * tq * ELEM;
+      uint32_t kw[8 * ELEM];  // this thread's 32 elements of the token row
+#pragma unroll
+      for (int v4 = 0; v4 < 2 * ELEM; ++v4) {
+        const uint4 r = *reinterpret_cast<const uint4*>(krow + 16 * v4);
+        kw[4 * v4 + 0] = r.x;
+        kw[4 * v4 + 1] = r.y;
+        kw[4 * v4 + 2] = r.z;
+        kw[4 * v4 + 3] = r.w;
+      }
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t b0, b1;
+        if constexpr (FP8) {
+          b0 = e4m3x2_to_f16x2(kw[ks] & 0xffffu);
+          b1 = e4m3x2_to_f16x2(kw[ks] >> 16);
+        } else {
+          b0 = kw[2 * ks];
+          b1 = kw[2 * ks + 1];
+        }
+        mma_16816<FP8>(cacc[nt], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
       }
     }
-    // ---- transposing butterfly over the 16 lanes of the half-warp
-    {
-      int n_cur = 8 * G;
+    const float sl2 = FP8 ? a.scale_log2 * a.k_scale : a.scale_log2;  // cached key = code * k_scale
+    float sc[4];
 #pragma unroll
-      for (int mask = 8; mask >= 1; mask >>= 1) {
-        if (n_cur >= 2) {
-          const int half = n_cur / 2;
-          const bool up = (c & mask) != 0;
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int k = 0; k < 8 * G / 2; ++k) {
-            if (k < half) {
-              const float send = up ? v[k] : v[half + k];
-              const float keep = up ? v[half + k] : v[k];
-              v[k] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
-            }
-          }
-          n_cur = half;
-        } else {
-          v[0] += __shfl_xor_sync(0xffffffffu, v[0], mask);
+      for (int j = 0; j < 2; ++j) {
+        const int tk = 8 * nt + 2 * tq + j;
+        sc[2 * nt + j] = (tk < n_valid) ? cacc[nt][j] * sl2 : -INFINITY;
+      }
+    float bm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+    const float m_new = fmaxf(m_run, bm);
+    const bool upd = (m_new - m_run) > RESCALE_THRESHOLD;
+    const float alpha = upd ? ex2_approx(m_run - m_new) : 1.f;
+    if (upd) m_run = m_new;
+    const float mo = (m_run == -INFINITY) ? 0.f : m_run;
+    float pr[4], rs = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      pr[j] = ex2_approx(sc[j] - mo);
+      rs += pr[j];
+    }
+    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+    l_run = l_run * alpha + rs;
+    if constexpr (MMA_PV) {
+      if (alpha != 1.f) {
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          ot[nt][0] *= alpha;
+          ot[nt][1] *= alpha;
         }
       }
-    }
-    // lane holds NF finished scores, global index base + k -> token 2*(idx/G) + hw, head idx%G
-    const int base = (G >= 2) ? NF * c : (c >> 1);
-#pragma unroll
-    for (int k = 0; k < NF; ++k) {
-      const int idx = base + k;
-      const int tk = 2 * (idx / G) + hw;
-      const int g = idx % G;
-      const float s = (tk < n_valid) ? v[k] * a.scale_log2 : -INFINITY;
-      sm.sc[warp][g][tk] = s;
-    }
-    __syncwarp();
-    // ---- online softmax, lane g owns head g
-    if (lane < G) {
-      float s[BS];
-#pragma unroll
-      for (int t4 = 0; t4 < BS / 4; ++t4) {
-        const float4 x = *reinterpret_cast<const float4*>(&sm.sc[warp][lane][t4 * 4]);
-        s[t4 * 4 + 0] = x.x;
-        s[t4 * 4 + 1] = x.y;
-        s[t4 * 4 + 2] = x.z;
-        s[t4 * 4 + 3] = x.w;
+      // A = P (head gq, tokens 2t, 2t+1 | 8+2t, 8+2t+1); padding heads are zero.
+      uint32_t pa0 = 0u, pa2 = 0u;
+      if (gq < G) {
+        if constexpr (FP8) {
+          __half2 h0 = __floats2half2_rn(pr[0], pr[1]), h2 = __floats2half2_rn(pr[2], pr[3]);
+          memcpy(&pa0, &h0, 4);
+          memcpy(&pa2, &h2, 4);
+        } else {
+          pa0 = pack_bf16x2(pr[0], pr[1]);
+          pa2 = pack_bf16x2(pr[2], pr[3]);
+        }
       }
-      float bm = s[0];
+      // B = V: rows 2t, 2t+1, 2t+8, 2t+9 (masked rows read as zero), elements 16 gq .. 16 gq + 15.
+      constexpr int WPR = 4 * ELEM;  // 32-bit words per 16-element row slice
+      uint32_t vr[4][WPR];
 #pragma unroll
-      for (int t = 1; t < BS; ++t) bm = fmaxf(bm, s[t]);
-      const float m_new = fmaxf(m_run, bm);
-      const bool upd = (m_new - m_run) > RESCALE_THRESHOLD;
-      const float alpha = upd ? ex2_approx(m_run - m_new) : 1.f;
-      if (upd) m_run = m_new;
-      const float mo = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
+      for (int r = 0; r < 4; ++r) {
+        const int tk = 2 * tq + (r & 1) + 8 * (r >> 1);
+        const bool keep = tk < n_valid;
 #pragma unroll
-      for (int t = 0; t < BS; ++t) {
-        const float p = ex2_approx(s[t] - mo);
-        rs += p;
-        sm.p[warp][t & 1][t >> 1][lane] = p;
+        for (int v4 = 0; v4 < ELEM; ++v4) {
+          uint4 x = *reinterpret_cast<const uint4*>(vblk + tk * ROW + 16 * gq * ELEM + 16 * v4);
+          if (!keep) x = make_uint4(0u, 0u, 0u, 0u);
+          vr[r][4 * v4 + 0] = x.x;
+          vr[r][4 * v4 + 1] = x.y;
+          vr[r][4 * v4 + 2] = x.z;
+          vr[r][4 * v4 + 3] = x.w;
+        }
       }
-      l_run = l_run * alpha + rs;
-      sm.alpha[warp][lane] = alpha;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        uint32_t b0, b1;
+        if constexpr (FP8) {  // byte nt of the two rows -> one E4M3 pair -> fp16 pair
+          const int w = nt >> 2, j = nt & 3;
+          const uint32_t sel = (uint32_t)(j | ((j + 4) << 4));
+          b0 = e4m3x2_to_f16x2(__byte_perm(vr[0][w], vr[1][w], sel));
+          b1 = e4m3x2_to_f16x2(__byte_perm(vr[2][w], vr[3][w], sel));
+        } else {  // half nt of the two rows -> one bf16 pair
+          const int w = nt >> 1;
+          const uint32_t sel = (nt & 1) ? 0x7632u : 0x5410u;
+          b0 = __byte_perm(vr[0][w], vr[1][w], sel);
+          b1 = __byte_perm(vr[2][w], vr[3][w], sel);
+        }
+        float acc[4] = {ot[nt][0], ot[nt][1], zpad[0], zpad[1]};
+        mma_16816<FP8>(acc, pa0, 0u, pa2, 0u, b0, b1);
+        ot[nt][0] = acc[0];
+        ot[nt][1] = acc[1];
+      }
+    } else {
+      if (gq < G) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int tk = 8 * nt + 2 * tq + j;
+            sm.p[warp][tk & 1][tk >> 1][gq] = pr[2 * nt + j];
+          }
+        if (tq == 0) sm.alpha[warp][gq] = alpha;
+      }
+      __syncwarp();
     }
-    __syncwarp();
-    // ---- O += p * v
-    {
+
+    // ---- O += p * v (CUDA cores)
+    if constexpr (!MMA_PV) {
       float al[G];
       bool any = false;
 #pragma unroll
@@ -288,10 +435,9 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int tk = 2 * i + hw;
-        uint4 vr = *reinterpret_cast<const uint4*>(vblk + tk * (D * 2) + c * 16);
-        if (!full && tk >= n_valid) vr = make_uint4(0u, 0u, 0u, 0u);  // never multiply masked values in
-        const float2 v0 = bf16x2_to_float2(vr.x), v1 = bf16x2_to_float2(vr.y), v2 = bf16x2_to_float2(vr.z),
-                     v3 = bf16x2_to_float2(vr.w);
+        float2 vx[4];
+        load_row8<FP8>(vblk + tk * ROW, c, !full && tk >= n_valid, vx);  // never multiply masked values in
+        const float2 v0 = vx[0], v1 = vx[1], v2 = vx[2], v3 = vx[3];
         float pg[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) pg[g] = sm.p[warp][hw][i][g];
@@ -308,22 +454,46 @@ __global__ void __launch_bounds__(WARPS * 32)
     __syncwarp();  // the slot is refilled by the next issue
   }
   cp_async_wait<0>();
+  if constexpr (FP8) {  // cached value = code * v_scale: applied to O once
+    const float2 vs = make_float2(a.v_scale, a.v_scale);
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) o2[g][m] = __fmul2_rn(o2[g][m], vs);
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      ot[nt][0] *= a.v_scale;
+      ot[nt][1] *= a.v_scale;
+    }
+  }
 
   // ---- merge the two half-warps (disjoint tokens, same running max)
+  if constexpr (!MMA_PV) {
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+    for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      o2[g][m].x += __shfl_xor_sync(0xffffffffu, o2[g][m].x, 16);
-      o2[g][m].y += __shfl_xor_sync(0xffffffffu, o2[g][m].y, 16);
-    }
+      for (int m = 0; m < 4; ++m) {
+        o2[g][m].x += __shfl_xor_sync(0xffffffffu, o2[g][m].x, 16);
+        o2[g][m].y += __shfl_xor_sync(0xffffffffu, o2[g][m].y, 16);
+      }
+  }
   __syncthreads();  // the KV ring is reused for the merge
   MergeSmem<G>& mg = *reinterpret_cast<MergeSmem<G>*>(smem_raw);
-  if (lane < G) {
-    mg.m[warp][lane] = m_run;
-    mg.l[warp][lane] = l_run;
+  if ((lane & 3) == 0 && (lane >> 2) < G) {
+    mg.m[warp][lane >> 2] = m_run;
+    mg.l[warp][lane >> 2] = l_run;
   }
-  if (hw == 0) {
+  if constexpr (MMA_PV) {
+    if ((lane >> 2) < G) {
+      float* dst = &mg.o[warp][lane >> 2][32 * (lane & 3)];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          *reinterpret_cast<float4*>(dst + 16 * j + 4 * q4) =
+              make_float4(ot[4 * q4][j], ot[4 * q4 + 1][j], ot[4 * q4 + 2][j], ot[4 * q4 + 3][j]);
+    }
+  } else if (hw == 0) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float4* dst = reinterpret_cast<float4*>(&mg.o[warp][g][c * 8]);
@@ -493,11 +663,11 @@ DecodePlan plan_decode(const attn_decode_params& p) {
   return plan;
 }
 
-template <int G>
+template <int G, bool FP8>
 static attn_status_t launch_decode_g(const decode::Args& a, const DecodePlan& plan, cudaStream_t stream) {
-  auto kern = decode::decode_split_kernel<G>;
-  const int smem = (int)sizeof(decode::Smem<G>);
-  static_assert(sizeof(decode::MergeSmem<G>) <= sizeof(decode::Smem<G>), "merge buffer fits");
+  auto kern = decode::decode_split_kernel<G, FP8, FP8>;  // P V on the tensor cores for FP8 caches
+  const int smem = (int)sizeof(decode::Smem<G, FP8>);
+  static_assert(sizeof(decode::MergeSmem<G>) <= sizeof(decode::Smem<G, FP8>), "merge buffer fits");
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -514,8 +684,11 @@ attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan,
   if (p.batch == 0) return ATTN_OK;
   decode::Args a;
   a.q = reinterpret_cast<const __nv_bfloat16*>(p.q);
-  a.k_cache = reinterpret_cast<const __nv_bfloat16*>(p.k_cache);
-  a.v_cache = reinterpret_cast<const __nv_bfloat16*>(p.v_cache);
+  a.k_cache = reinterpret_cast<const uint8_t*>(p.k_cache);
+  a.v_cache = reinterpret_cast<const uint8_t*>(p.v_cache);
+  const bool fp8 = p.kv_dtype == ATTN_DTYPE_FP8_E4M3;
+  a.k_scale = fp8 ? p.k_scale : 1.f;
+  a.v_scale = fp8 ? p.v_scale : 1.f;
   a.block_table = p.block_table;
   a.seq_lens = p.seq_lens;
   a.o = p.o;
@@ -537,10 +710,10 @@ attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan,
   a.error_flags = p.error_flags;
   attn_status_t st;
   switch (p.num_q_heads / p.num_kv_heads) {
-    case 1: st = launch_decode_g<1>(a, plan, stream); break;
-    case 2: st = launch_decode_g<2>(a, plan, stream); break;
-    case 4: st = launch_decode_g<4>(a, plan, stream); break;
-    case 8: st = launch_decode_g<8>(a, plan, stream); break;
+    case 1: st = fp8 ? launch_decode_g<1, true>(a, plan, stream) : launch_decode_g<1, false>(a, plan, stream); break;
+    case 2: st = fp8 ? launch_decode_g<2, true>(a, plan, stream) : launch_decode_g<2, false>(a, plan, stream); break;
+    case 4: st = fp8 ? launch_decode_g<4, true>(a, plan, stream) : launch_decode_g<4, false>(a, plan, stream); break;
+    case 8: st = fp8 ? launch_decode_g<8, true>(a, plan, stream) : launch_decode_g<8, false>(a, plan, stream); break;
     default: return ATTN_ERR_UNSUPPORTED;
   }
   if (st != ATTN_OK || plan.max_splits <= 1) return st;

@@ -257,20 +257,48 @@ def e4m3_codes(x) -> np.ndarray:
     return np.where(np.isnan(x), FP8_NAN, code).astype(np.uint8)
 
 
+def bf16_pool_to_e4m3(pool: np.ndarray, chunk: int = 1 << 24) -> tuple:
+    """Quantise a bf16 pool (uint16 bits) to E4M3 codes with one scale,
+    scale = max|x| / 448 over its finite entries; NaN entries get the NaN code.
+
+    Each of the 65536 bf16 bit patterns is rounded once (a lookup table), so
+    the pool itself is only gathered through the table, chunk by chunk.
+    """
+    flat = pool.reshape(-1)
+    starts = range(0, flat.size, chunk)
+
+    def chunk_amax(i):
+        a = flat[i:i + chunk] & np.uint16(0x7FFF)
+        return int(np.where(a < np.uint16(0x7F80), a, np.uint16(0)).max()) if a.size else 0  # finite only
+
+    with _cf.ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        amax_bits = max(ex.map(chunk_amax, starts), default=0)
+    amax = float(np.array([amax_bits << 16], dtype=np.uint32).view(np.float32)[0])
+    scale = amax / 448.0 if amax > 0 else 1.0
+    with np.errstate(invalid="ignore"):  # the NaN patterns stay NaN
+        values = (np.arange(1 << 16, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+        table = e4m3_codes(values / scale)
+    out = np.empty(flat.size, dtype=np.uint8)
+
+    def chunk_codes(i):
+        np.take(table, flat[i:i + chunk], out=out[i:i + chunk])
+
+    with _cf.ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        list(ex.map(chunk_codes, starts))
+    return out.reshape(pool.shape), scale
+
+
 def make_decode_fp8(cfg: DecodeConfig, kv_lens=None, identity: bool = False) -> dict:
     """Paged decode inputs with an FP8 E4M3 cache and one scale per tensor.
 
-    The N(0,1) bf16 pools of :func:`make_decode` are quantised to codes with
-    scale = max|x| / 448 over the valid entries (NaN sentinels in spare blocks
-    and tail slots become the NaN code). Returns the make_decode dict with
-    ``k_pool`` / ``v_pool`` as uint8 codes and ``k_scale`` / ``v_scale``.
+    The N(0,1) bf16 pools of :func:`make_decode` are quantised with
+    :func:`bf16_pool_to_e4m3` (NaN sentinels in spare blocks and tail slots
+    become the NaN code). Returns the make_decode dict with ``k_pool`` /
+    ``v_pool`` as uint8 codes and ``k_scale`` / ``v_scale``.
     """
     d = make_decode(cfg, kv_lens=kv_lens, identity=identity)
     for name in ("k", "v"):
-        f = (d[name + "_pool"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-        scale = float(np.nanmax(np.abs(f))) / 448.0 if np.isfinite(f).any() else 1.0
-        d[name + "_pool"] = e4m3_codes(f / scale)
-        d[name + "_scale"] = scale
+        d[name + "_pool"], d[name + "_scale"] = bf16_pool_to_e4m3(d[name + "_pool"])
     return d
 
 
@@ -289,12 +317,14 @@ def relayout_identity(pool: np.ndarray, table: np.ndarray, kv_lens) -> tuple:
     """Copy a paged pool into identity order (sequence 0's blocks first, ...).
 
     Returns ``(new_pool, new_table)`` holding the same logical tokens; used by
-    the bit-exact paging test. Unused slots stay NaN.
+    the bit-exact paging test. Unused slots stay NaN (bf16 bits, or the E4M3
+    NaN code for uint8 pools).
     """
     kv_lens = np.asarray(kv_lens, dtype=np.int64)
     nblk = (kv_lens + BLOCK_SIZE - 1) // BLOCK_SIZE
     used = int(nblk.sum())
-    new_pool = np.full((used + 1,) + pool.shape[1:], BF16_NAN, dtype=np.uint16)
+    fill = FP8_NAN if pool.dtype == np.uint8 else BF16_NAN
+    new_pool = np.full((used + 1,) + pool.shape[1:], fill, dtype=pool.dtype)
     new_table = np.full(table.shape, used, dtype=np.int32)
     off = 0
     for b, n in enumerate(nblk):

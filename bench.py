@@ -6,7 +6,8 @@ A step is one prefill call over the causal GQA workload (batch 4, 32 query /
 ``value`` is its throughput in TFLOP/s of algorithmic work (4 * head_dim per
 visible query-key pair and query head). The same JSON line also carries the
 paged split-KV decode workload (batch 64, lengths U[1024, 32768], 32/8 heads)
-timed the same way, in GB/s of algorithmic KV traffic, and the mixed batch
+timed the same way, in GB/s of algorithmic KV traffic (also on an FP8 E4M3
+copy of the cache, one scale per tensor), and the mixed batch
 (8 prefill chunks of 512 queries on cached context plus 128 decode rows over
 one paged cache) as a fraction of the combined tensor + HBM roofline.
 
@@ -19,6 +20,7 @@ max-over-ranks device time.
 from __future__ import annotations
 
 import argparse
+import functools
 import hashlib
 import json
 import os
@@ -177,6 +179,7 @@ def prefill_inputs(rank: int):
     return cfg, d, flops
 
 
+@functools.lru_cache(maxsize=2)
 def decode_inputs(rank: int, batch: int = 0):
     import dataclasses
     cfg = dataclasses.replace(DECODE_CFG, seed=DECODE_CFG.seed + 1000 * rank,
@@ -220,6 +223,8 @@ def run_ours(args, rank, world, local):
         result.update(bench_prefill(args, rank, world, local, attn, peaks, peak_src))
     if args.only in (None, "decode"):
         result["decode"] = bench_decode(args, rank, world, local, attn, peaks, peak_src)
+    if args.only in (None, "decodefp8"):
+        result["decode_fp8"] = bench_decode_fp8(args, rank, world, local, attn, peaks, peak_src)
     if args.only in (None, "mixed"):
         result["mixed"] = bench_mixed(args, rank, world, local, attn, peaks, peak_src)
     if args.only in (None, "prefill16k"):
@@ -334,6 +339,44 @@ def bench_decode(args, rank, world, local, attn, peaks, peak_src):
                          "peak_source": f"{peak_src} copy bandwidth", "traffic": profiled_traffic("decode"),
                          "algorithmic_bytes_per_launch": dbytes},
             "gpu_launches_per_step": 2, "clocks": dclk.summary()}
+
+
+def bench_decode_fp8(args, rank, world, local, attn, peaks, peak_src):
+    """The decode workload on an FP8 E4M3 cache (the bf16 pools quantised with one scale per tensor)."""
+    import torch
+    dcfg, dd, _ = decode_inputs(rank, args.decode_batch)
+    kq, k_scale = wl.bf16_pool_to_e4m3(dd["k_pool"])
+    vq, v_scale = wl.bf16_pool_to_e4m3(dd["v_pool"])
+    tokens = int(dd["kv_lens"].sum())
+    dbytes = float(tokens * dcfg.kv_heads * dcfg.head_dim * 1 * 2 + dcfg.batch * dcfg.q_heads * (dcfg.head_dim * 2 * 2 + 4))
+    dq = _dev_bf16(dd["q"])
+    kc, vc = torch.from_numpy(kq).cuda(), torch.from_numpy(vq).cuda()
+    del kq, vq
+    bt = torch.from_numpy(dd["block_table"]).cuda()
+    sl = torch.from_numpy(dd["kv_lens"]).cuda()
+    max_len = int(dd["kv_lens"].max())
+    dout = torch.empty_like(dq)
+    dlse = torch.empty(dq.shape[:2], dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(attn.decode_workspace_bytes(dq, kc, vc, bt, sl, max_seq_len=max_len), 1),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        attn.decode_paged(dq, kc, vc, bt, sl, dcfg.scale, max_seq_len=max_len, out=dout, lse=dlse, workspace=ws,
+                          k_scale=k_scale, v_scale=v_scale)
+
+    dsteps = max(args.steps, 5)
+    with ClockSampler(local) as clk:
+        ms = time_loop(step, dsteps, args.warmup, world)
+    peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    per_rank_gbs = dbytes / (ms * 1e-3) / 1e9
+    return {"workload": dcfg.name + "_fp8_e4m3", "value": round(per_rank_gbs * world, 1), "unit": "GB/s",
+            "ms_per_step": round(ms, 4), "steps": dsteps, "kv_tokens": tokens,
+            "kv_tokens_per_s": round(tokens * world / (ms * 1e-3), 1),
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<4,true>", "achieved": round(per_rank_gbs, 1),
+                         "peak": peak_h, "unit": "GB/s", "frac": round(per_rank_gbs / peak_h, 4),
+                         "peak_source": f"{peak_src} copy bandwidth", "traffic": None,
+                         "algorithmic_bytes_per_launch": dbytes},
+            "gpu_launches_per_step": 2, "clocks": clk.summary()}
 
 
 def bench_prefill_16k(args, rank, world, local, attn, peaks, peak_src):
@@ -482,7 +525,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--only", choices=["prefill", "decode", "mixed", "prefill16k"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decodefp8", "mixed", "prefill16k"], default=None,
                     help="profiling aid: run one workload only (the line is then marked partial)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="profiling aid: fewer decode sequences (default: the full 64)")

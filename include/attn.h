@@ -61,7 +61,7 @@ typedef enum {
   ATTN_ERR_NO_DEVICE = 7      /* no sm_100 device is current */
 } attn_status_t;
 
-typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1 } attn_dtype_t;
+typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1, ATTN_DTYPE_FP8_E4M3 = 2 } attn_dtype_t;
 
 /* Bits a kernel ORs into *error_flags. */
 #define ATTN_FAULT_TIMEOUT 0x1      /* a pipeline wait exceeded its bound; the tile was abandoned */
@@ -165,6 +165,15 @@ ATTN_API attn_status_t attn_prefill(const attn_prefill_params* p, attn_stream_t 
  * NULL to only query the size (returns ATTN_OK, enqueues nothing). If
  * workspace_bytes is too small the call returns ATTN_ERR_WORKSPACE and
  * enqueues nothing. A sequence with 0 keys gets O = 0 and LSE = -inf.
+ *
+ * FP8 cache ("5.2 推理加速的未来趋势：新算法、新硬件、新协同", 协同层: an FP8 KV
+ * cache halves its memory at almost no accuracy cost): kv_dtype =
+ * ATTN_DTYPE_FP8_E4M3 means k_cache / v_cache hold one-byte codes in the OCP
+ * E4M3 format without infinities (same [num_blocks, num_kv_heads, block_size,
+ * head_dim] layout), and the cached key (value) is code * k_scale (code *
+ * v_scale). One scale per tensor is this library's convention (the pages give
+ * none); k_scale and v_scale must be finite and > 0. kv_dtype = 0 (BF16, the
+ * zero-initialised default) ignores both scales. o stays bf16 or fp32.
  */
 typedef struct {
   const void* q;
@@ -186,6 +195,9 @@ typedef struct {
   float scale;
   attn_dtype_t o_dtype;
   int32_t* error_flags; /* nullable */
+  attn_dtype_t kv_dtype; /* ATTN_DTYPE_BF16 (0) or ATTN_DTYPE_FP8_E4M3 */
+  float k_scale;         /* FP8 only */
+  float v_scale;         /* FP8 only */
 } attn_decode_params;
 
 ATTN_API attn_status_t attn_decode_paged(const attn_decode_params* p, void* workspace, size_t workspace_bytes,

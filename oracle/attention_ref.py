@@ -206,12 +206,24 @@ def ref_decode_paged_fp8(q, k_pool, v_pool, k_scale, v_scale, block_table, seq_l
     """Decode over an FP8 E4M3 cache with one scale per tensor.
 
     Pools hold uint8 codes [NB, Hkv, 16, D]; the cached key (value) is
-    decode(code) * k_scale (v_scale). The decode definition above then applies
-    unchanged to those values.
+    decode(code) * k_scale (v_scale). Each sequence's codes are gathered and
+    decoded, then the decode definition above applies unchanged. Returns O
+    [B, Hq, D], LSE [B, Hq] (or arrays over ``rows`` = list of (b, h)).
     """
-    kf = e4m3_bits_to_f64(k_pool) * float(k_scale)
-    vf = e4m3_bits_to_f64(v_pool) * float(v_scale)
-    return ref_decode_paged(q, kf, vf, block_table, seq_lens, scale, rows)
+    q = np.asarray(q)
+    B, Hq, D = q.shape
+    G = Hq // np.asarray(k_pool).shape[1]
+    todo = rows if rows is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    O = np.zeros((len(todo), D))
+    L = np.zeros(len(todo))
+    for n, (b, h) in enumerate(todo):
+        kk = e4m3_bits_to_f64(gather_paged(k_pool, block_table[b], int(seq_lens[b]), h // G)) * float(k_scale)
+        vv = e4m3_bits_to_f64(gather_paged(v_pool, block_table[b], int(seq_lens[b]), h // G)) * float(v_scale)
+        o, lse = attention_rows(_as_f64(q[b, h][None]), kk, vv, scale, None)
+        O[n], L[n] = o[0], lse[0]
+    if rows is None:
+        return O.reshape(B, Hq, D), L.reshape(B, Hq)
+    return O, L
 
 
 def ref_prefill_paged(q, q_lens, k_pool, v_pool, block_table, k_lens, scale, causal, rows=None):

@@ -144,10 +144,20 @@ def test_decode_workspace_query_and_too_small(lib):
 @pytest.mark.parametrize("field,value,code", [
     ("head_dim", 64, 2), ("num_kv_heads", 3, 2), ("num_q_heads", 24, 2), ("block_size", 32, 2),
     ("scale", 0.0, 1), ("max_blocks_per_seq", 0, 1), ("batch", -1, 1), ("q", 0, 1), ("o", (1 << 20) + 4, 2),
-    ("num_splits", -2, 1),
+    ("num_splits", -2, 1), ("kv_dtype", 1, 1), ("kv_dtype", 7, 1),
 ])
 def test_decode_rejects_bad_arguments(lib, field, value, code):
     p = _decode_params(lib, **{field: value})
+    need = ctypes.c_size_t(0)
+    assert lib.LIB.attn_decode_paged(ctypes.byref(p), None, 0, ctypes.byref(need), None) == code
+
+
+@pytest.mark.parametrize("k_scale,v_scale,code", [
+    (0.01, 0.02, 0), (0.0, 0.02, 1), (0.01, -1.0, 1), (float("inf"), 0.02, 1), (0.01, float("nan"), 1),
+])
+def test_decode_fp8_scales_are_checked(lib, k_scale, v_scale, code):
+    """An FP8 E4M3 cache needs finite positive scales (checked before anything is enqueued)."""
+    p = _decode_params(lib, kv_dtype=lib.ATTN_DTYPE_FP8_E4M3, k_scale=k_scale, v_scale=v_scale)
     need = ctypes.c_size_t(0)
     assert lib.LIB.attn_decode_paged(ctypes.byref(p), None, 0, ctypes.byref(need), None) == code
 

@@ -44,6 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = {
     "prefill": ["attention_tiled_exact_b200/csrc/prefill_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
     "decode": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
+    "decode_fp8": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
 }
 
 
@@ -374,7 +375,7 @@ def bench_decode_fp8(args, rank, world, local, attn, peaks, peak_src):
             "kv_tokens_per_s": round(tokens * world / (ms * 1e-3), 1),
             "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<4,true>", "achieved": round(per_rank_gbs, 1),
                          "peak": peak_h, "unit": "GB/s", "frac": round(per_rank_gbs / peak_h, 4),
-                         "peak_source": f"{peak_src} copy bandwidth", "traffic": None,
+                         "peak_source": f"{peak_src} copy bandwidth", "traffic": profiled_traffic("decode_fp8"),
                          "algorithmic_bytes_per_launch": dbytes},
             "gpu_launches_per_step": 2, "clocks": clk.summary()}
 

@@ -84,6 +84,9 @@ def _load():
     lib.attn_decode_paged.restype = ctypes.c_int
     lib.attn_decode_paged_noalloc.argtypes = [ctypes.POINTER(DecodeParams), _vp]
     lib.attn_decode_paged_noalloc.restype = ctypes.c_int
+    lib.attn_decode_paged_shared_prefix.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_int32, _vp,
+                                                    ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t), _vp]
+    lib.attn_decode_paged_shared_prefix.restype = ctypes.c_int
     lib.splitkv_lse_combine.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp,
                                         ctypes.c_int, _vp, _vp]
     lib.splitkv_lse_combine.restype = ctypes.c_int
@@ -294,6 +297,58 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(LIB.attn_decode_paged(ctypes.byref(p), ws_ptr, ws_bytes, None, _stream(q.device)),
            "attn_decode_paged")
+    return out, lse
+
+
+def _check_decode_inputs(q, k_cache, v_cache, block_table, seq_lens, allow_fp8=True):
+    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
+    ok_cache = k_cache.dtype == torch.bfloat16 or (allow_fp8 and _is_fp8(k_cache))
+    _need(q.dtype == torch.bfloat16 and k_cache.dtype == v_cache.dtype and ok_cache,
+          "bf16 q; bf16 or FP8 E4M3 caches" if allow_fp8 else "bf16 q and caches")
+    _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
+    _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
+          "int32 block table [B, max_blocks]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "int32 seq_lens [B]")
+
+
+def decode_shared_prefix_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, prefix_len: int,
+                                         max_seq_len: int = 0, num_splits: int = 0) -> int:
+    """Bytes of workspace :func:`decode_paged_shared_prefix` needs for these shapes."""
+    p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, None, max_seq_len, num_splits, q, None, None)
+    need = ctypes.c_size_t(0)
+    _check(LIB.attn_decode_paged_shared_prefix(ctypes.byref(p), int(prefix_len), None, 0, ctypes.byref(need), None),
+           "attn_decode_paged_shared_prefix(size)")
+    return int(need.value)
+
+
+def decode_paged_shared_prefix(q, k_cache, v_cache, block_table, seq_lens, prefix_len: int,
+                               scale: float | None = None, max_seq_len: int = 0, num_splits: int = 0, out=None,
+                               lse=None, workspace=None, out_dtype=torch.bfloat16, want_lse: bool = True,
+                               error_flags=None):
+    """:func:`decode_paged` for sequences that all start with the same
+    ``prefix_len`` tokens (a multiple of 16), stored in the blocks listed
+    first in sequence 0's table; the prefix is attended once per batch.
+
+    Same tensors as :func:`decode_paged` (bf16 caches only). Returns
+    ``(O [B,Hq,D], LSE [B,Hq] or None)``.
+    """
+    _check_decode_inputs(q, k_cache, v_cache, block_table, seq_lens, allow_fp8=False)
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits, out, lse,
+                       error_flags)
+    need = ctypes.c_size_t(0)
+    _check(LIB.attn_decode_paged_shared_prefix(ctypes.byref(p), int(prefix_len), None, 0, ctypes.byref(need), None),
+           "attn_decode_paged_shared_prefix(size)")
+    if workspace is None and need.value > 0:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(LIB.attn_decode_paged_shared_prefix(ctypes.byref(p), int(prefix_len), ws_ptr, ws_bytes, None,
+                                               _stream(q.device)), "attn_decode_paged_shared_prefix")
     return out, lse
 
 

@@ -129,6 +129,26 @@ attn_status_t attn_decode_paged(const attn_decode_params* p, void* workspace, si
   return attn::launch_decode(*p, plan, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
+attn_status_t attn_decode_paged_shared_prefix(const attn_decode_params* p, int32_t prefix_len, void* workspace,
+                                             size_t workspace_bytes, size_t* workspace_needed,
+                                             attn_stream_t stream) {
+  attn_status_t st = attn::validate_decode(p);
+  if (st != ATTN_OK) return st;
+  if (prefix_len < 0 || prefix_len % 16 != 0 || (int64_t)prefix_len > (int64_t)p->max_blocks_per_seq * 16)
+    return ATTN_ERR_INVALID_ARG;
+  if (prefix_len == 0) return attn_decode_paged(p, workspace, workspace_bytes, workspace_needed, stream);
+  if (p->kv_dtype != ATTN_DTYPE_BF16) return ATTN_ERR_UNSUPPORTED;
+  const bool have_dev = attn::check_device() == ATTN_OK;
+  attn::CascadePlan plan = attn::plan_cascade(*p, prefix_len);
+  if (workspace_needed) *workspace_needed = plan.workspace_bytes;
+  if (workspace == nullptr && workspace_needed != nullptr) return ATTN_OK;  // size query only
+  if (workspace_bytes < plan.workspace_bytes) return ATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (p->batch == 0) return ATTN_OK;
+  if (!have_dev) return ATTN_ERR_NO_DEVICE;
+  return attn::launch_cascade(*p, plan, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
 attn_status_t splitkv_lse_combine(const float* part_o, const float* part_lse, int num_splits, int rows,
                                   int head_dim, const int32_t* splits_per_row, void* out_o, attn_dtype_t out_dtype,
                                   float* out_lse, attn_stream_t stream) {

@@ -36,4 +36,20 @@ attn_status_t launch_combine(const float* part_o, const float* part_lse, int num
                              int split_tokens, int rows_per_seq, void* out_o, attn_dtype_t out_dtype,
                              float* out_lse, cudaStream_t stream);
 
+// Shared-prefix (cascade) decode: key ranges of the prefix prefill, the suffix
+// decode (its parameters and split plan) and the workspace layout.
+struct CascadePlan {
+  int prefix_len;
+  int ranges;        // prefix key ranges (batch entries of the prefix prefill)
+  int range_blocks;  // cache blocks per range (the last range may hold fewer)
+  int suffix_cap;    // most tokens a sequence can hold past the prefix
+  attn_decode_params suffix;
+  DecodePlan suffix_plan;
+  size_t off_suffix_lens, off_range_lens, off_q_rep, off_pre_o, off_pre_lse, off_suf_o, off_suf_lse, off_decode;
+  size_t workspace_bytes;
+};
+CascadePlan plan_cascade(const attn_decode_params& p, int prefix_len);
+attn_status_t launch_cascade(const attn_decode_params& p, const CascadePlan& plan, void* workspace,
+                             cudaStream_t stream);
+
 }  // namespace attn

@@ -126,6 +126,27 @@ class DecodeConfig:
 
 
 @dataclasses.dataclass(frozen=True)
+class SharedPrefixConfig:
+    """Paged decode where every sequence starts with the same prefix_len
+    tokens (stored once), followed by suffix_lo..suffix_hi tokens of its own."""
+
+    name: str
+    batch: int
+    q_heads: int
+    kv_heads: int
+    head_dim: int
+    prefix_len: int
+    suffix_lo: int
+    suffix_hi: int
+    seed: int
+    spare_blocks: int = 64
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+
+@dataclasses.dataclass(frozen=True)
 class MixedConfig:
     """Chunked prefill on top of cached context, plus decode rows, paged KV."""
 
@@ -155,7 +176,10 @@ PAGED_DECODE = DecodeConfig("paged_decode_b64_h32kv8_d128_len1k_32k", 64, 32, 8,
 MIXED = MixedConfig("mixed_8x512chunks_ctx0_8k_plus_128dec_ctx512_16k",
                     8, 512, 0, 8192, 128, 512, 16384, 32, 8, 128, 4)
 
-WORKLOADS = {c.name: c for c in (TINY, CAUSAL_GQA_2K, CAUSAL_GQA_16K, PAGED_DECODE, MIXED)}
+SHARED_PREFIX_DECODE = SharedPrefixConfig("shared_prefix_decode_b64_h32kv8_d128_prefix8k_own64_2k",
+                                          64, 32, 8, 128, 8192, 64, 2048, 5)
+WORKLOADS = {c.name: c for c in (TINY, CAUSAL_GQA_2K, CAUSAL_GQA_16K, PAGED_DECODE, MIXED,
+                                  SHARED_PREFIX_DECODE)}
 
 
 # ----------------------------------------------------------------------------
@@ -311,6 +335,50 @@ def make_decode(cfg: DecodeConfig, kv_lens=None, identity: bool = False) -> dict
                         identity=identity)
     d.update(q=q, scale=cfg.scale)
     return d
+
+
+def make_shared_prefix_decode(cfg: SharedPrefixConfig, suffix_lens=None) -> dict:
+    """Paged decode inputs whose sequences share their first prefix_len tokens.
+
+    The prefix occupies prefix_len / 16 physical blocks that every row of the
+    block table lists first (aliased); each sequence's own tokens follow in
+    blocks of its own. Physical ids are a random permutation of the pool;
+    spare blocks and the tail slots past each sequence end hold NaN. Returns
+    q, k_pool, v_pool, block_table, kv_lens (= prefix_len + suffix),
+    suffix_lens, prefix_len, num_blocks, spare_ids, scale.
+    """
+    assert cfg.prefix_len % BLOCK_SIZE == 0
+    if suffix_lens is None:
+        suffix_lens = random_lengths(cfg.seed, cfg.batch, cfg.suffix_lo, cfg.suffix_hi)
+    suffix_lens = np.asarray(suffix_lens, dtype=np.int32)
+    pb = cfg.prefix_len // BLOCK_SIZE
+    own = (suffix_lens.astype(np.int64) + BLOCK_SIZE - 1) // BLOCK_SIZE
+    used = pb + int(own.sum())
+    num_blocks = used + cfg.spare_blocks
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([cfg.seed, 11])))
+    perm = rng.permutation(num_blocks)
+    spare = perm[used:]
+    max_blocks = max(1, pb + (int(own.max()) if len(own) else 0))
+    filler = int(spare[0]) if cfg.spare_blocks > 0 else 0
+    table = np.full((len(suffix_lens), max_blocks), filler, dtype=np.int32)
+    table[:, :pb] = perm[:pb]
+    off = pb
+    for b, n in enumerate(own):
+        table[b, pb:pb + n] = perm[off:off + n]
+        off += n
+    shape = (num_blocks, cfg.kv_heads, BLOCK_SIZE, cfg.head_dim)
+    k_pool = normal_bf16(cfg.seed, shape, 1)
+    v_pool = normal_bf16(cfg.seed, shape, 2)
+    kv_lens = (cfg.prefix_len + suffix_lens).astype(np.int32)
+    for pool in (k_pool, v_pool):
+        pool[spare] = BF16_NAN
+        for b, L in enumerate(kv_lens):
+            tail = int(L) % BLOCK_SIZE
+            if tail:
+                pool[table[b, (int(L) - 1) // BLOCK_SIZE], :, tail:, :] = BF16_NAN
+    q = normal_bf16(cfg.seed, (len(suffix_lens), cfg.q_heads, cfg.head_dim), 0)
+    return dict(q=q, k_pool=k_pool, v_pool=v_pool, block_table=table, kv_lens=kv_lens, suffix_lens=suffix_lens,
+                prefix_len=cfg.prefix_len, num_blocks=num_blocks, spare_ids=spare, scale=cfg.scale)
 
 
 def relayout_identity(pool: np.ndarray, table: np.ndarray, kv_lens) -> tuple:

@@ -230,6 +230,8 @@ def run_ours(args, rank, world, local):
         result["mixed"] = bench_mixed(args, rank, world, local, attn, peaks, peak_src)
     if args.only in (None, "prefill16k"):
         result["prefill_16k"] = bench_prefill_16k(args, rank, world, local, attn, peaks, peak_src)
+    if args.only in (None, "sharedprefix"):
+        result["shared_prefix"] = bench_shared_prefix(args, rank, world, local, attn, peaks, peak_src)
     if args.only is not None:
         result["partial"] = f"--only {args.only}: profiling run, not a bench line"
     if rank == 0 and args.only is None:
@@ -380,6 +382,56 @@ def bench_decode_fp8(args, rank, world, local, attn, peaks, peak_src):
             "gpu_launches_per_step": 2, "clocks": clk.summary()}
 
 
+def bench_shared_prefix(args, rank, world, local, attn, peaks, peak_src):
+    """Decode of 64 sequences that share an 8192-token prefix (its blocks aliased
+    in every table row) plus 64..2048 tokens of their own: the shared-prefix
+    call against the plain decode over the same tables."""
+    import dataclasses
+
+    import torch
+    cfg = dataclasses.replace(wl.SHARED_PREFIX_DECODE, seed=wl.SHARED_PREFIX_DECODE.seed + 1000 * rank)
+    d = wl.make_shared_prefix_decode(cfg)
+    q = _dev_bf16(d["q"])
+    kc, vc = _dev_bf16(d["k_pool"]), _dev_bf16(d["v_pool"])
+    bt = torch.from_numpy(d["block_table"]).cuda()
+    sl = torch.from_numpy(d["kv_lens"]).cuda()
+    max_len = int(d["kv_lens"].max())
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device="cuda")
+    ws_c = torch.empty(attn.decode_shared_prefix_workspace_bytes(q, kc, vc, bt, sl, cfg.prefix_len,
+                                                                 max_seq_len=max_len), dtype=torch.uint8,
+                       device="cuda")
+    ws_p = torch.empty(max(attn.decode_workspace_bytes(q, kc, vc, bt, sl, max_seq_len=max_len), 1),
+                       dtype=torch.uint8, device="cuda")
+
+    def cascade():
+        attn.decode_paged_shared_prefix(q, kc, vc, bt, sl, cfg.prefix_len, cfg.scale, max_seq_len=max_len,
+                                        out=out, lse=lse, workspace=ws_c)
+
+    def plain():
+        attn.decode_paged(q, kc, vc, bt, sl, cfg.scale, max_seq_len=max_len, out=out, lse=lse, workspace=ws_p)
+
+    steps = max(args.steps, 10)
+    with ClockSampler(local) as clk:
+        ms = time_loop(cascade, steps, args.warmup, world)
+    ms_plain = time_loop(plain, steps, args.warmup, world)
+    logical = int(d["kv_lens"].sum())                       # keys attended, summed over sequences
+    unique = cfg.prefix_len + int(d["suffix_lens"].sum())   # distinct cached tokens
+    ubytes = float(unique * cfg.kv_heads * cfg.head_dim * 2 * 2 + cfg.batch * cfg.q_heads * (cfg.head_dim * 4 + 4))
+    prefix_flops = 4.0 * cfg.batch * cfg.q_heads * cfg.prefix_len * cfg.head_dim
+    peak_h = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gbs = ubytes / (ms * 1e-3) / 1e9
+    max_splits = -(-(max_len - cfg.prefix_len) // 512)
+    return {"workload": cfg.name, "value": round(logical * world / (ms * 1e-3), 1), "unit": "kv_tokens/s",
+            "ms_per_step": round(ms, 4), "steps": steps, "kv_tokens": logical, "unique_kv_tokens": unique,
+            "plain_decode_ms_per_step": round(ms_plain, 4), "speedup_vs_plain_decode": round(ms_plain / ms, 3),
+            "roofline": {"bound": "hbm", "kernel": "whole call (prefix prefill + suffix decode + merge)",
+                         "achieved": round(gbs, 1), "peak": peak_h, "unit": "GB/s", "frac": round(gbs / peak_h, 4),
+                         "peak_source": f"{peak_src} copy bandwidth", "traffic": None,
+                         "algorithmic_bytes_per_launch": ubytes, "prefix_tensor_flops": prefix_flops},
+            "gpu_launches_per_step": 4 + (1 if max_splits > 1 else 0), "clocks": clk.summary()}
+
+
 def bench_prefill_16k(args, rank, world, local, attn, peaks, peak_src):
     """Long-context causal GQA prefill: batch 1, 32/8 heads, 16384 tokens, head_dim 128."""
     import dataclasses
@@ -526,7 +578,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--only", choices=["prefill", "decode", "decodefp8", "mixed", "prefill16k"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decodefp8", "mixed", "prefill16k", "sharedprefix"], default=None,
                     help="profiling aid: run one workload only (the line is then marked partial)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="profiling aid: fewer decode sequences (default: the full 64)")

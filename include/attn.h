@@ -204,6 +204,42 @@ ATTN_API attn_status_t attn_decode_paged(const attn_decode_params* p, void* work
                                 size_t* workspace_needed, attn_stream_t stream);
 
 /*
+ * attn_decode_paged for a batch whose sequences all begin with the same
+ * prefix_len tokens (a shared prompt): requests with a common prefix can share
+ * their KV blocks ("抱infra脚", Paged Attention), and a common prefix should
+ * not be processed once per request ("抱infra脚", RadixAttention).
+ *
+ * The prefix's keys/values are the blocks listed first in sequence 0's table,
+ * block_table[0][0 .. prefix_len / 16); the other sequences' entries for
+ * those positions are not read (they normally alias the same blocks). Each
+ * sequence b continues with its own blocks block_table[b][prefix_len / 16 ..]
+ * up to seq_lens[b] keys. The result is what attn_decode_paged returns when
+ * every sequence's first prefix_len keys/values are sequence 0's, up to fp32
+ * rounding (the prefix is merged in as separate log-sum-exp partials).
+ *
+ * The prefix is read once per batch instead of once per sequence: all batch
+ * queries of a query head run as the rows of one non-causal tcgen05 prefill
+ * over the prefix (cut into up to 16 key ranges when the batch is small),
+ * the split-KV decode covers each sequence's suffix, and one kernel merges
+ * the partials ("GPU Kernel 调度:大模型推理的拐点 2026", Flash Decoding
+ * section: partials merged by their log-sum-exp).
+ *
+ * Parameters as attn_decode_paged, plus prefix_len (host): a multiple of 16
+ * with 0 <= prefix_len <= max_blocks_per_seq * 16, else
+ * ATTN_ERR_INVALID_ARG; 0 runs attn_decode_paged itself (with its workspace
+ * size). kv_dtype must be ATTN_DTYPE_BF16 (ATTN_ERR_UNSUPPORTED otherwise).
+ * max_seq_len, if given, bounds seq_lens as in attn_decode_paged. Workspace
+ * rules as attn_decode_paged; the workspace is always needed (it holds the
+ * prefix and suffix partials) and its size depends on the device's SM count.
+ * A sequence with seq_lens[b] < prefix_len (or longer than its table) sets
+ * ATTN_FAULT_BAD_LENGTH in error_flags; its suffix is then taken as empty
+ * (or as the table's capacity).
+ */
+ATTN_API attn_status_t attn_decode_paged_shared_prefix(const attn_decode_params* p, int32_t prefix_len,
+                                                       void* workspace, size_t workspace_bytes,
+                                                       size_t* workspace_needed, attn_stream_t stream);
+
+/*
  * attn_decode_paged without a workspace argument, for callers that cannot
  * allocate device memory: a host program that only receives tensor pointers
  * from another component and has no allocator of its own to pass through this

@@ -162,6 +162,40 @@ def test_decode_fp8_scales_are_checked(lib, k_scale, v_scale, code):
     assert lib.LIB.attn_decode_paged(ctypes.byref(p), None, 0, ctypes.byref(need), None) == code
 
 
+@pytest.mark.parametrize("prefix_len,code", [(-16, 1), (8, 1), (2048 * 16 + 16, 1), (4096, 0), (2048 * 16, 0)])
+def test_shared_prefix_decode_checks_prefix_len(lib, prefix_len, code):
+    """prefix_len must be a multiple of 16 within the table capacity."""
+    p = _decode_params(lib)
+    need = ctypes.c_size_t(0)
+    assert lib.LIB.attn_decode_paged_shared_prefix(ctypes.byref(p), prefix_len, None, 0, ctypes.byref(need),
+                                                   None) == code
+    if code == 0:
+        assert need.value > 0 and need.value % 256 == 0
+
+
+def test_shared_prefix_decode_workspace_and_dtypes(lib):
+    p = _decode_params(lib)
+    need0, need = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    f = lib.LIB.attn_decode_paged_shared_prefix
+    # prefix_len 0 is the plain decode, with its workspace size
+    assert lib.LIB.attn_decode_paged(ctypes.byref(p), None, 0, ctypes.byref(need0), None) == 0
+    assert f(ctypes.byref(p), 0, None, 0, ctypes.byref(need), None) == 0 and need.value == need0.value
+    # a prefix needs room for its partials even with a single suffix split
+    p1 = _decode_params(lib, num_splits=1)
+    assert f(ctypes.byref(p1), 1024, None, 0, ctypes.byref(need), None) == 0
+    assert need.value >= 64 * 32 * 129 * 4 * 2
+    # too small: reported, nothing enqueued
+    need2 = ctypes.c_size_t(0)
+    assert f(ctypes.byref(p1), 1024, ctypes.c_void_p(1 << 20), need.value - 256, ctypes.byref(need2),
+             None) == lib.ATTN_ERR_WORKSPACE and need2.value == need.value
+    # the prefix runs on the bf16 prefill kernel: FP8 caches are not supported here
+    p8 = _decode_params(lib, kv_dtype=lib.ATTN_DTYPE_FP8_E4M3, k_scale=0.01, v_scale=0.01)
+    assert f(ctypes.byref(p8), 1024, None, 0, ctypes.byref(need), None) == lib.ATTN_ERR_UNSUPPORTED
+    # ordinary decode argument checks apply first
+    bad = _decode_params(lib, head_dim=64)
+    assert f(ctypes.byref(bad), 1024, None, 0, ctypes.byref(need), None) == lib.ATTN_ERR_UNSUPPORTED
+
+
 def test_combine_rejects_bad_arguments(lib):
     f = lib.LIB.splitkv_lse_combine
     assert f(1 << 20, 1 << 20, -1, 4, 128, None, 1 << 20, 0, None, None) == lib.ATTN_ERR_INVALID_ARG

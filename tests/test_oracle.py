@@ -369,3 +369,20 @@ def test_fp8_decode_oracle_matches_brute_force():
             vv = [[[dequant(d["v_pool"][p, kvh, s, j], d["v_scale"]) for j in range(8)] for p, s in toks]]
             Ob, Lbr = oracle.brute_attention([[[list(qf[b, h])]]], [kk], [vv], d["scale"], False)
             assert np.allclose(O[b, h], Ob[0][0][0], atol=1e-12) and abs(L[b, h] - Lbr[0][0][0]) < 1e-12
+
+
+def test_decode_over_a_shared_prefix_is_the_merge_of_prefix_and_suffix():
+    """Attention over prefix + own keys equals the log-sum-exp merge of the
+    attention over each part: the identity the shared-prefix decode relies on,
+    checked with the oracle's decode on the full, the prefix-only and the
+    suffix-only tables."""
+    cfg = wl.SharedPrefixConfig("t", 5, 4, 2, 32, 48, 0, 40, 7)
+    d = wl.make_shared_prefix_decode(cfg)
+    t, pb = d["block_table"], 3
+    O, L = ref.ref_decode_paged(d["q"], d["k_pool"], d["v_pool"], t, d["kv_lens"], d["scale"])
+    Op, Lp = ref.ref_decode_paged(d["q"], d["k_pool"], d["v_pool"], t[:, :pb], np.full(5, 48), d["scale"])
+    Os, Ls = ref.ref_decode_paged(d["q"], d["k_pool"], d["v_pool"], t[:, pb:], d["suffix_lens"], d["scale"])
+    Om, Lm = ref.combine_partials(np.stack([Op.reshape(20, 32), Os.reshape(20, 32)]),
+                                  np.stack([Lp.reshape(20), Ls.reshape(20)]))
+    assert np.abs(Om - O.reshape(20, 32)).max() < 1e-12 and np.abs(Lm - L.reshape(20)).max() < 1e-12
+    assert np.isneginf(Ls.reshape(20)[np.repeat(d["suffix_lens"] == 0, 4)]).all()

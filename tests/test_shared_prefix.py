@@ -75,3 +75,157 @@ def test_chunked_prefill_over_shared_prefix_blocks(lib):
     assert_o_close(outs[0][0], O_ref, False, "aliased prefix prefill")
     assert_lse_close(outs[0][1], L_ref, "aliased prefix prefill lse")
     assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+
+
+# ---------------------------------------------------------------------------
+# attn_decode_paged_shared_prefix: the shared prefix attended once per batch
+# (prefix prefill + suffix decode + log-sum-exp merge) against the fp64 oracle
+# of plain decode over the aliased tables.
+# ---------------------------------------------------------------------------
+
+
+def _cascade(lib, d, num_splits=0, out_dtype=None, table=None, seq_lens=None, flags=None, max_seq_len=0,
+             prefix_len=None):
+    import torch
+    o, lse = lib.decode_paged_shared_prefix(
+        to_dev_bf16(d["q"]), to_dev_bf16(d["k_pool"]), to_dev_bf16(d["v_pool"]),
+        to_dev_i32(d["block_table"] if table is None else table),
+        to_dev_i32(d["kv_lens"] if seq_lens is None else seq_lens),
+        d["prefix_len"] if prefix_len is None else prefix_len, d["scale"], max_seq_len=max_seq_len,
+        num_splits=num_splits, out_dtype=out_dtype or torch.float32, error_flags=flags)
+    torch.cuda.synchronize()
+    return to_f64(o), to_f64(lse)
+
+
+def _prefix_inputs(batch, G, prefix_len, lo, hi, seed, Hkv=2):
+    cfg = wl.SharedPrefixConfig("sp", batch, G * Hkv, Hkv, 128, prefix_len, lo, hi, seed)
+    return wl.make_shared_prefix_decode(cfg)
+
+
+@pytest.mark.parametrize("batch,G,prefix_len,lo,hi", [
+    (6, 4, 320, 0, 300),      # one prefix range
+    (1, 1, 16, 0, 40),        # a single sequence, a one-block prefix
+    (64, 4, 4096, 0, 700),    # the prefix cut into several key ranges
+    (130, 2, 512, 0, 100),    # two 128-row blocks of queries, ragged
+    (300, 8, 1024, 1, 2100),  # G = 8, three row blocks, split suffixes
+    (5, 1, 2048, 17, 17),     # G = 1 (single-head items), equal suffixes
+])
+def test_shared_prefix_decode_matches_oracle(lib, batch, G, prefix_len, lo, hi):
+    import torch
+    d = _prefix_inputs(batch, G, prefix_len, lo, hi, seed=80 + G + batch)
+    O_ref, L_ref = ref.ref_decode_paged(d["q"], d["k_pool"], d["v_pool"], d["block_table"], d["kv_lens"],
+                                        d["scale"])
+    for splits in (0, 1):
+        o, lse = _cascade(lib, d, num_splits=splits)
+        assert_o_close(o, O_ref, False, f"shared prefix splits={splits}")
+        assert_lse_close(lse, L_ref, f"shared prefix splits={splits}")
+    o16, _ = _cascade(lib, d, out_dtype=torch.bfloat16)
+    assert_o_close(o16, O_ref, True, "shared prefix bf16 out")
+
+
+def test_shared_prefix_reads_only_sequence_zero_prefix_entries(lib):
+    """Other sequences' table entries for the prefix positions are not read:
+    pointing them at a NaN spare block changes no bit of the result."""
+    d = _prefix_inputs(9, 4, 640, 0, 500, seed=90)
+    o1, l1 = _cascade(lib, d)
+    table = d["block_table"].copy()
+    table[1:, :640 // 16] = d["spare_ids"][0]
+    o2, l2 = _cascade(lib, d, table=table)
+    assert np.isfinite(o2).all() and np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_shared_prefix_filling_the_whole_table(lib):
+    """prefix_len = table capacity: every suffix is empty (no suffix decode)."""
+    d = _prefix_inputs(7, 2, 800, 0, 0, seed=91)
+    assert d["block_table"].shape[1] == 800 // 16
+    O_ref, L_ref = ref.ref_decode_paged(d["q"], d["k_pool"], d["v_pool"], d["block_table"], d["kv_lens"],
+                                        d["scale"])
+    o, lse = _cascade(lib, d)
+    assert_o_close(o, O_ref, False, "prefix only")
+    assert_lse_close(lse, L_ref, "prefix only")
+
+
+def test_shared_prefix_zero_is_plain_decode(lib):
+    """prefix_len = 0 runs the plain decode: identical bits."""
+    import torch
+    d = _prefix_inputs(5, 4, 0, 1, 900, seed=92)
+    o1, l1 = _cascade(lib, d)
+    o2, l2 = lib.decode_paged(to_dev_bf16(d["q"]), to_dev_bf16(d["k_pool"]), to_dev_bf16(d["v_pool"]),
+                              to_dev_i32(d["block_table"]), to_dev_i32(d["kv_lens"]), d["scale"],
+                              out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert np.array_equal(o1, to_f64(o2)) and np.array_equal(l1, to_f64(l2))
+
+
+def test_shared_prefix_short_sequence_is_flagged(lib):
+    """A sequence shorter than the prefix sets ATTN_FAULT_BAD_LENGTH; the
+    other sequences are unaffected."""
+    import torch
+    d = _prefix_inputs(4, 4, 320, 10, 200, seed=93)
+    lens = d["kv_lens"].copy()
+    lens[2] = 300
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = _cascade(lib, d, seq_lens=lens, flags=flags)
+    assert int(flags.item()) & lib.ATTN_FAULT_BAD_LENGTH
+    assert np.isfinite(o).all()
+    ok = [0, 1, 3]
+    O_ref, L_ref = ref.ref_decode_paged(d["q"][ok], d["k_pool"], d["v_pool"], d["block_table"][ok],
+                                        d["kv_lens"][ok], d["scale"])
+    assert_o_close(o[ok], O_ref, False, "unaffected rows")
+    assert_lse_close(lse[ok], L_ref, "unaffected rows")
+
+
+def test_shared_prefix_graph_replay(lib):
+    """Captured once with a caller-owned workspace, replayed with new own
+    tokens and lengths in the static buffers (the prefix stays)."""
+    import torch
+    cfg = wl.SharedPrefixConfig("g", 8, 8, 2, 128, 512, 0, 600, 94)
+    d0 = wl.make_shared_prefix_decode(cfg, suffix_lens=np.full(8, 600, dtype=np.int32))
+    q_s = to_dev_bf16(d0["q"])
+    k_s, v_s = to_dev_bf16(d0["k_pool"]), to_dev_bf16(d0["v_pool"])
+    bt_s, sl_s = to_dev_i32(d0["block_table"]), to_dev_i32(d0["kv_lens"])
+    o_s = torch.empty((8, 8, 128), dtype=torch.float32, device="cuda")
+    l_s = torch.empty((8, 8), dtype=torch.float32, device="cuda")
+    max_len = 512 + 600
+    ws = torch.empty(lib.decode_shared_prefix_workspace_bytes(q_s, k_s, v_s, bt_s, sl_s, 512, max_seq_len=max_len),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        lib.decode_paged_shared_prefix(q_s, k_s, v_s, bt_s, sl_s, 512, cfg.scale, max_seq_len=max_len, out=o_s,
+                                       lse=l_s, workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    rng = np.random.default_rng(95)
+    for it in range(3):
+        lens = 512 + rng.integers(0, 601, 8).astype(np.int32)
+        q_new = wl.normal_bf16(96 + it, (8, 8, 128))
+        q_s.copy_(to_dev_bf16(q_new))
+        sl_s.copy_(to_dev_i32(lens))
+        g.replay()
+        torch.cuda.synchronize()
+        O_ref, L_ref = ref.ref_decode_paged(q_new, d0["k_pool"], d0["v_pool"], d0["block_table"], lens, cfg.scale)
+        assert_o_close(to_f64(o_s), O_ref, False, f"replay {it}")
+        assert_lse_close(to_f64(l_s), L_ref, f"replay {it}")
+
+
+def test_shared_prefix_full_size_sampled_rows(lib):
+    """The bench's shared-prefix shape (64 sequences, 8192 shared tokens plus
+    64..2048 own tokens, 32/8 heads), checked on sampled rows."""
+    cfg = wl.SHARED_PREFIX_DECODE
+    d = wl.make_shared_prefix_decode(cfg)
+    o, lse = _cascade(lib, d)
+    rng = np.random.default_rng(97)
+    rows = [(0, 0), (cfg.batch - 1, cfg.q_heads - 1)] + [
+        (int(rng.integers(cfg.batch)), int(rng.integers(cfg.q_heads))) for _ in range(30)]
+    O_ref, L_ref = ref.ref_decode_paged(d["q"], d["k_pool"], d["v_pool"], d["block_table"], d["kv_lens"],
+                                        d["scale"], rows=rows)
+    assert_o_close(np.stack([o[b, h] for b, h in rows]), O_ref, False, "shared prefix full size")
+    assert_lse_close(np.array([lse[b, h] for b, h in rows]), L_ref, "shared prefix full size lse")

@@ -84,3 +84,20 @@ def test_e4m3_encoder_rounding():
     """Ties go to the even code, values past 448 saturate, NaN stays NaN."""
     x = np.array([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 500.0, -1e9, np.nan])
     assert [int(c) for c in wl.e4m3_codes(x)] == [0x38, 0x3A, 0x00, 0x02, 0x7E, 0xFE, 0x7F]
+
+
+def test_shared_prefix_tables_alias_the_prefix_blocks():
+    cfg = wl.SharedPrefixConfig("t", 7, 8, 2, 64, 96, 0, 50, 3)
+    d = wl.make_shared_prefix_decode(cfg)
+    t, pb = d["block_table"], 96 // 16
+    assert (t[:, :pb] == t[0, :pb]).all()  # every row lists the same prefix blocks first
+    own = [t[b, pb:pb + (int(s) + 15) // 16] for b, s in enumerate(d["suffix_lens"])]
+    ids = np.concatenate([t[0, :pb]] + own)
+    assert len(set(ids.tolist())) == len(ids)  # prefix and own blocks are distinct
+    assert not set(ids.tolist()) & set(d["spare_ids"].tolist())
+    assert (d["kv_lens"] == 96 + d["suffix_lens"]).all()
+    for pool in (d["k_pool"], d["v_pool"]):
+        assert (pool[d["spare_ids"]] == wl.BF16_NAN).all()
+        for b, L in enumerate(d["kv_lens"]):
+            if L % 16:
+                assert (pool[t[b, (L - 1) // 16], :, L % 16:] == wl.BF16_NAN).all()

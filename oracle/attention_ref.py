@@ -34,6 +34,22 @@ Attention 核心技术", the naive workflow S -> P -> O):
   Flash Decoding section: partial output / max / sum per chunk merged by the
   online-softmax formula, each partial carrying a log-sum-exp in FP32).
 
+Backward. The pages count a forward and a backward kernel for FlashAttention-2
+("GPU Kernel 调度:大模型推理的拐点 2026", the four-layer decomposition) and ask
+that both match a reference implementation (same page, checklist item 1),
+without writing the gradients out. They are the plain derivatives of the
+definition above for an upstream gradient dO (per query head, with P the
+normalised probabilities and masked entries 0):
+
+    dV = P^T dO            dP = dO V^T
+    D_i = sum_j P[i, j] dP[i, j]  ( = sum_d dO[i, d] O[i, d] )
+    dS = P * (dP - D)      dQ = scale * dS K      dK = scale * dS^T Q
+
+dK and dV of a key/value head sum the contributions of its G query heads.
+Pins: torch autograd in fp64 through a softmax written with torch ops,
+central finite differences, closed forms (one key; zero queries) and GQA vs
+MHA with repeated K/V.
+
 Pins (tests/test_oracle.py): brute-force ``math.fsum`` loops on tiny inputs,
 closed forms (one key, causal row 0, zero query, constant V, hand-derived
 weights), torch's fp64 CPU ``scaled_dot_product_attention`` with repeated
@@ -159,6 +175,43 @@ def ref_attention(q, k, v, scale, causal, rows=None):
             O[b, h], L[b, h] = attention_rows(q[b, h], k[b, h // G], v[b, h // G], scale,
                                               pos if causal else None)
     return O, L
+
+
+def ref_attention_backward(q, k, v, do, scale, causal):
+    """Gradients of O = softmax(scale Q K^T + causal mask) V for upstream dO.
+
+    q, do [B, Hq, Sq, D]; k, v [B, Hkv, Sk, D] (bf16 bits or floats). Returns
+    a dict of fp64 arrays: dq [B, Hq, Sq, D], dk and dv [B, Hkv, Sk, D], plus
+    the forward o, lse [B, Hq, Sq] and delta [B, Hq, Sq] (= rowsum(dO * O)).
+    Rows that see no key contribute nothing (P = 0).
+    """
+    q, k, v, do = (_as_f64(x) for x in (q, k, v, do))
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    pos = causal_positions(Sq, Sk) if causal else None
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    o = np.zeros_like(q)
+    lse = np.full((B, Hq, Sq), -np.inf)
+    delta = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            kvh = h // G
+            p, m, l = softmax_probs(q[b, h], k[b, kvh], scale, pos)
+            seen = l > 0.0
+            P = p / np.where(seen, l, 1.0)[:, None]
+            with np.errstate(divide="ignore"):
+                lse[b, h] = np.where(seen, m + np.log(np.where(seen, l, 1.0)), -np.inf)
+            o[b, h] = P @ v[b, kvh]
+            dv[b, kvh] += P.T @ do[b, h]
+            dP = do[b, h] @ v[b, kvh].T
+            delta[b, h] = (P * dP).sum(axis=1)
+            dS = P * (dP - delta[b, h][:, None])
+            dq[b, h] = scale * (dS @ k[b, kvh])
+            dk[b, kvh] += scale * (dS.T @ q[b, h])
+    return dict(dq=dq, dk=dk, dv=dv, o=o, lse=lse, delta=delta)
 
 
 def gather_paged(pool, block_table_row, length: int, kv_head: int) -> np.ndarray:

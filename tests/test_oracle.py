@@ -386,3 +386,128 @@ def test_decode_over_a_shared_prefix_is_the_merge_of_prefix_and_suffix():
                                   np.stack([Lp.reshape(20), Ls.reshape(20)]))
     assert np.abs(Om - O.reshape(20, 32)).max() < 1e-12 and np.abs(Lm - L.reshape(20)).max() < 1e-12
     assert np.isneginf(Ls.reshape(20)[np.repeat(d["suffix_lens"] == 0, 4)]).all()
+
+
+# ----------------------------------------------------------------------------
+# backward: gradients of the definition
+# ----------------------------------------------------------------------------
+
+
+def _autograd_backward(q, k, v, do, scale, causal):
+    """dQ, dK, dV by torch autograd in fp64 through the forward written with
+    torch ops (K/V repeated over each query-head group; masked softmax)."""
+    torch = pytest.importorskip("torch")
+    G = q.shape[1] // k.shape[1]
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    kk, vv = tk.repeat_interleave(G, dim=1), tv.repeat_interleave(G, dim=1)
+    s = scale * tq @ kk.transpose(-1, -2)
+    Sq, Sk = q.shape[2], k.shape[2]
+    if causal:
+        vis = torch.arange(Sk)[None, :] <= (torch.arange(Sq) + (Sk - Sq))[:, None]
+        s = s.masked_fill(~vis, float("-inf"))
+    p = torch.softmax(s, dim=-1).nan_to_num(0.0)  # rows with no key: P = 0
+    o = p @ vv
+    o.backward(torch.tensor(do, dtype=torch.float64))
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy(), o.detach().numpy()
+
+
+@pytest.mark.parametrize("Hq,Hkv,Sq,Sk,causal", [
+    (2, 2, 6, 6, False), (4, 2, 5, 9, True), (8, 2, 9, 4, True), (3, 1, 7, 7, True), (4, 4, 1, 12, False),
+])
+def test_backward_matches_torch_autograd(Hq, Hkv, Sq, Sk, causal):
+    rng = np.random.default_rng(400 + Hq * Sq + Sk)
+    q, do = _rand(rng, 2, Hq, Sq, 8), _rand(rng, 2, Hq, Sq, 8)
+    k, v = _rand(rng, 2, Hkv, Sk, 8), _rand(rng, 2, Hkv, Sk, 8)
+    r = ref.ref_attention_backward(q, k, v, do, 0.4, causal)
+    dq, dk, dv, o = _autograd_backward(q, k, v, do, 0.4, causal)
+    for name, a, b in (("dq", r["dq"], dq), ("dk", r["dk"], dk), ("dv", r["dv"], dv), ("o", r["o"], o)):
+        assert np.abs(a - b).max() < 1e-12, name
+    assert np.abs(r["delta"] - (do * o).sum(-1)).max() < 1e-12
+
+
+def test_backward_matches_finite_differences():
+    """Directional derivatives of f = sum(O * dO) by central differences."""
+    rng = np.random.default_rng(410)
+    q, do = _rand(rng, 1, 4, 5, 6), _rand(rng, 1, 4, 5, 6)
+    k, v = _rand(rng, 1, 2, 7, 6), _rand(rng, 1, 2, 7, 6)
+    r = ref.ref_attention_backward(q, k, v, do, 0.6, True)
+    eps = 1e-5
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        u = rng.standard_normal(x.shape)
+        args_p = dict(q=q, k=k, v=v)
+        args_m = dict(q=q, k=k, v=v)
+        args_p[name] = x + eps * u
+        args_m[name] = x - eps * u
+        fp = (ref.ref_attention(args_p["q"], args_p["k"], args_p["v"], 0.6, True)[0] * do).sum()
+        fm = (ref.ref_attention(args_m["q"], args_m["k"], args_m["v"], 0.6, True)[0] * do).sum()
+        fd = (fp - fm) / (2 * eps)
+        assert abs(fd - (r["d" + name] * u).sum()) < 1e-7 * max(1.0, abs(fd)), name
+
+
+def test_backward_closed_forms():
+    rng = np.random.default_rng(420)
+    # one key: O = v everywhere, so dV = sum of dO over the group's rows and dQ = dK = 0
+    q, do = _rand(rng, 1, 4, 6, 8), _rand(rng, 1, 4, 6, 8)
+    k, v = _rand(rng, 1, 2, 1, 8), _rand(rng, 1, 2, 1, 8)
+    r = ref.ref_attention_backward(q, k, v, do, 0.5, False)
+    assert np.abs(r["dq"]).max() < 1e-15 and np.abs(r["dk"]).max() < 1e-15
+    for kvh in range(2):
+        assert np.allclose(r["dv"][0, kvh, 0], do[0, 2 * kvh:2 * kvh + 2].sum(axis=(0, 1)), atol=1e-12)
+    # zero queries: uniform P over the visible keys and dK = scale * dS^T Q = 0
+    q0 = np.zeros((1, 2, 5, 8))
+    k, v, do = _rand(rng, 1, 2, 5, 8), _rand(rng, 1, 2, 5, 8), _rand(rng, 1, 2, 5, 8)
+    r = ref.ref_attention_backward(q0, k, v, do, 0.5, True)
+    assert np.abs(r["dk"]).max() == 0.0
+    n_vis = np.arange(1, 6)
+    for h in range(2):
+        want = np.stack([(do[0, h, j:] / n_vis[j:, None]).sum(0) for j in range(5)])
+        assert np.allclose(r["dv"][0, h], want, atol=1e-12)
+
+
+def test_backward_gqa_is_repeated_mha_summed():
+    rng = np.random.default_rng(430)
+    q, do = _rand(rng, 1, 6, 5, 4), _rand(rng, 1, 6, 5, 4)
+    k, v = _rand(rng, 1, 2, 8, 4), _rand(rng, 1, 2, 8, 4)
+    r = ref.ref_attention_backward(q, k, v, do, 0.7, True)
+    m = ref.ref_attention_backward(q, np.repeat(k, 3, axis=1), np.repeat(v, 3, axis=1), do, 0.7, True)
+    assert np.allclose(r["dq"], m["dq"], atol=1e-13)
+    assert np.allclose(r["dk"], m["dk"].reshape(1, 2, 3, 8, 4).sum(2), atol=1e-13)
+    assert np.allclose(r["dv"], m["dv"].reshape(1, 2, 3, 8, 4).sum(2), atol=1e-13)
+
+
+def _candidate_backward(q, k, v, do, scale, causal, mutant):
+    """A copy of the gradient formulas with one planted mistake (or none)."""
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            kvh = h // G
+            s = scale * q[b, h] @ k[b, kvh].T
+            if causal:
+                vis = np.arange(Sk)[None, :] <= (np.arange(Sq) + Sk - Sq)[:, None]
+                s = np.where(vis, s, -np.inf)
+            p = np.exp(s - s.max(1, keepdims=True))
+            p /= p.sum(1, keepdims=True)
+            dP = do[b, h] @ v[b, kvh].T
+            delta = (p * dP).sum(1, keepdims=True)
+            if mutant == "no_delta":
+                delta = 0.0
+            dS = p * (dP + delta) if mutant == "delta_sign" else p * (dP - delta)
+            dv[b, kvh] += (p @ do[b, h]) if mutant == "dv_untransposed" else (p.T @ do[b, h])
+            dq[b, h] = (1.0 if mutant == "dq_no_scale" else scale) * dS @ k[b, kvh]
+            dk[b, kvh] += scale * ((dS @ q[b, h]) if mutant == "dk_untransposed" else (dS.T @ q[b, h]))
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("mutant", ["no_delta", "delta_sign", "dv_untransposed", "dq_no_scale", "dk_untransposed"])
+def test_backward_pins_reject_planted_mistakes(mutant):
+    rng = np.random.default_rng(440)
+    q, do = _rand(rng, 1, 4, 6, 4), _rand(rng, 1, 4, 6, 4)
+    k, v = _rand(rng, 1, 2, 6, 4), _rand(rng, 1, 2, 6, 4)
+    want = _autograd_backward(q, k, v, do, 0.5, True)[:3]
+    good = _candidate_backward(q, k, v, do, 0.5, True, None)
+    assert all(np.allclose(a, b, atol=1e-12) for a, b in zip(good, want))
+    bad = _candidate_backward(q, k, v, do, 0.5, True, mutant)
+    assert not all(np.allclose(a, b, atol=1e-6) for a, b in zip(bad, want))

@@ -59,6 +59,21 @@ class PrefillParams(ctypes.Structure):
     ]
 
 
+class BackwardParams(ctypes.Structure):
+    """Mirror of ``attn_backward_params``."""
+
+    _fields_ = [
+        ("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp), ("dout", _vp),
+        ("dq", _vp), ("dk", _vp), ("dv", _vp),
+        ("batch", _i32), ("num_q_heads", _i32), ("num_kv_heads", _i32), ("head_dim", _i32),
+        ("seqlen_q", _i32), ("seqlen_k", _i32),
+    ] + [(f"{t}_{d}_stride", _i64) for t in ("q", "k", "v", "o", "do", "dq", "dk", "dv")
+         for d in ("batch", "head", "row")] + [
+        ("scale", ctypes.c_float), ("causal", _i32), ("o_dtype", _i32), ("grad_dtype", _i32),
+        ("error_flags", _vp),
+    ]
+
+
 class DecodeParams(ctypes.Structure):
     """Mirror of ``attn_decode_params``."""
 
@@ -87,6 +102,9 @@ def _load():
     lib.attn_decode_paged_shared_prefix.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_int32, _vp,
                                                     ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t), _vp]
     lib.attn_decode_paged_shared_prefix.restype = ctypes.c_int
+    lib.attn_prefill_backward.argtypes = [ctypes.POINTER(BackwardParams), _vp, ctypes.c_size_t,
+                                          ctypes.POINTER(ctypes.c_size_t), _vp]
+    lib.attn_prefill_backward.restype = ctypes.c_int
     lib.splitkv_lse_combine.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp,
                                         ctypes.c_int, _vp, _vp]
     lib.splitkv_lse_combine.restype = ctypes.c_int
@@ -183,6 +201,58 @@ def prefill(q, k, v, scale: float | None = None, causal: bool = False, out=None,
     p.seqlens_q, p.seqlens_k = _ptr(seqlens_q), _ptr(seqlens_k)
     _check(LIB.attn_prefill(ctypes.byref(p), _stream(q.device)), "attn_prefill")
     return out, lse
+
+
+def _backward_params(q, k, v, o, lse, dout, dq, dk, dv, scale, causal, error_flags):
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    p = BackwardParams()
+    p.q, p.k, p.v, p.o, p.lse, p.dout = _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout)
+    p.dq, p.dk, p.dv = _ptr(dq), _ptr(dk), _ptr(dv)
+    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.seqlen_q, p.seqlen_k = B, Hq, Hkv, D, Sq, Sk
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        setattr(p, f"{name}_batch_stride", t.stride(0))
+        setattr(p, f"{name}_head_stride", t.stride(1))
+        setattr(p, f"{name}_row_stride", t.stride(2))
+    p.scale = float(scale if scale is not None else 1.0 / math.sqrt(D))
+    p.causal, p.o_dtype, p.grad_dtype = int(bool(causal)), _out_code(o.dtype), _out_code(dq.dtype)
+    p.error_flags = _ptr(error_flags)
+    return p
+
+
+def prefill_backward(q, k, v, o, lse, dout, scale: float | None = None, causal: bool = False, dq=None, dk=None,
+                     dv=None, grad_dtype=torch.float32, workspace=None, error_flags=None):
+    """Gradients of :func:`prefill` (dense): returns ``(dQ, dK, dV)``.
+
+    q, dout [B,Hq,Sq,D] bf16; k, v [B,Hkv,Sk,D] bf16; o [B,Hq,Sq,D] (bf16 or
+    fp32) and lse [B,Hq,Sq] fp32 are the forward's outputs for the same
+    inputs. The gradients are ``grad_dtype`` (fp32 or bf16) unless given.
+    """
+    _need(q.dim() == 4 and k.dim() == 4 and v.dim() == 4 and dout.dim() == 4 and o.dim() == 4, "4-D tensors")
+    B, Hq, Sq, D = q.shape
+    _need(tuple(v.shape) == tuple(k.shape) and k.shape[0] == B and k.shape[3] == D, "k/v shape")
+    _need(tuple(o.shape) == tuple(q.shape) and tuple(dout.shape) == tuple(q.shape), "o/dout shape")
+    for t in (q, k, v, dout):
+        _need(t.dtype == torch.bfloat16 and t.is_cuda and t.stride(3) == 1, "bf16 CUDA, last dim contiguous")
+    _need(o.dtype in (torch.bfloat16, torch.float32) and o.stride(3) == 1, "o bf16 or fp32")
+    _need(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, Hq, Sq), "lse [B,Hq,Sq]")
+    if dq is None:
+        dq = torch.empty(q.shape, dtype=grad_dtype, device=q.device)
+    if dk is None:
+        dk = torch.empty(k.shape, dtype=grad_dtype, device=q.device)
+    if dv is None:
+        dv = torch.empty(v.shape, dtype=grad_dtype, device=q.device)
+    _need(dq.dtype == dk.dtype == dv.dtype, "one dtype for dq, dk, dv")
+    p = _backward_params(q, k, v, o, lse, dout, dq, dk, dv, scale, causal, error_flags)
+    need = ctypes.c_size_t(0)
+    _check(LIB.attn_prefill_backward(ctypes.byref(p), None, 0, ctypes.byref(need), None), "attn_prefill_backward(size)")
+    if workspace is None and need.value > 0:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(LIB.attn_prefill_backward(ctypes.byref(p), ws_ptr, ws_bytes, None, _stream(q.device)),
+           "attn_prefill_backward")
+    return dq, dk, dv
 
 
 def prefill_paged(q, k_cache, v_cache, block_table, seqlens_k, seqlens_q=None, scale: float | None = None,

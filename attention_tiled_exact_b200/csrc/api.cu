@@ -77,6 +77,36 @@ static attn_status_t validate_prefill(const attn_prefill_params* p) {
   return ATTN_OK;
 }
 
+static attn_status_t validate_backward(const attn_backward_params* p) {
+  if (!p) return ATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->num_q_heads < 0 || p->num_kv_heads < 0 || p->seqlen_q < 0 || p->seqlen_k < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (p->num_kv_heads == 0 || p->num_q_heads == 0) return ATTN_ERR_INVALID_ARG;
+  if (p->num_q_heads % p->num_kv_heads != 0) return ATTN_ERR_UNSUPPORTED;
+  if (p->head_dim != 64 && p->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!(p->scale > 0.f) || !isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
+  if (p->o_dtype != ATTN_DTYPE_BF16 && p->o_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  if (p->grad_dtype != ATTN_DTYPE_BF16 && p->grad_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  if (!p->q || !p->k || !p->v || !p->o || !p->lse || !p->dout || !p->dq || !p->dk || !p->dv)
+    return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {p->q, p->k, p->v, p->o, p->lse, p->dout, p->dq, p->dk, p->dv};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return ATTN_ERR_UNSUPPORTED;
+  const int64_t strides[] = {p->q_batch_stride,  p->q_head_stride,  p->q_row_stride,  p->k_batch_stride,
+                             p->k_head_stride,   p->k_row_stride,   p->v_batch_stride,  p->v_head_stride,
+                             p->v_row_stride,    p->o_batch_stride,  p->o_head_stride,  p->o_row_stride,
+                             p->do_batch_stride, p->do_head_stride, p->do_row_stride, p->dq_batch_stride,
+                             p->dq_head_stride,  p->dq_row_stride,  p->dk_batch_stride, p->dk_head_stride,
+                             p->dk_row_stride,   p->dv_batch_stride, p->dv_head_stride, p->dv_row_stride};
+  for (int64_t st : strides)
+    if (!mult8(st)) return ATTN_ERR_UNSUPPORTED;
+  const int64_t rows[] = {p->q_row_stride, p->k_row_stride, p->v_row_stride, p->o_row_stride,
+                          p->do_row_stride, p->dq_row_stride, p->dk_row_stride, p->dv_row_stride};
+  for (int64_t rs : rows)
+    if (rs < p->head_dim) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
 attn_status_t validate_decode(const attn_decode_params* p) {
   if (!p) return ATTN_ERR_INVALID_ARG;
   if (p->batch < 0 || p->batch > 65535) return ATTN_ERR_INVALID_ARG;
@@ -127,6 +157,21 @@ attn_status_t attn_decode_paged(const attn_decode_params* p, void* workspace, si
   if (p->batch == 0) return ATTN_OK;
   if (!have_dev) return ATTN_ERR_NO_DEVICE;
   return attn::launch_decode(*p, plan, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_prefill_backward(const attn_backward_params* p, void* workspace, size_t workspace_bytes,
+                                    size_t* workspace_needed, attn_stream_t stream) {
+  attn_status_t st = attn::validate_backward(p);
+  if (st != ATTN_OK) return st;
+  const size_t need = attn::backward_workspace_bytes(*p);
+  if (workspace_needed) *workspace_needed = need;
+  if (workspace == nullptr && workspace_needed != nullptr) return ATTN_OK;  // size query only
+  if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_UNSUPPORTED;
+  if (p->batch == 0) return ATTN_OK;
+  st = attn::check_device();
+  if (st != ATTN_OK) return st;
+  return attn::launch_backward(*p, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 attn_status_t attn_decode_paged_shared_prefix(const attn_decode_params* p, int32_t prefix_len, void* workspace,

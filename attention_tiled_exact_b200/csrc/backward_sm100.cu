@@ -1,0 +1,627 @@
+// Backward of exact attention for sm_100a: dQ, dK, dV from Q, K, V, the
+// forward's O and LSE, and the upstream gradient dO.
+//
+// What it computes (the plain derivatives of O = softmax(scale Q K^T + mask) V;
+// FlashAttention-2 has one forward and one backward kernel, "GPU Kernel 调度:
+// 大模型推理的拐点 2026", the four-layer decomposition): per query head, with
+// P = exp(scale Q K^T - LSE) (masked entries 0),
+//     dV = P^T dO,   dP = dO V^T,   D_i = rowsum(dO * O)_i,
+//     dS = P * (dP - D),   dQ = scale dS K,   dK = scale dS^T Q,
+// dK and dV of a key/value head summing its G query heads. Nothing of size
+// Sq x Sk goes to HBM: P and dS are rebuilt tile by tile from Q, K and the
+// forward's LSE, exactly as the forward builds S tile by tile.
+//
+// Three launches:
+//   * prep (one warp per query row): D = rowsum(dO * O), and LSE * log2(e)
+//     (+inf for rows that see no key, so that their P is exactly 0);
+//   * dK/dV kernel, one CTA per (batch, kv head, 128-key block j): K_j and V_j
+//     stay in shared memory; for every query head of the group and every
+//     query block i that sees block j, TMA streams Q_i and dO_i through a
+//     two-stage ring and one thread issues
+//         S^T = K_j Q_i^T, dP^T = V_j dO_i^T          (tcgen05, fp32 in TMEM)
+//     four warps (one key row per thread, the TMEM lane) turn them into
+//     P^T = exp2(S^T scale log2 e - LSE log2 e) and dS^T = P^T (dP^T - D),
+//     written back into TMEM as bf16 over S^T and dP^T, and the thread issues
+//         dV += P^T dO_i, dK += dS^T Q_i              (A from TMEM)
+//     into two accumulators that stay in TMEM for the whole CTA;
+//   * dQ kernel, one CTA per (batch, query head, 128-query block i): Q_i and
+//     dO_i stay in shared memory, K_j and V_j stream, S and dP are recomputed
+//     the same way and dQ += dS K_j accumulates in TMEM.
+// dQ is recomputed rather than accumulated with atomics from the dK/dV
+// kernel (7 products per tile pair instead of 5): the result is
+// deterministic, and TMEM has no room for a fifth 128-column accumulator
+// next to S^T, dP^T, dK and dV.
+//
+// Every operand form here is one the forward kernel also uses: K-major A and
+// B from shared memory for S-like products, A from TMEM with an MN-major B
+// tile (rows of the tile = the reduction) for the accumulating products.
+// Every mbarrier wait is bounded; on a timeout the CTA stops, drains and
+// reports ATTN_FAULT_TIMEOUT.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+namespace bwd {
+
+constexpr int BM = 128;  // rows of every tile (queries or keys)
+constexpr int NUM_THREADS = 192;  // warps 0-3: elementwise + epilogue; 4: TMA; 5: MMA
+constexpr int TMA_WARP = 4;
+constexpr int MMA_WARP = 5;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr long long WAIT_LIMIT = 2000000000LL;  // cycles (~1 s)
+constexpr float LOG2E = 1.4426950408889634f;
+
+struct Args {
+  int batch, hq, hkv, group, seqlen_q, seqlen_k, n_qb, n_kb;
+  int causal;
+  float scale, scale_log2;
+  const float* lse2;   // [B, Hq, Sq]: LSE * log2(e), +inf where the row sees no key
+  const float* delta;  // [B, Hq, Sq]: rowsum(dO * O)
+  void* dq;
+  void* dk;
+  void* dv;
+  long long dq_bs, dq_hs, dq_rs, dk_bs, dk_hs, dk_rs, dv_bs, dv_hs, dv_rs;
+  int grad_f32;
+  int32_t* error_flags;
+};
+
+template <int D>
+struct Layout {
+  static constexpr int CHUNKS = D / 64;  // 64-column (128-byte) boxes per row
+  static constexpr int TILE = BM * D * 2;
+  // Resident tiles A0, A1 (dK/dV kernel: K_j, V_j; dQ kernel: Q_i, dO_i) and
+  // a two-stage ring of streamed pairs B0, B1 (Q_i, dO_i or K_j, V_j).
+  static constexpr int A0_OFF = 0;
+  static constexpr int A1_OFF = TILE;
+  static constexpr int RING_OFF = 2 * TILE;          // stage s: B0 at + 2 s TILE, B1 at + (2 s + 1) TILE
+  static constexpr int VEC_OFF = RING_OFF + 4 * TILE;  // [stage][lse2, delta][BM] floats (dK/dV kernel)
+  static constexpr int BAR_OFF = VEC_OFF + 2 * 2 * BM * 4;
+  // a_full, ring_full[2], ring_empty[2], s_full, dp_full, ps_full, acc_full, mma_done
+  static constexpr int NUM_BARS = 10;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem address, abort flag
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
+};
+
+// TMEM columns: S (or S^T) at 0, dP (or dP^T) at 128, accumulators from 256
+// (dK/dV kernel: dV at 256, dK at 256 + D; dQ kernel: dQ at 256).
+constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC = 256;
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, WAIT_LIMIT));
+}
+
+// Stores one 32-column slice of a gradient row (fp32 or bf16).
+__device__ __forceinline__ void store_slice(void* base, long long off, int col0, const float* x, int f32) {
+  if (f32) {
+    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + off + col0);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dst[k] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + off + col0);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      dst[k] = make_uint4(pack_bf16x2(x[8 * k], x[8 * k + 1]), pack_bf16x2(x[8 * k + 2], x[8 * k + 3]),
+                          pack_bf16x2(x[8 * k + 4], x[8 * k + 5]), pack_bf16x2(x[8 * k + 6], x[8 * k + 7]));
+  }
+}
+
+// The work of one CTA.
+struct Work {
+  int b, kvh, h;   // h: the query head (dQ kernel)
+  int blk;         // the resident 128-row block (keys: j; queries: i)
+  int first;       // first streamed block
+  int per_head;    // streamed blocks per query head
+  int n_steps;     // total streamed blocks (dK/dV kernel: G heads x per_head)
+};
+
+template <bool KV>
+__device__ __forceinline__ Work decode_work(const Args& a) {
+  Work w;
+  const int off = a.seqlen_k - a.seqlen_q;  // bottom-right causal alignment
+  const int item = blockIdx.x;
+  if constexpr (KV) {
+    // Key block 0 first: under the causal mask it has the most query blocks.
+    const int bh = item % (a.batch * a.hkv);
+    w.blk = item / (a.batch * a.hkv);
+    w.b = bh / a.hkv;
+    w.kvh = bh - w.b * a.hkv;
+    w.h = 0;
+    // Query block i sees key block j when its last query (i BM + BM - 1) sits
+    // at or after the block's first key: i BM + BM - 1 + off >= j BM.
+    int first = 0;
+    if (a.causal) {
+      const int x = w.blk * BM - off - (BM - 1);
+      first = x > 0 ? (x + BM - 1) / BM : 0;
+    }
+    w.first = first;
+    w.per_head = a.n_qb > first ? a.n_qb - first : 0;
+    w.n_steps = a.group * w.per_head;
+  } else {
+    // The last query block first: under the causal mask it sees the most keys.
+    const int bh = item % (a.batch * a.hq);
+    w.blk = a.n_qb - 1 - item / (a.batch * a.hq);
+    w.b = bh / a.hq;
+    w.h = bh - w.b * a.hq;
+    w.kvh = w.h / a.group;
+    int n = a.n_kb;
+    if (a.causal) {
+      const int last = w.blk * BM + BM - 1 + off;  // the block's last query sees keys 0..last
+      const int nb = last >= 0 ? last / BM + 1 : 0;
+      n = nb < n ? nb : n;
+    }
+    w.first = 0;
+    w.per_head = n;
+    w.n_steps = n;
+  }
+  return w;
+}
+
+template <int D, bool KV>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Args a) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* a_full = bars;
+  uint64_t* ring_full = bars + 1;
+  uint64_t* ring_empty = bars + 3;
+  uint64_t* s_full = bars + 5;
+  uint64_t* dp_full = bars + 6;
+  uint64_t* ps_full = bars + 7;  // the elementwise warps wrote P / dS into TMEM
+  uint64_t* acc_full = bars + 8;
+  uint64_t* mma_done = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const Work w = decode_work<KV>(a);
+
+  if (threadIdx.x == 0) {
+    mbar_init(a_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ring_full[s], 1);
+      mbar_init(&ring_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(ps_full, 128);
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // Streamed step t: query head and block (dK/dV kernel) or key block (dQ kernel).
+  auto step_head = [&](int t) { return KV ? w.kvh * a.group + t / w.per_head : w.h; };
+  auto step_blk = [&](int t) { return KV ? w.first + t % w.per_head : t; };
+
+  if (warp == TMA_WARP) {
+    if (w.n_steps > 0) {
+      // ---------------------------------------------------------------- producer (whole warp)
+      // Lane 0 issues the copies. In the dK/dV kernel all lanes first write the
+      // step's per-column LSE and D into shared memory; the stage's full
+      // barrier, which the elementwise warps also wait on, publishes them.
+      float* vec = reinterpret_cast<float*>(smem + L::VEC_OFF);
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+        mbar_arrive_expect_tx(a_full, 2 * L::TILE);
+        for (int c = 0; c < L::CHUNKS; ++c) {
+          if constexpr (KV) {
+            tma_load_4d(smem + L::A0_OFF + c * (BM * 128), &tm_k, a_full, c * 64, w.blk * BM, w.kvh, w.b);
+            tma_load_4d(smem + L::A1_OFF + c * (BM * 128), &tm_v, a_full, c * 64, w.blk * BM, w.kvh, w.b);
+          } else {
+            tma_load_4d(smem + L::A0_OFF + c * (BM * 128), &tm_q, a_full, c * 64, w.blk * BM, w.h, w.b);
+            tma_load_4d(smem + L::A1_OFF + c * (BM * 128), &tm_do, a_full, c * 64, w.blk * BM, w.h, w.b);
+          }
+        }
+      }
+      int t = 0;
+      for (; t < w.n_steps; ++t) {
+        const int s = t & 1;
+        if (t >= 2 && !warp_wait(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag)) break;
+        const int h = step_head(t), blk = step_blk(t);
+        if constexpr (KV) {
+          // Queries past Sq get LSE = +inf (P = 0) and D = 0.
+          for (int k = lane; k < BM; k += 32) {
+            const int qpos = blk * BM + k;
+            const long long ro = ((long long)w.b * a.hq + h) * a.seqlen_q + qpos;
+            vec[(2 * s) * BM + k] = qpos < a.seqlen_q ? a.lse2[ro] : INFINITY;
+            vec[(2 * s + 1) * BM + k] = qpos < a.seqlen_q ? a.delta[ro] : 0.f;
+          }
+          __threadfence_block();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE);
+          uint8_t* b0 = smem + L::RING_OFF + (2 * s) * L::TILE;
+          uint8_t* b1 = b0 + L::TILE;
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            if constexpr (KV) {
+              tma_load_4d(b0 + c * (BM * 128), &tm_q, &ring_full[s], c * 64, blk * BM, h, w.b);
+              tma_load_4d(b1 + c * (BM * 128), &tm_do, &ring_full[s], c * 64, blk * BM, h, w.b);
+            } else {
+              tma_load_4d(b0 + c * (BM * 128), &tm_k, &ring_full[s], c * 64, blk * BM, w.kvh, w.b);
+              tma_load_4d(b1 + c * (BM * 128), &tm_v, &ring_full[s], c * 64, blk * BM, w.kvh, w.b);
+            }
+          }
+        }
+        __syncwarp();
+      }
+      // Drain: no copy may be in flight when the CTA exits (abort path).
+      if (lane == 0) {
+        mbar_wait_bounded(a_full, 0, abort_flag, WAIT_LIMIT);
+        for (int u = t - 2 > 0 ? t - 2 : 0; u < t; ++u)
+          mbar_wait_bounded(&ring_full[u & 1], (u >> 1) & 1, abort_flag, WAIT_LIMIT);
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0 && w.n_steps > 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      constexpr uint32_t ID_S = instr_desc_bf16(BM, BM, 0);   // S-like: both operands K-major
+      constexpr uint32_t ID_ACC = instr_desc_bf16(BM, D, 1);  // accumulate: B MN-major
+      const uint32_t hi = sw128_desc_hi(1024);
+      const uint32_t a0_lo = sw128_desc_lo(smem_addr(smem + L::A0_OFF), 16);
+      const uint32_t a1_lo = sw128_desc_lo(smem_addr(smem + L::A1_OFF), 16);
+      const uint32_t ring_k = sw128_desc_lo(smem_addr(smem + L::RING_OFF), 16);        // K-major
+      const uint32_t ring_mn = sw128_desc_lo(smem_addr(smem + L::RING_OFF), BM * 128);  // MN-major
+      const uint32_t id_s = ID_S, id_acc = ID_ACC;
+      // X (cols col) = A (BM x D) * B (BM x D)^T over head_dim.
+      auto issue_s = [&](uint32_t col, uint32_t a_lo, uint32_t b_lo) {
+        static_for<0, D / 16>([&](auto c) {
+          constexpr int kk = decltype(c)::value;
+          constexpr uint32_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+          mma_ss_lo<off, off>(tmem_base + col, a_lo, b_lo, hi, id_s, kk > 0 ? 1u : 0u);
+        });
+      };
+      // ACC (cols col) += X (bf16 in TMEM at a_col, BM x BM) * B (BM rows = the reduction, D columns).
+      auto issue_acc = [&](uint32_t col, uint32_t a_col, uint32_t b_lo, bool first) {
+        static_for<0, BM / 16>([&](auto c) {
+          constexpr int kk = decltype(c)::value;
+          constexpr uint32_t b_off = (kk * 16 * 128) >> 4;
+          mma_ts_lo<kk * 8, b_off>(tmem_base + col, tmem_base + a_col, b_lo, hi, id_acc,
+                                   (!first || kk > 0) ? 1u : 0u);
+        });
+      };
+      bool ok = mbar_wait_bounded(a_full, 0, abort_flag, WAIT_LIMIT);
+      for (int t = 0; t < w.n_steps && ok; ++t) {
+        const int s = t & 1;
+        ok = mbar_wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, WAIT_LIMIT);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t b0 = (uint32_t)(((2 * s) * L::TILE) >> 4);
+        const uint32_t b1 = (uint32_t)(((2 * s + 1) * L::TILE) >> 4);
+        // The previous step's accumulating MMAs read P / dS over these
+        // columns; MMAs from one thread run in issue order.
+        issue_s(COL_S, a0_lo, ring_k + b0);   // S^T = K Q^T  |  S = Q K^T
+        mma_commit(s_full);
+        issue_s(COL_DP, a1_lo, ring_k + b1);  // dP^T = V dO^T  |  dP = dO V^T
+        mma_commit(dp_full);
+        ok = mbar_wait_bounded(ps_full, t & 1, abort_flag, WAIT_LIMIT);
+        if (!ok) break;
+        tc_fence_after();
+        if constexpr (KV) {
+          issue_acc(COL_ACC, COL_S, ring_mn + b1, t == 0);       // dV += P^T dO
+          issue_acc(COL_ACC + D, COL_DP, ring_mn + b0, t == 0);  // dK += dS^T Q
+        } else {
+          issue_acc(COL_ACC, COL_DP, ring_mn + b0, t == 0);  // dQ += dS K
+        }
+        mma_commit(&ring_empty[s]);
+      }
+      if (ok) mma_commit(acc_full);
+      // Every MMA must have completed before tensor memory is released.
+      mma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, abort_flag, WAIT_LIMIT);
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise + epilogue
+    const int r = warp * 32 + lane;  // the resident tile's row == TMEM lane
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    const int off = a.seqlen_k - a.seqlen_q;
+    const float sl2 = a.scale_log2;
+    float* vec = reinterpret_cast<float*>(smem + L::VEC_OFF);
+    // dQ kernel: this row's LSE and D.
+    const int row_pos = w.blk * BM + r;  // key position (dK/dV) or query position (dQ)
+    float lse_r = INFINITY, delta_r = 0.f;
+    if constexpr (!KV) {
+      if (row_pos < a.seqlen_q) {
+        const long long ro = ((long long)w.b * a.hq + w.h) * a.seqlen_q + row_pos;
+        lse_r = a.lse2[ro];
+        delta_r = a.delta[ro];
+      }
+    }
+    bool ok = true;
+    for (int t = 0; t < w.n_steps && ok; ++t) {
+      const int s = t & 1;
+      const int blk = step_blk(t);
+      // Columns c < c_lim are visible.
+      int c_lim;
+      if constexpr (KV) {
+        // Column c = query i BM + c, at position i BM + c + off; this key row
+        // is visible to it when row_pos <= i BM + c + off. The producer wrote
+        // the step's per-column LSE and D before the stage's full barrier.
+        c_lim = row_pos < a.seqlen_k ? (a.causal ? row_pos - off - blk * BM : -BM) : BM;  // first visible column
+        ok = warp_wait(&ring_full[s], (t >> 1) & 1, abort_flag);
+        if (!ok) break;
+      } else {
+        // Column c = key blk BM + c; visible when < Sk and (causal) <= row_pos + off.
+        int lim = a.seqlen_k - blk * BM;
+        if (a.causal) {
+          const int cl = row_pos + off - blk * BM + 1;
+          lim = cl < lim ? cl : lim;
+        }
+        c_lim = lim;
+      }
+      const float* lse_c = vec + (2 * s) * BM;
+      const float* delta_c = vec + (2 * s + 1) * BM;
+      ok = warp_wait(s_full, t & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        uint32_t sv[32];
+        tmem_ld32(lane_base + COL_S + cc * 32, sv);
+        tmem_ld_wait();
+        float p[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int c = cc * 32 + jj;
+          const float lse = KV ? lse_c[c] : lse_r;
+          const bool vis = KV ? (c >= c_lim) : (c < c_lim);
+          p[jj] = vis ? ex2_approx(fmaf(__uint_as_float(sv[jj]), sl2, -lse)) : 0.f;
+        }
+        if (cc == 0) {
+          ok = warp_wait(dp_full, t & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        uint32_t dv[32];
+        tmem_ld32(lane_base + COL_DP + cc * 32, dv);
+        tmem_ld_wait();
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 2) {
+          const float d0 = KV ? delta_c[cc * 32 + jj] : delta_r;
+          const float d1 = KV ? delta_c[cc * 32 + jj + 1] : delta_r;
+          const float ds0 = p[jj] * (__uint_as_float(dv[jj]) - d0);
+          const float ds1 = p[jj + 1] * (__uint_as_float(dv[jj + 1]) - d1);
+          pk[jj / 2] = pack_bf16x2(p[jj], p[jj + 1]);
+          dk[jj / 2] = pack_bf16x2(ds0, ds1);
+        }
+        // bf16 pairs over the columns already read (chunk cc covers 16 cols).
+        if constexpr (KV) tmem_st16(lane_base + COL_S + cc * 16, pk);
+        tmem_st16(lane_base + COL_DP + cc * 16, dk);
+      }
+      if (!ok) break;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ps_full);
+    }
+    // ---- epilogue: this row of the accumulators, scaled where needed
+    const bool row_ok = row_pos < (KV ? a.seqlen_k : a.seqlen_q);
+    if (ok && w.n_steps > 0) ok = warp_wait(acc_full, 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const int n_out = KV ? 2 : 1;
+      for (int o = 0; o < n_out; ++o) {
+        // dK/dV kernel: o = 0 -> dV (unscaled), o = 1 -> dK (scale); dQ kernel: dQ (scale).
+        const bool is_dv = KV && o == 0;
+        void* base = KV ? (is_dv ? a.dv : a.dk) : a.dq;
+        const long long row_off =
+            KV ? (is_dv ? (long long)w.b * a.dv_bs + (long long)w.kvh * a.dv_hs + (long long)row_pos * a.dv_rs
+                        : (long long)w.b * a.dk_bs + (long long)w.kvh * a.dk_hs + (long long)row_pos * a.dk_rs)
+               : (long long)w.b * a.dq_bs + (long long)w.h * a.dq_hs + (long long)row_pos * a.dq_rs;
+        const float mul = is_dv ? 1.f : a.scale;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float x[32];
+          if (w.n_steps > 0) {
+            uint32_t v[32];
+            tmem_ld32(lane_base + COL_ACC + o * D + cc * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(v[k]) * mul;
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) x[k] = 0.f;  // no visible pair: the gradient is 0
+          }
+          if (row_ok) store_slice(base, row_off, cc * 32, x, a.grad_f32);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag && a.error_flags) atomicOr(a.error_flags, ATTN_FAULT_TIMEOUT);
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// D = rowsum(dO * O) and LSE * log2(e) per query row (one warp per row).
+template <int D>
+__global__ void __launch_bounds__(256)
+    bwd_prep_kernel(const void* o, int o_f32, long long o_bs, long long o_hs, long long o_rs,
+                    const __nv_bfloat16* dout, long long do_bs, long long do_hs, long long do_rs,
+                    const float* lse, int batch, int hq, int seqlen_q, float* lse2, float* delta) {
+  constexpr int PER = D / 32;
+  const long long row = (long long)blockIdx.x * 8 + warp_id();
+  const int lane = lane_id();
+  if (row >= (long long)batch * hq * seqlen_q) return;
+  const int q = (int)(row % seqlen_q);
+  const long long bh = row / seqlen_q;
+  const int h = (int)(bh % hq), b = (int)(bh / hq);
+  const __nv_bfloat16* dr = dout + b * do_bs + h * do_hs + q * do_rs + lane * PER;
+  float acc = 0.f;
+  if (o_f32) {
+    const float* orow = reinterpret_cast<const float*>(o) + b * o_bs + h * o_hs + q * o_rs + lane * PER;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc = fmaf(__bfloat162float(dr[k]), orow[k], acc);
+  } else {
+    const __nv_bfloat16* orow = reinterpret_cast<const __nv_bfloat16*>(o) + b * o_bs + h * o_hs + q * o_rs + lane * PER;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc = fmaf(__bfloat162float(dr[k]), __bfloat162float(orow[k]), acc);
+  }
+#pragma unroll
+  for (int sh = 16; sh >= 1; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  if (lane == 0) {
+    const float l = lse[row];
+    lse2[row] = l == -INFINITY ? INFINITY : l * LOG2E;
+    delta[row] = acc;
+  }
+}
+
+}  // namespace bwd
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*BwdEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static BwdEncodeFn bwd_encode_fn() {
+  static BwdEncodeFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<BwdEncodeFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 [d3][d2][d1][d0 = head_dim] with element strides s1..s3; box of 64
+// columns x 128 rows, 128-byte swizzle, zero fill out of bounds.
+static bool bwd_map(CUtensorMap* map, const void* base, int D, int rows, int heads, int batch, int64_t rs, int64_t hs,
+                    int64_t bs) {
+  BwdEncodeFn fn = bwd_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)rs * 2, (cuuint64_t)hs * 2, (cuuint64_t)bs * 2};
+  cuuint32_t box[4] = {64u, (cuuint32_t)bwd::BM, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t backward_workspace_bytes(const attn_backward_params& p) {
+  const size_t n = (size_t)p.batch * p.num_q_heads * p.seqlen_q * sizeof(float);
+  return 2 * ((n + 255) / 256 * 256);
+}
+
+template <int D, bool KV>
+static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const CUtensorMap& tdo, const bwd::Args& a, long long grid, cudaStream_t stream) {
+  using L = bwd::Layout<D>;
+  static_assert(L::SMEM_BYTES <= 232448, "shared memory budget");
+  auto kern = bwd::bwd_kernel<D, KV>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    configured = true;
+  }
+  if (grid <= 0) return ATTN_OK;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  kern<<<(unsigned)grid, bwd::NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t launch_backward(const attn_backward_params& p, void* workspace, cudaStream_t stream) {
+  if (p.batch == 0 || p.num_q_heads == 0 || (p.seqlen_q == 0 && p.seqlen_k == 0)) return ATTN_OK;
+  const int D = p.head_dim;
+  const size_t n = (size_t)p.batch * p.num_q_heads * p.seqlen_q;
+  float* lse2 = reinterpret_cast<float*>(workspace);
+  float* delta = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + (n * 4 + 255) / 256 * 256);
+  const bool o_f32 = p.o_dtype == ATTN_DTYPE_F32;
+  if (n > 0) {
+    const long long blocks = (long long)((n + 7) / 8);
+    if (blocks > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    if (D == 128)
+      bwd::bwd_prep_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
+          p.o, o_f32, p.o_batch_stride, p.o_head_stride, p.o_row_stride,
+          reinterpret_cast<const __nv_bfloat16*>(p.dout), p.do_batch_stride, p.do_head_stride, p.do_row_stride, p.lse,
+          p.batch, p.num_q_heads, p.seqlen_q, lse2, delta);
+    else
+      bwd::bwd_prep_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
+          p.o, o_f32, p.o_batch_stride, p.o_head_stride, p.o_row_stride,
+          reinterpret_cast<const __nv_bfloat16*>(p.dout), p.do_batch_stride, p.do_head_stride, p.do_row_stride, p.lse,
+          p.batch, p.num_q_heads, p.seqlen_q, lse2, delta);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  // Tensor maps need at least one row; an empty side is never loaded.
+  const int sq_map = p.seqlen_q > 0 ? p.seqlen_q : 1, sk_map = p.seqlen_k > 0 ? p.seqlen_k : 1;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!bwd_map(&tq, p.q, D, sq_map, p.num_q_heads, p.batch, p.q_row_stride, p.q_head_stride, p.q_batch_stride) ||
+      !bwd_map(&tdo, p.dout, D, sq_map, p.num_q_heads, p.batch, p.do_row_stride, p.do_head_stride,
+               p.do_batch_stride) ||
+      !bwd_map(&tk, p.k, D, sk_map, p.num_kv_heads, p.batch, p.k_row_stride, p.k_head_stride, p.k_batch_stride) ||
+      !bwd_map(&tv, p.v, D, sk_map, p.num_kv_heads, p.batch, p.v_row_stride, p.v_head_stride, p.v_batch_stride))
+    return ATTN_ERR_CUDA;
+  bwd::Args a;
+  memset(&a, 0, sizeof(a));
+  a.batch = p.batch;
+  a.hq = p.num_q_heads;
+  a.hkv = p.num_kv_heads;
+  a.group = p.num_q_heads / p.num_kv_heads;
+  a.seqlen_q = p.seqlen_q;
+  a.seqlen_k = p.seqlen_k;
+  a.n_qb = (p.seqlen_q + bwd::BM - 1) / bwd::BM;
+  a.n_kb = (p.seqlen_k + bwd::BM - 1) / bwd::BM;
+  a.causal = p.causal ? 1 : 0;
+  a.scale = p.scale;
+  a.scale_log2 = p.scale * bwd::LOG2E;
+  a.lse2 = lse2;
+  a.delta = delta;
+  a.dq = p.dq;
+  a.dk = p.dk;
+  a.dv = p.dv;
+  a.dq_bs = p.dq_batch_stride;
+  a.dq_hs = p.dq_head_stride;
+  a.dq_rs = p.dq_row_stride;
+  a.dk_bs = p.dk_batch_stride;
+  a.dk_hs = p.dk_head_stride;
+  a.dk_rs = p.dk_row_stride;
+  a.dv_bs = p.dv_batch_stride;
+  a.dv_hs = p.dv_head_stride;
+  a.dv_rs = p.dv_row_stride;
+  a.grad_f32 = p.grad_dtype == ATTN_DTYPE_F32;
+  a.error_flags = p.error_flags;
+  const long long kv_items = (long long)a.n_kb * p.batch * p.num_kv_heads;
+  const long long q_items = (long long)a.n_qb * p.batch * p.num_q_heads;
+  attn_status_t st;
+  if (D == 128) {
+    st = launch_bwd<128, true>(tq, tk, tv, tdo, a, kv_items, stream);
+    if (st == ATTN_OK) st = launch_bwd<128, false>(tq, tk, tv, tdo, a, q_items, stream);
+  } else {
+    st = launch_bwd<64, true>(tq, tk, tv, tdo, a, kv_items, stream);
+    if (st == ATTN_OK) st = launch_bwd<64, false>(tq, tk, tv, tdo, a, q_items, stream);
+  }
+  return st;
+}
+
+}  // namespace attn

@@ -36,6 +36,10 @@ attn_status_t launch_combine(const float* part_o, const float* part_lse, int num
                              int split_tokens, int rows_per_seq, void* out_o, attn_dtype_t out_dtype,
                              float* out_lse, cudaStream_t stream);
 
+// Backward (dQ, dK, dV). Arguments were validated by the caller.
+size_t backward_workspace_bytes(const attn_backward_params& p);
+attn_status_t launch_backward(const attn_backward_params& p, void* workspace, cudaStream_t stream);
+
 // Shared-prefix (cascade) decode: key ranges of the prefix prefill, the suffix
 // decode (its parameters and split plan) and the workspace layout.
 struct CascadePlan {

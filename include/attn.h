@@ -204,6 +204,71 @@ ATTN_API attn_status_t attn_decode_paged(const attn_decode_params* p, void* work
                                 size_t* workspace_needed, attn_stream_t stream);
 
 /*
+ * Backward of attn_prefill (dense, non-paged): the gradients dQ, dK, dV of
+ * O = softmax(scale Q K^T + causal mask) V for an upstream gradient dO. These
+ * are the plain derivatives of that definition; the pages count one backward
+ * kernel next to the forward one for FlashAttention-2 and ask both to match a
+ * reference ("GPU Kernel 调度:大模型推理的拐点 2026", the four-layer
+ * decomposition and checklist item 1). With P = exp(scale Q K^T - LSE)
+ * (masked entries 0), per query head:
+ *   dV = P^T dO;  dP = dO V^T;  D = rowsum(dO * O);  dS = P * (dP - D);
+ *   dQ = scale dS K;  dK = scale dS^T Q
+ * and dK, dV of a key/value head sum over its num_q_heads / num_kv_heads
+ * query heads. The causal mask and its bottom-right alignment are those of
+ * attn_prefill. P and dS are rebuilt tile by tile (never stored); P and dS
+ * enter the tensor-core products in bf16 with fp32 accumulation.
+ *
+ * Layout (element strides; the last dimension contiguous):
+ *   q, dout [batch, num_q_heads, seqlen_q, head_dim] bf16
+ *   k, v [batch, num_kv_heads, seqlen_k, head_dim] bf16
+ *   o [batch, num_q_heads, seqlen_q, head_dim] o_dtype: attn_prefill's output
+ *   lse [batch, num_q_heads, seqlen_q] fp32, contiguous: attn_prefill's LSE
+ *   dq like q, dk and dv like k, all grad_dtype (BF16 or F32)
+ * Requirements: head_dim 64 or 128; num_q_heads % num_kv_heads == 0; every
+ * pointer 16-byte aligned and every stride a multiple of 8 elements.
+ * All buffers are the caller's device memory; dq, dk, dv are overwritten
+ * (rows that see no key get 0). Deterministic: no atomics.
+ *
+ * Workspace: at least *workspace_needed bytes of device memory, 256-byte
+ * aligned (two fp32 values per query row). workspace = NULL only queries the
+ * size (returns ATTN_OK, enqueues nothing); a smaller workspace returns
+ * ATTN_ERR_WORKSPACE and enqueues nothing. Asynchronous on `stream`.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const float* lse;
+  const void* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  int batch;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int seqlen_q;
+  int seqlen_k;
+  int64_t q_batch_stride, q_head_stride, q_row_stride;
+  int64_t k_batch_stride, k_head_stride, k_row_stride;
+  int64_t v_batch_stride, v_head_stride, v_row_stride;
+  int64_t o_batch_stride, o_head_stride, o_row_stride;
+  int64_t do_batch_stride, do_head_stride, do_row_stride;
+  int64_t dq_batch_stride, dq_head_stride, dq_row_stride;
+  int64_t dk_batch_stride, dk_head_stride, dk_row_stride;
+  int64_t dv_batch_stride, dv_head_stride, dv_row_stride;
+  float scale;
+  int causal;
+  attn_dtype_t o_dtype;    /* dtype of o: BF16 or F32 */
+  attn_dtype_t grad_dtype; /* dtype of dq, dk, dv: BF16 or F32 */
+  int32_t* error_flags;    /* nullable */
+} attn_backward_params;
+
+ATTN_API attn_status_t attn_prefill_backward(const attn_backward_params* p, void* workspace, size_t workspace_bytes,
+                                             size_t* workspace_needed, attn_stream_t stream);
+
+/*
  * attn_decode_paged for a batch whose sequences all begin with the same
  * prefix_len tokens (a shared prompt): requests with a common prefix can share
  * their KV blocks ("抱infra脚", Paged Attention), and a common prefix should

@@ -43,13 +43,17 @@ def test_struct_layouts_match_the_header(lib):
     """Compile a C probe against attn.h and compare sizes/offsets with ctypes."""
     fields_p = [f for f, _ in lib.PrefillParams._fields_]
     fields_d = [f for f, _ in lib.DecodeParams._fields_]
+    fields_b = [f for f, _ in lib.BackwardParams._fields_]
     body = ['#include <stdio.h>', '#include <stddef.h>', '#include "attn.h"', "int main(void){"]
     body.append('printf("P %zu\\n", sizeof(attn_prefill_params));')
     body.append('printf("D %zu\\n", sizeof(attn_decode_params));')
+    body.append('printf("B %zu\\n", sizeof(attn_backward_params));')
     for f in fields_p:
         body.append(f'printf("p.{f} %zu\\n", offsetof(attn_prefill_params, {f}));')
     for f in fields_d:
         body.append(f'printf("d.{f} %zu\\n", offsetof(attn_decode_params, {f}));')
+    for f in fields_b:
+        body.append(f'printf("b.{f} %zu\\n", offsetof(attn_backward_params, {f}));')
     body.append("return 0;}")
     with tempfile.TemporaryDirectory() as d:
         c = os.path.join(d, "probe.c")
@@ -63,6 +67,9 @@ def test_struct_layouts_match_the_header(lib):
         assert int(got[f"p.{f}"]) == getattr(lib.PrefillParams, f).offset, f
     for f in fields_d:
         assert int(got[f"d.{f}"]) == getattr(lib.DecodeParams, f).offset, f
+    assert int(got["B"]) == ctypes.sizeof(lib.BackwardParams)
+    for f in fields_b:
+        assert int(got[f"b.{f}"]) == getattr(lib.BackwardParams, f).offset, f
 
 
 def test_status_strings(lib):
@@ -194,6 +201,47 @@ def test_shared_prefix_decode_workspace_and_dtypes(lib):
     # ordinary decode argument checks apply first
     bad = _decode_params(lib, head_dim=64)
     assert f(ctypes.byref(bad), 1024, None, 0, ctypes.byref(need), None) == lib.ATTN_ERR_UNSUPPORTED
+
+
+def _backward_params(lib, **kw):
+    p = lib.BackwardParams()
+    fake = 1 << 20
+    for f in ("q", "k", "v", "o", "lse", "dout", "dq", "dk", "dv"):
+        setattr(p, f, fake)
+    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.seqlen_q, p.seqlen_k = 2, 8, 2, 128, 300, 300
+    for t, (bs, hs) in (("q", (8 * 300 * 128, 300 * 128)), ("do", (8 * 300 * 128, 300 * 128)),
+                        ("o", (8 * 300 * 128, 300 * 128)), ("dq", (8 * 300 * 128, 300 * 128)),
+                        ("k", (2 * 300 * 128, 300 * 128)), ("v", (2 * 300 * 128, 300 * 128)),
+                        ("dk", (2 * 300 * 128, 300 * 128)), ("dv", (2 * 300 * 128, 300 * 128))):
+        setattr(p, f"{t}_batch_stride", bs)
+        setattr(p, f"{t}_head_stride", hs)
+        setattr(p, f"{t}_row_stride", 128)
+    p.scale, p.causal, p.o_dtype, p.grad_dtype = 0.088, 1, 0, 1
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_backward_workspace_query(lib):
+    p = _backward_params(lib)
+    need = ctypes.c_size_t(0)
+    f = lib.LIB.attn_prefill_backward
+    assert f(ctypes.byref(p), None, 0, ctypes.byref(need), None) == 0
+    assert need.value == 2 * ((2 * 8 * 300 * 4 + 255) // 256 * 256)
+    need2 = ctypes.c_size_t(0)
+    assert f(ctypes.byref(p), ctypes.c_void_p(1 << 20), need.value - 256, ctypes.byref(need2),
+             None) == lib.ATTN_ERR_WORKSPACE and need2.value == need.value
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 96, 2), ("num_kv_heads", 3, 2), ("scale", float("nan"), 1), ("lse", 0, 1), ("dv", 0, 1),
+    ("dq", (1 << 20) + 8, 2), ("k_row_stride", 132, 2), ("o_dtype", 2, 1), ("grad_dtype", 5, 1),
+    ("dk_row_stride", 64, 1), ("seqlen_q", -1, 1),
+])
+def test_backward_rejects_bad_arguments(lib, field, value, code):
+    p = _backward_params(lib, **{field: value})
+    need = ctypes.c_size_t(0)
+    assert lib.LIB.attn_prefill_backward(ctypes.byref(p), None, 0, ctypes.byref(need), None) == code
 
 
 def test_combine_rejects_bad_arguments(lib):

@@ -50,10 +50,11 @@ namespace attn {
 
 namespace bwd {
 
-constexpr int BM = 128;  // rows of every tile (queries or keys)
-constexpr int NUM_THREADS = 192;  // warps 0-3: elementwise + epilogue; 4: TMA; 5: MMA
-constexpr int TMA_WARP = 4;
-constexpr int MMA_WARP = 5;
+constexpr int BM = 128;              // rows of every tile (queries or keys)
+constexpr int EW_WARPS = 8;          // two elementwise warpgroups, one per 64-column half
+constexpr int TMA_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int NUM_THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_LIMIT = 2000000000LL;  // cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
@@ -62,8 +63,9 @@ struct Args {
   int batch, hq, hkv, group, seqlen_q, seqlen_k, n_qb, n_kb;
   int causal;
   float scale, scale_log2;
-  const float* lse2;   // [B, Hq, Sq]: LSE * log2(e), +inf where the row sees no key
-  const float* delta;  // [B, Hq, Sq]: rowsum(dO * O)
+  // Per query row, padded to whole 128-row blocks: [B, Hq, n_qb * 128].
+  const float* lse2;   // LSE * log2(e); +inf where the row sees no key and past Sq
+  const float* delta;  // rowsum(dO * O); 0 past Sq
   void* dq;
   void* dk;
   void* dv;
@@ -80,21 +82,31 @@ struct Layout {
   // a two-stage ring of streamed pairs B0, B1 (Q_i, dO_i or K_j, V_j).
   static constexpr int A0_OFF = 0;
   static constexpr int A1_OFF = TILE;
-  static constexpr int RING_OFF = 2 * TILE;          // stage s: B0 at + 2 s TILE, B1 at + (2 s + 1) TILE
+  static constexpr int RING_OFF = 2 * TILE;            // stage s: B0 at + 2 s TILE, B1 at + (2 s + 1) TILE
   static constexpr int VEC_OFF = RING_OFF + 4 * TILE;  // [stage][lse2, delta][BM] floats (dK/dV kernel)
   static constexpr int BAR_OFF = VEC_OFF + 2 * 2 * BM * 4;
-  // a_full, ring_full[2], ring_empty[2], s_full, dp_full, ps_full, acc_full, mma_done
-  static constexpr int NUM_BARS = 10;
+  // a_full, ring_full[2], ring_empty[2], sdp_full[2], ps_full[2], acc_full, mma_done
+  static constexpr int NUM_BARS = 11;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem address, abort flag
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
 };
 
-// TMEM columns: S (or S^T) at 0, dP (or dP^T) at 128, accumulators from 256
-// (dK/dV kernel: dV at 256, dK at 256 + D; dQ kernel: dQ at 256).
+// TMEM columns: S (or S^T) at 0, dP (or dP^T) at 128, each in two 64-column
+// halves; accumulators from 256 (dK/dV kernel: dV at 256, dK at 256 + D; dQ
+// kernel: dQ at 256). Half g's bf16 P / dS pairs go over the first 32
+// columns of that half.
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC = 256;
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, WAIT_LIMIT));
+}
+
+// Contiguous global -> shared copy completing on an mbarrier (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_addr(dst)),
+               "l"(src), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
 }
 
 // Stores one 32-column slice of a gradient row (fp32 or bf16).
@@ -110,6 +122,32 @@ __device__ __forceinline__ void store_slice(void* base, long long off, int col0,
       dst[k] = make_uint4(pack_bf16x2(x[8 * k], x[8 * k + 1]), pack_bf16x2(x[8 * k + 2], x[8 * k + 3]),
                           pack_bf16x2(x[8 * k + 4], x[8 * k + 5]), pack_bf16x2(x[8 * k + 6], x[8 * k + 7]));
   }
+}
+
+// X[:, half] = A (BM x D) * B[half rows] (64 x D)^T over head_dim: both
+// operands K-major; the B half starts 64 rows (8 KB) into each column box.
+template <int D, int HALF>
+__device__ __forceinline__ void issue_s_half(uint32_t d_col, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                             uint32_t idesc) {
+  static_for<0, D / 16>([&](auto c) {
+    constexpr int kk = decltype(c)::value;
+    constexpr uint32_t a_off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+    constexpr uint32_t b_off = a_off + ((HALF * 64 * 128) >> 4);
+    mma_ss_lo<a_off, b_off>(d_col, a_lo, b_lo, hi, idesc, kk > 0 ? 1u : 0u);
+  });
+}
+
+// ACC += X[:, half] (bf16 in TMEM) * B[half rows] (64 rows = the reduction x D),
+// B MN-major.
+template <int HALF>
+__device__ __forceinline__ void issue_acc_half(uint32_t d_col, uint32_t a_col, uint32_t b_lo, uint32_t hi,
+                                               uint32_t idesc, bool first) {
+  static_for<0, 4>([&](auto c) {
+    constexpr int k = decltype(c)::value;
+    constexpr int kk = HALF * 4 + k;  // 16-row step of B
+    constexpr uint32_t b_off = (kk * 16 * 128) >> 4;
+    mma_ts_lo<HALF * 64 + k * 8, b_off>(d_col, a_col, b_lo, hi, idesc, (first && HALF == 0 && k == 0) ? 0u : 1u);
+  });
 }
 
 // The work of one CTA.
@@ -174,11 +212,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* a_full = bars;
   uint64_t* ring_full = bars + 1;
   uint64_t* ring_empty = bars + 3;
-  uint64_t* s_full = bars + 5;
-  uint64_t* dp_full = bars + 6;
-  uint64_t* ps_full = bars + 7;  // the elementwise warps wrote P / dS into TMEM
-  uint64_t* acc_full = bars + 8;
-  uint64_t* mma_done = bars + 9;
+  uint64_t* sdp_full = bars + 5;  // per half: S and dP of that half are in TMEM
+  uint64_t* ps_full = bars + 7;   // per half: its warpgroup wrote P / dS into TMEM
+  uint64_t* acc_full = bars + 9;
+  uint64_t* mma_done = bars + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   const int warp = warp_id();
@@ -190,10 +227,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_empty[s], 1);
+      mbar_init(&sdp_full[s], 1);
+      mbar_init(&ps_full[s], 4);  // one arrival per warp of the half's warpgroup
     }
-    mbar_init(s_full, 1);
-    mbar_init(dp_full, 1);
-    mbar_init(ps_full, 128);
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -211,119 +247,107 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Streamed step t: query head and block (dK/dV kernel) or key block (dQ kernel).
   auto step_head = [&](int t) { return KV ? w.kvh * a.group + t / w.per_head : w.h; };
   auto step_blk = [&](int t) { return KV ? w.first + t % w.per_head : t; };
+  // Padded per-row vectors of query block i of head h.
+  auto vec_row = [&](int h, int i) { return (((long long)w.b * a.hq + h) * a.n_qb + i) * BM; };
 
   if (warp == TMA_WARP) {
-    if (w.n_steps > 0) {
-      // ---------------------------------------------------------------- producer (whole warp)
-      // Lane 0 issues the copies. In the dK/dV kernel all lanes first write the
-      // step's per-column LSE and D into shared memory; the stage's full
-      // barrier, which the elementwise warps also wait on, publishes them.
+    if (lane == 0 && w.n_steps > 0) {
+      // ---------------------------------------------------------------- producer
       float* vec = reinterpret_cast<float*>(smem + L::VEC_OFF);
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-        tma_prefetch_desc(&tm_do);
-        mbar_arrive_expect_tx(a_full, 2 * L::TILE);
-        for (int c = 0; c < L::CHUNKS; ++c) {
-          if constexpr (KV) {
-            tma_load_4d(smem + L::A0_OFF + c * (BM * 128), &tm_k, a_full, c * 64, w.blk * BM, w.kvh, w.b);
-            tma_load_4d(smem + L::A1_OFF + c * (BM * 128), &tm_v, a_full, c * 64, w.blk * BM, w.kvh, w.b);
-          } else {
-            tma_load_4d(smem + L::A0_OFF + c * (BM * 128), &tm_q, a_full, c * 64, w.blk * BM, w.h, w.b);
-            tma_load_4d(smem + L::A1_OFF + c * (BM * 128), &tm_do, a_full, c * 64, w.blk * BM, w.h, w.b);
-          }
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(a_full, 2 * L::TILE);
+      for (int c = 0; c < L::CHUNKS; ++c) {
+        if constexpr (KV) {
+          tma_load_4d(smem + L::A0_OFF + c * (BM * 128), &tm_k, a_full, c * 64, w.blk * BM, w.kvh, w.b);
+          tma_load_4d(smem + L::A1_OFF + c * (BM * 128), &tm_v, a_full, c * 64, w.blk * BM, w.kvh, w.b);
+        } else {
+          tma_load_4d(smem + L::A0_OFF + c * (BM * 128), &tm_q, a_full, c * 64, w.blk * BM, w.h, w.b);
+          tma_load_4d(smem + L::A1_OFF + c * (BM * 128), &tm_do, a_full, c * 64, w.blk * BM, w.h, w.b);
         }
       }
       int t = 0;
       for (; t < w.n_steps; ++t) {
         const int s = t & 1;
-        if (t >= 2 && !warp_wait(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag)) break;
+        if (t >= 2 && !mbar_wait_bounded(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag, WAIT_LIMIT)) break;
         const int h = step_head(t), blk = step_blk(t);
+        uint8_t* b0 = smem + L::RING_OFF + (2 * s) * L::TILE;
+        uint8_t* b1 = b0 + L::TILE;
         if constexpr (KV) {
-          // Queries past Sq get LSE = +inf (P = 0) and D = 0.
-          for (int k = lane; k < BM; k += 32) {
-            const int qpos = blk * BM + k;
-            const long long ro = ((long long)w.b * a.hq + h) * a.seqlen_q + qpos;
-            vec[(2 * s) * BM + k] = qpos < a.seqlen_q ? a.lse2[ro] : INFINITY;
-            vec[(2 * s + 1) * BM + k] = qpos < a.seqlen_q ? a.delta[ro] : 0.f;
-          }
-          __threadfence_block();
-        }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE);
-          uint8_t* b0 = smem + L::RING_OFF + (2 * s) * L::TILE;
-          uint8_t* b1 = b0 + L::TILE;
+          // The step's per-column LSE and D ride on the same barrier.
+          mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE + 2 * BM * 4);
+          const long long vr = vec_row(h, blk);
+          bulk_load(vec + (2 * s) * BM, a.lse2 + vr, BM * 4, &ring_full[s]);
+          bulk_load(vec + (2 * s + 1) * BM, a.delta + vr, BM * 4, &ring_full[s]);
           for (int c = 0; c < L::CHUNKS; ++c) {
-            if constexpr (KV) {
-              tma_load_4d(b0 + c * (BM * 128), &tm_q, &ring_full[s], c * 64, blk * BM, h, w.b);
-              tma_load_4d(b1 + c * (BM * 128), &tm_do, &ring_full[s], c * 64, blk * BM, h, w.b);
-            } else {
-              tma_load_4d(b0 + c * (BM * 128), &tm_k, &ring_full[s], c * 64, blk * BM, w.kvh, w.b);
-              tma_load_4d(b1 + c * (BM * 128), &tm_v, &ring_full[s], c * 64, blk * BM, w.kvh, w.b);
-            }
+            tma_load_4d(b0 + c * (BM * 128), &tm_q, &ring_full[s], c * 64, blk * BM, h, w.b);
+            tma_load_4d(b1 + c * (BM * 128), &tm_do, &ring_full[s], c * 64, blk * BM, h, w.b);
+          }
+        } else {
+          mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE);
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_4d(b0 + c * (BM * 128), &tm_k, &ring_full[s], c * 64, blk * BM, w.kvh, w.b);
+            tma_load_4d(b1 + c * (BM * 128), &tm_v, &ring_full[s], c * 64, blk * BM, w.kvh, w.b);
           }
         }
-        __syncwarp();
       }
       // Drain: no copy may be in flight when the CTA exits (abort path).
-      if (lane == 0) {
-        mbar_wait_bounded(a_full, 0, abort_flag, WAIT_LIMIT);
-        for (int u = t - 2 > 0 ? t - 2 : 0; u < t; ++u)
-          mbar_wait_bounded(&ring_full[u & 1], (u >> 1) & 1, abort_flag, WAIT_LIMIT);
-      }
+      mbar_wait_bounded(a_full, 0, abort_flag, WAIT_LIMIT);
+      for (int u = t - 2 > 0 ? t - 2 : 0; u < t; ++u)
+        mbar_wait_bounded(&ring_full[u & 1], (u >> 1) & 1, abort_flag, WAIT_LIMIT);
     }
   } else if (warp == MMA_WARP) {
     if (lane == 0 && w.n_steps > 0) {
       // ---------------------------------------------------------------- MMA issuer
-      constexpr uint32_t ID_S = instr_desc_bf16(BM, BM, 0);   // S-like: both operands K-major
-      constexpr uint32_t ID_ACC = instr_desc_bf16(BM, D, 1);  // accumulate: B MN-major
+      // Per step: S-like products of half 0, then of half 1 (so half 0's
+      // elementwise work overlaps half 1's products), then the accumulating
+      // products of half 0 and of half 1 as their warpgroups finish.
+      constexpr uint32_t ID_S = instr_desc_bf16(BM, 64, 0);   // both operands K-major, N = 64
+      constexpr uint32_t ID_ACC = instr_desc_bf16(BM, D, 1);  // B MN-major
       const uint32_t hi = sw128_desc_hi(1024);
       const uint32_t a0_lo = sw128_desc_lo(smem_addr(smem + L::A0_OFF), 16);
       const uint32_t a1_lo = sw128_desc_lo(smem_addr(smem + L::A1_OFF), 16);
       const uint32_t ring_k = sw128_desc_lo(smem_addr(smem + L::RING_OFF), 16);        // K-major
       const uint32_t ring_mn = sw128_desc_lo(smem_addr(smem + L::RING_OFF), BM * 128);  // MN-major
       const uint32_t id_s = ID_S, id_acc = ID_ACC;
-      // X (cols col) = A (BM x D) * B (BM x D)^T over head_dim.
-      auto issue_s = [&](uint32_t col, uint32_t a_lo, uint32_t b_lo) {
-        static_for<0, D / 16>([&](auto c) {
-          constexpr int kk = decltype(c)::value;
-          constexpr uint32_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
-          mma_ss_lo<off, off>(tmem_base + col, a_lo, b_lo, hi, id_s, kk > 0 ? 1u : 0u);
-        });
-      };
-      // ACC (cols col) += X (bf16 in TMEM at a_col, BM x BM) * B (BM rows = the reduction, D columns).
-      auto issue_acc = [&](uint32_t col, uint32_t a_col, uint32_t b_lo, bool first) {
-        static_for<0, BM / 16>([&](auto c) {
-          constexpr int kk = decltype(c)::value;
-          constexpr uint32_t b_off = (kk * 16 * 128) >> 4;
-          mma_ts_lo<kk * 8, b_off>(tmem_base + col, tmem_base + a_col, b_lo, hi, id_acc,
-                                   (!first || kk > 0) ? 1u : 0u);
-        });
-      };
+      const uint32_t tS = tmem_base + COL_S, tDP = tmem_base + COL_DP, tA = tmem_base + COL_ACC;
       bool ok = mbar_wait_bounded(a_full, 0, abort_flag, WAIT_LIMIT);
       for (int t = 0; t < w.n_steps && ok; ++t) {
         const int s = t & 1;
         ok = mbar_wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, WAIT_LIMIT);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t b0 = (uint32_t)(((2 * s) * L::TILE) >> 4);
-        const uint32_t b1 = (uint32_t)(((2 * s + 1) * L::TILE) >> 4);
-        // The previous step's accumulating MMAs read P / dS over these
+        const uint32_t b0k = ring_k + (uint32_t)(((2 * s) * L::TILE) >> 4);
+        const uint32_t b1k = ring_k + (uint32_t)(((2 * s + 1) * L::TILE) >> 4);
+        const uint32_t b0m = ring_mn + (uint32_t)(((2 * s) * L::TILE) >> 4);
+        const uint32_t b1m = ring_mn + (uint32_t)(((2 * s + 1) * L::TILE) >> 4);
+        // The previous step's accumulating products read P / dS over these
         // columns; MMAs from one thread run in issue order.
-        issue_s(COL_S, a0_lo, ring_k + b0);   // S^T = K Q^T  |  S = Q K^T
-        mma_commit(s_full);
-        issue_s(COL_DP, a1_lo, ring_k + b1);  // dP^T = V dO^T  |  dP = dO V^T
-        mma_commit(dp_full);
-        ok = mbar_wait_bounded(ps_full, t & 1, abort_flag, WAIT_LIMIT);
+        issue_s_half<D, 0>(tS, a0_lo, b0k, hi, id_s);   // S^T = K Q^T  |  S = Q K^T
+        issue_s_half<D, 0>(tDP, a1_lo, b1k, hi, id_s);  // dP^T = V dO^T  |  dP = dO V^T
+        mma_commit(&sdp_full[0]);
+        issue_s_half<D, 1>(tS + 64, a0_lo, b0k, hi, id_s);
+        issue_s_half<D, 1>(tDP + 64, a1_lo, b1k, hi, id_s);
+        mma_commit(&sdp_full[1]);
+        ok = mbar_wait_bounded(&ps_full[0], t & 1, abort_flag, WAIT_LIMIT);
         if (!ok) break;
         tc_fence_after();
         if constexpr (KV) {
-          issue_acc(COL_ACC, COL_S, ring_mn + b1, t == 0);       // dV += P^T dO
-          issue_acc(COL_ACC + D, COL_DP, ring_mn + b0, t == 0);  // dK += dS^T Q
+          issue_acc_half<0>(tA, tS, b1m, hi, id_acc, t == 0);       // dV += P^T dO
+          issue_acc_half<0>(tA + D, tDP, b0m, hi, id_acc, t == 0);  // dK += dS^T Q
         } else {
-          issue_acc(COL_ACC, COL_DP, ring_mn + b0, t == 0);  // dQ += dS K
+          issue_acc_half<0>(tA, tDP, b0m, hi, id_acc, t == 0);  // dQ += dS K
+        }
+        ok = mbar_wait_bounded(&ps_full[1], t & 1, abort_flag, WAIT_LIMIT);
+        if (!ok) break;
+        tc_fence_after();
+        if constexpr (KV) {
+          issue_acc_half<1>(tA, tS, b1m, hi, id_acc, t == 0);
+          issue_acc_half<1>(tA + D, tDP, b0m, hi, id_acc, t == 0);
+        } else {
+          issue_acc_half<1>(tA, tDP, b0m, hi, id_acc, t == 0);
         }
         mma_commit(&ring_empty[s]);
       }
@@ -334,36 +358,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------------ elementwise + epilogue
-    const int r = warp * 32 + lane;  // the resident tile's row == TMEM lane
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    const int wq = warp & 3;
+    const int half = warp >> 2;      // this warpgroup's 64 columns
+    const int r = wq * 32 + lane;    // the resident tile's row == TMEM lane
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
     const int off = a.seqlen_k - a.seqlen_q;
     const float sl2 = a.scale_log2;
-    float* vec = reinterpret_cast<float*>(smem + L::VEC_OFF);
-    // dQ kernel: this row's LSE and D.
+    const float* vec = reinterpret_cast<const float*>(smem + L::VEC_OFF);
     const int row_pos = w.blk * BM + r;  // key position (dK/dV) or query position (dQ)
     float lse_r = INFINITY, delta_r = 0.f;
     if constexpr (!KV) {
-      if (row_pos < a.seqlen_q) {
-        const long long ro = ((long long)w.b * a.hq + w.h) * a.seqlen_q + row_pos;
-        lse_r = a.lse2[ro];
-        delta_r = a.delta[ro];
-      }
+      const long long vr = vec_row(w.h, w.blk) + r;  // padded: +inf / 0 past Sq
+      lse_r = a.lse2[vr];
+      delta_r = a.delta[vr];
     }
     bool ok = true;
     for (int t = 0; t < w.n_steps && ok; ++t) {
       const int s = t & 1;
       const int blk = step_blk(t);
-      // Columns c < c_lim are visible.
+      // KV: columns c >= c_lim are visible (query blk BM + c sits at position
+      // blk BM + c + off and sees this key when row_pos <= that). Q: columns
+      // c < c_lim are visible (key blk BM + c, below Sk and, causal, at most
+      // row_pos + off).
       int c_lim;
       if constexpr (KV) {
-        // Column c = query i BM + c, at position i BM + c + off; this key row
-        // is visible to it when row_pos <= i BM + c + off. The producer wrote
-        // the step's per-column LSE and D before the stage's full barrier.
-        c_lim = row_pos < a.seqlen_k ? (a.causal ? row_pos - off - blk * BM : -BM) : BM;  // first visible column
+        c_lim = row_pos < a.seqlen_k ? (a.causal ? row_pos - off - blk * BM : -BM) : BM;
+        // The producer's LSE / D copies complete on the stage's full barrier.
         ok = warp_wait(&ring_full[s], (t >> 1) & 1, abort_flag);
         if (!ok) break;
       } else {
-        // Column c = key blk BM + c; visible when < Sk and (causal) <= row_pos + off.
         int lim = a.seqlen_k - blk * BM;
         if (a.causal) {
           const int cl = row_pos + off - blk * BM + 1;
@@ -373,50 +396,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const float* lse_c = vec + (2 * s) * BM;
       const float* delta_c = vec + (2 * s + 1) * BM;
-      ok = warp_wait(s_full, t & 1, abort_flag);
+      ok = warp_wait(&sdp_full[half], t & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int cc = 0; cc < BM / 32; ++cc) {
-        uint32_t sv[32];
-        tmem_ld32(lane_base + COL_S + cc * 32, sv);
-        tmem_ld_wait();
-        float p[32];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int c = cc * 32 + jj;
-          const float lse = KV ? lse_c[c] : lse_r;
-          const bool vis = KV ? (c >= c_lim) : (c < c_lim);
-          p[jj] = vis ? ex2_approx(fmaf(__uint_as_float(sv[jj]), sl2, -lse)) : 0.f;
-        }
-        if (cc == 0) {
-          ok = warp_wait(dp_full, t & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        uint32_t dv[32];
-        tmem_ld32(lane_base + COL_DP + cc * 32, dv);
+      for (int cc = 0; cc < 2; ++cc) {
+        const int col = half * 64 + cc * 32;
+        uint32_t sv[32], dv[32];
+        tmem_ld32(lane_base + COL_S + col, sv);
+        tmem_ld32(lane_base + COL_DP + col, dv);
         tmem_ld_wait();
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 2) {
-          const float d0 = KV ? delta_c[cc * 32 + jj] : delta_r;
-          const float d1 = KV ? delta_c[cc * 32 + jj + 1] : delta_r;
-          const float ds0 = p[jj] * (__uint_as_float(dv[jj]) - d0);
-          const float ds1 = p[jj + 1] * (__uint_as_float(dv[jj + 1]) - d1);
-          pk[jj / 2] = pack_bf16x2(p[jj], p[jj + 1]);
-          dk[jj / 2] = pack_bf16x2(ds0, ds1);
+        for (int j4 = 0; j4 < 32; j4 += 4) {
+          float l4[4], d4[4];
+          if constexpr (KV) {
+            const float4 lv = *reinterpret_cast<const float4*>(lse_c + col + j4);
+            const float4 dv4 = *reinterpret_cast<const float4*>(delta_c + col + j4);
+            l4[0] = lv.x, l4[1] = lv.y, l4[2] = lv.z, l4[3] = lv.w;
+            d4[0] = dv4.x, d4[1] = dv4.y, d4[2] = dv4.z, d4[3] = dv4.w;
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) l4[u] = lse_r, d4[u] = delta_r;
+          }
+          float p[4], ds[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = col + j4 + u;
+            const bool vis = KV ? (c >= c_lim) : (c < c_lim);
+            p[u] = vis ? ex2_approx(fmaf(__uint_as_float(sv[j4 + u]), sl2, -l4[u])) : 0.f;
+            ds[u] = p[u] * (__uint_as_float(dv[j4 + u]) - d4[u]);
+          }
+          pk[j4 / 2] = pack_bf16x2(p[0], p[1]);
+          pk[j4 / 2 + 1] = pack_bf16x2(p[2], p[3]);
+          dk[j4 / 2] = pack_bf16x2(ds[0], ds[1]);
+          dk[j4 / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        // bf16 pairs over the columns already read (chunk cc covers 16 cols).
-        if constexpr (KV) tmem_st16(lane_base + COL_S + cc * 16, pk);
-        tmem_st16(lane_base + COL_DP + cc * 16, dk);
+        // bf16 pairs over this half's first 32 columns, all read already.
+        if constexpr (KV) tmem_st16(lane_base + COL_S + half * 64 + cc * 16, pk);
+        tmem_st16(lane_base + COL_DP + half * 64 + cc * 16, dk);
       }
-      if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ps_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ps_full[half]);
     }
-    // ---- epilogue: this row of the accumulators, scaled where needed
+    // ---- epilogue: each warpgroup stores half of the columns of its rows
     const bool row_ok = row_pos < (KV ? a.seqlen_k : a.seqlen_q);
     if (ok && w.n_steps > 0) ok = warp_wait(acc_full, 0, abort_flag);
     if (ok) {
@@ -432,7 +457,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                : (long long)w.b * a.dq_bs + (long long)w.h * a.dq_hs + (long long)row_pos * a.dq_rs;
         const float mul = is_dv ? 1.f : a.scale;
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int cc = half * (D / 64); cc < (half + 1) * (D / 64); ++cc) {
           float x[32];
           if (w.n_steps > 0) {
             uint32_t v[32];
@@ -459,34 +484,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// D = rowsum(dO * O) and LSE * log2(e) per query row (one warp per row).
+// Per query row, padded to whole 128-row blocks: D = rowsum(dO * O) and
+// LSE * log2(e) (+inf for rows that see no key and for padding rows, whose D
+// is 0). One warp per row, vector loads.
 template <int D>
 __global__ void __launch_bounds__(256)
     bwd_prep_kernel(const void* o, int o_f32, long long o_bs, long long o_hs, long long o_rs,
-                    const __nv_bfloat16* dout, long long do_bs, long long do_hs, long long do_rs,
-                    const float* lse, int batch, int hq, int seqlen_q, float* lse2, float* delta) {
-  constexpr int PER = D / 32;
+                    const __nv_bfloat16* dout, long long do_bs, long long do_hs, long long do_rs, const float* lse,
+                    int batch, int hq, int seqlen_q, int n_qb, float* lse2, float* delta) {
+  constexpr int PER = D / 32;  // 4 (head_dim 128) or 2 (64)
+  const long long padded = (long long)n_qb * 128;
   const long long row = (long long)blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
-  if (row >= (long long)batch * hq * seqlen_q) return;
-  const int q = (int)(row % seqlen_q);
-  const long long bh = row / seqlen_q;
+  if (row >= (long long)batch * hq * padded) return;
+  const int q = (int)(row % padded);
+  const long long bh = row / padded;
+  if (q >= seqlen_q) {
+    if (lane == 0) {
+      lse2[row] = INFINITY;
+      delta[row] = 0.f;
+    }
+    return;
+  }
   const int h = (int)(bh % hq), b = (int)(bh / hq);
   const __nv_bfloat16* dr = dout + b * do_bs + h * do_hs + q * do_rs + lane * PER;
-  float acc = 0.f;
+  float dov[PER], ov[PER];
+  if constexpr (PER == 4) {
+    const uint2 x = *reinterpret_cast<const uint2*>(dr);
+    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
+    const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
+    dov[0] = a0.x, dov[1] = a0.y, dov[2] = a1.x, dov[3] = a1.y;
+  } else {
+    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dr));
+    dov[0] = a0.x, dov[1] = a0.y;
+  }
   if (o_f32) {
     const float* orow = reinterpret_cast<const float*>(o) + b * o_bs + h * o_hs + q * o_rs + lane * PER;
-#pragma unroll
-    for (int k = 0; k < PER; ++k) acc = fmaf(__bfloat162float(dr[k]), orow[k], acc);
+    if constexpr (PER == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(orow);
+      ov[0] = x.x, ov[1] = x.y, ov[2] = x.z, ov[3] = x.w;
+    } else {
+      const float2 x = *reinterpret_cast<const float2*>(orow);
+      ov[0] = x.x, ov[1] = x.y;
+    }
   } else {
-    const __nv_bfloat16* orow = reinterpret_cast<const __nv_bfloat16*>(o) + b * o_bs + h * o_hs + q * o_rs + lane * PER;
-#pragma unroll
-    for (int k = 0; k < PER; ++k) acc = fmaf(__bfloat162float(dr[k]), __bfloat162float(orow[k]), acc);
+    const __nv_bfloat16* orow =
+        reinterpret_cast<const __nv_bfloat16*>(o) + b * o_bs + h * o_hs + q * o_rs + lane * PER;
+    if constexpr (PER == 4) {
+      const uint2 x = *reinterpret_cast<const uint2*>(orow);
+      const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
+      const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
+      ov[0] = a0.x, ov[1] = a0.y, ov[2] = a1.x, ov[3] = a1.y;
+    } else {
+      const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(orow));
+      ov[0] = a0.x, ov[1] = a0.y;
+    }
   }
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) acc = fmaf(dov[k], ov[k], acc);
 #pragma unroll
   for (int sh = 16; sh >= 1; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
   if (lane == 0) {
-    const float l = lse[row];
+    const float l = lse[bh * seqlen_q + q];
     lse2[row] = l == -INFINITY ? INFINITY : l * LOG2E;
     delta[row] = acc;
   }
@@ -528,8 +588,13 @@ static bool bwd_map(CUtensorMap* map, const void* base, int D, int rows, int hea
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Two fp32 values per query row, rows padded to whole 128-row blocks.
+static size_t padded_rows(const attn_backward_params& p) {
+  return (size_t)p.batch * p.num_q_heads * ((p.seqlen_q + bwd::BM - 1) / bwd::BM) * bwd::BM;
+}
+
 size_t backward_workspace_bytes(const attn_backward_params& p) {
-  const size_t n = (size_t)p.batch * p.num_q_heads * p.seqlen_q * sizeof(float);
+  const size_t n = padded_rows(p) * sizeof(float);
   return 2 * ((n + 255) / 256 * 256);
 }
 
@@ -554,7 +619,8 @@ static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, co
 attn_status_t launch_backward(const attn_backward_params& p, void* workspace, cudaStream_t stream) {
   if (p.batch == 0 || p.num_q_heads == 0 || (p.seqlen_q == 0 && p.seqlen_k == 0)) return ATTN_OK;
   const int D = p.head_dim;
-  const size_t n = (size_t)p.batch * p.num_q_heads * p.seqlen_q;
+  const size_t n = padded_rows(p);
+  const int n_qb = (p.seqlen_q + bwd::BM - 1) / bwd::BM;
   float* lse2 = reinterpret_cast<float*>(workspace);
   float* delta = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + (n * 4 + 255) / 256 * 256);
   const bool o_f32 = p.o_dtype == ATTN_DTYPE_F32;
@@ -565,12 +631,12 @@ attn_status_t launch_backward(const attn_backward_params& p, void* workspace, cu
       bwd::bwd_prep_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
           p.o, o_f32, p.o_batch_stride, p.o_head_stride, p.o_row_stride,
           reinterpret_cast<const __nv_bfloat16*>(p.dout), p.do_batch_stride, p.do_head_stride, p.do_row_stride, p.lse,
-          p.batch, p.num_q_heads, p.seqlen_q, lse2, delta);
+          p.batch, p.num_q_heads, p.seqlen_q, n_qb, lse2, delta);
     else
       bwd::bwd_prep_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
           p.o, o_f32, p.o_batch_stride, p.o_head_stride, p.o_row_stride,
           reinterpret_cast<const __nv_bfloat16*>(p.dout), p.do_batch_stride, p.do_head_stride, p.do_row_stride, p.lse,
-          p.batch, p.num_q_heads, p.seqlen_q, lse2, delta);
+          p.batch, p.num_q_heads, p.seqlen_q, n_qb, lse2, delta);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   // Tensor maps need at least one row; an empty side is never loaded.

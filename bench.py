@@ -232,6 +232,8 @@ def run_ours(args, rank, world, local):
         result["prefill_16k"] = bench_prefill_16k(args, rank, world, local, attn, peaks, peak_src)
     if args.only in (None, "sharedprefix"):
         result["shared_prefix"] = bench_shared_prefix(args, rank, world, local, attn, peaks, peak_src)
+    if args.only in (None, "backward"):
+        result["backward"] = bench_backward(args, rank, world, local, attn, peaks, peak_src)
     if args.only is not None:
         result["partial"] = f"--only {args.only}: profiling run, not a bench line"
     if rank == 0 and args.only is None:
@@ -432,6 +434,36 @@ def bench_shared_prefix(args, rank, world, local, attn, peaks, peak_src):
             "gpu_launches_per_step": 4 + (1 if max_splits > 1 else 0), "clocks": clk.summary()}
 
 
+def bench_backward(args, rank, world, local, attn, peaks, peak_src):
+    """Backward of the causal GQA prefill workload (4 x 32/8 heads x 2048 x 128):
+    dQ, dK, dV from the library's own forward O (bf16) and LSE, bf16 gradients."""
+    import torch
+    cfg, d, fwd_flops = prefill_inputs(rank)
+    q, k, v = _dev_bf16(d["q"]), _dev_bf16(d["k"]), _dev_bf16(d["v"])
+    do = _dev_bf16(wl.normal_bf16(cfg.seed + 1000 * rank, q.shape, 43))
+    o, lse = attn.prefill(q, k, v, cfg.scale, cfg.causal)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(2 * cfg.batch * cfg.q_heads * (-(-cfg.seqlen_q // 128) * 128) * 4 + 512, dtype=torch.uint8,
+                     device="cuda")
+
+    def step():
+        attn.prefill_backward(q, k, v, o, lse, do, cfg.scale, cfg.causal, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    steps = max(5, min(args.steps, 20))
+    with ClockSampler(local) as clk:
+        ms = time_loop(step, steps, args.warmup, world)
+    flops = 2.5 * fwd_flops  # five products per visible pair (S, dP, dV, dK, dQ) against the forward's two
+    tf = flops / (ms * 1e-3) / 1e12
+    peak_t = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    return {"workload": cfg.name + "_backward", "value": round(tf * world, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "steps": steps,
+            "roofline": {"bound": "tensor", "kernel": "whole call (prep + dK/dV + dQ)", "achieved": round(tf, 2),
+                         "peak": peak_t, "unit": "TFLOP/s", "frac": round(tf / peak_t, 4),
+                         "peak_source": f"{peak_src} bf16 GEMM", "algorithmic_flops_per_launch": flops,
+                         "executed_flops_per_launch": 3.5 * fwd_flops},
+            "gpu_launches_per_step": 3, "clocks": clk.summary()}
+
+
 def bench_prefill_16k(args, rank, world, local, attn, peaks, peak_src):
     """Long-context causal GQA prefill: batch 1, 32/8 heads, 16384 tokens, head_dim 128."""
     import dataclasses
@@ -578,7 +610,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--only", choices=["prefill", "decode", "decodefp8", "mixed", "prefill16k", "sharedprefix"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decodefp8", "mixed", "prefill16k", "sharedprefix", "backward"], default=None,
                     help="profiling aid: run one workload only (the line is then marked partial)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="profiling aid: fewer decode sequences (default: the full 64)")

@@ -230,7 +230,8 @@ ATTN_API attn_status_t attn_decode_paged(const attn_decode_params* p, void* work
  * (rows that see no key get 0). Deterministic: no atomics.
  *
  * Workspace: at least *workspace_needed bytes of device memory, 256-byte
- * aligned (two fp32 values per query row). workspace = NULL only queries the
+ * aligned (two fp32 values per query row, rows padded to a multiple of 128
+ * per head). workspace = NULL only queries the
  * size (returns ATTN_OK, enqueues nothing); a smaller workspace returns
  * ATTN_ERR_WORKSPACE and enqueues nothing. Asynchronous on `stream`.
  */

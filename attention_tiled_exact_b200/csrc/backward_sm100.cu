@@ -55,6 +55,7 @@ constexpr int EW_WARPS = 8;          // two elementwise warpgroups, one per 64-c
 constexpr int TMA_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int NUM_THREADS = 320;
+static_assert(TMA_WARP == EW_WARPS && MMA_WARP == EW_WARPS + 1 && NUM_THREADS == (EW_WARPS + 2) * 32, "warp roles");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_LIMIT = 2000000000LL;  // cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
@@ -313,43 +314,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t ring_mn = sw128_desc_lo(smem_addr(smem + L::RING_OFF), BM * 128);  // MN-major
       const uint32_t id_s = ID_S, id_acc = ID_ACC;
       const uint32_t tS = tmem_base + COL_S, tDP = tmem_base + COL_DP, tA = tmem_base + COL_ACC;
+      // Stage addresses of step t's streamed tiles (K-major and MN-major views).
+      auto b_k = [&](int t, int which) { return ring_k + (uint32_t)(((2 * (t & 1) + which) * L::TILE) >> 4); };
+      auto b_m = [&](int t, int which) { return ring_mn + (uint32_t)(((2 * (t & 1) + which) * L::TILE) >> 4); };
+      // S-like products of one half of step t (S^T = K Q^T, dP^T = V dO^T, or
+      // S = Q K^T, dP = dO V^T), then its barrier.
+      auto s_half = [&](int t, int half) {
+        if (half == 0) {
+          issue_s_half<D, 0>(tS, a0_lo, b_k(t, 0), hi, id_s);
+          issue_s_half<D, 0>(tDP, a1_lo, b_k(t, 1), hi, id_s);
+        } else {
+          issue_s_half<D, 1>(tS + 64, a0_lo, b_k(t, 0), hi, id_s);
+          issue_s_half<D, 1>(tDP + 64, a1_lo, b_k(t, 1), hi, id_s);
+        }
+        mma_commit(&sdp_full[half]);
+      };
+      // Accumulating products of one half of step t, once its warpgroup has
+      // written P / dS.
+      auto acc_half = [&](int t, int half) {
+        if (half == 0) {
+          if constexpr (KV) {
+            issue_acc_half<0>(tA, tS, b_m(t, 1), hi, id_acc, t == 0);       // dV += P^T dO
+            issue_acc_half<0>(tA + D, tDP, b_m(t, 0), hi, id_acc, t == 0);  // dK += dS^T Q
+          } else {
+            issue_acc_half<0>(tA, tDP, b_m(t, 0), hi, id_acc, t == 0);  // dQ += dS K
+          }
+        } else {
+          if constexpr (KV) {
+            issue_acc_half<1>(tA, tS, b_m(t, 1), hi, id_acc, t == 0);
+            issue_acc_half<1>(tA + D, tDP, b_m(t, 0), hi, id_acc, t == 0);
+          } else {
+            issue_acc_half<1>(tA, tDP, b_m(t, 0), hi, id_acc, t == 0);
+          }
+        }
+      };
+      // Ping-pong over the two halves: half h's products of step t + 1 are
+      // issued right after its accumulating products of step t (they reuse its
+      // TMEM columns; MMAs from one thread run in issue order), so while one
+      // warpgroup works the tensor core runs the other half's products.
       bool ok = mbar_wait_bounded(a_full, 0, abort_flag, WAIT_LIMIT);
-      for (int t = 0; t < w.n_steps && ok; ++t) {
-        const int s = t & 1;
-        ok = mbar_wait_bounded(&ring_full[s], (t >> 1) & 1, abort_flag, WAIT_LIMIT);
-        if (!ok) break;
+      if (ok) ok = mbar_wait_bounded(&ring_full[0], 0, abort_flag, WAIT_LIMIT);
+      if (ok) {
         tc_fence_after();
-        const uint32_t b0k = ring_k + (uint32_t)(((2 * s) * L::TILE) >> 4);
-        const uint32_t b1k = ring_k + (uint32_t)(((2 * s + 1) * L::TILE) >> 4);
-        const uint32_t b0m = ring_mn + (uint32_t)(((2 * s) * L::TILE) >> 4);
-        const uint32_t b1m = ring_mn + (uint32_t)(((2 * s + 1) * L::TILE) >> 4);
-        // The previous step's accumulating products read P / dS over these
-        // columns; MMAs from one thread run in issue order.
-        issue_s_half<D, 0>(tS, a0_lo, b0k, hi, id_s);   // S^T = K Q^T  |  S = Q K^T
-        issue_s_half<D, 0>(tDP, a1_lo, b1k, hi, id_s);  // dP^T = V dO^T  |  dP = dO V^T
-        mma_commit(&sdp_full[0]);
-        issue_s_half<D, 1>(tS + 64, a0_lo, b0k, hi, id_s);
-        issue_s_half<D, 1>(tDP + 64, a1_lo, b1k, hi, id_s);
-        mma_commit(&sdp_full[1]);
+        s_half(0, 0);
+        s_half(0, 1);
+      }
+      for (int t = 0; t < w.n_steps && ok; ++t) {
+        const bool next = t + 1 < w.n_steps;
         ok = mbar_wait_bounded(&ps_full[0], t & 1, abort_flag, WAIT_LIMIT);
         if (!ok) break;
         tc_fence_after();
-        if constexpr (KV) {
-          issue_acc_half<0>(tA, tS, b1m, hi, id_acc, t == 0);       // dV += P^T dO
-          issue_acc_half<0>(tA + D, tDP, b0m, hi, id_acc, t == 0);  // dK += dS^T Q
-        } else {
-          issue_acc_half<0>(tA, tDP, b0m, hi, id_acc, t == 0);  // dQ += dS K
+        acc_half(t, 0);
+        if (next) {
+          ok = mbar_wait_bounded(&ring_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag, WAIT_LIMIT);
+          if (!ok) break;
+          tc_fence_after();
+          s_half(t + 1, 0);
         }
         ok = mbar_wait_bounded(&ps_full[1], t & 1, abort_flag, WAIT_LIMIT);
         if (!ok) break;
         tc_fence_after();
-        if constexpr (KV) {
-          issue_acc_half<1>(tA, tS, b1m, hi, id_acc, t == 0);
-          issue_acc_half<1>(tA + D, tDP, b0m, hi, id_acc, t == 0);
-        } else {
-          issue_acc_half<1>(tA, tDP, b0m, hi, id_acc, t == 0);
-        }
-        mma_commit(&ring_empty[s]);
+        acc_half(t, 1);
+        mma_commit(&ring_empty[t & 1]);  // step t's tiles are free once these have run
+        if (next) s_half(t + 1, 1);
       }
       if (ok) mma_commit(acc_full);
       // Every MMA must have completed before tensor memory is released.

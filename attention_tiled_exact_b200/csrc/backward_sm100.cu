@@ -12,8 +12,9 @@
 // forward's LSE, exactly as the forward builds S tile by tile.
 //
 // Three launches:
-//   * prep (one warp per query row): D = rowsum(dO * O), and LSE * log2(e)
-//     (+inf for rows that see no key, so that their P is exactly 0);
+//   * prep (one warp per query row): -D = -rowsum(dO * O) and -LSE log2(e)
+//     (-inf for rows that see no key, so that their P is exactly 0), padded
+//     to whole 128-row blocks;
 //   * dK/dV kernel, one CTA per (batch, kv head, 128-key block j): K_j and V_j
 //     stay in shared memory; for every query head of the group and every
 //     query block i that sees block j, TMA streams Q_i and dO_i through a
@@ -64,9 +65,11 @@ struct Args {
   int batch, hq, hkv, group, seqlen_q, seqlen_k, n_qb, n_kb;
   int causal;
   float scale, scale_log2;
-  // Per query row, padded to whole 128-row blocks: [B, Hq, n_qb * 128].
-  const float* lse2;   // LSE * log2(e); +inf where the row sees no key and past Sq
-  const float* delta;  // rowsum(dO * O); 0 past Sq
+  // Per query row, padded to whole 128-row blocks: [B, Hq, n_qb * 128],
+  // both negated so that the elementwise step is one packed FMA and one
+  // packed add per pair.
+  const float* lse2;   // -LSE * log2(e); -inf where the row sees no key and past Sq
+  const float* delta;  // -rowsum(dO * O); 0 past Sq
   void* dq;
   void* dk;
   void* dv;
@@ -393,12 +396,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float sl2 = a.scale_log2;
     const float* vec = reinterpret_cast<const float*>(smem + L::VEC_OFF);
     const int row_pos = w.blk * BM + r;  // key position (dK/dV) or query position (dQ)
-    float lse_r = INFINITY, delta_r = 0.f;
+    float nlse_r = -INFINITY, ndelta_r = 0.f;
     if constexpr (!KV) {
-      const long long vr = vec_row(w.h, w.blk) + r;  // padded: +inf / 0 past Sq
-      lse_r = a.lse2[vr];
-      delta_r = a.delta[vr];
+      const long long vr = vec_row(w.h, w.blk) + r;  // padded: -inf / 0 past Sq
+      nlse_r = a.lse2[vr];
+      ndelta_r = a.delta[vr];
     }
+    const float2 sl2x2 = make_float2(sl2, sl2);
     bool ok = true;
     for (int t = 0; t < w.n_steps && ok; ++t) {
       const int s = t & 1;
@@ -426,6 +430,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ok = warp_wait(&sdp_full[half], t & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
+      // The whole half is visible on all but the diagonal and ragged tiles:
+      // no per-element mask there.
+      const bool all_vis = KV ? (c_lim <= half * 64) : (c_lim >= half * 64 + 64);
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const int col = half * 64 + cc * 32;
@@ -436,28 +443,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int j4 = 0; j4 < 32; j4 += 4) {
-          float l4[4], d4[4];
+          float2 nl[2], nd[2];
           if constexpr (KV) {
             const float4 lv = *reinterpret_cast<const float4*>(lse_c + col + j4);
             const float4 dv4 = *reinterpret_cast<const float4*>(delta_c + col + j4);
-            l4[0] = lv.x, l4[1] = lv.y, l4[2] = lv.z, l4[3] = lv.w;
-            d4[0] = dv4.x, d4[1] = dv4.y, d4[2] = dv4.z, d4[3] = dv4.w;
+            nl[0] = make_float2(lv.x, lv.y), nl[1] = make_float2(lv.z, lv.w);
+            nd[0] = make_float2(dv4.x, dv4.y), nd[1] = make_float2(dv4.z, dv4.w);
           } else {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) l4[u] = lse_r, d4[u] = delta_r;
+            nl[0] = nl[1] = make_float2(nlse_r, nlse_r);
+            nd[0] = nd[1] = make_float2(ndelta_r, ndelta_r);
           }
-          float p[4], ds[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = col + j4 + u;
-            const bool vis = KV ? (c >= c_lim) : (c < c_lim);
-            p[u] = vis ? ex2_approx(fmaf(__uint_as_float(sv[j4 + u]), sl2, -l4[u])) : 0.f;
-            ds[u] = p[u] * (__uint_as_float(dv[j4 + u]) - d4[u]);
+          for (int u = 0; u < 2; ++u) {
+            const int j = j4 + 2 * u;
+            // P = 2^(S scale log2 e - LSE log2 e); dS = P (dP - D).
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nl[u]);
+            float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (!all_vis) {
+              const int c = col + j;
+              const bool v0 = KV ? (c >= c_lim) : (c < c_lim);
+              const bool v1 = KV ? (c + 1 >= c_lim) : (c + 1 < c_lim);
+              p.x = v0 ? p.x : 0.f;
+              p.y = v1 ? p.y : 0.f;
+            }
+            const float2 ds =
+                __fmul2_rn(p, __fadd2_rn(make_float2(__uint_as_float(dv[j]), __uint_as_float(dv[j + 1])), nd[u]));
+            pk[j / 2] = pack_bf16x2(p.x, p.y);
+            dk[j / 2] = pack_bf16x2(ds.x, ds.y);
           }
-          pk[j4 / 2] = pack_bf16x2(p[0], p[1]);
-          pk[j4 / 2 + 1] = pack_bf16x2(p[2], p[3]);
-          dk[j4 / 2] = pack_bf16x2(ds[0], ds[1]);
-          dk[j4 / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
         // bf16 pairs over this half's first 32 columns, all read already.
         if constexpr (KV) tmem_st16(lane_base + COL_S + half * 64 + cc * 16, pk);
@@ -511,8 +524,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// Per query row, padded to whole 128-row blocks: D = rowsum(dO * O) and
-// LSE * log2(e) (+inf for rows that see no key and for padding rows, whose D
+// Per query row, padded to whole 128-row blocks: -D = -rowsum(dO * O) and
+// -LSE * log2(e) (-inf for rows that see no key and for padding rows, whose D
 // is 0). One warp per row, vector loads.
 template <int D>
 __global__ void __launch_bounds__(256)
@@ -528,7 +541,7 @@ __global__ void __launch_bounds__(256)
   const long long bh = row / padded;
   if (q >= seqlen_q) {
     if (lane == 0) {
-      lse2[row] = INFINITY;
+      lse2[row] = -INFINITY;
       delta[row] = 0.f;
     }
     return;
@@ -574,8 +587,8 @@ __global__ void __launch_bounds__(256)
   for (int sh = 16; sh >= 1; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
   if (lane == 0) {
     const float l = lse[bh * seqlen_q + q];
-    lse2[row] = l == -INFINITY ? INFINITY : l * LOG2E;
-    delta[row] = acc;
+    lse2[row] = l == -INFINITY ? -INFINITY : -l * LOG2E;
+    delta[row] = -acc;
   }
 }
 

@@ -50,6 +50,12 @@ Pins: torch autograd in fp64 through a softmax written with torch ops,
 central finite differences, closed forms (one key; zero queries) and GQA vs
 MHA with repeated K/V.
 
+Block-sparse attention (BSR: query blocks see listed key blocks, the
+FlashInfer abstraction, "抱infra脚", FlashInfer) is the same definition with
+S = -inf outside the listed blocks. Pins: every block listed equals dense
+attention, and each query block equals dense attention over its gathered
+key blocks.
+
 Pins (tests/test_oracle.py): brute-force ``math.fsum`` loops on tiny inputs,
 closed forms (one key, causal row 0, zero query, constant V, hand-derived
 weights), torch's fp64 CPU ``scaled_dot_product_attention`` with repeated
@@ -212,6 +218,42 @@ def ref_attention_backward(q, k, v, do, scale, causal):
             dq[b, h] = scale * (dS @ k[b, kvh])
             dk[b, kvh] += scale * (dS.T @ q[b, h])
     return dict(dq=dq, dk=dk, dv=dv, o=o, lse=lse, delta=delta)
+
+
+def ref_block_sparse_attention(q, k, v, indptr, indices, row_block, col_block, scale):
+    """Attention with a block-sparse mask in BSR form, for one sequence.
+
+    q [Hq, Sq, D]; k, v [Hkv, Sk, D]. Query rows are grouped in blocks of
+    ``row_block`` rows and keys in blocks of ``col_block`` keys; query block r
+    sees exactly the key blocks ``indices[indptr[r]:indptr[r + 1]]`` (every
+    key of those blocks below Sk) and no other key. The block-sparse format
+    is the FlashInfer unified abstraction ("抱infra脚", FlashInfer). Written
+    out as the dense definition with S = -inf outside the mask. Returns
+    O [Hq, Sq, D] and LSE [Hq, Sq] (a row with no visible key: 0 and -inf).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[0], k.shape[1]
+    G = Hq // Hkv
+    visible = np.zeros((Sq, Sk), dtype=bool)
+    for i in range(Sq):
+        r = i // row_block
+        for c in indices[indptr[r]:indptr[r + 1]]:
+            visible[i, c * col_block:min((c + 1) * col_block, Sk)] = True
+    O = np.zeros((Hq, Sq, D))
+    L = np.full((Hq, Sq), -np.inf)
+    for h in range(Hq):
+        s = scale * (q[h] @ k[h // G].T)
+        s = np.where(visible, s, -np.inf)
+        for i in range(Sq):
+            if not visible[i].any():
+                continue
+            m = s[i].max()
+            p = np.exp(s[i] - m)
+            l = p.sum()
+            O[h, i] = (p @ v[h // G]) / l
+            L[h, i] = m + np.log(l)
+    return O, L
 
 
 def gather_paged(pool, block_table_row, length: int, kv_head: int) -> np.ndarray:

@@ -511,3 +511,40 @@ def test_backward_pins_reject_planted_mistakes(mutant):
     assert all(np.allclose(a, b, atol=1e-12) for a, b in zip(good, want))
     bad = _candidate_backward(q, k, v, do, 0.5, True, mutant)
     assert not all(np.allclose(a, b, atol=1e-6) for a, b in zip(bad, want))
+
+
+# ----------------------------------------------------------------------------
+# block-sparse (BSR) attention
+# ----------------------------------------------------------------------------
+
+
+def test_block_sparse_with_every_block_is_dense():
+    rng = np.random.default_rng(450)
+    q, k, v = _rand(rng, 4, 37, 8), _rand(rng, 2, 50, 8), _rand(rng, 2, 50, 8)
+    n_rb, n_cb = 5, 4  # row blocks of 8, column blocks of 16 (the last one ragged)
+    indptr = np.arange(n_rb + 1) * n_cb
+    indices = np.tile(np.arange(n_cb)[::-1], n_rb)  # every block, in reverse order
+    O, L = ref.ref_block_sparse_attention(q, k, v, indptr, indices, 8, 16, 0.3)
+    Od, Ld = ref.ref_attention(q[None], k[None], v[None], 0.3, False)
+    assert np.abs(O - Od[0]).max() < 1e-12 and np.abs(L - Ld[0]).max() < 1e-12
+
+
+def test_block_sparse_is_dense_attention_over_the_gathered_blocks():
+    """Each query block against the concatenation of its listed key blocks,
+    through the brute-force fsum definition (a different computation)."""
+    rng = np.random.default_rng(451)
+    q, k, v = _rand(rng, 2, 10, 4), _rand(rng, 1, 40, 4), _rand(rng, 1, 40, 4)
+    indptr = np.array([0, 2, 2, 5])  # row block 1 sees nothing
+    indices = np.array([2, 0, 1, 2, 0])
+    O, L = ref.ref_block_sparse_attention(q, k, v, indptr, indices, 4, 16, 0.5)
+    for r in range(3):
+        rows = slice(4 * r, min(4 * r + 4, 10))
+        cols = indices[indptr[r]:indptr[r + 1]]
+        if len(cols) == 0:
+            assert (O[:, rows] == 0).all() and np.isneginf(L[:, rows]).all()
+            continue
+        keys = np.concatenate([np.arange(c * 16, min(c * 16 + 16, 40)) for c in cols])
+        Ob, Lb = oracle.brute_attention(_nested(q[None, :, rows]), _nested(k[None][:, :, keys]),
+                                        _nested(v[None][:, :, keys]), 0.5, False)
+        assert np.abs(O[:, rows] - np.asarray(Ob)[0]).max() < 1e-12
+        assert np.abs(L[:, rows] - np.asarray(Lb)[0]).max() < 1e-12

@@ -381,6 +381,76 @@ def make_shared_prefix_decode(cfg: SharedPrefixConfig, suffix_lens=None) -> dict
                 prefix_len=cfg.prefix_len, num_blocks=num_blocks, spare_ids=spare, scale=cfg.scale)
 
 
+def make_block_sparse(seed: int, q_heads: int, kv_heads: int, seqlen_q: int, seqlen_k: int, head_dim: int,
+                      row_block: int, window: int, extra: int, spare_blocks: int = 8) -> dict:
+    """A block-sparse (BSR) pattern over one sequence, with its keys/values paged.
+
+    Query block r (``row_block`` rows) sees a window of ``window`` key blocks
+    (16 keys each) around its own position plus ``extra`` random other key
+    blocks, listed in random order (``indptr`` / ``indices``, logical key
+    blocks). q [Hq, Sq, D], k/v [Hkv, Sk, D] are N(0,1) bf16; the pools
+    [NB, Hkv, 16, D] hold logical key block c in physical block ``phys[c]``
+    (a random permutation); spare blocks and the tail slots past Sk hold NaN.
+    """
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 60])))
+    n_rb = -(-seqlen_q // row_block)
+    n_cb = -(-seqlen_k // BLOCK_SIZE)
+    indptr = [0]
+    indices = []
+    for r in range(n_rb):
+        centre = (r * row_block * seqlen_k) // max(seqlen_q, 1) // BLOCK_SIZE
+        lo = max(0, centre - window // 2)
+        cols = set(range(lo, min(n_cb, lo + window)))
+        others = [c for c in range(n_cb) if c not in cols]
+        if others and extra:
+            cols |= set(rng.choice(others, size=min(extra, len(others)), replace=False).tolist())
+        cols = np.array(sorted(cols), dtype=np.int32)
+        rng.shuffle(cols)
+        indices.extend(cols.tolist())
+        indptr.append(len(indices))
+    q = normal_bf16(seed, (q_heads, seqlen_q, head_dim), 61)
+    k = normal_bf16(seed, (kv_heads, seqlen_k, head_dim), 62)
+    v = normal_bf16(seed, (kv_heads, seqlen_k, head_dim), 63)
+    nb = n_cb + spare_blocks
+    phys = rng.permutation(nb).astype(np.int32)
+    pools = []
+    for x in (k, v):
+        pool = np.full((nb, kv_heads, BLOCK_SIZE, head_dim), BF16_NAN, dtype=np.uint16)
+        for c in range(n_cb):
+            t1 = min((c + 1) * BLOCK_SIZE, seqlen_k)
+            pool[phys[c], :, :t1 - c * BLOCK_SIZE] = x[:, c * BLOCK_SIZE:t1]
+        pools.append(pool)
+    return dict(q=q, k=k, v=v, k_pool=pools[0], v_pool=pools[1], phys=phys[:n_cb], spare_ids=phys[n_cb:],
+                indptr=np.array(indptr, dtype=np.int64), indices=np.array(indices, dtype=np.int32),
+                row_block=row_block, num_blocks=nb)
+
+
+def bsr_tables(d: dict, seqlen_k: int) -> tuple:
+    """Block tables that express a BSR pattern from :func:`make_block_sparse`:
+    one row per query block listing the physical blocks of its key blocks.
+
+    The kernels mask each table row by its token count, so a partial last key
+    block (Sk not a multiple of 16), when listed, is moved to the end of its
+    row and the count stops at Sk. Returns ``(table [n_rb, max_n] int32,
+    seqlens_k [n_rb] int32)``; unused entries point at a spare block.
+    """
+    indptr, indices, phys = d["indptr"], d["indices"], d["phys"]
+    n_rb = len(indptr) - 1
+    tail = seqlen_k % BLOCK_SIZE
+    last = (seqlen_k - 1) // BLOCK_SIZE
+    width = max(1, int(np.diff(indptr).max()) if n_rb else 1)
+    table = np.full((n_rb, width), int(d["spare_ids"][0]), dtype=np.int32)
+    lens = np.zeros(n_rb, dtype=np.int32)
+    for r in range(n_rb):
+        cols = [int(c) for c in indices[indptr[r]:indptr[r + 1]]]
+        partial = tail and last in cols
+        if partial:
+            cols = [c for c in cols if c != last] + [last]
+        table[r, :len(cols)] = phys[cols]
+        lens[r] = BLOCK_SIZE * len(cols) - ((BLOCK_SIZE - tail) if partial else 0)
+    return table, lens
+
+
 def relayout_identity(pool: np.ndarray, table: np.ndarray, kv_lens) -> tuple:
     """Copy a paged pool into identity order (sequence 0's blocks first, ...).
 

@@ -548,3 +548,24 @@ def test_block_sparse_is_dense_attention_over_the_gathered_blocks():
                                         _nested(v[None][:, :, keys]), 0.5, False)
         assert np.abs(O[:, rows] - np.asarray(Ob)[0]).max() < 1e-12
         assert np.abs(L[:, rows] - np.asarray(Lb)[0]).max() < 1e-12
+
+
+def test_block_sparse_via_block_tables_is_the_bsr_definition():
+    """The paged-prefill oracle over the per-query-block tables of
+    workloads.bsr_tables (the form the kernels take) equals the BSR
+    definition, including a listed partial last key block."""
+    d = wl.make_block_sparse(72, 4, 2, 70, 200, 8, 16, 3, 2)
+    table, lens = wl.bsr_tables(d, 200)
+    n_rb = len(d["indptr"]) - 1
+    qb = np.zeros((n_rb, 4, 16, 8), dtype=np.uint16)
+    q_lens = np.zeros(n_rb, dtype=np.int32)
+    for r in range(n_rb):
+        rows = d["q"][:, 16 * r:16 * r + 16]
+        qb[r, :, :rows.shape[1]] = rows
+        q_lens[r] = rows.shape[1]
+    O, L = ref.ref_prefill_paged(qb, q_lens, d["k_pool"], d["v_pool"], table, lens, 0.35, False)
+    Ob, Lb = ref.ref_block_sparse_attention(d["q"], d["k"], d["v"], d["indptr"], d["indices"], 16, 16, 0.35)
+    got = np.concatenate([O[r, :, :q_lens[r]] for r in range(n_rb)], axis=1)
+    got_l = np.concatenate([L[r, :, :q_lens[r]] for r in range(n_rb)], axis=1)
+    assert (200 - 1) // 16 in set(d["indices"].tolist())  # the partial block is exercised
+    assert np.abs(got - Ob).max() < 1e-12 and np.abs(got_l - Lb).max() < 1e-12

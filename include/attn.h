@@ -103,6 +103,14 @@ typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1, ATTN_DTYPE_FP8_E4M3 = 2 
  * max_blocks_per_seq * block_size; seqlen_k must then be the maximum of
  * seqlens_k (an upper bound is fine). The causal alignment uses the
  * per-sequence lengths.
+ *
+ * Block-sparse attention (BSR: query block r sees only the key blocks listed
+ * for it, the block-sparse format of the FlashInfer section of "抱infra脚")
+ * is this paged mode, non-causal, with one batch entry per query block whose
+ * table row lists the physical blocks of its key blocks, in any order. A
+ * table row is masked by its token count seqlens_k[r], so a partial block
+ * (fewer than 16 valid keys) may only be the last one of a row. Decode takes
+ * a BSR pattern the same way (one table row per query).
  */
 typedef struct {
   const void* q;

@@ -569,3 +569,46 @@ def test_block_sparse_via_block_tables_is_the_bsr_definition():
     got_l = np.concatenate([L[r, :, :q_lens[r]] for r in range(n_rb)], axis=1)
     assert (200 - 1) // 16 in set(d["indices"].tolist())  # the partial block is exercised
     assert np.abs(got - Ob).max() < 1e-12 and np.abs(got_l - Lb).max() < 1e-12
+
+
+# ----------------------------------------------------------------------------
+# randomised shapes (hypothesis): backward and block-sparse pins
+# ----------------------------------------------------------------------------
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(G=st.sampled_from([1, 2, 3]), Hkv=st.integers(1, 2), Sq=st.integers(1, 9), Sk=st.integers(1, 9),
+       D=st.sampled_from([2, 5]), causal=st.booleans(), seed=st.integers(0, 10_000))
+def test_backward_random_shapes_match_autograd(G, Hkv, Sq, Sk, D, causal, seed):
+    rng = np.random.default_rng(seed)
+    q, do = _rand(rng, 1, G * Hkv, Sq, D), _rand(rng, 1, G * Hkv, Sq, D)
+    k, v = _rand(rng, 1, Hkv, Sk, D), _rand(rng, 1, Hkv, Sk, D)
+    r = ref.ref_attention_backward(q, k, v, do, 0.7, causal)
+    dq, dk, dv, _ = _autograd_backward(q, k, v, do, 0.7, causal)
+    assert np.abs(r["dq"] - dq).max() < 1e-11
+    assert np.abs(r["dk"] - dk).max() < 1e-11
+    assert np.abs(r["dv"] - dv).max() < 1e-11
+
+
+@settings(max_examples=25, deadline=None)
+@given(Sq=st.integers(1, 20), Sk=st.integers(1, 40), rb=st.sampled_from([1, 4, 8]), seed=st.integers(0, 10_000))
+def test_block_sparse_random_patterns_match_gathered_dense(Sq, Sk, rb, seed):
+    """Random BSR patterns (possibly empty rows, any order) against dense
+    attention over each row block's gathered keys."""
+    rng = np.random.default_rng(seed)
+    q, k, v = _rand(rng, 2, Sq, 3), _rand(rng, 1, Sk, 3), _rand(rng, 1, Sk, 3)
+    n_rb, n_cb = -(-Sq // rb), -(-Sk // 16)
+    lists = [rng.permutation(n_cb)[:rng.integers(0, n_cb + 1)] for _ in range(n_rb)]
+    indptr = np.concatenate([[0], np.cumsum([len(c) for c in lists])])
+    indices = np.concatenate(lists).astype(np.int64) if indptr[-1] else np.zeros(0, dtype=np.int64)
+    O, L = ref.ref_block_sparse_attention(q, k, v, indptr, indices, rb, 16, 0.4)
+    for r, cols in enumerate(lists):
+        rows = slice(r * rb, min(r * rb + rb, Sq))
+        if len(cols) == 0:
+            assert (O[:, rows] == 0).all() and np.isneginf(L[:, rows]).all()
+            continue
+        keys = np.concatenate([np.arange(c * 16, min(c * 16 + 16, Sk)) for c in cols])
+        Od, Ld = ref.ref_attention(q[None, :, rows], k[None][:, :, keys], v[None][:, :, keys], 0.4, False)
+        assert np.abs(O[:, rows] - Od[0]).max() < 1e-12 and np.abs(L[:, rows] - Ld[0]).max() < 1e-12

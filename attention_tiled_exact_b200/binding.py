@@ -325,6 +325,17 @@ def _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_le
     return p
 
 
+def _check_decode_inputs(q, k_cache, v_cache, block_table, seq_lens, allow_fp8=True):
+    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
+    ok_cache = k_cache.dtype == torch.bfloat16 or (allow_fp8 and _is_fp8(k_cache))
+    _need(q.dtype == torch.bfloat16 and k_cache.dtype == v_cache.dtype and ok_cache,
+          "bf16 q; bf16 or FP8 E4M3 caches" if allow_fp8 else "bf16 q and caches")
+    _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
+    _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
+          "int32 block table [B, max_blocks]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "int32 seq_lens [B]")
+
+
 def decode_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int = 0,
                            num_splits: int = 0) -> int:
     """Bytes of workspace :func:`decode_paged` needs for these shapes."""
@@ -345,13 +356,7 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None
     CUDA). ``max_seq_len`` is a host-side upper bound of seq_lens used for the
     split plan (0 = table capacity). Returns ``(O [B,Hq,D], LSE [B,Hq] or None)``.
     """
-    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
-    _need(q.dtype == torch.bfloat16 and k_cache.dtype == v_cache.dtype and
-          (k_cache.dtype == torch.bfloat16 or _is_fp8(k_cache)), "bf16 q; bf16 or FP8 E4M3 caches")
-    _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
-    _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
-          "int32 block table [B, max_blocks]")
-    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "int32 seq_lens [B]")
+    _check_decode_inputs(q, k_cache, v_cache, block_table, seq_lens)
     B, Hq, D = q.shape
     if out is None:
         out = torch.empty((B, Hq, D), dtype=out_dtype, device=q.device)
@@ -368,17 +373,6 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale: float | None
     _check(LIB.attn_decode_paged(ctypes.byref(p), ws_ptr, ws_bytes, None, _stream(q.device)),
            "attn_decode_paged")
     return out, lse
-
-
-def _check_decode_inputs(q, k_cache, v_cache, block_table, seq_lens, allow_fp8=True):
-    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
-    ok_cache = k_cache.dtype == torch.bfloat16 or (allow_fp8 and _is_fp8(k_cache))
-    _need(q.dtype == torch.bfloat16 and k_cache.dtype == v_cache.dtype and ok_cache,
-          "bf16 q; bf16 or FP8 E4M3 caches" if allow_fp8 else "bf16 q and caches")
-    _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
-    _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
-          "int32 block table [B, max_blocks]")
-    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "int32 seq_lens [B]")
 
 
 def decode_shared_prefix_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, prefix_len: int,
@@ -431,13 +425,7 @@ def decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, out, lse=No
     array that the library owns on each GPU, so nothing is allocated here or in
     the library. Calls that overlap on the GPU race on that array.
     """
-    _need(q.dim() == 3 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
-    _need(q.dtype == torch.bfloat16 and k_cache.dtype == v_cache.dtype and
-          (k_cache.dtype == torch.bfloat16 or _is_fp8(k_cache)), "bf16 q; bf16 or FP8 E4M3 caches")
-    _need(q.is_contiguous() and k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous q and caches")
-    _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.dim() == 2,
-          "int32 block table [B, max_blocks]")
-    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "int32 seq_lens [B]")
+    _check_decode_inputs(q, k_cache, v_cache, block_table, seq_lens)
     _need(out is not None and tuple(out.shape) == tuple(q.shape) and out.is_contiguous(), "out [B, Hq, D]")
     p = _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits, out, lse,
                        error_flags, k_scale, v_scale)

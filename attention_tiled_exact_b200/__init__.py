@@ -1,18 +1,27 @@
 """Exact scaled-dot-product attention for B200 (sm_100a).
 
-Three calls, each a thin marshalling layer over the C-ABI library
-``libattn_b200.so`` (every step of the computation runs in its CUDA kernels):
+A thin marshalling layer over the C-ABI library ``libattn_b200.so`` (every
+step of the computation runs in its CUDA kernels):
 
 * :func:`prefill` -- tiled causal / non-causal GQA prefill with online softmax;
 * :func:`prefill_paged` -- the same over a block-table KV cache (chunked prefill);
-* :func:`decode_paged` -- split-KV decode over a block-table KV cache;
-* :func:`splitkv_lse_combine` -- log-sum-exp merge of split partials.
+* :func:`prefill_backward` -- dQ, dK, dV of the dense prefill;
+* :func:`decode_paged` -- split-KV decode over a block-table KV cache (bf16 or
+  FP8 E4M3 cache), with :func:`decode_workspace_bytes` for its workspace;
+* :func:`decode_paged_shared_prefix` -- decode of a batch sharing a prefix,
+  which is attended once per batch (:func:`decode_shared_prefix_workspace_bytes`);
+* :func:`decode_paged_noalloc` -- decode for callers that cannot allocate;
+* :func:`splitkv_lse_combine` -- log-sum-exp merge of split partials;
+* :func:`sync_error_flags` / :func:`status_from_flags` -- the device error
+  word as a status.
 
 The library is loaded on first use of one of these names; if it is missing
 the import fails with an error that says how to build it. There is no CPU
 fallback.
 """
-_API = ("prefill", "prefill_paged", "decode_paged", "decode_paged_noalloc", "splitkv_lse_combine", "decode_workspace_bytes",
+_API = ("prefill", "prefill_paged", "prefill_backward", "decode_paged", "decode_workspace_bytes",
+        "decode_paged_shared_prefix", "decode_shared_prefix_workspace_bytes", "decode_paged_noalloc",
+        "splitkv_lse_combine", "sync_error_flags", "status_from_flags", "set_wait_limit", "selftest_exp2",
         "AttnError", "library_path", "status_string")
 
 

@@ -35,6 +35,7 @@ ATTN_DTYPE_FP8_E4M3 = 2
 ATTN_FAULT_TIMEOUT = 0x1
 ATTN_FAULT_BAD_BLOCK = 0x2
 ATTN_FAULT_BAD_LENGTH = 0x4
+ATTN_FAULT_PREFIX_MISMATCH = 0x8
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
@@ -112,6 +113,14 @@ def _load():
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_version.argtypes = []
     lib.attn_version.restype = ctypes.c_int
+    lib.attn_status_from_flags.argtypes = [ctypes.c_int32]
+    lib.attn_status_from_flags.restype = ctypes.c_int
+    lib.attn_sync_error_flags.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.attn_sync_error_flags.restype = ctypes.c_int
+    lib.attn_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.attn_set_wait_limit.restype = None
+    lib.attn_selftest_exp2.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp]
+    lib.attn_selftest_exp2.restype = ctypes.c_int
     return lib
 
 
@@ -135,6 +144,41 @@ class AttnError(RuntimeError):
 def _check(status: int, where: str):
     if status != ATTN_OK:
         raise AttnError(status, where)
+
+
+def status_from_flags(flags: int) -> int:
+    """The status an error word maps to (ATTN_ERR_TIMEOUT, ATTN_ERR_DEVICE_FAULT or ATTN_OK)."""
+    return int(LIB.attn_status_from_flags(int(flags)))
+
+
+def sync_error_flags(error_flags) -> tuple[int, int]:
+    """Wait for the current stream, read the int32 device error word and map it.
+
+    Returns ``(status, word)``; the word is left as it is.
+    """
+    _need(error_flags.dtype == torch.int32 and error_flags.is_cuda and error_flags.numel() >= 1, "int32 error word")
+    word = ctypes.c_int32(0)
+    st = LIB.attn_sync_error_flags(_ptr(error_flags), _stream(error_flags.device), ctypes.byref(word))
+    if st == ATTN_ERR_CUDA or st == ATTN_ERR_INVALID_ARG:
+        raise AttnError(st, "attn_sync_error_flags")
+    return int(st), int(word.value)
+
+
+def set_wait_limit(cycles: int = 0) -> None:
+    """Diagnostic: clock-cycle bound of the prefill/backward pipeline waits (0 = the ~1 s default)."""
+    LIB.attn_set_wait_limit(int(cycles))
+
+
+def selftest_exp2(x):
+    """Diagnostic: the prefill kernel's FMA-pipe 2^x and MUFU ex2.approx of an fp32 CUDA tensor.
+
+    Returns ``(y_poly, y_mufu)``, fp32 tensors shaped like ``x``.
+    """
+    _need(x.dtype == torch.float32 and x.is_cuda and x.is_contiguous(), "contiguous fp32 CUDA tensor")
+    y_poly, y_mufu = torch.empty_like(x), torch.empty_like(x)
+    _check(LIB.attn_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), x.numel(), _stream(x.device)),
+           "attn_selftest_exp2")
+    return y_poly, y_mufu
 
 
 def _ptr(t):

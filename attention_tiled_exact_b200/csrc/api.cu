@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "attn.h"
@@ -13,13 +14,20 @@
 namespace attn {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// About one second at the B200's 1.9 GHz boost clock.
+constexpr long long kDefaultWaitLimit = 2000000000LL;
+static std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+
+long long pipeline_wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
+
 static bool mult8(int64_t s) { return (s % 8) == 0; }
 
 int device_sm_count() {
   static std::mutex mu;
-  static int cache[64] = {0};
+  static int cache[kMaxDevices] = {0};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
   std::lock_guard<std::mutex> lock(mu);
   if (cache[dev] == 0) {
     int n = 0;
@@ -207,6 +215,29 @@ attn_status_t splitkv_lse_combine(const float* part_o, const float* part_lse, in
   if (st != ATTN_OK) return st;
   return attn::launch_combine(part_o, part_lse, num_splits, rows, head_dim, splits_per_row, nullptr, 1, 1, out_o,
                               out_dtype, out_lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+void attn_set_wait_limit(long long cycles) {
+  attn::g_wait_limit.store(cycles > 0 ? cycles : attn::kDefaultWaitLimit, std::memory_order_relaxed);
+}
+
+attn_status_t attn_status_from_flags(int32_t flags) {
+  if (flags & ATTN_FAULT_TIMEOUT) return ATTN_ERR_TIMEOUT;
+  if (flags != 0) return ATTN_ERR_DEVICE_FAULT;
+  return ATTN_OK;
+}
+
+attn_status_t attn_sync_error_flags(const int32_t* error_flags, attn_stream_t stream, int32_t* flags_out) {
+  if (!error_flags) return ATTN_ERR_INVALID_ARG;
+  int32_t word = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&word, error_flags, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  if (flags_out) *flags_out = word;
+  return attn_status_from_flags(word);
 }
 
 const char* attn_status_string(attn_status_t status) {

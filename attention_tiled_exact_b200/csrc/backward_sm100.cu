@@ -58,7 +58,6 @@ constexpr int MMA_WARP = 9;
 constexpr int NUM_THREADS = 320;
 static_assert(TMA_WARP == EW_WARPS && MMA_WARP == EW_WARPS + 1 && NUM_THREADS == (EW_WARPS + 2) * 32, "warp roles");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr long long WAIT_LIMIT = 2000000000LL;  // cycles (~1 s)
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct Args {
@@ -76,6 +75,7 @@ struct Args {
   long long dq_bs, dq_hs, dq_rs, dk_bs, dk_hs, dk_rs, dv_bs, dv_hs, dv_rs;
   int grad_f32;
   int32_t* error_flags;
+  long long wait_limit;  // cycle bound of every pipeline wait
 };
 
 template <int D>
@@ -101,8 +101,8 @@ struct Layout {
 // columns of that half.
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC = 256;
 
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, WAIT_LIMIT));
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
+  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, limit));
 }
 
 // Contiguous global -> shared copy completing on an mbarrier (no multicast).
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int t = 0;
       for (; t < w.n_steps; ++t) {
         const int s = t & 1;
-        if (t >= 2 && !mbar_wait_bounded(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        if (t >= 2 && !mbar_wait_bounded(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag, a.wait_limit)) break;
         const int h = step_head(t), blk = step_blk(t);
         uint8_t* b0 = smem + L::RING_OFF + (2 * s) * L::TILE;
         uint8_t* b1 = b0 + L::TILE;
@@ -297,10 +297,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      // Drain: no copy may be in flight when the CTA exits (abort path).
-      mbar_wait_bounded(a_full, 0, abort_flag, WAIT_LIMIT);
-      for (int u = t - 2 > 0 ? t - 2 : 0; u < t; ++u)
-        mbar_wait_bounded(&ring_full[u & 1], (u >> 1) & 1, abort_flag, WAIT_LIMIT);
+      // Drain: no copy may be in flight when the CTA exits. The last two
+      // steps' copies are the only ones that can still run (a stage's earlier
+      // copy completed before its empty barrier let the next one start); on
+      // the abort path they still land by themselves, so these waits ignore
+      // the abort flag.
+      mbar_wait_drain(a_full, 0);
+      for (int u = t - 2 > 0 ? t - 2 : 0; u < t; ++u) mbar_wait_drain(&ring_full[u & 1], (u >> 1) & 1);
     }
   } else if (warp == MMA_WARP) {
     if (lane == 0 && w.n_steps > 0) {
@@ -355,8 +358,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // issued right after its accumulating products of step t (they reuse its
       // TMEM columns; MMAs from one thread run in issue order), so while one
       // warpgroup works the tensor core runs the other half's products.
-      bool ok = mbar_wait_bounded(a_full, 0, abort_flag, WAIT_LIMIT);
-      if (ok) ok = mbar_wait_bounded(&ring_full[0], 0, abort_flag, WAIT_LIMIT);
+      bool ok = mbar_wait_bounded(a_full, 0, abort_flag, a.wait_limit);
+      if (ok) ok = mbar_wait_bounded(&ring_full[0], 0, abort_flag, a.wait_limit);
       if (ok) {
         tc_fence_after();
         s_half(0, 0);
@@ -364,17 +367,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int t = 0; t < w.n_steps && ok; ++t) {
         const bool next = t + 1 < w.n_steps;
-        ok = mbar_wait_bounded(&ps_full[0], t & 1, abort_flag, WAIT_LIMIT);
+        ok = mbar_wait_bounded(&ps_full[0], t & 1, abort_flag, a.wait_limit);
         if (!ok) break;
         tc_fence_after();
         acc_half(t, 0);
         if (next) {
-          ok = mbar_wait_bounded(&ring_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag, WAIT_LIMIT);
+          ok = mbar_wait_bounded(&ring_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag, a.wait_limit);
           if (!ok) break;
           tc_fence_after();
           s_half(t + 1, 0);
         }
-        ok = mbar_wait_bounded(&ps_full[1], t & 1, abort_flag, WAIT_LIMIT);
+        ok = mbar_wait_bounded(&ps_full[1], t & 1, abort_flag, a.wait_limit);
         if (!ok) break;
         tc_fence_after();
         acc_half(t, 1);
@@ -382,9 +385,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (next) s_half(t + 1, 1);
       }
       if (ok) mma_commit(acc_full);
-      // Every MMA must have completed before tensor memory is released.
+      // Every MMA issued must have completed before tensor memory is released
+      // (on the abort path too: they finish by themselves).
       mma_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0, abort_flag, WAIT_LIMIT);
+      mbar_wait_drain(mma_done, 0);
     }
   } else {
     // ------------------------------------------------------------------ elementwise + epilogue
@@ -415,7 +419,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if constexpr (KV) {
         c_lim = row_pos < a.seqlen_k ? (a.causal ? row_pos - off - blk * BM : -BM) : BM;
         // The producer's LSE / D copies complete on the stage's full barrier.
-        ok = warp_wait(&ring_full[s], (t >> 1) & 1, abort_flag);
+        ok = warp_wait(&ring_full[s], (t >> 1) & 1, abort_flag, a.wait_limit);
         if (!ok) break;
       } else {
         int lim = a.seqlen_k - blk * BM;
@@ -427,7 +431,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const float* lse_c = vec + (2 * s) * BM;
       const float* delta_c = vec + (2 * s + 1) * BM;
-      ok = warp_wait(&sdp_full[half], t & 1, abort_flag);
+      ok = warp_wait(&sdp_full[half], t & 1, abort_flag, a.wait_limit);
       if (!ok) break;
       tc_fence_after();
       // The whole half is visible on all but the diagonal and ragged tiles:
@@ -483,7 +487,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     // ---- epilogue: each warpgroup stores half of the columns of its rows
     const bool row_ok = row_pos < (KV ? a.seqlen_k : a.seqlen_q);
-    if (ok && w.n_steps > 0) ok = warp_wait(acc_full, 0, abort_flag);
+    if (ok && w.n_steps > 0) ok = warp_wait(acc_full, 0, abort_flag, a.wait_limit);
     if (ok) {
       tc_fence_after();
       const int n_out = KV ? 2 : 1;
@@ -602,14 +606,15 @@ typedef CUresult (*BwdEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, v
                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static BwdEncodeFn bwd_encode_fn() {
-  static BwdEncodeFn fn = nullptr;
-  if (!fn) {
+  static const BwdEncodeFn fn = []() -> BwdEncodeFn {  // process-wide; initialised once, thread-safely
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<BwdEncodeFn>(ptr);
-  }
+      return reinterpret_cast<BwdEncodeFn>(ptr);
+    cudaGetLastError();
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -644,12 +649,15 @@ static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   using L = bwd::Layout<D>;
   static_assert(L::SMEM_BYTES <= 232448, "shared memory budget");
   auto kern = bwd::bwd_kernel<D, KV>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES) != cudaSuccess)
+  static DeviceOnce setup;  // the shared-memory attribute, once per device
+  const attn_status_t st = setup.run([&]() -> attn_status_t {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES) != cudaSuccess) {
+      cudaGetLastError();
       return ATTN_ERR_CUDA;
-    configured = true;
-  }
+    }
+    return ATTN_OK;
+  });
+  if (st != ATTN_OK) return st;
   if (grid <= 0) return ATTN_OK;
   if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   kern<<<(unsigned)grid, bwd::NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
@@ -717,6 +725,7 @@ attn_status_t launch_backward(const attn_backward_params& p, void* workspace, cu
   a.dv_rs = p.dv_row_stride;
   a.grad_f32 = p.grad_dtype == ATTN_DTYPE_F32;
   a.error_flags = p.error_flags;
+  a.wait_limit = pipeline_wait_limit();
   const long long kv_items = (long long)a.n_kb * p.batch * p.num_kv_heads;
   const long long q_items = (long long)a.n_qb * p.batch * p.num_q_heads;
   attn_status_t st;

@@ -26,7 +26,8 @@
 //      seq_lens[b] - prefix_len), giving one more partial per row;
 //   3. merge: one warp per (sequence, head) row combines the S + 1 partials.
 // A small kernel before step 1 writes the suffix lengths (flagging sequences
-// shorter than the prefix), the per-range prefix lengths and the q copies.
+// shorter than the prefix), the per-range prefix lengths and the q copies,
+// and flags table rows whose prefix entries differ from row 0's.
 #include <cuda_bf16.h>
 #include <stdint.h>
 #include <string.h>
@@ -45,9 +46,19 @@ __global__ void __launch_bounds__(256)
     prepare_kernel(const int32_t* __restrict__ seq_lens, int batch, int prefix_len, int suffix_cap,
                    int32_t* __restrict__ suffix_lens, int32_t* __restrict__ range_lens, int ranges, int range_len,
                    const uint4* __restrict__ q, uint4* __restrict__ q_rep, int hq, int row_vecs,
-                   int32_t* __restrict__ error_flags) {
+                   const int32_t* __restrict__ block_table, int max_blocks, int32_t* __restrict__ error_flags) {
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long stride = (long long)gridDim.x * blockDim.x;
+  // Every row's prefix entries must alias row 0's (the prefix is read from
+  // row 0 only): a row that lists other blocks there is flagged.
+  const int prefix_blocks = prefix_len / 16;
+  bool mismatch = false;
+  for (long long i = tid + prefix_blocks; i < (long long)batch * prefix_blocks; i += stride) {
+    const long long b = i / prefix_blocks;
+    const int j = (int)(i - b * prefix_blocks);
+    mismatch |= block_table[b * max_blocks + j] != block_table[j];
+  }
+  if (mismatch && error_flags) atomicOr(error_flags, ATTN_FAULT_PREFIX_MISMATCH);
   for (long long i = tid; i < batch; i += stride) {
     const int L = seq_lens[i];
     int s = L - prefix_len;
@@ -222,7 +233,8 @@ attn_status_t launch_cascade(const attn_decode_params& p, const CascadePlan& c, 
     prepare_kernel<<<(int)blocks, 256, 0, stream>>>(p.seq_lens, p.batch, c.prefix_len, c.suffix_cap, suffix_lens,
                                                    range_lens, c.ranges, c.range_blocks * 16,
                                                    reinterpret_cast<const uint4*>(p.q), reinterpret_cast<uint4*>(q_rep),
-                                                   p.num_q_heads, row_vecs, p.error_flags);
+                                                   p.num_q_heads, row_vecs, p.block_table, p.max_blocks_per_seq,
+                                                   p.error_flags);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
 

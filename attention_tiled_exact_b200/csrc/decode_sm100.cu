@@ -668,12 +668,15 @@ static attn_status_t launch_decode_g(const decode::Args& a, const DecodePlan& pl
   auto kern = decode::decode_split_kernel<G, FP8, FP8>;  // P V on the tensor cores for FP8 caches
   const int smem = (int)sizeof(decode::Smem<G, FP8>);
   static_assert(sizeof(decode::MergeSmem<G>) <= sizeof(decode::Smem<G, FP8>), "merge buffer fits");
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  static DeviceOnce setup;  // the shared-memory attribute, once per device
+  const attn_status_t st = setup.run([&]() -> attn_status_t {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
       return ATTN_ERR_CUDA;
-    configured = true;
-  }
+    }
+    return ATTN_OK;
+  });
+  if (st != ATTN_OK) return st;
   dim3 grid(plan.max_splits, a.hkv, a.batch);
   kern<<<grid, decode::WARPS * 32, smem, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

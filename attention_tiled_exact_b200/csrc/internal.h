@@ -3,9 +3,49 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "attn.h"
 
 namespace attn {
+
+constexpr int kMaxDevices = 64;
+
+// One-time setup of a kernel (its attributes), done once per device and
+// thread-safe. cudaFuncSetAttribute applies to the current device only, so a
+// process that drives several GPUs needs it on each of them. `fn` runs with
+// the device current, under a lock, until it returns something other than
+// ATTN_ERR_CUDA; that status is then returned by every later call on that
+// device without taking the lock.
+class DeviceOnce {
+ public:
+  template <class F>
+  attn_status_t run(F&& fn) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_NO_DEVICE;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+    int st = state_[dev].load(std::memory_order_acquire);
+    if (st != 0) return static_cast<attn_status_t>(st - 1);
+    std::lock_guard<std::mutex> lock(mu_);
+    st = state_[dev].load(std::memory_order_relaxed);
+    if (st != 0) return static_cast<attn_status_t>(st - 1);
+    const attn_status_t r = fn();
+    if (r != ATTN_ERR_CUDA) state_[dev].store(static_cast<int>(r) + 1, std::memory_order_release);
+    return r;
+  }
+
+ private:
+  std::mutex mu_;
+  std::atomic<int> state_[kMaxDevices] = {};  // 0: not done; else the status + 1
+};
+
+// Cycle bound of every pipeline wait of the prefill and backward kernels
+// (attn_set_wait_limit; about one second by default).
+long long pipeline_wait_limit();
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

@@ -46,6 +46,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include "exp2_poly.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
@@ -70,7 +71,6 @@ constexpr int REG_SOFTMAX = 216;
 constexpr int REG_OTHER = 72;
 static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_OTHER == NUM_THREADS * REG_LAUNCH, "register split");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr long long WAIT_LIMIT = 2000000000LL;  // cycles (~1 s)
 constexpr float RESCALE_THRESHOLD = 8.0f;        // log2 units: rescale only when the max grows by > 2^8
 // Variable-length launches with at most SORT_MAX_ITEMS items sort the items by
 // cost before the snake assignment; a CTA then keeps at most LIST_MAX of them.
@@ -110,6 +110,7 @@ struct Args {
   int sort_items;  // order items by cost (variable lengths) instead of row block
   long long o_bs, o_hs, o_rs;
   int32_t* error_flags;
+  long long wait_limit;  // cycle bound of every pipeline wait
   // paged keys/values (PAGED kernels only)
   const int32_t* block_table;
   int max_blocks;
@@ -256,30 +257,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair of inputs on the FMA pipe (the MUFU unit is the scarce
-// resource of this kernel). Range reduction rounds x to the nearest integer n
-// by adding 1.5 * 2^23 (the integer lands in the low mantissa bits), so
-// x = n + f with |f| <= 1/2; 2^f comes from a degree-3 polynomial fitted for
-// this kernel (minimax in relative error on [-1/2, 1/2] by Lawson's
-// iteratively reweighted least squares; max relative error 7.5e-5, far below
-// the 2^-9 rounding of the bf16 P it feeds); n is then added to the exponent
-// field. Inputs are clamped at -126, so tiny results come out as ~2^-126
-// instead of 0, and must stay below 128.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float C0 = 0.9999280571937561f, C1 = 0.6932609677314758f, C2 = 0.2426111251115799f,
-                  C3 = 0.0551716648042202f;
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(make_float2(C3, C3), f, make_float2(C2, C2));
-  p = __ffma2_rn(p, f, make_float2(C1, C1));
-  p = __ffma2_rn(p, f, make_float2(C0, C0));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // Exponentials of one row block of scores (s[]), their sum, and the packed
 // bf16 P stored to TMEM 16 columns at a time. EMU8: in every 8 consecutive
 // pairs, a spread-out EMU8 of them take exp2 on the FMA pipe (exp2_poly2), the
@@ -398,8 +375,8 @@ __device__ __forceinline__ void store_rows_tma(const CUtensorMap* tm_o, uint8_t*
 
 // All lanes of the warp get the same answer (a timeout seen by one lane is
 // seen by all), so warp-collective instructions after it stay converged.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, WAIT_LIMIT));
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
+  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, limit));
 }
 
 // Persistent: CTA c processes work items in the snake order of snake_item
@@ -491,7 +468,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (PAGED && args.seqlens_k[w.b] > args.max_blocks * 16 && args.error_flags)
           atomicOr(args.error_flags, ATTN_FAULT_BAD_LENGTH);
         // Q tiles: wait until the last S MMA of the previous item has read them.
-        if (nq > 0 && !mbar_wait_bounded(q_empty, (nq - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        if (nq > 0 && !mbar_wait_bounded(q_empty, (nq - 1) & 1, abort_flag, args.wait_limit)) break;
         mbar_arrive_expect_tx(q_full, (w.active[0] + w.active[1]) * L::Q_TILE);
         for (int t = 0; t < 2; ++t) {
           if (!w.active[t]) continue;
@@ -543,7 +520,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint64_t* full = is_v ? v_full : k_full;
           uint64_t* empty = is_v ? v_empty : k_empty;
           const int s = cnt % stages;
-          if (cnt >= stages && !mbar_wait_bounded(&empty[s], ((cnt / stages) - 1) & 1, abort_flag, WAIT_LIMIT))
+          if (cnt >= stages && !mbar_wait_bounded(&empty[s], ((cnt / stages) - 1) & 1, abort_flag, args.wait_limit))
             return false;
           mbar_arrive_expect_tx(&full[s], L::KV_TILE);
           uint8_t* dst = smem + (is_v ? L::V_OFF : L::K_OFF) + s * L::KV_TILE;
@@ -567,13 +544,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (ok) ok = load(true, i);
         }
       }
-      // Drain: wait for the last copy issued into each slot, so no copy is in
-      // flight when the CTA exits (matters only on the abort path).
-      for (int i = max(0, nk - KSTAGES); i < nk; ++i)
-        mbar_wait_bounded(&k_full[i % KSTAGES], (i / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
-      for (int i = max(0, nv - VSTAGES); i < nv; ++i)
-        mbar_wait_bounded(&v_full[i % VSTAGES], (i / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
-      if (nq > 0) mbar_wait_bounded(q_full, (nq - 1) & 1, abort_flag, WAIT_LIMIT);
+      // Drain: wait for the last copy issued into each slot (a slot's earlier
+      // copy completed before its empty barrier let the next one start), so no
+      // copy is in flight when the CTA exits. On the abort path the consumers
+      // have stopped, but every copy issued still lands by itself, so these
+      // waits ignore the abort flag.
+      for (int i = max(0, nk - KSTAGES); i < nk; ++i) mbar_wait_drain(&k_full[i % KSTAGES], (i / KSTAGES) & 1);
+      for (int i = max(0, nv - VSTAGES); i < nv; ++i) mbar_wait_drain(&v_full[i % VSTAGES], (i / VSTAGES) & 1);
+      if (nq > 0) mbar_wait_drain(q_full, (nq - 1) & 1);
     } else if (warp == MMA_WARP && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer (both tiles)
       // One thread issues every MMA in the fixed order S_0(0), S_1(0), then per
@@ -624,7 +602,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // S of block i for every tile that has it; then K_i can be released.
         auto s_blocks = [&](int i) -> bool {
           const int kg = kb + i;
-          if (!mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, WAIT_LIMIT)) return false;
+          if (!mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, args.wait_limit)) return false;
           tc_fence_after();
           for (int t = 0; t < 2; ++t) {
             if (i >= w.n_kv[t]) continue;
@@ -635,17 +613,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (i == n_kv - 1) mma_commit(q_empty);  // the item's last S MMA has been issued
           return true;
         };
-        ok = mbar_wait_bounded(q_full, nq & 1, abort_flag, WAIT_LIMIT);
+        ok = mbar_wait_bounded(q_full, nq & 1, abort_flag, args.wait_limit);
         if (ok) ok = s_blocks(0);
         for (int i = 0; i < n_kv && ok; ++i) {
           const int vg = kb + i;  // V_i is the (kb + i)-th V block
-          ok = mbar_wait_bounded(&v_full[vg % VSTAGES], (vg / VSTAGES) & 1, abort_flag, WAIT_LIMIT);
+          ok = mbar_wait_bounded(&v_full[vg % VSTAGES], (vg / VSTAGES) & 1, abort_flag, args.wait_limit);
           const bool next = i + 1 < n_kv;
           const int kg = kb + i + 1;
-          if (ok && next) ok = mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, WAIT_LIMIT);
+          if (ok && next) ok = mbar_wait_bounded(&k_full[kg % KSTAGES], (kg / KSTAGES) & 1, abort_flag, args.wait_limit);
           for (int t = 0; t < 2 && ok; ++t) {
             if (i >= w.n_kv[t]) continue;
-            ok = mbar_wait_bounded(&p_full[t], (gb[t] + i) & 1, abort_flag, WAIT_LIMIT);
+            ok = mbar_wait_bounded(&p_full[t], (gb[t] + i) & 1, abort_flag, args.wait_limit);
             if (!ok) break;
             tc_fence_after();
             issue_pv(t, vg, i == 0);
@@ -669,10 +647,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         kb += n_kv;
         ++nq;
       }
-      // Wait until every MMA has completed before tensor memory can be
-      // released (bounded; matters on the abort path).
+      // Wait until every MMA issued has completed before tensor memory can be
+      // released (on the abort path too: the issued MMAs finish by themselves).
       mma_commit(mma_done);
-      mbar_wait_bounded(mma_done, 0, abort_flag, WAIT_LIMIT);
+      mbar_wait_drain(mma_done, 0);
     }
   } else {
     regs_inc<REG_SOFTMAX>();
@@ -707,7 +685,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float l = 0.f;         // running sum of 2^(s*scale*log2e - m2)
       for (int i = 0; i < nt; ++i) {
         const int g = gb + i;
-        ok = warp_wait(&s_full[t], g & 1, abort_flag);
+        ok = warp_wait(&s_full[t], g & 1, abort_flag, args.wait_limit);
         if (!ok) break;
         tc_fence_after();
         uint32_t sb[BK];
@@ -761,8 +739,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         l = l * alpha + (acc.x + acc.y);
         if (v_fix && i == nt - 1) {
           const int vg = kb + i, vs = vg % VSTAGES;
-          ok = warp_wait(&v_full[vs], (vg / VSTAGES) & 1, abort_flag);
-          if (!ok) break;
+          ok = warp_wait(&v_full[vs], (vg / VSTAGES) & 1, abort_flag, args.wait_limit);
+          if (!ok) {
+            tmem_st_wait();  // this block's P stores, before tensor memory can be freed
+            break;
+          }
           uint8_t* vblk = smem + L::V_OFF + vs * L::KV_TILE;
           const int r0 = w.sk - k0;  // first row past the sequence end
           const int units = (BK - r0) * L::CHUNKS * 8;  // 16-byte units to clear
@@ -791,7 +772,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const bool has_keys = nt > 0;
       if (has_keys) {
-        ok = warp_wait(&o_full[t], nf & 1, abort_flag);
+        ok = warp_wait(&o_full[t], nf & 1, abort_flag, args.wait_limit);
         ++nf;
         if (!ok) break;
       }
@@ -863,14 +844,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  // The driver entry point is process-wide; a function-local static is
+  // initialised once, thread-safely.
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    cudaGetLastError();
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -897,8 +881,8 @@ static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk
   using L = Layout<D>;
   static_assert(L::SMEM_BYTES <= 232448, "shared memory budget");
   auto kern = prefill_fwd_kernel<D, EMU8, PAGED>;
-  static int state = 0;  // 0 = unchecked, 1 = ready, -1 = unusable
-  if (state == 0) {
+  static DeviceOnce setup;
+  const attn_status_t st = setup.run([&]() -> attn_status_t {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
       cudaGetLastError();
@@ -906,17 +890,14 @@ static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk
     }
     // The in-kernel register split assumes exactly REG_LAUNCH registers per
     // thread at launch; anything else could make setmaxnreg.inc wait forever.
-    if (fa.numRegs != REG_LAUNCH) {
-      state = -1;
-    } else if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES) !=
-               cudaSuccess) {
+    if (fa.numRegs != REG_LAUNCH) return ATTN_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES) != cudaSuccess) {
       cudaGetLastError();
       return ATTN_ERR_CUDA;
-    } else {
-      state = 1;
     }
-  }
-  if (state != 1) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+  });
+  if (st != ATTN_OK) return st;
   const int grid = items < device_sm_count() ? items : device_sm_count();
   Args ak = a;
   // Sort only when lengths vary per sequence and every CTA's share fits its list.
@@ -992,6 +973,7 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
                 : 0;
   if (!a.o_tma) to = tq;  // never read
   a.error_flags = p.error_flags;
+  a.wait_limit = pipeline_wait_limit();
   if (paged) {
     a.block_table = p.block_table;
     a.max_blocks = p.max_blocks_per_seq;

@@ -65,6 +65,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Cycle bound of the drain waits below (~1 s at 2 GHz).
+constexpr long long DRAIN_LIMIT = 2000000000LL;
+
+// A wait for work that is already in flight and completes by itself (a TMA
+// copy that was issued, or the MMAs tracked by a commit). Used on the way out
+// of a kernel, abort path included: it ignores the abort flag, so a CTA never
+// frees tensor memory or exits while its copies or MMAs still run. Bounded by
+// DRAIN_LIMIT all the same; returns false if that ran out.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > DRAIN_LIMIT) return false;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (no multicast)
 // ---------------------------------------------------------------------------

@@ -56,8 +56,8 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = 2,   /* head_dim not 64/128, Hq % Hkv != 0, misaligned pointer/stride */
   ATTN_ERR_WORKSPACE = 3,     /* workspace too small; *workspace_needed says how much */
   ATTN_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
-  ATTN_ERR_DEVICE_FAULT = 5,  /* reserved for callers mapping error_flags to a status */
-  ATTN_ERR_TIMEOUT = 6,       /* reserved for callers mapping error_flags to a status */
+  ATTN_ERR_DEVICE_FAULT = 5,  /* error_flags holds a fault bit other than ATTN_FAULT_TIMEOUT (attn_sync_error_flags) */
+  ATTN_ERR_TIMEOUT = 6,       /* error_flags holds ATTN_FAULT_TIMEOUT (attn_sync_error_flags) */
   ATTN_ERR_NO_DEVICE = 7      /* no sm_100 device is current */
 } attn_status_t;
 
@@ -67,6 +67,7 @@ typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1, ATTN_DTYPE_FP8_E4M3 = 2 
 #define ATTN_FAULT_TIMEOUT 0x1      /* a pipeline wait exceeded its bound; the tile was abandoned */
 #define ATTN_FAULT_BAD_BLOCK 0x2    /* a block-table entry was outside [0, num_blocks) */
 #define ATTN_FAULT_BAD_LENGTH 0x4   /* a sequence length exceeded its block table or was negative */
+#define ATTN_FAULT_PREFIX_MISMATCH 0x8 /* attn_decode_paged_shared_prefix: a table row's prefix blocks differ from row 0's */
 
 /*
  * Prefill: tiled attention over a whole query block, one pass over K/V with
@@ -285,7 +286,10 @@ ATTN_API attn_status_t attn_prefill_backward(const attn_backward_params* p, void
  *
  * The prefix's keys/values are the blocks listed first in sequence 0's table,
  * block_table[0][0 .. prefix_len / 16); the other sequences' entries for
- * those positions are not read (they normally alias the same blocks). Each
+ * those positions must alias the same blocks. They are only compared with
+ * row 0's: a row that lists different blocks there sets
+ * ATTN_FAULT_PREFIX_MISMATCH in error_flags, and its prefix is still taken
+ * from row 0 (the result does not depend on those entries). Each
  * sequence b continues with its own blocks block_table[b][prefix_len / 16 ..]
  * up to seq_lens[b] keys. The result is what attn_decode_paged returns when
  * every sequence's first prefix_len keys/values are sequence 0's, up to fp32
@@ -330,6 +334,9 @@ ATTN_API attn_status_t attn_decode_paged_shared_prefix(const attn_decode_params*
  * device, with that device current); make that first call before any stream
  * capture. All calls share the one array: calls whose kernels overlap on the
  * GPU, e.g. on two streams, race and must be serialised by the caller.
+ * The looked-up address stays cached for the life of the process: after
+ * cudaDeviceReset on a device, this call must not be used on that device
+ * again (the cached address would point into the destroyed context).
  */
 ATTN_API attn_status_t attn_decode_paged_noalloc(const attn_decode_params* p, attn_stream_t stream);
 
@@ -350,6 +357,40 @@ ATTN_API attn_status_t attn_decode_paged_noalloc(const attn_decode_params* p, at
 ATTN_API attn_status_t splitkv_lse_combine(const float* part_o, const float* part_lse, int num_splits, int rows,
                                   int head_dim, const int32_t* splits_per_row, void* out_o,
                                   attn_dtype_t out_dtype, float* out_lse, attn_stream_t stream);
+
+/*
+ * Error word helpers. The kernels OR ATTN_FAULT_* bits into a caller's
+ * error_flags word instead of aborting; these turn the word into a status.
+ * attn_status_from_flags: ATTN_ERR_TIMEOUT if ATTN_FAULT_TIMEOUT is set, else
+ * ATTN_ERR_DEVICE_FAULT if any bit is set, else ATTN_OK.
+ * attn_sync_error_flags: waits for `stream` (cudaStreamSynchronize), copies
+ * the device word error_flags to *flags_out (nullable, host) and returns
+ * attn_status_from_flags of it; ATTN_ERR_INVALID_ARG for a NULL word,
+ * ATTN_ERR_CUDA if the copy or the synchronisation failed. The word is left
+ * as it is (the caller clears it before reusing it).
+ */
+ATTN_API attn_status_t attn_status_from_flags(int32_t flags);
+ATTN_API attn_status_t attn_sync_error_flags(const int32_t* error_flags, attn_stream_t stream, int32_t* flags_out);
+
+/*
+ * Diagnostics (not part of the method; for tests and bring-up).
+ *
+ * attn_set_wait_limit: the clock-cycle bound of every pipeline wait in the
+ * prefill and backward kernels launched after the call (process-wide;
+ * cycles <= 0 restores the default of 2e9 cycles, about one second). A wait
+ * that runs out makes its CTA stop, wait for the copies and tensor-core
+ * products it already issued (those waits keep their own ~1 s bound), free
+ * its tensor memory and OR ATTN_FAULT_TIMEOUT into error_flags; the outputs of
+ * that call are then undefined. A tiny bound exercises that path on purpose.
+ *
+ * attn_selftest_exp2: y_poly[i] = the prefill kernel's FMA-pipe 2^x[i] (a
+ * cubic on the reduced argument; relative error about 7.5e-5 for x in
+ * [-125, 127], inputs below -126 clamped to -126) and, if y_mufu is not NULL,
+ * y_mufu[i] = the MUFU ex2.approx.ftz result, for 0 <= i < n. x, y_poly,
+ * y_mufu: device fp32 arrays of n elements. Asynchronous on `stream`.
+ */
+ATTN_API void attn_set_wait_limit(long long cycles);
+ATTN_API attn_status_t attn_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int n, attn_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 ATTN_API const char* attn_status_string(attn_status_t status);

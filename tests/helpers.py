@@ -29,13 +29,15 @@ def bf16_half_ulp(x):
 
 
 def assert_o_close(o_gpu, o_ref, bf16_out: bool, what=""):
-    """|dO| <= 1e-2 (fp32 output); bf16 output adds its own rounding half-ulp."""
+    """|dO| <= 1e-2 on fp32 output; on bf16 output |dO| <= max(1e-2, half a bf16
+    ulp of the reference value), since for |O| >= 4 the correctly rounded bf16
+    value alone can be 0.0156 away."""
     o_gpu = np.asarray(o_gpu, dtype=np.float64)
     o_ref = np.asarray(o_ref, dtype=np.float64)
     assert o_gpu.shape == o_ref.shape, (o_gpu.shape, o_ref.shape)
     assert np.isfinite(o_gpu).all(), f"{what}: non-finite output"
     err = np.abs(o_gpu - o_ref)
-    tol = TOL_O + (bf16_half_ulp(o_ref) if bf16_out else 0.0)
+    tol = np.maximum(TOL_O, bf16_half_ulp(o_ref)) if bf16_out else TOL_O
     bad = err > tol
     assert not bad.any(), (f"{what}: max|dO|={err.max():.3g} at {np.unravel_index(err.argmax(), err.shape)}, "
                            f"{bad.sum()} elements over tolerance")

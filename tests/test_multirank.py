@@ -52,3 +52,30 @@ def test_two_gloo_ranks_take_max_time_and_own_distinct_batches():
     assert res[0][1] == res[1][1] > 0             # same per-rank work (weak scaling)
     digests = res[0][3]
     assert digests[0] != digests[1]               # each rank generated its own batch
+
+
+def _bench(*argv, env=None):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    e = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    e.update(env or {})
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *argv], capture_output=True, text=True,
+                       env=e, timeout=300)
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return r.returncode, (json.loads(lines[-1]) if lines else None), r.stdout + r.stderr
+
+
+def test_bench_starts_its_own_ranks():
+    """`bench.py --gpus 2` outside torchrun launches two ranks itself (gloo on a
+    CPU-only host); rank 0 alone prints one line, which counts both ranks."""
+    rc, line, log = _bench("--gpus", "2", "--only", "launcher", "--steps", "3", "--warmup", "3")
+    assert rc == 0, log
+    assert line is not None and line["n_gpus"] == 2, log
+    assert log.count('"n_gpus"') == 1, log
+
+
+def test_bench_refuses_a_rank_count_that_does_not_match():
+    rc, line, log = _bench("--gpus", "2", "--only", "launcher", env={"WORLD_SIZE": "1", "RANK": "0"})
+    assert rc != 0 and line is None, log

@@ -118,17 +118,18 @@ def test_paged_bad_block_is_flagged(lib):
     assert np.isfinite(o).all()
 
 
-def _mixed_run(lib, d, cfg):
+def _mixed_run(lib, d, cfg, out_dtype=None):
     """One step of the mixed batch: paged prefill of the chunks, then decode of the rest."""
     import torch
+    out_dtype = out_dtype or torch.float32
     kc, vc = to_dev_bf16(d["k_pool"]), to_dev_bf16(d["v_pool"])
     table = to_dev_i32(d["block_table"])
     lens = to_dev_i32(d["kv_lens"])
     nc = cfg.chunks
     o_p, l_p = lib.prefill_paged(to_dev_bf16(d["q_chunk"]), kc, vc, table[:nc], lens[:nc], None, cfg.scale, True,
-                                 out_dtype=torch.float32)
+                                 out_dtype=out_dtype)
     o_d, l_d = lib.decode_paged(to_dev_bf16(d["q_dec"]), kc, vc, table[nc:].contiguous(), lens[nc:].contiguous(),
-                                cfg.scale, max_seq_len=int(d["kv_lens"][nc:].max()), out_dtype=torch.float32)
+                                cfg.scale, max_seq_len=int(d["kv_lens"][nc:].max()), out_dtype=out_dtype)
     torch.cuda.synchronize()
     return to_f64(o_p), to_f64(l_p), to_f64(o_d), to_f64(l_d)
 
@@ -148,21 +149,24 @@ def test_mixed_batch_small(lib):
     assert_lse_close(l_d, Ld, "mixed decode")
 
 
-def test_mixed_full_size_sampled_rows(lib):
-    """8 chunks x 512 queries on context U[0, 8192] + 128 decode rows on U[512, 16384]."""
+def test_mixed_full_size_every_row(lib):
+    """8 chunks x 512 queries on context U[0, 8192] + 128 decode rows on
+    U[512, 16384]: every prefill row and every decode row against the oracle
+    (fp32 output, strict bound), then the bench's bf16-output step."""
+    import torch
+    from tests.oracle_all_rows import decode_all_rows, prefill_paged_all_rows
     cfg = wl.MIXED
     d = wl.make_mixed(cfg)
-    o_p, l_p, o_d, l_d = _mixed_run(lib, d, cfg)
-    assert np.isfinite(o_p).all() and np.isfinite(o_d).all()
-    rng = np.random.default_rng(1)
     nc = cfg.chunks
-    rows = [(b, int(rng.integers(cfg.q_heads)), int(i)) for b in range(nc) for i in (0, 511, rng.integers(512))]
-    Op, Lp = ref.ref_prefill_paged(d["q_chunk"], [cfg.chunk_len] * nc, d["k_pool"], d["v_pool"],
-                                   d["block_table"][:nc], d["kv_lens"][:nc], cfg.scale, True, rows=rows)
-    assert_o_close(np.stack([o_p[b, h, i] for b, h, i in rows]), Op, False, "mixed prefill rows")
-    assert_lse_close(np.array([l_p[b, h, i] for b, h, i in rows]), Lp, "mixed prefill rows")
-    drows = [(b, int(rng.integers(cfg.q_heads))) for b in range(0, cfg.decodes, 4)]
-    Od, Ld = ref.ref_decode_paged(d["q_dec"], d["k_pool"], d["v_pool"], d["block_table"][nc:], d["kv_lens"][nc:],
-                                  cfg.scale, rows=drows)
-    assert_o_close(np.stack([o_d[b, h] for b, h in drows]), Od, False, "mixed decode rows")
-    assert_lse_close(np.array([l_d[b, h] for b, h in drows]), Ld, "mixed decode rows")
+    Op, Lp = prefill_paged_all_rows(d["q_chunk"], np.full(nc, cfg.chunk_len, dtype=np.int32), d["k_pool"],
+                                    d["v_pool"], d["block_table"][:nc], d["kv_lens"][:nc], cfg.scale, True)
+    Od, Ld = decode_all_rows(d["q_dec"], d["k_pool"], d["v_pool"], d["block_table"][nc:], d["kv_lens"][nc:],
+                             cfg.scale)
+    o_p, l_p, o_d, l_d = _mixed_run(lib, d, cfg)
+    assert_o_close(o_p, Op, False, "mixed prefill")
+    assert_lse_close(l_p, Lp, "mixed prefill")
+    assert_o_close(o_d, Od, False, "mixed decode")
+    assert_lse_close(l_d, Ld, "mixed decode")
+    o_p, l_p, o_d, l_d = _mixed_run(lib, d, cfg, out_dtype=torch.bfloat16)
+    assert_o_close(o_p, Op, True, "mixed prefill bf16 out")
+    assert_o_close(o_d, Od, True, "mixed decode bf16 out")

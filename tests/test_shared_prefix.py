@@ -124,14 +124,25 @@ def test_shared_prefix_decode_matches_oracle(lib, batch, G, prefix_len, lo, hi):
 
 
 def test_shared_prefix_reads_only_sequence_zero_prefix_entries(lib):
-    """Other sequences' table entries for the prefix positions are not read:
-    pointing them at a NaN spare block changes no bit of the result."""
+    """The prefix is read from sequence 0's table entries only: pointing the
+    other sequences' prefix entries at a NaN spare block changes no bit of the
+    result, and the mismatch is flagged (ATTN_FAULT_PREFIX_MISMATCH); aliased
+    entries leave the error word clear."""
+    import torch
     d = _prefix_inputs(9, 4, 640, 0, 500, seed=90)
-    o1, l1 = _cascade(lib, d)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o1, l1 = _cascade(lib, d, flags=flags)
+    assert int(flags.item()) == 0
     table = d["block_table"].copy()
     table[1:, :640 // 16] = d["spare_ids"][0]
-    o2, l2 = _cascade(lib, d, table=table)
+    o2, l2 = _cascade(lib, d, table=table, flags=flags)
+    assert int(flags.item()) == lib.ATTN_FAULT_PREFIX_MISMATCH
     assert np.isfinite(o2).all() and np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    flags.zero_()
+    table = d["block_table"].copy()
+    table[8, 639 // 16] = d["spare_ids"][1]  # one entry of the last row, the last prefix block
+    _cascade(lib, d, table=table, flags=flags)
+    assert int(flags.item()) == lib.ATTN_FAULT_PREFIX_MISMATCH
 
 
 def test_shared_prefix_filling_the_whole_table(lib):
@@ -216,16 +227,13 @@ def test_shared_prefix_graph_replay(lib):
         assert_lse_close(to_f64(l_s), L_ref, f"replay {it}")
 
 
-def test_shared_prefix_full_size_sampled_rows(lib):
+def test_shared_prefix_full_size_every_row(lib):
     """The bench's shared-prefix shape (64 sequences, 8192 shared tokens plus
-    64..2048 own tokens, 32/8 heads), checked on sampled rows."""
+    64..2048 own tokens, 32/8 heads), every row against the oracle."""
+    from tests.oracle_all_rows import decode_all_rows
     cfg = wl.SHARED_PREFIX_DECODE
     d = wl.make_shared_prefix_decode(cfg)
+    O_ref, L_ref = decode_all_rows(d["q"], d["k_pool"], d["v_pool"], d["block_table"], d["kv_lens"], d["scale"])
     o, lse = _cascade(lib, d)
-    rng = np.random.default_rng(97)
-    rows = [(0, 0), (cfg.batch - 1, cfg.q_heads - 1)] + [
-        (int(rng.integers(cfg.batch)), int(rng.integers(cfg.q_heads))) for _ in range(30)]
-    O_ref, L_ref = ref.ref_decode_paged(d["q"], d["k_pool"], d["v_pool"], d["block_table"], d["kv_lens"],
-                                        d["scale"], rows=rows)
-    assert_o_close(np.stack([o[b, h] for b, h in rows]), O_ref, False, "shared prefix full size")
-    assert_lse_close(np.array([lse[b, h] for b, h in rows]), L_ref, "shared prefix full size lse")
+    assert_o_close(o, O_ref, False, "shared prefix full size")
+    assert_lse_close(lse, L_ref, "shared prefix full size lse")

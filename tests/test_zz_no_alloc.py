@@ -38,6 +38,40 @@ def test_noalloc_decode_matches_workspace_decode_twice(lib):
 
 
 @pytest.mark.gpu
+def test_noalloc_after_a_larger_plan_and_without_allocating(lib):
+    """A call with more splits over longer sequences leaves its partials in the
+    shared array; a smaller call right after must not read any of them. Around
+    that call neither torch's allocator nor the device's free memory moves."""
+    import torch
+    big_lens = np.array([30000, 17, 25000, 9000, 31000, 1], dtype=np.int32)
+    small_lens = np.array([300, 1, 2000, 64, 65, 1000], dtype=np.int32)
+    cfg = wl.DecodeConfig("noalloc2", 6, 32, 8, 128, 1, 1, 22)
+    d_big = wl.make_decode(cfg, kv_lens=big_lens)
+    d_small = wl.make_decode(wl.DecodeConfig("noalloc3", 6, 32, 8, 128, 1, 1, 23), kv_lens=small_lens)
+    dev = {k: (to_dev_bf16(v) if k in ("q", "k_pool", "v_pool") else to_dev_i32(v))
+           for k, v in d_big.items() if k in ("q", "k_pool", "v_pool", "block_table", "kv_lens")}
+    small = {k: (to_dev_bf16(v) if k in ("q", "k_pool", "v_pool") else to_dev_i32(v))
+             for k, v in d_small.items() if k in ("q", "k_pool", "v_pool", "block_table", "kv_lens")}
+    out_big = torch.empty((6, 32, 128), dtype=torch.float32, device="cuda")
+    lib.decode_paged_noalloc(dev["q"], dev["k_pool"], dev["v_pool"], dev["block_table"], dev["kv_lens"], out_big,
+                             None, cfg.scale, max_seq_len=int(big_lens.max()), num_splits=32)
+    ref_o, ref_l = lib.decode_paged(small["q"], small["k_pool"], small["v_pool"], small["block_table"],
+                                    small["kv_lens"], cfg.scale, max_seq_len=int(small_lens.max()), num_splits=3,
+                                    out_dtype=torch.float32)
+    out = torch.full((6, 32, 128), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((6, 32), float("nan"), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    allocated, (free, _) = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()
+    lib.decode_paged_noalloc(small["q"], small["k_pool"], small["v_pool"], small["block_table"], small["kv_lens"],
+                             out, lse, cfg.scale, max_seq_len=int(small_lens.max()), num_splits=3)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == allocated
+    assert torch.cuda.mem_get_info()[0] == free
+    assert_o_close(to_f64(out), to_f64(ref_o), False, "noalloc after a larger plan")
+    assert_lse_close(to_f64(lse), to_f64(ref_l), "noalloc after a larger plan")
+
+
+@pytest.mark.gpu
 def test_noalloc_rejects_a_plan_larger_than_its_array(lib):
     import torch
     B, Hq, Hkv = 512, 64, 8

@@ -614,7 +614,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           return true;
         };
         ok = mbar_wait_bounded(q_full, nq & 1, abort_flag, args.wait_limit);
-        if (ok) ok = s_blocks(0);
+        if (ok && n_kv == 0) {
+          // Every row of the item sees no key: no K/V block was loaded and no
+          // MMA reads Q. Hand the Q buffer back at once (the epilogue writes
+          // O = 0 and LSE = -inf without tensor memory).
+          mma_commit(q_empty);
+        } else if (ok) {
+          ok = s_blocks(0);
+        }
         for (int i = 0; i < n_kv && ok; ++i) {
           const int vg = kb + i;  // V_i is the (kb + i)-th V block
           ok = mbar_wait_bounded(&v_full[vg % VSTAGES], (vg / VSTAGES) & 1, abort_flag, args.wait_limit);

@@ -26,12 +26,18 @@ def _chunks(ctx, q_len, Hq, Hkv, D, seed, identity=False):
 
 
 def _run(lib, d, out_dtype=None, flags=None, table=None):
+    """One paged prefill call; without a caller's error word, its own must stay clear."""
     import torch
+    own = flags is None
+    if own:
+        flags = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, lse = lib.prefill_paged(to_dev_bf16(d["q"]), to_dev_bf16(d["k_pool"]), to_dev_bf16(d["v_pool"]),
                                to_dev_i32(d["block_table"] if table is None else table), to_dev_i32(d["kv_lens"]),
                                to_dev_i32(d["q_lens"]), d["scale"], True, out_dtype=out_dtype or torch.float32,
                                error_flags=flags)
     torch.cuda.synchronize()
+    if own:
+        assert lib.sync_error_flags(flags) == (lib.ATTN_OK, 0)
     return to_f64(o), to_f64(lse)
 
 

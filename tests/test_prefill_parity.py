@@ -15,10 +15,15 @@ pytestmark = pytest.mark.gpu
 
 
 def _run(lib, d, out_dtype=None, **kw):
+    """One prefill call; its error word must stay clear (no block, length or
+    timeout fault: a wait that ran out would still leave a correct-looking O)."""
     import torch
     q, k, v = to_dev_bf16(d["q"]), to_dev_bf16(d["k"]), to_dev_bf16(d["v"])
-    o, lse = lib.prefill(q, k, v, d["scale"], d["causal"], out_dtype=out_dtype or torch.bfloat16, **kw)
-    torch.cuda.synchronize()
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = lib.prefill(q, k, v, d["scale"], d["causal"], out_dtype=out_dtype or torch.bfloat16, error_flags=flags,
+                         **kw)
+    status, word = lib.sync_error_flags(flags)
+    assert word == 0 and status == lib.ATTN_OK, f"error word {word:#x}"
     return to_f64(o), to_f64(lse)
 
 
@@ -71,8 +76,9 @@ def test_no_keys_gives_zero_and_minus_inf(lib):
     d["v"] = d["v"][:, :, :0]
     q = to_dev_bf16(d["q"])
     k = torch.empty((1, 1, 0, 128), dtype=torch.bfloat16, device="cuda")
-    o, lse = lib.prefill(q, k, k, d["scale"], False, out_dtype=torch.float32)
-    torch.cuda.synchronize()
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = lib.prefill(q, k, k, d["scale"], False, out_dtype=torch.float32, error_flags=flags)
+    assert lib.sync_error_flags(flags) == (lib.ATTN_OK, 0)
     assert (to_f64(o) == 0).all() and np.isneginf(to_f64(lse)).all()
 
 
@@ -111,8 +117,10 @@ def test_dense_varlen_padded_batch(lib, Hq, Hkv, D, causal):
     q, k, v = to_dev_bf16(d["q"]), to_dev_bf16(d["k"]), to_dev_bf16(d["v"])
     out = torch.full((B, Hq, Sq, D), 7.0, dtype=torch.float32, device="cuda")
     lse = torch.full((B, Hq, Sq), 7.0, dtype=torch.float32, device="cuda")
-    lib.prefill(q, k, v, d["scale"], causal, out=out, lse=lse, seqlens_q=to_dev_i32(lq), seqlens_k=to_dev_i32(lk))
-    torch.cuda.synchronize()
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lib.prefill(q, k, v, d["scale"], causal, out=out, lse=lse, seqlens_q=to_dev_i32(lq), seqlens_k=to_dev_i32(lk),
+                error_flags=flags)
+    assert lib.sync_error_flags(flags) == (lib.ATTN_OK, 0)
     o, l = to_f64(out), to_f64(lse)
     for b in range(B):
         nq, nk = int(lq[b]), min(int(lk[b]), Sk)

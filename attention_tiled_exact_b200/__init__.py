@@ -11,6 +11,8 @@ step of the computation runs in its CUDA kernels):
 * :func:`decode_paged_shared_prefix` -- decode of a batch sharing a prefix,
   which is attended once per batch (:func:`decode_shared_prefix_workspace_bytes`);
 * :func:`decode_paged_noalloc` -- decode for callers that cannot allocate;
+* :class:`PersistentDecode` -- a resident decode kernel driven step by step;
+* :class:`DecodeGraphPool` -- CUDA graphs of the decode step per static shape;
 * :func:`splitkv_lse_combine` -- log-sum-exp merge of split partials;
 * :func:`sync_error_flags` / :func:`status_from_flags` -- the device error
   word as a status.
@@ -22,6 +24,7 @@ fallback.
 _API = ("prefill", "prefill_paged", "prefill_backward", "decode_paged", "decode_workspace_bytes",
         "decode_paged_shared_prefix", "decode_shared_prefix_workspace_bytes", "decode_paged_noalloc",
         "splitkv_lse_combine", "sync_error_flags", "status_from_flags", "set_wait_limit", "selftest_exp2",
+        "PersistentDecode", "DecodeGraphPool",
         "AttnError", "library_path", "status_string")
 
 

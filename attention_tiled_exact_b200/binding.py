@@ -88,6 +88,13 @@ class DecodeParams(ctypes.Structure):
     ]
 
 
+class PersistentCmd(ctypes.Structure):
+    """Mirror of ``attn_persistent_cmd`` (host memory shared with the persistent kernel)."""
+
+    _fields_ = [("seq", _i32), ("batch", _i32), ("max_seq_len", _i32), ("stop", _i32), ("done", _i32),
+                ("status", _i32), ("running", _i32), ("reserved", _i32)]
+
+
 def _load():
     if not os.path.exists(_LIB_FILE):
         raise ImportError(f"{_LIB_FILE} is missing: build it with "
@@ -121,6 +128,28 @@ def _load():
     lib.attn_set_wait_limit.restype = None
     lib.attn_selftest_exp2.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp]
     lib.attn_selftest_exp2.restype = ctypes.c_int
+    lib.attn_decode_persistent_workspace.argtypes = [ctypes.POINTER(DecodeParams), ctypes.POINTER(ctypes.c_size_t)]
+    lib.attn_decode_persistent_workspace.restype = ctypes.c_int
+    lib.attn_decode_persistent_launch.argtypes = [ctypes.POINTER(DecodeParams), _vp, _vp, ctypes.c_size_t,
+                                                  ctypes.c_longlong, _vp]
+    lib.attn_decode_persistent_launch.restype = ctypes.c_int
+    lib.attn_decode_persistent_submit.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
+    lib.attn_decode_persistent_submit.restype = ctypes.c_int
+    lib.attn_decode_persistent_wait.argtypes = [_vp, ctypes.c_int32, ctypes.c_longlong]
+    lib.attn_decode_persistent_wait.restype = ctypes.c_int
+    lib.attn_decode_persistent_stop.argtypes = [_vp]
+    lib.attn_decode_persistent_stop.restype = None
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lib.attn_decode_graph_pool_workspace.argtypes = [ctypes.POINTER(DecodeParams), i32p, ctypes.c_int, i32p,
+                                                     ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+    lib.attn_decode_graph_pool_workspace.restype = ctypes.c_int
+    lib.attn_decode_graph_pool_create.argtypes = [ctypes.POINTER(DecodeParams), i32p, ctypes.c_int, i32p,
+                                                  ctypes.c_int, _vp, ctypes.c_size_t, ctypes.POINTER(_vp)]
+    lib.attn_decode_graph_pool_create.restype = ctypes.c_int
+    lib.attn_decode_graph_pool_replay.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, i32p, i32p]
+    lib.attn_decode_graph_pool_replay.restype = ctypes.c_int
+    lib.attn_decode_graph_pool_destroy.argtypes = [_vp]
+    lib.attn_decode_graph_pool_destroy.restype = None
     return lib
 
 
@@ -503,3 +532,122 @@ def splitkv_lse_combine(part_o, part_lse, splits_per_row=None, out=None, out_lse
                                    _out_code(out.dtype), _ptr(out_lse), _stream(part_o.device)),
            "splitkv_lse_combine")
     return out, out_lse
+
+
+# ----------------------------------------------------------------------------
+# persistent decode and the decode graph pool
+# ----------------------------------------------------------------------------
+
+
+class PersistentDecode:
+    """A resident decode kernel driven step by step from the host.
+
+    The tensors are the static buffers every step reads and writes (as for
+    :func:`decode_paged`; ``out`` and, optionally, ``lse`` are written). The
+    buffers hold up to ``q.shape[0]`` sequences; ``max_seq_len`` bounds every
+    step's lengths (0: the table capacity). The kernel is launched on
+    ``stream`` (a non-blocking torch stream by default) and runs until
+    :meth:`stop`, or until ``idle_cycles`` SM cycles pass without a step.
+    While it runs it holds every SM, so kernels of other streams wait; fill
+    the static buffers with copies (copy engines), not kernels.
+    """
+
+    def __init__(self, q, k_cache, v_cache, block_table, seq_lens, out, lse=None, scale=None, max_seq_len=0,
+                 num_splits=0, idle_cycles=2_000_000_000, error_flags=None, k_scale=None, v_scale=None,
+                 stream=None):
+        _check_decode_inputs(q, k_cache, v_cache, block_table, seq_lens)
+        _need(out is not None and tuple(out.shape) == tuple(q.shape) and out.is_contiguous(), "out [B, Hq, D]")
+        self._keep = (q, k_cache, v_cache, block_table, seq_lens, out, lse, error_flags)
+        self.params = _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, max_seq_len, num_splits,
+                                     out, lse, error_flags, k_scale, v_scale)
+        need = ctypes.c_size_t(0)
+        _check(LIB.attn_decode_persistent_workspace(ctypes.byref(self.params), ctypes.byref(need)),
+               "attn_decode_persistent_workspace")
+        self.workspace = torch.empty(max(int(need.value), 256), dtype=torch.uint8, device=q.device)
+        self.cmd_buf = torch.zeros(ctypes.sizeof(PersistentCmd) // 4, dtype=torch.int32, pin_memory=True)
+        self.cmd = PersistentCmd.from_address(self.cmd_buf.data_ptr())
+        self.stream = stream if stream is not None else torch.cuda.Stream(device=q.device)
+        self._cmd_ptr = ctypes.c_void_p(self.cmd_buf.data_ptr())
+        _check(LIB.attn_decode_persistent_launch(ctypes.byref(self.params), self._cmd_ptr, _ptr(self.workspace),
+                                                 self.workspace.numel(), int(idle_cycles),
+                                                 ctypes.c_void_p(self.stream.cuda_stream)),
+               "attn_decode_persistent_launch")
+
+    def submit(self, batch: int, max_seq_len: int = 0) -> int:
+        """Start a step over the first ``batch`` sequences of the static buffers; returns its number."""
+        step = ctypes.c_int32(0)
+        _check(LIB.attn_decode_persistent_submit(self._cmd_ptr, int(batch), int(max_seq_len), ctypes.byref(step)),
+               "attn_decode_persistent_submit")
+        return int(step.value)
+
+    def wait(self, step: int, timeout_s: float = 10.0) -> None:
+        """Block the host until step ``step`` is complete (its outputs are in HBM)."""
+        _check(LIB.attn_decode_persistent_wait(self._cmd_ptr, int(step), int(timeout_s * 1e6)),
+               "attn_decode_persistent_wait")
+
+    def step(self, batch: int, max_seq_len: int = 0, timeout_s: float = 10.0) -> int:
+        s = self.submit(batch, max_seq_len)
+        self.wait(s, timeout_s)
+        return s
+
+    @property
+    def status(self) -> int:
+        return int(self.cmd.status)
+
+    @property
+    def running(self) -> bool:
+        return bool(self.cmd.running)
+
+    def stop(self) -> None:
+        """Ask the kernel to exit and wait for its stream."""
+        LIB.attn_decode_persistent_stop(self._cmd_ptr)
+        self.stream.synchronize()
+
+
+class DecodeGraphPool:
+    """CUDA graphs of the decode step, one per (batch bucket, length bucket).
+
+    The tensors are the static buffers every replay reads and writes (as for
+    :func:`decode_paged`); the buckets are ascending lists. :meth:`replay`
+    launches the smallest bucket covering a step on the current stream; rows
+    of the static buffers past the step's batch must keep seq_lens 0.
+    """
+
+    def __init__(self, q, k_cache, v_cache, block_table, seq_lens, out, lse, batch_buckets, len_buckets,
+                 scale=None, num_splits=0, error_flags=None, k_scale=None, v_scale=None):
+        _check_decode_inputs(q, k_cache, v_cache, block_table, seq_lens)
+        _need(out is not None and tuple(out.shape) == tuple(q.shape) and out.is_contiguous(), "out [B, Hq, D]")
+        self._keep = (q, k_cache, v_cache, block_table, seq_lens, out, lse, error_flags)
+        self.params = _decode_params(q, k_cache, v_cache, block_table, seq_lens, scale, 0, num_splits, out, lse,
+                                     error_flags, k_scale, v_scale)
+        bb = (ctypes.c_int32 * len(batch_buckets))(*batch_buckets)
+        lb = (ctypes.c_int32 * len(len_buckets))(*len_buckets)
+        need = ctypes.c_size_t(0)
+        _check(LIB.attn_decode_graph_pool_workspace(ctypes.byref(self.params), bb, len(batch_buckets), lb,
+                                                    len(len_buckets), ctypes.byref(need)),
+               "attn_decode_graph_pool_workspace")
+        self.workspace = torch.empty(max(int(need.value), 256), dtype=torch.uint8, device=q.device)
+        handle = ctypes.c_void_p(0)
+        _check(LIB.attn_decode_graph_pool_create(ctypes.byref(self.params), bb, len(batch_buckets), lb,
+                                                 len(len_buckets), _ptr(self.workspace), self.workspace.numel(),
+                                                 ctypes.byref(handle)), "attn_decode_graph_pool_create")
+        self._handle = handle
+
+    def replay(self, batch: int, max_seq_len: int = 0):
+        """Replay the bucket covering (batch, max_seq_len) on the current stream; returns that bucket."""
+        bb, bl = ctypes.c_int32(0), ctypes.c_int32(0)
+        _check(LIB.attn_decode_graph_pool_replay(self._handle, int(batch), int(max_seq_len),
+                                                 _stream(self._keep[0].device), ctypes.byref(bb), ctypes.byref(bl)),
+               "attn_decode_graph_pool_replay")
+        return int(bb.value), int(bl.value)
+
+    def close(self) -> None:
+        if self._handle:
+            LIB.attn_decode_graph_pool_destroy(self._handle)
+            self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

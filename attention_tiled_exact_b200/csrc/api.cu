@@ -5,7 +5,10 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <string.h>
+
 #include <atomic>
+#include <chrono>
 #include <mutex>
 
 #include "attn.h"
@@ -215,6 +218,64 @@ attn_status_t splitkv_lse_combine(const float* part_o, const float* part_lse, in
   if (st != ATTN_OK) return st;
   return attn::launch_combine(part_o, part_lse, num_splits, rows, head_dim, splits_per_row, nullptr, 1, 1, out_o,
                               out_dtype, out_lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_decode_persistent_workspace(const attn_decode_params* p, size_t* bytes) {
+  attn_status_t st = attn::validate_decode(p);
+  if (st != ATTN_OK) return st;
+  if (!bytes) return ATTN_ERR_INVALID_ARG;
+  if (attn::check_device() != ATTN_OK) return ATTN_ERR_NO_DEVICE;  // the size depends on the SM count
+  *bytes = attn::decode_persistent_workspace_bytes(*p);
+  return ATTN_OK;
+}
+
+attn_status_t attn_decode_persistent_launch(const attn_decode_params* p, attn_persistent_cmd* cmd, void* workspace,
+                                            size_t workspace_bytes, long long idle_cycles, attn_stream_t stream) {
+  attn_status_t st = attn::validate_decode(p);
+  if (st != ATTN_OK) return st;
+  if (!cmd || !workspace || p->batch <= 0 || idle_cycles <= 0) return ATTN_ERR_INVALID_ARG;
+  st = attn::check_device();
+  if (st != ATTN_OK) return st;
+  if (workspace_bytes < attn::decode_persistent_workspace_bytes(*p)) return ATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_UNSUPPORTED;
+  // The command block is host memory the device must reach: pinned and mapped.
+  void* dev = nullptr;
+  if (cudaHostGetDevicePointer(&dev, cmd, 0) != cudaSuccess || dev == nullptr) {
+    cudaGetLastError();
+    return ATTN_ERR_INVALID_ARG;
+  }
+  memset(cmd, 0, sizeof(*cmd));
+  std::atomic_thread_fence(std::memory_order_seq_cst);
+  return attn::launch_decode_persistent(*p, reinterpret_cast<int32_t*>(dev), workspace, idle_cycles,
+                                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_decode_persistent_submit(attn_persistent_cmd* cmd, int32_t batch, int32_t max_seq_len,
+                                            int32_t* step) {
+  if (!cmd || batch < 0 || max_seq_len < 0) return ATTN_ERR_INVALID_ARG;
+  const int32_t seq = __atomic_load_n(&cmd->seq, __ATOMIC_ACQUIRE);
+  if (__atomic_load_n(&cmd->done, __ATOMIC_ACQUIRE) != seq) return ATTN_ERR_INVALID_ARG;  // previous step pending
+  __atomic_store_n(&cmd->batch, batch, __ATOMIC_RELAXED);
+  __atomic_store_n(&cmd->max_seq_len, max_seq_len, __ATOMIC_RELAXED);
+  __atomic_store_n(&cmd->seq, seq + 1, __ATOMIC_RELEASE);  // publishes batch and max_seq_len with it
+  if (step) *step = seq + 1;
+  return ATTN_OK;
+}
+
+attn_status_t attn_decode_persistent_wait(const attn_persistent_cmd* cmd, int32_t step, long long timeout_us) {
+  if (!cmd) return ATTN_ERR_INVALID_ARG;
+  const auto t0 = std::chrono::steady_clock::now();
+  while (true) {
+    if (__atomic_load_n(&cmd->done, __ATOMIC_ACQUIRE) >= step) return ATTN_OK;
+    if (__atomic_load_n(&cmd->status, __ATOMIC_ACQUIRE) != 0) return ATTN_ERR_TIMEOUT;  // the kernel gave up
+    const long long us =
+        std::chrono::duration_cast<std::chrono::microseconds>(std::chrono::steady_clock::now() - t0).count();
+    if (us > timeout_us) return ATTN_ERR_TIMEOUT;
+  }
+}
+
+void attn_decode_persistent_stop(attn_persistent_cmd* cmd) {
+  if (cmd) __atomic_store_n(&cmd->stop, 1, __ATOMIC_RELEASE);
 }
 
 void attn_set_wait_limit(long long cycles) {

@@ -163,8 +163,20 @@ __device__ __forceinline__ void load_row8(const uint8_t* row, int c, bool zero, 
 }
 
 // Sequence length clamped to the block table's capacity (flagging a fault).
+// A 32-bit or 16-byte load of an input that the host may rewrite between the
+// steps of the persistent decode kernel (q, the block table, the lengths):
+// there it bypasses L1 (__ldcg), which is not coherent with those writes; the
+// per-launch kernels keep L1 (a block-table entry sits on the path to every
+// copy, and an L1 hit keeps that short).
+template <bool COHERENT, typename T>
+__device__ __forceinline__ T ld_input(const T* p) {
+  if constexpr (COHERENT) return __ldcg(p);
+  return *p;
+}
+
+template <bool COHERENT = false>
 __device__ __forceinline__ int checked_len(const Args& a, int b) {
-  int L = a.seq_lens[b];
+  int L = ld_input<COHERENT>(a.seq_lens + b);
   if (L < 0 || L > a.max_blocks * BS) {
     if (a.error_flags) atomicOr(a.error_flags, ATTN_FAULT_BAD_LENGTH);
     L = L < 0 ? 0 : a.max_blocks * BS;
@@ -187,25 +199,26 @@ __device__ __forceinline__ int checked_len(const Args& a, int b) {
 // j, column n reads element 16 n + j: each thread then gathers its 4 token rows
 // (2t, 2t+1, 2t+8, 2t+9) as 16 contiguous elements and holds the output of
 // head lane / 4 for the 32 contiguous elements 32 (lane % 4) + 0..31.
-template <int G, bool FP8, bool MMA_PV>
-__global__ void __launch_bounds__(WARPS * 32)
-    decode_split_kernel(const Args a) {
+// One (split, kv head, sequence) task of the split-KV decode, by one CTA of
+// WARPS warps (all threads call it together; smem_raw holds Smem<G, FP8>).
+// max_splits is the plan's split count: a longer sequence is cut there.
+template <int G, bool FP8, bool MMA_PV, bool COHERENT = false>
+__device__ __forceinline__ void split_task(const Args& a, int split, int kvh, int b, int max_splits,
+                                           uint8_t* smem_raw) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   constexpr int ELEM = FP8 ? 1 : 2;              // bytes per cache element
   constexpr int ROW = D * ELEM;                  // bytes per cached token row
   constexpr int CHUNKS16 = BS * ROW / (16 * 32);  // 16-byte copies per lane per block
-  extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem<G, FP8>& sm = *reinterpret_cast<Smem<G, FP8>*>(smem_raw);
 
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = warp_id(), lane = lane_id();
   const int hw = lane >> 4, c = lane & 15;  // half-warp, 16-byte chunk of head_dim
 
   const int T = a.split_tokens;
-  int L = checked_len(a, b);
-  if (L > (int)gridDim.x * T) {  // longer than the caller's max_seq_len bound
+  int L = checked_len<COHERENT>(a, b);
+  if (L > max_splits * T) {  // longer than the caller's max_seq_len bound
     if (a.error_flags && split == 0 && threadIdx.x == 0) atomicOr(a.error_flags, ATTN_FAULT_BAD_LENGTH);
-    L = gridDim.x * T;
+    L = max_splits * T;
   }
   const int n_splits = max(1, (L + T - 1) / T);
   if (split >= n_splits) return;
@@ -225,7 +238,7 @@ __global__ void __launch_bounds__(WARPS * 32)
     for (int w = 0; w < 4; ++w) {
       uint4 r = make_uint4(0u, 0u, 0u, 0u);
       if (gq < G)
-        r = *reinterpret_cast<const uint4*>(a.q + ((long long)b * a.hq + kvh * G + gq) * D + 32 * tq + 8 * w);
+        r = ld_input<COHERENT>(reinterpret_cast<const uint4*>(a.q + ((long long)b * a.hq + kvh * G + gq) * D + 32 * tq + 8 * w));
       qa[2 * w][0] = FP8 ? bf16x2_to_f16x2(r.x) : r.x;
       qa[2 * w][1] = FP8 ? bf16x2_to_f16x2(r.y) : r.y;
       qa[2 * w + 1][0] = FP8 ? bf16x2_to_f16x2(r.z) : r.z;
@@ -249,7 +262,7 @@ __global__ void __launch_bounds__(WARPS * 32)
   const int n_mine = (blk_end - blk_begin - warp + WARPS - 1) / WARPS;
   auto block_of = [&](int n) { return blk_begin + warp + n * WARPS; };
   auto phys_of = [&](int blk, bool& valid) {
-    const int ph = table[blk];
+    const int ph = ld_input<COHERENT>(table + blk);
     valid = (ph >= 0) && (ph < a.num_blocks);
     return ph;
   };
@@ -536,6 +549,13 @@ __global__ void __launch_bounds__(WARPS * 32)
   }
 }
 
+template <int G, bool FP8, bool MMA_PV>
+__global__ void __launch_bounds__(WARPS * 32)
+    decode_split_kernel(const Args a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  split_task<G, FP8, MMA_PV>(a, blockIdx.x, blockIdx.y, blockIdx.z, gridDim.x, smem_raw);
+}
+
 }  // namespace decode
 
 // ---------------------------------------------------------------------------
@@ -548,23 +568,20 @@ namespace combine {
 // n = max(1, ceil(L / split_tokens)) from its sequence length; on the decode
 // path rows with n == 1 were written by the decode kernel and are skipped.
 template <int HD>
-__global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restrict__ part_o,
-                                                          const float* __restrict__ part_lse, int num_splits,
-                                                          int rows, const int32_t* __restrict__ splits_per_row,
-                                                          const int32_t* __restrict__ seq_lens, int split_tokens,
-                                                          int max_len, int rows_per_seq, void* out_o, int out_f32,
-                                                          float* out_lse) {
+__device__ __forceinline__ void combine_row(int row, const float* __restrict__ part_o,
+                                            const float* __restrict__ part_lse, int num_splits, int rows,
+                                            const int32_t* __restrict__ splits_per_row,
+                                            const int32_t* __restrict__ seq_lens, int split_tokens, int max_len,
+                                            int rows_per_seq, void* out_o, int out_f32, float* out_lse) {
   constexpr int PER = HD / 32;  // floats per lane
-  const int row = blockIdx.x * (blockDim.x / 32) + warp_id();
   const int lane = lane_id();
-  if (row >= rows) return;
   int n;
   if (splits_per_row) {  // standalone call with per-row counts
-    n = min(max(splits_per_row[row], 0), num_splits);
+    n = min(max(__ldcg(splits_per_row + row), 0), num_splits);
   } else if (seq_lens == nullptr) {  // standalone call: every row has num_splits partials
     n = num_splits;
   } else {  // decode path
-    int L = seq_lens[row / rows_per_seq];
+    int L = __ldcg(seq_lens + row / rows_per_seq);
     L = min(max(L, 0), max_len);
     n = max(1, (L + split_tokens - 1) / split_tokens);
     if (n == 1) return;
@@ -573,7 +590,7 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restric
   constexpr float LOG2E = 1.4426950408889634f;
   // max and sum of exp over the splits, lanes strided over s
   float M = -INFINITY;
-  for (int s = lane; s < n; s += 32) M = fmaxf(M, part_lse[(long long)s * rows + row]);
+  for (int s = lane; s < n; s += 32) M = fmaxf(M, __ldcg(part_lse + (long long)s * rows + row));
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float out[PER];
@@ -582,23 +599,23 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restric
   float lse = -INFINITY;
   if (M != -INFINITY) {
     float sum = 0.f;
-    for (int s = lane; s < n; s += 32) sum += ex2_approx((part_lse[(long long)s * rows + row] - M) * LOG2E);
+    for (int s = lane; s < n; s += 32) sum += ex2_approx((__ldcg(part_lse + (long long)s * rows + row) - M) * LOG2E);
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     lse = M + logf(sum);
     for (int s = 0; s < n; ++s) {
-      const float ls = part_lse[(long long)s * rows + row];
+      const float ls = __ldcg(part_lse + (long long)s * rows + row);
       if (ls == -INFINITY) continue;  // weight 0: its partial is not read
       const float wgt = ex2_approx((ls - lse) * LOG2E);
       const float* src = part_o + ((long long)s * rows + row) * HD + lane * PER;
       if constexpr (PER == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(src));
         out[0] = fmaf(wgt, x.x, out[0]);
         out[1] = fmaf(wgt, x.y, out[1]);
         out[2] = fmaf(wgt, x.z, out[2]);
         out[3] = fmaf(wgt, x.w, out[3]);
       } else {
-        const float2 x = *reinterpret_cast<const float2*>(src);
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
         out[0] = fmaf(wgt, x.x, out[0]);
         out[1] = fmaf(wgt, x.y, out[1]);
       }
@@ -616,6 +633,19 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restric
   if (lane == 0 && out_lse) out_lse[row] = lse;
 }
 
+template <int HD>
+__global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restrict__ part_o,
+                                                          const float* __restrict__ part_lse, int num_splits,
+                                                          int rows, const int32_t* __restrict__ splits_per_row,
+                                                          const int32_t* __restrict__ seq_lens, int split_tokens,
+                                                          int max_len, int rows_per_seq, void* out_o, int out_f32,
+                                                          float* out_lse) {
+  const int row = blockIdx.x * (blockDim.x / 32) + warp_id();
+  if (row >= rows) return;
+  combine_row<HD>(row, part_o, part_lse, num_splits, rows, splits_per_row, seq_lens, split_tokens, max_len,
+                  rows_per_seq, out_o, out_f32, out_lse);
+}
+
 }  // namespace combine
 
 // ---------------------------------------------------------------------------
@@ -626,41 +656,86 @@ static int env_int(const char* name, int dflt) {
   return (e && *e) ? atoi(e) : dflt;
 }
 
-DecodePlan plan_decode(const attn_decode_params& p) {
-  DecodePlan plan;
-  const int cap = p.max_blocks_per_seq * decode::BS;
-  const int max_len = (p.max_seq_len > 0 && p.max_seq_len < cap) ? p.max_seq_len : cap;
-  const int unit = decode::BS * decode::WARPS;  // 64 tokens
+namespace decode {
+
+// Tokens per split (a multiple of 64) and the number of splits a sequence of
+// max_len keys is cut into. num_splits > 0 fixes the count; forced > 0 fixes
+// the tokens; otherwise enough CTAs for many waves (good balance across
+// sequences of mixed lengths) while each split still streams at least 512
+// tokens. The same arithmetic runs on the host (attn_decode_paged) and in the
+// persistent decode kernel, so both cut a step identically.
+__host__ __device__ inline void split_plan(int batch, int hkv, int max_len, int num_splits, int sm_count, int forced,
+                                           int* split_tokens, int* max_splits) {
+  const int unit = BS * WARPS;  // 64 tokens
   int T;
-  const int forced = env_int("ATTN_DECODE_SPLIT_TOKENS", 0);
   if (forced > 0) {
     T = forced;
-  } else if (p.num_splits > 0) {
-    T = (max_len + p.num_splits - 1) / p.num_splits;
+  } else if (num_splits > 0) {
+    T = (max_len + num_splits - 1) / num_splits;
   } else {
-    // Enough CTAs for many waves (good balance across sequences of mixed
-    // lengths) while each split still streams at least 512 tokens.
-    const long long pairs = (long long)p.batch * p.num_kv_heads;
-    const long long target = 32LL * device_sm_count();
-    long long per_seq = (target + pairs - 1) / pairs;
+    const long long pairs = (long long)batch * hkv;
+    const long long target = 32LL * sm_count;
+    long long per_seq = pairs > 0 ? (target + pairs - 1) / pairs : 1;
     if (per_seq < 1) per_seq = 1;
     T = (int)((max_len + per_seq - 1) / per_seq);
     if (T < 512) T = 512;
   }
   T = ((T + unit - 1) / unit) * unit;
   if (T <= 0) T = unit;
-  plan.split_tokens = T;
-  plan.max_splits = max_len > 0 ? (max_len + T - 1) / T : 1;
-  if (plan.max_splits < 1) plan.max_splits = 1;
-  const size_t rows = (size_t)p.batch * p.num_q_heads;
-  size_t bytes = 0;
-  if (plan.max_splits > 1) {
-    const size_t po = plan.max_splits * rows * p.head_dim * sizeof(float);
-    const size_t pl = plan.max_splits * rows * sizeof(float);
-    bytes = ((po + 255) / 256) * 256 + ((pl + 255) / 256) * 256;
+  int n = max_len > 0 ? (max_len + T - 1) / T : 1;
+  *split_tokens = T;
+  *max_splits = n < 1 ? 1 : n;
+}
+
+// Bytes of the partials (O then LSE, each 256-byte aligned) for a plan.
+__host__ __device__ inline size_t partial_bytes(int max_splits, size_t rows, int head_dim, size_t* lse_offset) {
+  if (max_splits <= 1) {
+    if (lse_offset) *lse_offset = 0;
+    return 0;
   }
-  plan.workspace_bytes = bytes;
+  const size_t po = (size_t)max_splits * rows * head_dim * sizeof(float);
+  const size_t pl = (size_t)max_splits * rows * sizeof(float);
+  if (lse_offset) *lse_offset = ((po + 255) / 256) * 256;
+  return ((po + 255) / 256) * 256 + ((pl + 255) / 256) * 256;
+}
+
+}  // namespace decode
+
+DecodePlan plan_decode(const attn_decode_params& p) {
+  DecodePlan plan;
+  const int cap = p.max_blocks_per_seq * decode::BS;
+  const int max_len = (p.max_seq_len > 0 && p.max_seq_len < cap) ? p.max_seq_len : cap;
+  decode::split_plan(p.batch, p.num_kv_heads, max_len, p.num_splits, device_sm_count(),
+                     env_int("ATTN_DECODE_SPLIT_TOKENS", 0), &plan.split_tokens, &plan.max_splits);
+  plan.workspace_bytes =
+      decode::partial_bytes(plan.max_splits, (size_t)p.batch * p.num_q_heads, p.head_dim, nullptr);
   return plan;
+}
+
+// The split kernel's one-time set-up (its shared-memory attribute), once per device.
+template <int G, bool FP8>
+static attn_status_t setup_decode_g() {
+  auto kern = decode::decode_split_kernel<G, FP8, FP8>;  // P V on the tensor cores for FP8 caches
+  const int smem = (int)sizeof(decode::Smem<G, FP8>);
+  static DeviceOnce setup;
+  return setup.run([&]() -> attn_status_t {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+  });
+}
+
+attn_status_t prepare_decode(const attn_decode_params& p) {
+  const bool fp8 = p.kv_dtype == ATTN_DTYPE_FP8_E4M3;
+  switch (p.num_q_heads / p.num_kv_heads) {
+    case 1: return fp8 ? setup_decode_g<1, true>() : setup_decode_g<1, false>();
+    case 2: return fp8 ? setup_decode_g<2, true>() : setup_decode_g<2, false>();
+    case 4: return fp8 ? setup_decode_g<4, true>() : setup_decode_g<4, false>();
+    case 8: return fp8 ? setup_decode_g<8, true>() : setup_decode_g<8, false>();
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
 }
 
 template <int G, bool FP8>
@@ -668,14 +743,7 @@ static attn_status_t launch_decode_g(const decode::Args& a, const DecodePlan& pl
   auto kern = decode::decode_split_kernel<G, FP8, FP8>;  // P V on the tensor cores for FP8 caches
   const int smem = (int)sizeof(decode::Smem<G, FP8>);
   static_assert(sizeof(decode::MergeSmem<G>) <= sizeof(decode::Smem<G, FP8>), "merge buffer fits");
-  static DeviceOnce setup;  // the shared-memory attribute, once per device
-  const attn_status_t st = setup.run([&]() -> attn_status_t {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
-      cudaGetLastError();
-      return ATTN_ERR_CUDA;
-    }
-    return ATTN_OK;
-  });
+  const attn_status_t st = setup_decode_g<G, FP8>();
   if (st != ATTN_OK) return st;
   dim3 grid(plan.max_splits, a.hkv, a.batch);
   kern<<<grid, decode::WARPS * 32, smem, stream>>>(a);
@@ -741,6 +809,285 @@ attn_status_t launch_combine(const float* part_o, const float* part_lse, int num
         part_o, part_lse, num_splits, rows, splits_per_row, seq_lens, split_tokens, max_len, rows_per_seq, out_o,
         out_dtype == ATTN_DTYPE_F32, out_lse);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Persistent decode: one resident kernel runs a stream of decode steps over
+// static buffers, commanded from the host through a block of host memory that
+// is mapped into the device ("GPU Kernel 调度:大模型推理的拐点 2026", Persistent
+// Kernel section: a resident kernel pulls work instead of paying a launch per
+// step). A step is the same computation as attn_decode_paged: the same split
+// plan, the same split task per (split, kv head, sequence) and the same
+// log-sum-exp combine, so its results are bit for bit those of a launch.
+//
+//   * CTA 0 polls the command block (system-scope acquire loads) for the next
+//     step number, or a stop request, and posts the step's batch and length
+//     bound in a mailbox in device memory; the other CTAs wait on the mailbox.
+//   * every CTA takes (split, kv head, sequence) tasks in turn; the CTA whose
+//     split is the last one of its (sequence, kv head) to finish merges that
+//     group's partials (a per-group counter, no grid-wide barrier).
+//   * the last CTA to finish the step writes its number back to the command
+//     block (system-scope release).
+//   * every wait is bounded: with no command for idle_limit cycles (or, for the
+//     other CTAs, no mailbox post for idle_limit + wait_limit) the kernel exits,
+//     raising ATTN_FAULT_TIMEOUT in the command block's status and error_flags.
+// ---------------------------------------------------------------------------
+namespace decode {
+
+// Words of the command block (attn_persistent_cmd) and of the mailbox.
+enum { CMD_SEQ = 0, CMD_BATCH, CMD_MAXLEN, CMD_STOP, CMD_DONE, CMD_STATUS, CMD_RUNNING };
+enum { MB_STEP = 0, MB_BATCH, MB_MAXLEN, MB_STATE, MB_DONE_CTAS, MB_COUNTERS = 8 };
+enum { ST_WAIT = 0, ST_RUN, ST_STOP, ST_IDLE };
+
+struct PersistArgs {
+  Args base;           // static buffers; batch, split_tokens and the partials are set per step
+  int* cmd;            // device address of the host command block
+  float* partials;     // workspace: the partials of the largest step
+  int* sync;           // workspace: mailbox, finished-CTA count, per-(sequence, kv head) counters
+  int max_batch, cap_len, num_splits, sm_count, forced;
+  long long idle_limit, wait_limit;
+};
+
+__device__ __forceinline__ int ld_acquire_sys(const int* p) {
+  int v;
+  asm volatile("ld.acquire.sys.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_sys(int* p, int v) {
+  asm volatile("st.release.sys.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <int G, bool FP8>
+__global__ void __launch_bounds__(WARPS * 32) decode_persistent_kernel(const PersistArgs pa) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  __shared__ int s_state, s_batch, s_maxlen, s_last;
+  int* const cmd = pa.cmd;
+  int* const sync = pa.sync;
+  const int hkv = pa.base.hkv, hq = pa.base.hq;
+  if (blockIdx.x == 0 && threadIdx.x == 0) st_release_sys(cmd + CMD_RUNNING, 1);
+  for (int step = 1;; ++step) {
+    // ---- the step's command
+    if (threadIdx.x == 0) {
+      int state = ST_WAIT, batch = 0, maxlen = 0;
+      const long long t0 = clock64();
+      if (blockIdx.x == 0) {
+        while (state == ST_WAIT) {
+          if (ld_acquire_sys(cmd + CMD_SEQ) >= step) {
+            state = ST_RUN;
+            batch = ld_acquire_sys(cmd + CMD_BATCH);
+            maxlen = ld_acquire_sys(cmd + CMD_MAXLEN);
+          } else if (ld_acquire_sys(cmd + CMD_STOP)) {
+            state = ST_STOP;
+          } else if (clock64() - t0 > pa.idle_limit) {
+            state = ST_IDLE;
+          } else {
+            __nanosleep(256);
+          }
+        }
+        sync[MB_BATCH] = batch;
+        sync[MB_MAXLEN] = maxlen;
+        sync[MB_STATE] = state;
+        st_release_gpu(sync + MB_STEP, step);
+      } else {
+        while (ld_acquire_gpu(sync + MB_STEP) < step) {
+          if (clock64() - t0 > pa.idle_limit + pa.wait_limit) {
+            state = ST_IDLE;
+            break;
+          }
+          __nanosleep(256);
+        }
+        if (state == ST_WAIT) {
+          state = ld_acquire_gpu(sync + MB_STATE);
+          batch = ld_acquire_gpu(sync + MB_BATCH);
+          maxlen = ld_acquire_gpu(sync + MB_MAXLEN);
+        }
+      }
+      s_state = state;
+      s_batch = batch;
+      s_maxlen = maxlen;
+    }
+    __syncthreads();
+    if (s_state != ST_RUN) {
+      if (threadIdx.x == 0 && s_state == ST_IDLE) {
+        atomicOr(cmd + CMD_STATUS, ATTN_FAULT_TIMEOUT);
+        if (pa.base.error_flags) atomicOr(pa.base.error_flags, ATTN_FAULT_TIMEOUT);
+      }
+      if (blockIdx.x == 0 && threadIdx.x == 0) {
+        __threadfence_system();
+        st_release_sys(cmd + CMD_RUNNING, 0);
+      }
+      break;
+    }
+    // ---- the step: the split plan of attn_decode_paged for this batch and bound
+    int batch = s_batch, maxlen = s_maxlen;
+    if (batch < 0 || batch > pa.max_batch) {
+      if (threadIdx.x == 0 && blockIdx.x == 0 && pa.base.error_flags)
+        atomicOr(pa.base.error_flags, ATTN_FAULT_BAD_LENGTH);
+      batch = batch < 0 ? 0 : pa.max_batch;
+    }
+    if (maxlen <= 0 || maxlen > pa.cap_len) maxlen = pa.cap_len;
+    int T, nsplit;
+    split_plan(batch, hkv, maxlen, pa.num_splits, pa.sm_count, pa.forced, &T, &nsplit);
+    Args a = pa.base;
+    a.batch = batch;
+    a.split_tokens = T;
+    size_t lse_off = 0;
+    partial_bytes(nsplit, (size_t)batch * hq, D, &lse_off);
+    a.part_o = pa.partials;
+    a.part_lse = nsplit > 1 ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(pa.partials) + lse_off) : nullptr;
+    const int tasks = nsplit * hkv * batch;
+    for (int t = blockIdx.x; t < tasks; t += gridDim.x) {
+      const int split = t % nsplit, r = t / nsplit, kvh = r % hkv, b = r / hkv;
+      split_task<G, FP8, FP8, true>(a, split, kvh, b, nsplit, smem_raw);
+      __syncthreads();  // shared memory is refilled by the next task
+      if (nsplit == 1) continue;
+      int L = __ldcg(a.seq_lens + b);  // clamped exactly as split_task clamps it
+      L = L < 0 ? 0 : (L > a.max_blocks * BS ? a.max_blocks * BS : L);
+      if (L > nsplit * T) L = nsplit * T;
+      const int n = max(1, (L + T - 1) / T);
+      if (n == 1 || split >= n) continue;  // O written directly, or an empty split
+      if (threadIdx.x == 0) {
+        __threadfence();  // this split's partial, before its arrival
+        s_last = atomicAdd(sync + MB_COUNTERS + b * hkv + kvh, 1) == n - 1;
+      }
+      __syncthreads();
+      if (s_last) {  // every split of (b, kvh) has arrived: merge its G rows
+        __threadfence();
+        for (int g = warp_id(); g < G; g += WARPS)
+          combine::combine_row<D>((b * hq) + kvh * G + g, a.part_o, a.part_lse, nsplit, batch * hq, nullptr,
+                                  a.seq_lens, T, nsplit * T, hq, a.o, a.o_f32, a.lse);
+        if (threadIdx.x == 0) sync[MB_COUNTERS + b * hkv + kvh] = 0;  // ready for the next step
+      }
+      __syncthreads();
+    }
+    // ---- the last CTA out reports the step
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(sync + MB_DONE_CTAS, 1) == (int)gridDim.x - 1) {
+        sync[MB_DONE_CTAS] = 0;
+        __threadfence_system();
+        st_release_sys(cmd + CMD_DONE, step);
+      }
+    }
+  }
+}
+
+}  // namespace decode
+
+// Workspace of the persistent decode: the partials of the largest step (any
+// batch up to p.batch at the length bound), then the mailbox and counters.
+static void persistent_layout(const attn_decode_params& p, int cap_len, size_t* sync_off, size_t* total) {
+  size_t part = 0;
+  const int sms = device_sm_count();
+  const int forced = env_int("ATTN_DECODE_SPLIT_TOKENS", 0);
+  for (int b = 1; b <= p.batch; ++b) {
+    int T, n;
+    decode::split_plan(b, p.num_kv_heads, cap_len, p.num_splits, sms, forced, &T, &n);
+    const size_t need = decode::partial_bytes(n, (size_t)b * p.num_q_heads, p.head_dim, nullptr);
+    if (need > part) part = need;
+  }
+  *sync_off = (part + 255) / 256 * 256;
+  const size_t words = decode::MB_COUNTERS + (size_t)p.batch * p.num_kv_heads;
+  *total = *sync_off + (words * sizeof(int) + 255) / 256 * 256;
+}
+
+static int persistent_cap_len(const attn_decode_params& p) {
+  const int cap = p.max_blocks_per_seq * decode::BS;
+  return (p.max_seq_len > 0 && p.max_seq_len < cap) ? p.max_seq_len : cap;
+}
+
+size_t decode_persistent_workspace_bytes(const attn_decode_params& p) {
+  size_t off, total;
+  persistent_layout(p, persistent_cap_len(p), &off, &total);
+  return total;
+}
+
+template <int G, bool FP8>
+static attn_status_t launch_persistent_g(const decode::PersistArgs& pa, cudaStream_t stream) {
+  auto kern = decode::decode_persistent_kernel<G, FP8>;
+  const int smem = (int)sizeof(decode::Smem<G, FP8>);
+  static DeviceOnce setup;  // the shared-memory attribute, once per device
+  attn_status_t st = setup.run([&]() -> attn_status_t {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+  });
+  if (st != ATTN_OK) return st;
+  // Every CTA must be resident at once (CTAs wait on CTA 0's mailbox): a
+  // cooperative launch of as many CTAs as fit.
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, decode::WARPS * 32, smem) != cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  const int grid = per_sm * pa.sm_count;
+  void* args[] = {const_cast<decode::PersistArgs*>(&pa)};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(decode::WARPS * 32), args,
+                                  smem, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+attn_status_t launch_decode_persistent(const attn_decode_params& p, int32_t* cmd_dev, void* workspace,
+                                       long long idle_cycles, cudaStream_t stream) {
+  const int cap_len = persistent_cap_len(p);
+  size_t sync_off, total;
+  persistent_layout(p, cap_len, &sync_off, &total);
+  int* sync = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(workspace) + sync_off);
+  if (cudaMemsetAsync(sync, 0, total - sync_off, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  decode::PersistArgs pa;
+  memset(&pa, 0, sizeof(pa));
+  decode::Args& a = pa.base;
+  a.q = reinterpret_cast<const __nv_bfloat16*>(p.q);
+  a.k_cache = reinterpret_cast<const uint8_t*>(p.k_cache);
+  a.v_cache = reinterpret_cast<const uint8_t*>(p.v_cache);
+  const bool fp8 = p.kv_dtype == ATTN_DTYPE_FP8_E4M3;
+  a.k_scale = fp8 ? p.k_scale : 1.f;
+  a.v_scale = fp8 ? p.v_scale : 1.f;
+  a.block_table = p.block_table;
+  a.seq_lens = p.seq_lens;
+  a.o = p.o;
+  a.lse = p.lse;
+  a.o_f32 = p.o_dtype == ATTN_DTYPE_F32;
+  a.hq = p.num_q_heads;
+  a.hkv = p.num_kv_heads;
+  a.max_blocks = p.max_blocks_per_seq;
+  a.num_blocks = p.num_blocks;
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  a.error_flags = p.error_flags;
+  pa.cmd = cmd_dev;
+  pa.partials = reinterpret_cast<float*>(workspace);
+  pa.sync = sync;
+  pa.max_batch = p.batch;
+  pa.cap_len = cap_len;
+  pa.num_splits = p.num_splits;
+  pa.sm_count = device_sm_count();
+  pa.forced = env_int("ATTN_DECODE_SPLIT_TOKENS", 0);
+  pa.idle_limit = idle_cycles;
+  pa.wait_limit = 2000000000LL;
+  switch (p.num_q_heads / p.num_kv_heads) {
+    case 1: return fp8 ? launch_persistent_g<1, true>(pa, stream) : launch_persistent_g<1, false>(pa, stream);
+    case 2: return fp8 ? launch_persistent_g<2, true>(pa, stream) : launch_persistent_g<2, false>(pa, stream);
+    case 4: return fp8 ? launch_persistent_g<4, true>(pa, stream) : launch_persistent_g<4, false>(pa, stream);
+    case 8: return fp8 ? launch_persistent_g<8, true>(pa, stream) : launch_persistent_g<8, false>(pa, stream);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace attn

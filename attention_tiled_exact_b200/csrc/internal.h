@@ -71,10 +71,20 @@ DecodePlan plan_decode(const attn_decode_params& p);
 attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan, void* workspace,
                             cudaStream_t stream);
 
+// The decode kernels' one-time set-up for these parameters (kernel
+// attributes), without launching anything: to be done before a stream capture.
+attn_status_t prepare_decode(const attn_decode_params& p);
+
 attn_status_t launch_combine(const float* part_o, const float* part_lse, int num_splits, int rows,
                              int head_dim, const int32_t* splits_per_row, const int32_t* seq_lens,
                              int split_tokens, int rows_per_seq, void* out_o, attn_dtype_t out_dtype,
                              float* out_lse, cudaStream_t stream);
+
+// Persistent decode: workspace size and launch (arguments validated by the
+// caller; cmd_dev is the device address of the host command block).
+size_t decode_persistent_workspace_bytes(const attn_decode_params& p);
+attn_status_t launch_decode_persistent(const attn_decode_params& p, int32_t* cmd_dev, void* workspace,
+                                       long long idle_cycles, cudaStream_t stream);
 
 // Backward (dQ, dK, dV). Arguments were validated by the caller.
 size_t backward_workspace_bytes(const attn_backward_params& p);

@@ -17,7 +17,9 @@ per other workload, each timed the same way:
   rows over one paged cache, as a fraction of the combined tensor + HBM
   roofline;
 * ``shared_prefix``: decode of 64 sequences sharing an 8192-token prefix;
-* ``backward``: dQ, dK, dV of the headline workload.
+* ``backward``: dQ, dK, dV of the headline workload;
+* ``decode_step_latency``: one small decode step (8 sequences) with the host
+  in the loop: direct launch, CUDA-graph replay and persistent kernel.
 
 On rank 0 of a 1-GPU run every workload also times the fp64 CPU oracle on a
 bounded sample of the same inputs (``cpu_baseline``) and reports the largest
@@ -64,7 +66,7 @@ KERNEL_SOURCES = {
     "decode": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
     "decode_fp8": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
 }
-LEGS = ("tiny", "prefill", "prefill16k", "decode", "decodefp8", "mixed", "sharedprefix", "backward")
+LEGS = ("tiny", "prefill", "prefill16k", "decode", "decodefp8", "mixed", "sharedprefix", "backward", "decodesteps")
 
 
 def kernel_hash(kind: str) -> str:
@@ -848,6 +850,70 @@ def bench_mixed(c: Ctx):
     return res
 
 
+def bench_decode_steps(c: Ctx):
+    """Latency of one small decode step (8 sequences of U[512, 2048] tokens,
+    32/8 heads) with the host in the loop, three ways: a direct call
+    (split kernel + combine launched), a replay from the CUDA graph pool, and a
+    step of the persistent decode kernel. Each is timed on the host around
+    call + synchronisation (or submit + wait), median over the steps."""
+    import torch
+    attn = c.attn
+    cfg = _with_rank_seed(wl.DecodeConfig("decode_step_b8_h32kv8_d128_len512_2k", 8, 32, 8, 128, 512, 2048, 6), c.rank)
+    d = wl.make_decode(cfg)
+    q = _dev_bf16(d["q"])
+    kc, vc = _dev_bf16(d["k_pool"]), _dev_bf16(d["v_pool"])
+    bt = torch.from_numpy(d["block_table"]).cuda()
+    sl = torch.from_numpy(d["kv_lens"]).cuda()
+    max_len = int(d["kv_lens"].max())
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(attn.decode_workspace_bytes(q, kc, vc, bt, sl, max_seq_len=max_len), 1), dtype=torch.uint8,
+                     device="cuda")
+    n = max(200, c.args.steps)
+
+    def host_median(fn):
+        for _ in range(20):
+            fn()
+        ts = []
+        for _ in range(n):
+            t0 = time.perf_counter()
+            fn()
+            ts.append((time.perf_counter() - t0) * 1e6)
+        ts.sort()
+        return {"median_us": round(ts[n // 2], 2), "p10_us": round(ts[n // 10], 2), "p90_us": round(ts[(9 * n) // 10], 2)}
+
+    def direct():
+        attn.decode_paged(q, kc, vc, bt, sl, cfg.scale, max_seq_len=max_len, out=out, lse=lse, workspace=ws)
+        torch.cuda.synchronize()
+
+    res = {"workload": cfg.name, "unit": "us per step (host round trip: call + synchronise)", "steps": n,
+           "kv_tokens": int(d["kv_lens"].sum())}
+    res["direct"] = host_median(direct)
+    dev_ms = time_loop(lambda: attn.decode_paged(q, kc, vc, bt, sl, cfg.scale, max_seq_len=max_len, out=out,
+                                                 lse=lse, workspace=ws), n, c.args.warmup, c.world)
+    res["direct_device_back_to_back_us"] = round(dev_ms * 1e3, 2)
+    pool = attn.DecodeGraphPool(q, kc, vc, bt, sl, out, lse, [1, 2, 4, 8], [512, 1024, 2048, 4096], cfg.scale)
+    try:
+        stream = torch.cuda.current_stream()
+
+        def graph():
+            pool.replay(cfg.batch, max_len)
+            stream.synchronize()
+
+        res["graph"] = host_median(graph)
+        res["graph_bucket"] = list(pool.replay(cfg.batch, max_len))
+    finally:
+        pool.close()
+    torch.cuda.synchronize()
+    pd = attn.PersistentDecode(q, kc, vc, bt, sl, out, lse, cfg.scale)
+    try:
+        res["persistent"] = host_median(lambda: pd.step(cfg.batch, max_len))
+    finally:
+        pd.stop()
+    res["gpu_launches_per_step"] = {"direct": 2, "graph": 1, "persistent": 0}
+    return res
+
+
 def bench_launcher_stub(c: Ctx):
     """Host-only check of the N-rank launch (no GPU work): every rank reports in."""
     t0 = time.perf_counter()
@@ -868,7 +934,7 @@ def run_ours(args, rank, world, local):
     legs = {"tiny": ("tiny", bench_tiny), "prefill16k": ("prefill_16k", bench_prefill_16k),
             "decode": ("decode", bench_decode), "decodefp8": ("decode_fp8", bench_decode_fp8),
             "mixed": ("mixed", bench_mixed), "sharedprefix": ("shared_prefix", bench_shared_prefix),
-            "backward": ("backward", bench_backward)}
+            "backward": ("backward", bench_backward), "decodesteps": ("decode_step_latency", bench_decode_steps)}
     if args.only in (None, "prefill"):
         result.update(bench_prefill(c))
         parity.update(result.pop("parity", {}))

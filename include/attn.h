@@ -341,6 +341,107 @@ ATTN_API attn_status_t attn_decode_paged_shared_prefix(const attn_decode_params*
 ATTN_API attn_status_t attn_decode_paged_noalloc(const attn_decode_params* p, attn_stream_t stream);
 
 /*
+ * Persistent decode: one resident kernel executes a stream of decode steps
+ * over static buffers, commanded from the host through a small block of host
+ * memory, instead of launching kernels for every step ("GPU Kernel 调度:大模型推
+ * 理的拐点 2026", Persistent Kernel section: a kernel that stays resident and
+ * pulls work removes the per-step launch cost that shows at small batch).
+ * Every step computes exactly what attn_decode_paged computes for the same
+ * buffers, batch and max_seq_len: the same split plan and kernels' arithmetic,
+ * bit for bit.
+ *
+ * attn_persistent_cmd is host memory shared with the kernel: it must be
+ * page-locked and mapped into the device (cudaHostAlloc with
+ * cudaHostAllocMapped, or any pinned memory on a system with unified
+ * addressing). Fields marked host are written by the caller (through
+ * attn_decode_persistent_submit / _stop), fields marked device by the kernel.
+ *
+ * attn_decode_persistent_launch: p describes the static buffers exactly as for
+ * attn_decode_paged (q, o, lse, block_table, seq_lens, caches, error_flags),
+ * with p->batch the largest batch a step may have and p->max_seq_len the
+ * largest bound a step may give (0: the table capacity). The call zeroes
+ * *cmd, zeroes the control words of the workspace (cudaMemsetAsync on
+ * `stream`) and launches the kernel cooperatively on `stream` (one CTA per
+ * resident slot of every SM); it returns at once. While the kernel runs it
+ * holds every SM: kernels of other streams wait, copies do not. Workspace:
+ * attn_decode_persistent_workspace bytes of device memory, 256-byte aligned,
+ * owned by the caller and not touched by anyone else while the kernel runs.
+ * idle_cycles (> 0): the kernel exits, with ATTN_FAULT_TIMEOUT in cmd->status
+ * and error_flags, after that many SM clock cycles without a command.
+ *
+ * A step: write its inputs (q rows, block-table rows, seq_lens) into the
+ * static buffers and make them visible (e.g. synchronise the stream that
+ * copied them), then attn_decode_persistent_submit(cmd, batch, max_seq_len,
+ * &step) (max_seq_len 0: the launch bound), then
+ * attn_decode_persistent_wait(cmd, step, timeout_us) before reading o / lse or
+ * rewriting the inputs. Submit returns ATTN_ERR_INVALID_ARG while a step is
+ * still running. Wait returns ATTN_OK, or ATTN_ERR_TIMEOUT when the step did
+ * not finish within timeout_us or the kernel gave up. attn_decode_persistent_stop
+ * asks the kernel to exit once idle; the caller then synchronises `stream`.
+ * The host-side calls make no CUDA call.
+ */
+typedef struct {
+  int32_t seq;          /* host: number of the last step submitted (1, 2, ...) */
+  int32_t batch;        /* host: sequences in that step (<= the launch's batch) */
+  int32_t max_seq_len;  /* host: bound of that step's seq_lens (0: the launch bound) */
+  int32_t stop;         /* host: nonzero asks the kernel to exit once idle */
+  int32_t done;         /* device: number of the last step completed */
+  int32_t status;       /* device: ATTN_FAULT_* bits when the kernel gave up */
+  int32_t running;      /* device: 1 from the kernel's start until it exits */
+  int32_t reserved;
+} attn_persistent_cmd;
+
+ATTN_API attn_status_t attn_decode_persistent_workspace(const attn_decode_params* p, size_t* bytes);
+ATTN_API attn_status_t attn_decode_persistent_launch(const attn_decode_params* p, attn_persistent_cmd* cmd,
+                                                     void* workspace, size_t workspace_bytes, long long idle_cycles,
+                                                     attn_stream_t stream);
+ATTN_API attn_status_t attn_decode_persistent_submit(attn_persistent_cmd* cmd, int32_t batch, int32_t max_seq_len,
+                                                     int32_t* step);
+ATTN_API attn_status_t attn_decode_persistent_wait(const attn_persistent_cmd* cmd, int32_t step, long long timeout_us);
+ATTN_API void attn_decode_persistent_stop(attn_persistent_cmd* cmd);
+
+/*
+ * A pool of CUDA graphs of the decode step, one per static shape ("GPU Kernel
+ * 调度:大模型推理的拐点 2026", CUDA Graph section: capture the shapes a server
+ * sees up front and replay the nearest one, so a step costs one graph launch
+ * instead of one launch per kernel).
+ *
+ * attn_decode_graph_pool_create captures attn_decode_paged once for every
+ * (batch bucket, length bucket) pair, over the static buffers p describes
+ * (q, o, lse, block_table, seq_lens, caches and error_flags as for
+ * attn_decode_paged; p->batch is the rows those buffers hold, at least the
+ * largest batch bucket). Buckets are host arrays of strictly ascending
+ * positive values (at most 1024 each); a length bucket is a max_seq_len bound
+ * (up to the table capacity). workspace: at least attn_decode_graph_pool_workspace
+ * bytes of device memory, 256-byte aligned, owned by the caller and shared by
+ * every graph of the pool. The capture runs on an internal stream and does
+ * not touch the buffers.
+ *
+ * attn_decode_graph_pool_replay(pool, batch, max_seq_len, stream, ...) launches
+ * the graph of the smallest batch bucket >= batch and the smallest length
+ * bucket >= max_seq_len (0: the largest), and reports the chosen bucket in
+ * *bucket_batch / *bucket_len (nullable). The graph reads the buffers as they
+ * are when it runs: the caller has written this step's q rows, table rows and
+ * seq_lens, and keeps seq_lens of the rows from batch up to the bucket's batch
+ * at 0 (those rows get O = 0, LSE = -inf). The result is attn_decode_paged
+ * with batch = the bucket's batch and max_seq_len = the bucket's length, bit
+ * for bit. ATTN_ERR_INVALID_ARG when no bucket covers the step. Replays share
+ * the workspace: replays that overlap on the GPU race.
+ */
+typedef struct attn_decode_graph_pool attn_decode_graph_pool;
+
+ATTN_API attn_status_t attn_decode_graph_pool_workspace(const attn_decode_params* p, const int32_t* batch_buckets,
+                                                        int n_batch, const int32_t* len_buckets, int n_len,
+                                                        size_t* bytes);
+ATTN_API attn_status_t attn_decode_graph_pool_create(const attn_decode_params* p, const int32_t* batch_buckets,
+                                                     int n_batch, const int32_t* len_buckets, int n_len,
+                                                     void* workspace, size_t workspace_bytes,
+                                                     attn_decode_graph_pool** pool);
+ATTN_API attn_status_t attn_decode_graph_pool_replay(attn_decode_graph_pool* pool, int32_t batch, int32_t max_seq_len,
+                                                     attn_stream_t stream, int32_t* bucket_batch, int32_t* bucket_len);
+ATTN_API void attn_decode_graph_pool_destroy(attn_decode_graph_pool* pool);
+
+/*
  * Split-KV log-sum-exp combine ("GPU Kernel 调度:大模型推理的拐点 2026",
  * Flash Decoding section: partials merged with the online-softmax formula,
  * each carrying a log-sum-exp accumulated in FP32). For each row r:

@@ -48,6 +48,9 @@ def test_struct_layouts_match_the_header(lib):
     body.append('printf("P %zu\\n", sizeof(attn_prefill_params));')
     body.append('printf("D %zu\\n", sizeof(attn_decode_params));')
     body.append('printf("B %zu\\n", sizeof(attn_backward_params));')
+    body.append('printf("C %zu\\n", sizeof(attn_persistent_cmd));')
+    for f, _ in lib.PersistentCmd._fields_:
+        body.append(f'printf("c.{f} %zu\\n", offsetof(attn_persistent_cmd, {f}));')
     for f in fields_p:
         body.append(f'printf("p.{f} %zu\\n", offsetof(attn_prefill_params, {f}));')
     for f in fields_d:
@@ -67,6 +70,9 @@ def test_struct_layouts_match_the_header(lib):
         assert int(got[f"p.{f}"]) == getattr(lib.PrefillParams, f).offset, f
     for f in fields_d:
         assert int(got[f"d.{f}"]) == getattr(lib.DecodeParams, f).offset, f
+    assert int(got["C"]) == ctypes.sizeof(lib.PersistentCmd)
+    for f, _ in lib.PersistentCmd._fields_:
+        assert int(got[f"c.{f}"]) == getattr(lib.PersistentCmd, f).offset, f
     assert int(got["B"]) == ctypes.sizeof(lib.BackwardParams)
     for f in fields_b:
         assert int(got[f"b.{f}"]) == getattr(lib.BackwardParams, f).offset, f

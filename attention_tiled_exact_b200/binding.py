@@ -56,7 +56,7 @@ class PrefillParams(ctypes.Structure):
         ("scale", ctypes.c_float), ("causal", _i32), ("o_dtype", _i32),
         ("seqlens_q", _vp), ("seqlens_k", _vp), ("k_cache", _vp), ("v_cache", _vp),
         ("block_table", _vp), ("max_blocks_per_seq", _i32), ("num_blocks", _i32),
-        ("block_size", _i32), ("error_flags", _vp),
+        ("block_size", _i32), ("error_flags", _vp), ("cu_seqlens_q", _vp), ("total_q", _i32),
     ]
 
 
@@ -236,37 +236,70 @@ def _need(cond, msg):
 # ----------------------------------------------------------------------------
 
 
+def _queries(p, q, out, lse, out_dtype, want_lse, batch, cu_seqlens_q, max_seqlen_q):
+    """Fill the query / output / LSE fields of PrefillParams for a padded
+    [B,Hq,Sq,D] or a packed [total_q,Hq,D] layout; returns (out, lse)."""
+    if cu_seqlens_q is None:
+        _need(q.dim() == 4 and q.shape[0] == batch, "q must be [B, Hq, Sq, D]")
+        B, Hq, Sq, D = q.shape
+        o_shape, lse_shape = (B, Hq, Sq, D), (B, Hq, Sq)
+    else:
+        _need(q.dim() == 3, "packed q must be [total_q, Hq, D]")
+        _need(cu_seqlens_q.dtype == torch.int32 and cu_seqlens_q.is_cuda and cu_seqlens_q.is_contiguous() and
+              cu_seqlens_q.numel() == batch + 1, "int32 cu_seqlens_q [B + 1]")
+        _need(max_seqlen_q is not None and int(max_seqlen_q) >= 0, "max_seqlen_q (an upper bound of the rows of a sequence)")
+        total, Hq, D = q.shape
+        Sq = int(max_seqlen_q)
+        o_shape, lse_shape = (total, Hq, D), (Hq, total)
+    _need(q.dtype == torch.bfloat16 and q.is_cuda and q.stride(-1) == 1, "bf16 CUDA q, last dim contiguous")
+    if out is None:
+        out = torch.empty(o_shape, dtype=out_dtype, device=q.device)
+    _need(tuple(out.shape) == o_shape and out.stride(-1) == 1, f"out {o_shape}")
+    if lse is None and want_lse:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse.is_contiguous() and lse.dtype == torch.float32 and tuple(lse.shape) == lse_shape, f"lse {lse_shape}")
+    p.q, p.o, p.lse = _ptr(q), _ptr(out), _ptr(lse)
+    p.num_q_heads, p.head_dim, p.seqlen_q = Hq, D, Sq
+    if cu_seqlens_q is None:
+        p.q_batch_stride, p.q_head_stride, p.q_row_stride = q.stride(0), q.stride(1), q.stride(2)
+        p.o_batch_stride, p.o_head_stride, p.o_row_stride = out.stride(0), out.stride(1), out.stride(2)
+    else:
+        p.q_batch_stride, p.q_head_stride, p.q_row_stride = 0, q.stride(1), q.stride(0)
+        p.o_batch_stride, p.o_head_stride, p.o_row_stride = 0, out.stride(1), out.stride(0)
+        p.cu_seqlens_q, p.total_q = _ptr(cu_seqlens_q), q.shape[0]
+    p.o_dtype = _out_code(out.dtype)
+    return out, lse
+
+
 def prefill(q, k, v, scale: float | None = None, causal: bool = False, out=None, lse=None,
-            out_dtype=torch.bfloat16, want_lse: bool = True, error_flags=None, seqlens_q=None, seqlens_k=None):
+            out_dtype=torch.bfloat16, want_lse: bool = True, error_flags=None, seqlens_q=None, seqlens_k=None,
+            cu_seqlens_q=None, max_seqlen_q=None):
     """Tiled prefill attention. q [B,Hq,Sq,D], k/v [B,Hkv,Sk,D] bf16 CUDA tensors.
 
     seqlens_q / seqlens_k (int32 [B] CUDA tensors, optional): valid query rows
     and keys of each sequence of a padded batch (rows past seqlens_q[b] are
     not written).
-    Returns ``(O [B,Hq,Sq,D], LSE [B,Hq,Sq] fp32 or None)``.
+    Packed queries: with cu_seqlens_q (int32 [B + 1] CUDA) and max_seqlen_q
+    (host int), q is [total_q, Hq, D], sequence b owning rows
+    cu_seqlens_q[b] .. cu_seqlens_q[b+1] - 1; O is then [total_q, Hq, D] and
+    the LSE [Hq, total_q].
+    Returns ``(O [B,Hq,Sq,D], LSE [B,Hq,Sq] fp32 or None)`` (padded).
     """
-    _need(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be 4-D [B, H, S, D]")
-    B, Hq, Sq, D = q.shape
-    Hkv, Sk = k.shape[1], k.shape[2]
-    _need(tuple(v.shape) == tuple(k.shape) and k.shape[0] == B and k.shape[3] == D, "shape mismatch")
-    for t in (q, k, v):
+    _need(k.dim() == 4 and v.dim() == 4, "k, v must be 4-D [B, H, S, D]")
+    B, Hkv, Sk, D = k.shape
+    _need(tuple(v.shape) == tuple(k.shape) and q.shape[-1] == D, "shape mismatch")
+    for t in (k, v):
         _need(t.dtype == torch.bfloat16 and t.is_cuda and t.stride(3) == 1, "bf16 CUDA, last dim contiguous")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty((B, Hq, Sq, D), dtype=out_dtype, device=q.device)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    if lse is not None:
-        _need(lse.is_contiguous() and lse.dtype == torch.float32 and tuple(lse.shape) == (B, Hq, Sq), "lse")
     p = PrefillParams()
-    p.q, p.k, p.v, p.o, p.lse = _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse)
-    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.seqlen_q, p.seqlen_k = B, Hq, Hkv, D, Sq, Sk
-    p.q_batch_stride, p.q_head_stride, p.q_row_stride = q.stride(0), q.stride(1), q.stride(2)
+    out, lse = _queries(p, q, out, lse, out_dtype, want_lse, B, cu_seqlens_q, max_seqlen_q)
+    p.k, p.v = _ptr(k), _ptr(v)
+    p.batch, p.num_kv_heads, p.seqlen_k = B, Hkv, Sk
     p.k_batch_stride, p.k_head_stride, p.k_row_stride = k.stride(0), k.stride(1), k.stride(2)
     p.v_batch_stride, p.v_head_stride, p.v_row_stride = v.stride(0), v.stride(1), v.stride(2)
-    p.o_batch_stride, p.o_head_stride, p.o_row_stride = out.stride(0), out.stride(1), out.stride(2)
-    p.scale, p.causal, p.o_dtype = float(scale), int(bool(causal)), _out_code(out.dtype)
+    p.scale, p.causal = float(scale), int(bool(causal))
     p.error_flags = _ptr(error_flags)
     for name, t in (("seqlens_q", seqlens_q), ("seqlens_k", seqlens_k)):
         if t is not None:
@@ -330,19 +363,20 @@ def prefill_backward(q, k, v, o, lse, dout, scale: float | None = None, causal: 
 
 def prefill_paged(q, k_cache, v_cache, block_table, seqlens_k, seqlens_q=None, scale: float | None = None,
                   causal: bool = True, out=None, lse=None, out_dtype=torch.bfloat16, want_lse: bool = True,
-                  error_flags=None):
+                  error_flags=None, cu_seqlens_q=None, max_seqlen_q=None):
     """Prefill of query chunks against a paged KV cache (chunked prefill).
 
-    q [B,Hq,Sq,D] bf16 (rows past seqlens_q[b] are not written);
+    q [B,Hq,Sq,D] bf16 (rows past seqlens_q[b] are not written), or packed
+    [total_q,Hq,D] with cu_seqlens_q / max_seqlen_q as in :func:`prefill`;
     k_cache/v_cache [NB,Hkv,16,D] bf16; block_table [B,max_blocks] int32;
     seqlens_k [B] int32: cached keys of each sequence, the chunk's own keys
     included (bottom-right causal alignment). Returns ``(O, LSE)``.
     """
-    _need(q.dim() == 4 and k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
-    B, Hq, Sq, D = q.shape
-    NB, Hkv, BS, D2 = k_cache.shape
-    _need(D2 == D and q.dtype == torch.bfloat16 and k_cache.dtype == torch.bfloat16 and
-          v_cache.dtype == torch.bfloat16 and q.stride(3) == 1, "bf16 q and caches, last dim contiguous")
+    _need(k_cache.dim() == 4 and v_cache.shape == k_cache.shape, "shapes")
+    NB, Hkv, BS, D = k_cache.shape
+    B = block_table.shape[0]
+    _need(q.shape[-1] == D and k_cache.dtype == torch.bfloat16 and v_cache.dtype == torch.bfloat16,
+          "bf16 caches of q's head_dim")
     _need(k_cache.is_contiguous() and v_cache.is_contiguous(), "contiguous caches")
     _need(block_table.dtype == torch.int32 and block_table.is_contiguous() and block_table.shape[0] == B,
           "int32 block table [B, max_blocks]")
@@ -351,20 +385,14 @@ def prefill_paged(q, k_cache, v_cache, block_table, seqlens_k, seqlens_q=None, s
         _need(seqlens_q.dtype == torch.int32 and seqlens_q.numel() == B, "int32 seqlens_q [B]")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty((B, Hq, Sq, D), dtype=out_dtype, device=q.device)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     p = PrefillParams()
-    p.q, p.o, p.lse = _ptr(q), _ptr(out), _ptr(lse)
+    out, lse = _queries(p, q, out, lse, out_dtype, want_lse, B, cu_seqlens_q, max_seqlen_q)
     p.k_cache, p.v_cache, p.block_table = _ptr(k_cache), _ptr(v_cache), _ptr(block_table)
     p.seqlens_k, p.seqlens_q = _ptr(seqlens_k), _ptr(seqlens_q)
-    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.seqlen_q = B, Hq, Hkv, D, Sq
+    p.batch, p.num_kv_heads = B, Hkv
     p.seqlen_k = block_table.shape[1] * BS  # upper bound of seqlens_k
     p.max_blocks_per_seq, p.num_blocks, p.block_size = block_table.shape[1], NB, BS
-    p.q_batch_stride, p.q_head_stride, p.q_row_stride = q.stride(0), q.stride(1), q.stride(2)
-    p.o_batch_stride, p.o_head_stride, p.o_row_stride = out.stride(0), out.stride(1), out.stride(2)
-    p.scale, p.causal, p.o_dtype = float(scale), int(bool(causal)), _out_code(out.dtype)
+    p.scale, p.causal = float(scale), int(bool(causal))
     p.error_flags = _ptr(error_flags)
     _check(LIB.attn_prefill(ctypes.byref(p), _stream(q.device)), "attn_prefill(paged)")
     return out, lse

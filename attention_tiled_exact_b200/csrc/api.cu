@@ -65,6 +65,7 @@ static attn_status_t validate_prefill(const attn_prefill_params* p) {
   if (p->head_dim != 64 && p->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
   if (!(p->scale > 0.f) || !isfinite(p->scale)) return ATTN_ERR_INVALID_ARG;
   if (p->o_dtype != ATTN_DTYPE_BF16 && p->o_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID_ARG;
+  if (p->cu_seqlens_q && (p->seqlens_q || p->total_q < 0)) return ATTN_ERR_INVALID_ARG;
   const bool paged = p->k_cache != nullptr || p->v_cache != nullptr;
   if (!p->q || !p->o) return ATTN_ERR_INVALID_ARG;
   if (paged) {
@@ -149,7 +150,7 @@ extern "C" {
 attn_status_t attn_prefill(const attn_prefill_params* p, attn_stream_t stream) {
   attn_status_t st = attn::validate_prefill(p);
   if (st != ATTN_OK) return st;
-  if (p->batch == 0 || p->seqlen_q == 0) return ATTN_OK;
+  if (p->batch == 0 || p->seqlen_q == 0 || (p->cu_seqlens_q && p->total_q == 0)) return ATTN_OK;
   st = attn::check_device();
   if (st != ATTN_OK) return st;
   return attn::launch_prefill(*p, reinterpret_cast<cudaStream_t>(stream));

@@ -103,12 +103,15 @@ struct Args {
   int n_row_blocks;
   const int32_t* seqlens_q;
   const int32_t* seqlens_k;
+  const int32_t* cu_seqlens_q;  // packed queries: sequence b's rows are [cu[b], cu[b+1]) of total_q
+  int total_q;
   void* o;
   float* lse;
   int o_f32;
   int o_tma;  // O rows of a full 32-row warp slice go out through the tm_o tile store
   int sort_items;  // order items by cost (variable lengths) instead of row block
   long long o_bs, o_hs, o_rs;
+  long long lse_rows;  // rows per (batch, head) of the LSE tensor: seqlen_q, or total_q when packed
   int32_t* error_flags;
   long long wait_limit;  // cycle bound of every pipeline wait
   // paged keys/values (PAGED kernels only)
@@ -141,6 +144,7 @@ struct Layout {
 
 struct Work {
   int b, kvh;
+  int qoff, qb;  // the sequence's first row and batch coordinate in the Q / O / LSE tensors
   int head[2];
   int row0[2];
   int active[2];
@@ -177,7 +181,18 @@ __device__ __forceinline__ Work decode_work(const Args& a, int item) {
     w.row0[0] = 2 * p * BM;
     w.row0[1] = (2 * p + 1) * BM;
   }
-  w.sq = a.seqlens_q ? a.seqlens_q[w.b] : a.seqlen_q;
+  if (a.cu_seqlens_q) {  // packed: rows [s0, s1) of the [total_q, Hq, D] tensors
+    int s0 = a.cu_seqlens_q[w.b], s1 = a.cu_seqlens_q[w.b + 1];
+    s0 = min(max(s0, 0), a.total_q);
+    s1 = min(max(s1, s0), a.total_q);
+    w.qoff = s0;
+    w.qb = 0;
+    w.sq = s1 - s0;
+  } else {
+    w.qoff = 0;
+    w.qb = w.b;
+    w.sq = a.seqlens_q ? a.seqlens_q[w.b] : a.seqlen_q;
+  }
   w.sk = a.seqlens_k ? a.seqlens_k[w.b] : a.seqlen_k;
   if (w.sq > a.seqlen_q) w.sq = a.seqlen_q;
   if (w.sq < 0) w.sq = 0;
@@ -473,8 +488,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < 2; ++t) {
           if (!w.active[t]) continue;
           for (int c = 0; c < L::CHUNKS; ++c)
-            tma_load_4d(smem + L::Q_OFF + t * L::Q_TILE + c * (BM * 128), &tm_q, q_full, c * 64, w.row0[t],
-                        w.head[t], w.b);
+            tma_load_4d(smem + L::Q_OFF + t * L::Q_TILE + c * (BM * 128), &tm_q, q_full, c * 64,
+                        w.qoff + w.row0[t], w.head[t], w.qb);
         }
         ++nq;
         // Bring the next item's Q tiles into L2 now, so that its shared-memory
@@ -485,7 +500,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const Work wn = decode_work(args, nxt);
             for (int t = 0; t < 2; ++t) {
               if (!wn.active[t]) continue;
-              for (int c = 0; c < L::CHUNKS; ++c) tma_prefetch_l2_4d(&tm_q, c * 64, wn.row0[t], wn.head[t], wn.b);
+              for (int c = 0; c < L::CHUNKS; ++c)
+                tma_prefetch_l2_4d(&tm_q, c * 64, wn.qoff + wn.row0[t], wn.head[t], wn.qb);
             }
           }
         }
@@ -775,7 +791,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float inv_l = empty ? 0.f : 1.f / l;
       if (args.lse && store) {
         const float lse = empty ? -INFINITY : (m2 + log2f(l)) * 0.69314718055994530942f;
-        args.lse[((long long)w.b * args.hq + w.head[t]) * args.seqlen_q + qrow] = lse;
+        args.lse[((long long)w.qb * args.hq + w.head[t]) * args.lse_rows + w.qoff + qrow] = lse;
       }
       const bool has_keys = nt > 0;
       if (has_keys) {
@@ -783,16 +799,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++nf;
         if (!ok) break;
       }
-      const long long obase =
-          (long long)w.b * args.o_bs + (long long)w.head[t] * args.o_hs + (long long)qrow * args.o_rs;
+      const long long obase = (long long)w.qb * args.o_bs + (long long)w.head[t] * args.o_hs +
+                              (long long)(w.qoff + qrow) * args.o_rs;
       if (has_keys) tc_fence_after();
       if (args.o_tma && w.row0[t] + sub * 32 + 32 <= w.sq) {  // warp-uniform
         uint8_t* stage = smem + L::O_OFF + warp * L::W_STAGE;
-        const int r0 = w.row0[t] + sub * 32;
+        const int r0 = w.qoff + w.row0[t] + sub * 32;
         if (args.o_f32)
-          store_rows_tma<D, true>(&tm_o, stage, tO, has_keys, inv_l, r0, w.head[t], w.b);
+          store_rows_tma<D, true>(&tm_o, stage, tO, has_keys, inv_l, r0, w.head[t], w.qb);
         else
-          store_rows_tma<D, false>(&tm_o, stage, tO, has_keys, inv_l, r0, w.head[t], w.b);
+          store_rows_tma<D, false>(&tm_o, stage, tO, has_keys, inv_l, r0, w.head[t], w.qb);
         continue;
       }
 #pragma unroll
@@ -908,7 +924,8 @@ static attn_status_t launch_variant(const CUtensorMap& tq, const CUtensorMap& tk
   const int grid = items < device_sm_count() ? items : device_sm_count();
   Args ak = a;
   // Sort only when lengths vary per sequence and every CTA's share fits its list.
-  ak.sort_items = (a.seqlens_q || a.seqlens_k) && items <= SORT_MAX_ITEMS && (items + grid - 1) / grid <= LIST_MAX;
+  ak.sort_items = (a.seqlens_q || a.seqlens_k || a.cu_seqlens_q) && items <= SORT_MAX_ITEMS &&
+                  (items + grid - 1) / grid <= LIST_MAX;
   kern<<<grid, NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, to, ak, items);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -920,9 +937,16 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
   if (p.batch == 0 || p.seqlen_q == 0 || p.num_q_heads == 0) return ATTN_OK;
   const bool paged = p.k_cache != nullptr;
   const int D = p.head_dim;
+  // Packed queries ([total_q, Hq, D] rows addressed through cu_seqlens_q) are
+  // one "batch" of total_q rows to the tensor maps.
+  const bool packed = p.cu_seqlens_q != nullptr;
+  const uint64_t q_rows = packed ? (uint64_t)p.total_q : (uint64_t)p.seqlen_q;
+  const uint64_t q_batches = packed ? 1 : (uint64_t)p.batch;
+  const int64_t q_bs = packed ? p.q_row_stride * (int64_t)p.total_q : p.q_batch_stride;
+  const int64_t o_bs = packed ? p.o_row_stride * (int64_t)p.total_q : p.o_batch_stride;
   CUtensorMap tq, tk, tv;
-  if (!encode_4d(&tq, p.q, D, p.seqlen_q, p.num_q_heads, p.batch, p.q_row_stride * 2, p.q_head_stride * 2,
-                 p.q_batch_stride * 2, BM))
+  if (!encode_4d(&tq, p.q, D, q_rows, p.num_q_heads, q_batches, p.q_row_stride * 2, p.q_head_stride * 2, q_bs * 2,
+                 BM))
     return ATTN_ERR_CUDA;
   if (paged) {
     // Pools [num_blocks, Hkv, 16, D]: one 16-row box per cache block and D chunk.
@@ -964,18 +988,21 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
   a.n_row_blocks = (p.seqlen_q + BM - 1) / BM;
   a.seqlens_q = p.seqlens_q;
   a.seqlens_k = p.seqlens_k;
+  a.cu_seqlens_q = p.cu_seqlens_q;
+  a.total_q = packed ? p.total_q : 0;
+  a.lse_rows = packed ? p.total_q : p.seqlen_q;
   a.o = p.o;
   a.lse = p.lse;
   a.o_f32 = p.o_dtype == ATTN_DTYPE_F32;
-  a.o_bs = p.o_batch_stride;
+  a.o_bs = o_bs;
   a.o_hs = p.o_head_stride;
   a.o_rs = p.o_row_stride;
   // O goes out through tile stores when its map encodes (the API's alignment
   // rules make that the normal case); otherwise every row is stored directly.
   const int esz = a.o_f32 ? 4 : 2;
   CUtensorMap to;
-  a.o_tma = encode_4d(&to, p.o, D, p.seqlen_q, p.num_q_heads, p.batch, p.o_row_stride * esz,
-                      p.o_head_stride * esz, p.o_batch_stride * esz, 32, a.o_f32 != 0)
+  a.o_tma = encode_4d(&to, p.o, D, q_rows, p.num_q_heads, q_batches, p.o_row_stride * esz, p.o_head_stride * esz,
+                      o_bs * esz, 32, a.o_f32 != 0)
                 ? 1
                 : 0;
   if (!a.o_tma) to = tq;  // never read

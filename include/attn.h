@@ -105,6 +105,19 @@ typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1, ATTN_DTYPE_FP8_E4M3 = 2 
  * seqlens_k (an upper bound is fine). The causal alignment uses the
  * per-sequence lengths.
  *
+ * Packed variable-length queries (a batch of chunks of different lengths
+ * without padding, "抱infra脚" Chunked Prefill): set cu_seqlens_q (device,
+ * [batch + 1], nondecreasing, cu_seqlens_q[0] == 0) and total_q (host, the
+ * rows of the packed tensors, >= cu_seqlens_q[batch]). Then q and o are
+ * [total_q, num_q_heads, head_dim] with strides q_row_stride / q_head_stride
+ * (o_row_stride / o_head_stride; the batch strides are ignored), sequence b
+ * owns rows cu_seqlens_q[b] .. cu_seqlens_q[b+1] - 1, lse is [num_q_heads,
+ * total_q] fp32 contiguous, and seqlen_q is an upper bound on a sequence's
+ * rows (rows past it are not computed). seqlens_q must then be NULL. Keys and
+ * values are dense per sequence or paged exactly as above, with the same
+ * bottom-right causal alignment per sequence. A packed call gives every valid
+ * row the same bits as the padded layout would.
+ *
  * Block-sparse attention (BSR: query block r sees only the key blocks listed
  * for it, the block-sparse format of the FlashInfer section of "抱infra脚")
  * is this paged mode, non-causal, with one batch entry per query block whose
@@ -142,6 +155,9 @@ typedef struct {
   int num_blocks;
   int block_size;
   int32_t* error_flags; /* nullable */
+  /* optional packed queries (see above) */
+  const int32_t* cu_seqlens_q;
+  int total_q;
 } attn_prefill_params;
 
 ATTN_API attn_status_t attn_prefill(const attn_prefill_params* p, attn_stream_t stream);

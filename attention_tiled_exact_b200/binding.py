@@ -6,7 +6,9 @@ kernels. The names follow the C ABI declared in include/attn.h.
 
 Importing this module loads the library and fails loudly if it is missing
 (build it with ``python -m attention_tiled_exact_b200.build``). There is no
-CPU fallback.
+CPU fallback. With ``ATTN_B200_DEBUG_BOUNDS=1`` in the environment it loads
+the debug build ``libattn_b200_debug.so`` instead, whose kernels check their
+shared-memory, tensor-memory and output indices (``ATTN_FAULT_BOUNDS``).
 """
 from __future__ import annotations
 
@@ -17,7 +19,8 @@ import os
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_FILE = os.path.join(HERE, "libattn_b200.so")
+DEBUG_BOUNDS = os.environ.get("ATTN_B200_DEBUG_BOUNDS", "0") not in ("", "0")
+_LIB_FILE = os.path.join(HERE, "libattn_b200_debug.so" if DEBUG_BOUNDS else "libattn_b200.so")
 
 ATTN_OK = 0
 ATTN_ERR_INVALID_ARG = 1
@@ -36,6 +39,19 @@ ATTN_FAULT_TIMEOUT = 0x1
 ATTN_FAULT_BAD_BLOCK = 0x2
 ATTN_FAULT_BAD_LENGTH = 0x4
 ATTN_FAULT_PREFIX_MISMATCH = 0x8
+ATTN_FAULT_BOUNDS = 0x10
+
+# Bounds-check sites of the debug build (attn_bounds_site_t).
+BOUNDS_SITES = {
+    "PREFILL_SMEM_Q": 1, "PREFILL_SMEM_KV": 2, "PREFILL_TABLE": 3, "PREFILL_TMEM_S": 4, "PREFILL_TMEM_O": 5,
+    "PREFILL_SMEM_STAGE": 6, "PREFILL_SMEM_VFIX": 7, "PREFILL_OUT": 8, "DECODE_TABLE": 9, "DECODE_SMEM": 10,
+    "DECODE_PARTIAL": 11, "COMBINE": 12, "BWD_SMEM": 13, "BWD_TMEM": 14, "BWD_OUT": 15,
+}
+
+
+def fault_site(word: int) -> int:
+    """The site of the first failed bounds check recorded in an error word (0: none)."""
+    return (int(word) >> 16) & 0xFF
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
@@ -128,6 +144,10 @@ def _load():
     lib.attn_set_wait_limit.restype = None
     lib.attn_selftest_exp2.argtypes = [_vp, _vp, _vp, ctypes.c_int, _vp]
     lib.attn_selftest_exp2.restype = ctypes.c_int
+    lib.attn_debug_bounds_enabled.argtypes = []
+    lib.attn_debug_bounds_enabled.restype = ctypes.c_int
+    lib.attn_debug_plant_bounds.argtypes = [ctypes.c_int]
+    lib.attn_debug_plant_bounds.restype = ctypes.c_int
     lib.attn_decode_persistent_workspace.argtypes = [ctypes.POINTER(DecodeParams), ctypes.POINTER(ctypes.c_size_t)]
     lib.attn_decode_persistent_workspace.restype = ctypes.c_int
     lib.attn_decode_persistent_launch.argtypes = [ctypes.POINTER(DecodeParams), _vp, _vp, ctypes.c_size_t,
@@ -196,6 +216,17 @@ def sync_error_flags(error_flags) -> tuple[int, int]:
 def set_wait_limit(cycles: int = 0) -> None:
     """Diagnostic: clock-cycle bound of the prefill/backward pipeline waits (0 = the ~1 s default)."""
     LIB.attn_set_wait_limit(int(cycles))
+
+
+def debug_bounds_enabled() -> bool:
+    """True when the loaded library is the bounds-checking debug build."""
+    return bool(LIB.attn_debug_bounds_enabled())
+
+
+def debug_plant_bounds(site: int) -> None:
+    """Debug build: kernels launched from now on report a failed check at ``site``
+    (0 turns it off) while their accesses keep their real, checked indices."""
+    _check(LIB.attn_debug_plant_bounds(int(site)), "attn_debug_plant_bounds")
 
 
 def selftest_exp2(x):

@@ -13,6 +13,7 @@
 
 #include "attn.h"
 #include "internal.h"
+#include "bounds_check.cuh"
 
 namespace attn {
 
@@ -23,6 +24,10 @@ constexpr long long kDefaultWaitLimit = 2000000000LL;
 static std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
 long long pipeline_wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
+
+static std::atomic<int> g_planted_site{0};
+
+int planted_bounds_site() { return g_planted_site.load(std::memory_order_relaxed); }
 
 static bool mult8(int64_t s) { return (s % 8) == 0; }
 
@@ -281,6 +286,15 @@ void attn_decode_persistent_stop(attn_persistent_cmd* cmd) {
 
 void attn_set_wait_limit(long long cycles) {
   attn::g_wait_limit.store(cycles > 0 ? cycles : attn::kDefaultWaitLimit, std::memory_order_relaxed);
+}
+
+int attn_debug_bounds_enabled(void) { return ATTN_DEBUG_BOUNDS ? 1 : 0; }
+
+attn_status_t attn_debug_plant_bounds(int site) {
+  if (!ATTN_DEBUG_BOUNDS) return ATTN_ERR_UNSUPPORTED;
+  if (site < 0 || site > 255) return ATTN_ERR_INVALID_ARG;
+  attn::g_planted_site.store(site, std::memory_order_relaxed);
+  return ATTN_OK;
 }
 
 attn_status_t attn_status_from_flags(int32_t flags) {

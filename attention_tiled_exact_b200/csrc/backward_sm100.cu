@@ -44,6 +44,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include "bounds_check.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
@@ -76,6 +77,7 @@ struct Args {
   int grad_f32;
   int32_t* error_flags;
   long long wait_limit;  // cycle bound of every pipeline wait
+  int planted;           // debug build: bounds-check site reported as failed
 };
 
 template <int D>
@@ -279,10 +281,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int h = step_head(t), blk = step_blk(t);
         uint8_t* b0 = smem + L::RING_OFF + (2 * s) * L::TILE;
         uint8_t* b1 = b0 + L::TILE;
+        // The stage's two tiles and its per-row vectors stay inside the ring
+        // and the vector area.
+        if (!ATTN_IN_BOUNDS(s >= 0 && s < 2 && L::RING_OFF + (2 * s + 2) * L::TILE <= L::VEC_OFF &&
+                                L::VEC_OFF + (2 * s + 2) * BM * 4 <= L::BAR_OFF,
+                            ATTN_SITE_BWD_SMEM, a.error_flags, a.planted))
+          continue;
         if constexpr (KV) {
           // The step's per-column LSE and D ride on the same barrier.
           mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE + 2 * BM * 4);
           const long long vr = vec_row(h, blk);
+          if (!ATTN_IN_BOUNDS(h >= 0 && h < a.hq && blk >= 0 && blk < a.n_qb, ATTN_SITE_BWD_OUT, a.error_flags,
+                              a.planted))
+            continue;
           bulk_load(vec + (2 * s) * BM, a.lse2 + vr, BM * 4, &ring_full[s]);
           bulk_load(vec + (2 * s + 1) * BM, a.delta + vr, BM * 4, &ring_full[s]);
           for (int c = 0; c < L::CHUNKS; ++c) {
@@ -403,10 +414,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float nlse_r = -INFINITY, ndelta_r = 0.f;
     if constexpr (!KV) {
       const long long vr = vec_row(w.h, w.blk) + r;  // padded: -inf / 0 past Sq
-      nlse_r = a.lse2[vr];
-      ndelta_r = a.delta[vr];
+      if (ATTN_IN_BOUNDS(w.h >= 0 && w.h < a.hq && w.blk >= 0 && w.blk < a.n_qb && r >= 0 && r < BM,
+                         ATTN_SITE_BWD_OUT, a.error_flags, a.planted)) {
+        nlse_r = a.lse2[vr];
+        ndelta_r = a.delta[vr];
+      }
     }
     const float2 sl2x2 = make_float2(sl2, sl2);
+    // This warpgroup's S / dP columns and the accumulators stay inside the
+    // allocation.
+    const bool cols_ok = ATTN_IN_BOUNDS(half >= 0 && half < 2 && COL_DP + half * 64 + 64 <= COL_ACC &&
+                                            COL_ACC + (KV ? 2 : 1) * D <= TMEM_COLS,
+                                        ATTN_SITE_BWD_TMEM, a.error_flags, a.planted);
+    (void)cols_ok;
     bool ok = true;
     for (int t = 0; t < w.n_steps && ok; ++t) {
       const int s = t & 1;
@@ -441,8 +461,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int cc = 0; cc < 2; ++cc) {
         const int col = half * 64 + cc * 32;
         uint32_t sv[32], dv[32];
-        tmem_ld32(lane_base + COL_S + col, sv);
-        tmem_ld32(lane_base + COL_DP + col, dv);
+        if (cols_ok) {
+          tmem_ld32(lane_base + COL_S + col, sv);
+          tmem_ld32(lane_base + COL_DP + col, dv);
+        }
         tmem_ld_wait();
         uint32_t pk[16], dk[16];
 #pragma unroll
@@ -477,8 +499,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         // bf16 pairs over this half's first 32 columns, all read already.
-        if constexpr (KV) tmem_st16(lane_base + COL_S + half * 64 + cc * 16, pk);
-        tmem_st16(lane_base + COL_DP + half * 64 + cc * 16, dk);
+        if (cols_ok) {
+          if constexpr (KV) tmem_st16(lane_base + COL_S + half * 64 + cc * 16, pk);
+          tmem_st16(lane_base + COL_DP + half * 64 + cc * 16, dk);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
@@ -503,7 +527,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
         for (int cc = half * (D / 64); cc < (half + 1) * (D / 64); ++cc) {
           float x[32];
-          if (w.n_steps > 0) {
+          if (w.n_steps > 0 && cols_ok) {
             uint32_t v[32];
             tmem_ld32(lane_base + COL_ACC + o * D + cc * 32, v);
             tmem_ld_wait();
@@ -513,7 +537,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k < 32; ++k) x[k] = 0.f;  // no visible pair: the gradient is 0
           }
-          if (row_ok) store_slice(base, row_off, cc * 32, x, a.grad_f32);
+          if (row_ok && ATTN_IN_BOUNDS(w.b >= 0 && w.b < a.batch && (KV ? w.kvh < a.hkv : w.h < a.hq),
+                                       ATTN_SITE_BWD_OUT, a.error_flags, a.planted))
+            store_slice(base, row_off, cc * 32, x, a.grad_f32);
         }
       }
     }
@@ -726,6 +752,7 @@ attn_status_t launch_backward(const attn_backward_params& p, void* workspace, cu
   a.grad_f32 = p.grad_dtype == ATTN_DTYPE_F32;
   a.error_flags = p.error_flags;
   a.wait_limit = pipeline_wait_limit();
+  a.planted = planted_bounds_site();
   const long long kv_items = (long long)a.n_kb * p.batch * p.num_kv_heads;
   const long long q_items = (long long)a.n_qb * p.batch * p.num_q_heads;
   attn_status_t st;

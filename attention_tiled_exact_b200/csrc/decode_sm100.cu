@@ -43,6 +43,7 @@
 #include <string.h>
 #include <stdint.h>
 
+#include "bounds_check.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
@@ -72,6 +73,7 @@ struct Args {
   int batch, hq, hkv, max_blocks, num_blocks, split_tokens;
   float scale_log2;
   int32_t* error_flags;
+  int planted;  // debug build: bounds-check site reported as failed
 };
 
 template <int G, bool FP8 = false>
@@ -262,6 +264,10 @@ __device__ __forceinline__ void split_task(const Args& a, int split, int kvh, in
   const int n_mine = (blk_end - blk_begin - warp + WARPS - 1) / WARPS;
   auto block_of = [&](int n) { return blk_begin + warp + n * WARPS; };
   auto phys_of = [&](int blk, bool& valid) {
+    if (!ATTN_IN_BOUNDS(blk >= 0 && blk < a.max_blocks, ATTN_SITE_DECODE_TABLE, a.error_flags, a.planted)) {
+      valid = false;
+      return -1;
+    }
     const int ph = ld_input<COHERENT>(table + blk);
     valid = (ph >= 0) && (ph < a.num_blocks);
     return ph;
@@ -270,7 +276,9 @@ __device__ __forceinline__ void split_task(const Args& a, int split, int kvh, in
     if (n < n_mine) {
       bool valid;
       const int ph = phys_of(block_of(n), valid);
-      if (valid) {
+      [[maybe_unused]] constexpr int SLOT = (int)sizeof(sm.kv[0][0][0]);
+      if (valid && ATTN_IN_BOUNDS(warp >= 0 && warp < WARPS && n % NST >= 0 && ((CHUNKS16 - 1) * 32 + 31) * 16 + 16 <= SLOT,
+                                  ATTN_SITE_DECODE_SMEM, a.error_flags, a.planted)) {
         const long long off = ((long long)ph * a.hkv + kvh) * (BS * ROW);  // bytes
         const uint8_t* ksrc = a.k_cache + off;
         const uint8_t* vsrc = a.v_cache + off;
@@ -543,8 +551,11 @@ __device__ __forceinline__ void split_task(const Args& a, int split, int kvh, in
       if (d == 0 && a.lse) a.lse[row] = lse;
     } else {
       const long long rows = (long long)a.batch * a.hq;
-      a.part_o[((long long)split * rows + row) * D + d] = out;
-      if (d == 0) a.part_lse[(long long)split * rows + row] = lse;
+      if (ATTN_IN_BOUNDS(split >= 0 && split < max_splits && row >= 0 && row < rows, ATTN_SITE_DECODE_PARTIAL,
+                         a.error_flags, a.planted)) {
+        a.part_o[((long long)split * rows + row) * D + d] = out;
+        if (d == 0) a.part_lse[(long long)split * rows + row] = lse;
+      }
     }
   }
 }
@@ -572,7 +583,8 @@ __device__ __forceinline__ void combine_row(int row, const float* __restrict__ p
                                             const float* __restrict__ part_lse, int num_splits, int rows,
                                             const int32_t* __restrict__ splits_per_row,
                                             const int32_t* __restrict__ seq_lens, int split_tokens, int max_len,
-                                            int rows_per_seq, void* out_o, int out_f32, float* out_lse) {
+                                            int rows_per_seq, void* out_o, int out_f32, float* out_lse,
+                                            int32_t* flags = nullptr, int planted = 0) {
   constexpr int PER = HD / 32;  // floats per lane
   const int lane = lane_id();
   int n;
@@ -604,6 +616,7 @@ __device__ __forceinline__ void combine_row(int row, const float* __restrict__ p
     for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     lse = M + logf(sum);
     for (int s = 0; s < n; ++s) {
+      if (!ATTN_IN_BOUNDS(s < num_splits, ATTN_SITE_COMBINE, flags, planted)) break;
       const float ls = __ldcg(part_lse + (long long)s * rows + row);
       if (ls == -INFINITY) continue;  // weight 0: its partial is not read
       const float wgt = ex2_approx((ls - lse) * LOG2E);
@@ -639,11 +652,11 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float* __restric
                                                           int rows, const int32_t* __restrict__ splits_per_row,
                                                           const int32_t* __restrict__ seq_lens, int split_tokens,
                                                           int max_len, int rows_per_seq, void* out_o, int out_f32,
-                                                          float* out_lse) {
+                                                          float* out_lse, int32_t* flags, int planted) {
   const int row = blockIdx.x * (blockDim.x / 32) + warp_id();
   if (row >= rows) return;
   combine_row<HD>(row, part_o, part_lse, num_splits, rows, splits_per_row, seq_lens, split_tokens, max_len,
-                  rows_per_seq, out_o, out_f32, out_lse);
+                  rows_per_seq, out_o, out_f32, out_lse, flags, planted);
 }
 
 }  // namespace combine
@@ -779,6 +792,7 @@ attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan,
   a.split_tokens = plan.split_tokens;
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.error_flags = p.error_flags;
+  a.planted = planted_bounds_site();
   attn_status_t st;
   switch (p.num_q_heads / p.num_kv_heads) {
     case 1: st = fp8 ? launch_decode_g<1, true>(a, plan, stream) : launch_decode_g<1, false>(a, plan, stream); break;
@@ -789,25 +803,26 @@ attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan,
   }
   if (st != ATTN_OK || plan.max_splits <= 1) return st;
   return launch_combine(a.part_o, a.part_lse, plan.max_splits, (int)rows, p.head_dim, nullptr, p.seq_lens,
-                        plan.split_tokens, p.num_q_heads, p.o, p.o_dtype, p.lse, stream);
+                        plan.split_tokens, p.num_q_heads, p.o, p.o_dtype, p.lse, stream, p.error_flags);
 }
 
 attn_status_t launch_combine(const float* part_o, const float* part_lse, int num_splits, int rows, int head_dim,
                              const int32_t* splits_per_row, const int32_t* seq_lens, int split_tokens,
                              int rows_per_seq, void* out_o, attn_dtype_t out_dtype, float* out_lse,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, int32_t* error_flags) {
   if (rows == 0) return ATTN_OK;
+  const int planted = planted_bounds_site();
   const int warps = 8;
   const int grid = (rows + warps - 1) / warps;
   const int max_len = num_splits * split_tokens;
   if (head_dim == 128)
     combine::lse_combine_kernel<128><<<grid, warps * 32, 0, stream>>>(
         part_o, part_lse, num_splits, rows, splits_per_row, seq_lens, split_tokens, max_len, rows_per_seq, out_o,
-        out_dtype == ATTN_DTYPE_F32, out_lse);
+        out_dtype == ATTN_DTYPE_F32, out_lse, error_flags, planted);
   else
     combine::lse_combine_kernel<64><<<grid, warps * 32, 0, stream>>>(
         part_o, part_lse, num_splits, rows, splits_per_row, seq_lens, split_tokens, max_len, rows_per_seq, out_o,
-        out_dtype == ATTN_DTYPE_F32, out_lse);
+        out_dtype == ATTN_DTYPE_F32, out_lse, error_flags, planted);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -963,7 +978,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_persistent_kernel(const Per
         __threadfence();
         for (int g = warp_id(); g < G; g += WARPS)
           combine::combine_row<D>((b * hq) + kvh * G + g, a.part_o, a.part_lse, nsplit, batch * hq, nullptr,
-                                  a.seq_lens, T, nsplit * T, hq, a.o, a.o_f32, a.lse);
+                                  a.seq_lens, T, nsplit * T, hq, a.o, a.o_f32, a.lse, a.error_flags, a.planted);
         if (threadIdx.x == 0) sync[MB_COUNTERS + b * hkv + kvh] = 0;  // ready for the next step
       }
       __syncthreads();
@@ -1071,6 +1086,7 @@ attn_status_t launch_decode_persistent(const attn_decode_params& p, int32_t* cmd
   a.num_blocks = p.num_blocks;
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.error_flags = p.error_flags;
+  a.planted = planted_bounds_site();
   pa.cmd = cmd_dev;
   pa.partials = reinterpret_cast<float*>(workspace);
   pa.sync = sync;

@@ -47,6 +47,10 @@ class DeviceOnce {
 // (attn_set_wait_limit; about one second by default).
 long long pipeline_wait_limit();
 
+// The bounds-check site that debug kernels launched now report as failed
+// (attn_debug_plant_bounds; 0: none).
+int planted_bounds_site();
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 
@@ -78,7 +82,7 @@ attn_status_t prepare_decode(const attn_decode_params& p);
 attn_status_t launch_combine(const float* part_o, const float* part_lse, int num_splits, int rows,
                              int head_dim, const int32_t* splits_per_row, const int32_t* seq_lens,
                              int split_tokens, int rows_per_seq, void* out_o, attn_dtype_t out_dtype,
-                             float* out_lse, cudaStream_t stream);
+                             float* out_lse, cudaStream_t stream, int32_t* error_flags = nullptr);
 
 // Persistent decode: workspace size and launch (arguments validated by the
 // caller; cmd_dev is the device address of the host command block).

@@ -47,6 +47,7 @@
 #include <string.h>
 
 #include "exp2_poly.cuh"
+#include "bounds_check.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
@@ -114,6 +115,8 @@ struct Args {
   long long lse_rows;  // rows per (batch, head) of the LSE tensor: seqlen_q, or total_q when packed
   int32_t* error_flags;
   long long wait_limit;  // cycle bound of every pipeline wait
+  int planted;           // debug build: bounds-check site reported as failed
+  long long out_rows;    // rows per (batch, head) of O: seqlen_q, or total_q when packed
   // paged keys/values (PAGED kernels only)
   const int32_t* block_table;
   int max_blocks;
@@ -487,9 +490,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive_expect_tx(q_full, (w.active[0] + w.active[1]) * L::Q_TILE);
         for (int t = 0; t < 2; ++t) {
           if (!w.active[t]) continue;
-          for (int c = 0; c < L::CHUNKS; ++c)
-            tma_load_4d(smem + L::Q_OFF + t * L::Q_TILE + c * (BM * 128), &tm_q, q_full, c * 64,
-                        w.qoff + w.row0[t], w.head[t], w.qb);
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            const int off = L::Q_OFF + t * L::Q_TILE + c * (BM * 128);
+            if (ATTN_IN_BOUNDS(off >= L::Q_OFF && off + BM * 128 <= L::Q_OFF + 2 * L::Q_TILE,
+                               ATTN_SITE_PREFILL_SMEM_Q, args.error_flags, args.planted))
+              tma_load_4d(smem + off, &tm_q, q_full, c * 64, w.qoff + w.row0[t], w.head[t], w.qb);
+          }
         }
         ++nq;
         // Bring the next item's Q tiles into L2 now, so that its shared-memory
@@ -519,7 +525,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < BK / 16; ++j) {
               const int tok = blk * BK + j * 16;
-              e[j] = tok < w.sk ? table[tok >> 4] : args.num_blocks;
+              e[j] = args.num_blocks;
+              if (tok < w.sk && ATTN_IN_BOUNDS((tok >> 4) < args.max_blocks, ATTN_SITE_PREFILL_TABLE,
+                                               args.error_flags, args.planted))
+                e[j] = table[tok >> 4];
             }
 #pragma unroll
             for (int j = 0; j < BK / 16; ++j) {
@@ -539,15 +548,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (cnt >= stages && !mbar_wait_bounded(&empty[s], ((cnt / stages) - 1) & 1, abort_flag, args.wait_limit))
             return false;
           mbar_arrive_expect_tx(&full[s], L::KV_TILE);
-          uint8_t* dst = smem + (is_v ? L::V_OFF : L::K_OFF) + s * L::KV_TILE;
+          const int ring = is_v ? L::V_OFF : L::K_OFF;
+          uint8_t* dst = smem + ring + s * L::KV_TILE;
           const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
           if constexpr (!PAGED) {
             for (int c = 0; c < L::CHUNKS; ++c)
-              tma_load_4d(dst + c * (BK * 128), tm, &full[s], c * 64, blk * BK, w.kvh, w.b);
+              if (ATTN_IN_BOUNDS(s >= 0 && s < stages && (s * L::KV_TILE + c * (BK * 128) + BK * 128 <=
+                                                          stages * L::KV_TILE),
+                                 ATTN_SITE_PREFILL_SMEM_KV, args.error_flags, args.planted))
+                tma_load_4d(dst + c * (BK * 128), tm, &full[s], c * 64, blk * BK, w.kvh, w.b);
           } else {
             for (int j = 0; j < BK / 16; ++j)
               for (int c = 0; c < L::CHUNKS; ++c)
-                tma_load_4d(dst + c * (BK * 128) + j * (16 * 128), tm, &full[s], c * 64, 0, w.kvh, phys[j]);
+                if (ATTN_IN_BOUNDS(s >= 0 && s < stages && (s * L::KV_TILE + c * (BK * 128) + j * (16 * 128) +
+                                                                16 * 128 <= stages * L::KV_TILE),
+                                   ATTN_SITE_PREFILL_SMEM_KV, args.error_flags, args.planted))
+                  tma_load_4d(dst + c * (BK * 128) + j * (16 * 128), tm, &full[s], c * 64, 0, w.kvh, phys[j]);
           }
           ++cnt;
           return true;
@@ -589,6 +605,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t qa = q_lo + (uint32_t)((t * L::Q_TILE) >> 4);
         const uint32_t ka = k_lo + (uint32_t)(((kg % KSTAGES) * L::KV_TILE) >> 4);
         const uint32_t d = tmem_base + t * 128;
+        if (!ATTN_IN_BOUNDS(t >= 0 && t < 2 && t * 128 + BK <= 256, ATTN_SITE_PREFILL_TMEM_S, args.error_flags,
+                            args.planted))
+          return;
         static_for<0, D / 16>([&](auto c) {
           constexpr int kk = decltype(c)::value;
           constexpr uint32_t a_off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
@@ -601,6 +620,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto issue_pv = [&](int t, int vg, bool first) {
         const uint32_t va = v_lo + (uint32_t)(((vg % VSTAGES) * L::KV_TILE) >> 4);
         const uint32_t d = tmem_base + 256 + t * 128, a = tmem_base + t * 128;
+        if (!ATTN_IN_BOUNDS(t >= 0 && t < 2 && 256 + t * 128 + D <= (int)TMEM_COLS, ATTN_SITE_PREFILL_TMEM_O,
+                            args.error_flags, args.planted))
+          return;
         static_for<0, BK / 16>([&](auto c) {
           constexpr int kk = decltype(c)::value;
           constexpr uint32_t b_off = (kk * 16 * 128) >> 4;
@@ -685,6 +707,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tS = lane_base + t * 128;
     const uint32_t tO = lane_base + 256 + t * 128;
     const float sl2 = args.scale_log2;
+    // This warp's S / P and O columns stay inside the allocation.
+    const bool s_cols = ATTN_IN_BOUNDS(t >= 0 && t < 2 && t * 128 + BK <= 256, ATTN_SITE_PREFILL_TMEM_S,
+                                       args.error_flags, args.planted);
+    const bool o_cols = ATTN_IN_BOUNDS(t >= 0 && t < 2 && 256 + t * 128 + D <= (int)TMEM_COLS,
+                                       ATTN_SITE_PREFILL_TMEM_O, args.error_flags, args.planted);
+    (void)s_cols;
+    (void)o_cols;
     int gb = 0;  // this tile's blocks so far (all items)
     int kb = 0;  // K / V blocks loaded before the current item
     int nf = 0;  // items this tile finished (o_full phases)
@@ -713,7 +742,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         uint32_t sb[BK];
 #pragma unroll
-        for (int c = 0; c < BK / 32; ++c) tmem_ld32(tS + c * 32, &sb[c * 32]);
+        for (int c = 0; c < BK / 32; ++c)
+          if (s_cols) tmem_ld32(tS + c * 32, &sb[c * 32]);
         tmem_ld_wait();
         float s[BK];
 #pragma unroll
@@ -740,7 +770,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float alpha = upd ? ex2_approx(m2 - m_new) : 1.f;
         if (upd) m2 = m_new;
         const float m_off = (m2 == -INFINITY) ? 0.f : m2;
-        if (i > 0 && __any_sync(0xffffffffu, upd)) {
+        if (i > 0 && __any_sync(0xffffffffu, upd) && o_cols) {
           // Rescale O in place. Its last writer, P V of the previous block,
           // has completed: the commit that signalled this S tracks every
           // earlier MMA of the issuer.
@@ -754,11 +784,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_st32(tO + c * 32, o);
           }
         }
-        float2 acc;
-        if (need_mask)
+        float2 acc = make_float2(0.f, 0.f);
+        if (!s_cols) {
+        } else if (need_mask) {
           exp_pack_store<EMU8, true>(s, sl2, m_off, tS, acc);
-        else
+        } else {
           exp_pack_store<EMU8>(s, sl2, m_off, tS, acc);
+        }
         l = l * alpha + (acc.x + acc.y);
         if (v_fix && i == nt - 1) {
           const int vg = kb + i, vs = vg % VSTAGES;
@@ -773,7 +805,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int u = r; u < units; u += 128) {
             const int unit = u & 7, rc = u >> 3;
             const int row = r0 + rc % (BK - r0), c = rc / (BK - r0);
-            *reinterpret_cast<uint4*>(vblk + c * (BK * 128) + row * 128 + unit * 16) = make_uint4(0u, 0u, 0u, 0u);
+            const int off = c * (BK * 128) + row * 128 + unit * 16;
+            if (ATTN_IN_BOUNDS(vs >= 0 && vs < VSTAGES && row >= 0 && row < BK && off >= 0 && off + 16 <= L::KV_TILE,
+                               ATTN_SITE_PREFILL_SMEM_VFIX, args.error_flags, args.planted))
+              *reinterpret_cast<uint4*>(vblk + off) = make_uint4(0u, 0u, 0u, 0u);
           }
           fence_proxy_async_smem();
         }
@@ -789,7 +824,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool store = qrow < w.sq;
       const bool empty = !(l > 0.f);
       const float inv_l = empty ? 0.f : 1.f / l;
-      if (args.lse && store) {
+      // The row, head and batch coordinates of this row's O and LSE (rows
+      // past the sequence end are not stored).
+      const bool out_ok =
+          !store || ATTN_IN_BOUNDS(w.qoff + qrow >= 0 && w.qoff + qrow < args.out_rows && w.head[t] >= 0 &&
+                                       w.head[t] < args.hq && w.qb >= 0 && w.qb < (args.cu_seqlens_q ? 1 : args.batch),
+                                   ATTN_SITE_PREFILL_OUT, args.error_flags, args.planted);
+      if (args.lse && store && out_ok) {
         const float lse = empty ? -INFINITY : (m2 + log2f(l)) * 0.69314718055994530942f;
         args.lse[((long long)w.qb * args.hq + w.head[t]) * args.lse_rows + w.qoff + qrow] = lse;
       }
@@ -805,23 +846,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (args.o_tma && w.row0[t] + sub * 32 + 32 <= w.sq) {  // warp-uniform
         uint8_t* stage = smem + L::O_OFF + warp * L::W_STAGE;
         const int r0 = w.qoff + w.row0[t] + sub * 32;
-        if (args.o_f32)
-          store_rows_tma<D, true>(&tm_o, stage, tO, has_keys, inv_l, r0, w.head[t], w.qb);
-        else
-          store_rows_tma<D, false>(&tm_o, stage, tO, has_keys, inv_l, r0, w.head[t], w.qb);
+        // The warp's staging area (one 4 KB box per round) and its 32 output
+        // rows.
+        if (ATTN_IN_BOUNDS(warp >= 0 && warp < SOFTMAX_WARPS &&
+                               L::O_OFF + (warp + 1) * L::W_STAGE <= L::BAR_OFF && 4096 <= L::W_STAGE &&
+                               r0 >= 0 && r0 + 32 <= args.out_rows,
+                           ATTN_SITE_PREFILL_SMEM_STAGE, args.error_flags, args.planted)) {
+          if (args.o_f32)
+            store_rows_tma<D, true>(&tm_o, stage, tO, has_keys && o_cols, inv_l, r0, w.head[t], w.qb);
+          else
+            store_rows_tma<D, false>(&tm_o, stage, tO, has_keys && o_cols, inv_l, r0, w.head[t], w.qb);
+        }
         continue;
       }
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        if (has_keys) {  // warp-uniform: every lane issues the collective load
+        if (has_keys && o_cols) {  // warp-uniform: every lane issues the collective load
           tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
         } else {
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
-        if (!store) continue;
+        if (!store || !out_ok) continue;
         if (args.o_f32) {
           float* dst = reinterpret_cast<float*>(args.o) + obase + c * 32;
 #pragma unroll
@@ -1008,6 +1056,8 @@ attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream) 
   if (!a.o_tma) to = tq;  // never read
   a.error_flags = p.error_flags;
   a.wait_limit = pipeline_wait_limit();
+  a.planted = planted_bounds_site();
+  a.out_rows = a.lse_rows;
   if (paged) {
     a.block_table = p.block_table;
     a.max_blocks = p.max_blocks_per_seq;

@@ -68,6 +68,38 @@ typedef enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1, ATTN_DTYPE_FP8_E4M3 = 2 
 #define ATTN_FAULT_BAD_BLOCK 0x2    /* a block-table entry was outside [0, num_blocks) */
 #define ATTN_FAULT_BAD_LENGTH 0x4   /* a sequence length exceeded its block table or was negative */
 #define ATTN_FAULT_PREFIX_MISMATCH 0x8 /* attn_decode_paged_shared_prefix: a table row's prefix blocks differ from row 0's */
+#define ATTN_FAULT_BOUNDS 0x10      /* debug build only: an index failed its bounds check (site in bits 16..23) */
+/* The site (attn_bounds_site_t) of the first failed bounds check of a debug
+ * build, 0 if none; the word's other bits are the ATTN_FAULT_* flags. */
+#define ATTN_FAULT_SITE(word) (((word) >> 16) & 0xff)
+
+/*
+ * Bounds-check sites of the debug build (libattn_b200_debug.so, compiled with
+ * ATTN_DEBUG_BOUNDS=1). Before each of these accesses the debug kernels check
+ * the computed index against the extent it must stay within; a failed check
+ * skips the access (no trap), ORs ATTN_FAULT_BOUNDS into error_flags and, if
+ * it is the first, records its site in bits 16..23. A skipped copy can leave a
+ * pipeline wait unfinished, which then also reports ATTN_FAULT_TIMEOUT. The
+ * release library carries none of these checks.
+ */
+typedef enum {
+  ATTN_SITE_NONE = 0,
+  ATTN_SITE_PREFILL_SMEM_Q = 1,      /* Q tile copy: destination inside the Q buffer */
+  ATTN_SITE_PREFILL_SMEM_KV = 2,     /* K / V tile copy: ring slot inside its ring */
+  ATTN_SITE_PREFILL_TABLE = 3,       /* paged prefill: block-table column < max_blocks */
+  ATTN_SITE_PREFILL_TMEM_S = 4,      /* S / P columns (load, store, MMA target) inside the allocation */
+  ATTN_SITE_PREFILL_TMEM_O = 5,      /* O columns (rescale, epilogue, MMA target) inside the allocation */
+  ATTN_SITE_PREFILL_SMEM_STAGE = 6,  /* output staging inside the warp's staging area */
+  ATTN_SITE_PREFILL_SMEM_VFIX = 7,   /* zeroing of V rows past the sequence end inside the V slot */
+  ATTN_SITE_PREFILL_OUT = 8,         /* O / LSE row, head and batch inside the output tensors */
+  ATTN_SITE_DECODE_TABLE = 9,        /* decode: block-table column < max_blocks */
+  ATTN_SITE_DECODE_SMEM = 10,        /* decode: K / V staging inside the split's shared buffer */
+  ATTN_SITE_DECODE_PARTIAL = 11,     /* decode: split index < the workspace's splits per row */
+  ATTN_SITE_COMBINE = 12,            /* combine: split index < num_splits */
+  ATTN_SITE_BWD_SMEM = 13,           /* backward: ring stage and per-row vectors inside shared memory */
+  ATTN_SITE_BWD_TMEM = 14,           /* backward: S / dP / accumulator columns inside the allocation */
+  ATTN_SITE_BWD_OUT = 15             /* backward: gradient row / vector row inside its tensor */
+} attn_bounds_site_t;
 
 /*
  * Prefill: tiled attention over a whole query block, one pass over K/V with
@@ -508,6 +540,20 @@ ATTN_API attn_status_t attn_sync_error_flags(const int32_t* error_flags, attn_st
  */
 ATTN_API void attn_set_wait_limit(long long cycles);
 ATTN_API attn_status_t attn_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int n, attn_stream_t stream);
+
+/*
+ * attn_debug_bounds_enabled: 1 in the debug build (bounds checks compiled
+ * in), 0 in the release library.
+ *
+ * attn_debug_plant_bounds: debug build only. Every kernel launched after the
+ * call reports a failed check at `site` (attn_bounds_site_t) each time it
+ * reaches that site, as if its index were out of range, while the access
+ * itself still uses the real, checked index: it shows that the site's check
+ * is wired and recorded, without touching anything out of range. site 0 turns
+ * it off. Process-wide. The release library returns ATTN_ERR_UNSUPPORTED.
+ */
+ATTN_API int attn_debug_bounds_enabled(void);
+ATTN_API attn_status_t attn_debug_plant_bounds(int site);
 
 /* Static, human-readable name of a status code. */
 ATTN_API const char* attn_status_string(attn_status_t status);

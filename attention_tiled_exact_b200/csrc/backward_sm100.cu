@@ -80,28 +80,54 @@ struct Args {
   int planted;           // debug build: bounds-check site reported as failed
 };
 
+// dK/dV kernel shared memory: K_j and V_j resident; a two-stage ring of
+// (Q_i, dO_i) pairs with that query block's -LSE log2 e and -D per column.
 template <int D>
-struct Layout {
+struct KvLayout {
   static constexpr int CHUNKS = D / 64;  // 64-column (128-byte) boxes per row
   static constexpr int TILE = BM * D * 2;
-  // Resident tiles A0, A1 (dK/dV kernel: K_j, V_j; dQ kernel: Q_i, dO_i) and
-  // a two-stage ring of streamed pairs B0, B1 (Q_i, dO_i or K_j, V_j).
-  static constexpr int A0_OFF = 0;
-  static constexpr int A1_OFF = TILE;
-  static constexpr int RING_OFF = 2 * TILE;            // stage s: B0 at + 2 s TILE, B1 at + (2 s + 1) TILE
-  static constexpr int VEC_OFF = RING_OFF + 4 * TILE;  // [stage][lse2, delta][BM] floats (dK/dV kernel)
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = TILE;
+  static constexpr int RING_OFF = 2 * TILE;            // stage s: Q at + 2 s TILE, dO at + (2 s + 1) TILE
+  static constexpr int VEC_OFF = RING_OFF + 4 * TILE;  // [stage][lse2, delta][BM] floats
   static constexpr int BAR_OFF = VEC_OFF + 2 * 2 * BM * 4;
-  // a_full, ring_full[2], ring_empty[2], sdp_full[2], ps_full[2], acc_full, mma_done
+  // a_full, ring_full[2], ring_empty[2], s_full, dp_full, p_full, ds_full, acc_full, mma_done
   static constexpr int NUM_BARS = 11;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem address, abort flag
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
 };
 
-// TMEM columns: S (or S^T) at 0, dP (or dP^T) at 128, each in two 64-column
-// halves; accumulators from 256 (dK/dV kernel: dV at 256, dK at 256 + D; dQ
-// kernel: dQ at 256). Half g's bf16 P / dS pairs go over the first 32
-// columns of that half.
-constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC = 256;
+// dQ kernel shared memory: Q_i and dO_i resident; K_j in a three-slot ring
+// (S_j is issued two steps ahead and dQ += dS_j K_j reads K_j last), V_j in a
+// two-slot ring.
+template <int D>
+struct QLayout {
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int TILE = BM * D * 2;
+  static constexpr int K_SLOTS = 3;
+  static constexpr int V_SLOTS = 2;
+  static constexpr int Q_OFF = 0;
+  static constexpr int DO_OFF = TILE;
+  static constexpr int K_OFF = 2 * TILE;
+  static constexpr int V_OFF = K_OFF + K_SLOTS * TILE;
+  static constexpr int BAR_OFF = V_OFF + V_SLOTS * TILE;
+  // a_full, k_full[3], k_empty[3], v_full[2], v_empty[2], sdp_full, ps_full, acc_full, mma_done
+  static constexpr int NUM_BARS = 1 + 2 * K_SLOTS + 2 * V_SLOTS + 4;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+};
+
+// Tensor memory (512 columns). Every S-like product is one 128 x 128 tile
+// (N = 128: a tcgen05.mma of N = 64 costs nearly as long as one of N = 128,
+// measured), so the buffers are whole tiles:
+//   dK/dV kernel: S^T and dP^T of a step alternate between buffers X (0) and
+//   Y (128); dV at 256, dK at 256 + D. The S^T buffer then holds P^T (bf16
+//   pairs) over the first 32 columns of each 64-column half and dS^T over the
+//   last 32.
+//   dQ kernel: S and dP of step t are products 2t and 2t + 1, product p in
+//   buffer p mod 3 (columns 0, 128, 256); dQ at 384. The dP buffer then holds
+//   dS (bf16 pairs) over the first 32 columns of each half.
+constexpr uint32_t COL_ACC_KV = 256, COL_ACC_Q = 384;
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
   return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, limit));
@@ -113,6 +139,16 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                    smem_addr(dst)),
                "l"(src), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
+}
+
+// Four consecutive floats from shared memory (32-bit shared address). Not
+// ordered against the mbarrier waits by a memory clobber: every use sits after
+// the wait that made the data visible, in the same thread, and volatile asm
+// keeps its place among the other volatile asm statements.
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
 }
 
 // Stores one 32-column slice of a gradient row (fp32 or bf16).
@@ -130,29 +166,26 @@ __device__ __forceinline__ void store_slice(void* base, long long off, int col0,
   }
 }
 
-// X[:, half] = A (BM x D) * B[half rows] (64 x D)^T over head_dim: both
-// operands K-major; the B half starts 64 rows (8 KB) into each column box.
-template <int D, int HALF>
-__device__ __forceinline__ void issue_s_half(uint32_t d_col, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
-                                             uint32_t idesc) {
+// X (128 x 128) = A (BM x D) * B (BM x D)^T over head_dim, both operands
+// K-major 128-row tiles.
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t d_col, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc) {
   static_for<0, D / 16>([&](auto c) {
     constexpr int kk = decltype(c)::value;
-    constexpr uint32_t a_off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
-    constexpr uint32_t b_off = a_off + ((HALF * 64 * 128) >> 4);
-    mma_ss_lo<a_off, b_off>(d_col, a_lo, b_lo, hi, idesc, kk > 0 ? 1u : 0u);
+    constexpr uint32_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+    mma_ss_lo<off, off>(d_col, a_lo, b_lo, hi, idesc, kk > 0 ? 1u : 0u);
   });
 }
 
-// ACC += X[:, half] (bf16 in TMEM) * B[half rows] (64 rows = the reduction x D),
-// B MN-major.
-template <int HALF>
-__device__ __forceinline__ void issue_acc_half(uint32_t d_col, uint32_t a_col, uint32_t b_lo, uint32_t hi,
-                                               uint32_t idesc, bool first) {
-  static_for<0, 4>([&](auto c) {
-    constexpr int k = decltype(c)::value;
-    constexpr int kk = HALF * 4 + k;  // 16-row step of B
+// ACC += X (bf16 pairs in TMEM: half h's 64 reduction rows over columns
+// a_col + 64 h + [0, 32)) * B (128 reduction rows x D, MN-major), both halves.
+__device__ __forceinline__ void issue_acc(uint32_t d_col, uint32_t a_col, uint32_t b_lo, uint32_t hi,
+                                          uint32_t idesc, bool first) {
+  static_for<0, 8>([&](auto c) {
+    constexpr int kk = decltype(c)::value;   // 16-row step of B
+    constexpr int a_off = (kk >> 2) * 64 + (kk & 3) * 8;
     constexpr uint32_t b_off = (kk * 16 * 128) >> 4;
-    mma_ts_lo<HALF * 64 + k * 8, b_off>(d_col, a_col, b_lo, hi, idesc, (first && HALF == 0 && k == 0) ? 0u : 1u);
+    mma_ts_lo<a_off, b_off>(d_col, a_col, b_lo, hi, idesc, (first && kk == 0) ? 0u : 1u);
   });
 }
 
@@ -207,35 +240,92 @@ __device__ __forceinline__ Work decode_work(const Args& a) {
   return w;
 }
 
+// Stores this warpgroup's half of the columns of n_out accumulators of its
+// rows (gradient rows past the sequence end are not written).
 template <int D, bool KV>
+__device__ __forceinline__ void store_grads(const Args& a, const Work& w, uint32_t lane_base, uint32_t col_acc,
+                                            int half, int row_pos, bool has_acc) {
+  const bool row_ok = row_pos < (KV ? a.seqlen_k : a.seqlen_q);
+  const int n_out = KV ? 2 : 1;
+  for (int o = 0; o < n_out; ++o) {
+    // dK/dV kernel: o = 0 -> dV (unscaled), o = 1 -> dK (scale); dQ kernel: dQ (scale).
+    const bool is_dv = KV && o == 0;
+    void* base = KV ? (is_dv ? a.dv : a.dk) : a.dq;
+    const long long row_off =
+        KV ? (is_dv ? (long long)w.b * a.dv_bs + (long long)w.kvh * a.dv_hs + (long long)row_pos * a.dv_rs
+                    : (long long)w.b * a.dk_bs + (long long)w.kvh * a.dk_hs + (long long)row_pos * a.dk_rs)
+           : (long long)w.b * a.dq_bs + (long long)w.h * a.dq_hs + (long long)row_pos * a.dq_rs;
+    const float mul = is_dv ? 1.f : a.scale;
+#pragma unroll 1
+    for (int cc = half * (D / 64); cc < (half + 1) * (D / 64); ++cc) {
+      float x[32];
+      if (has_acc) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + col_acc + o * D + cc * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(v[k]) * mul;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) x[k] = 0.f;  // no visible pair: the gradient is 0
+      }
+      if (row_ok && ATTN_IN_BOUNDS(w.b >= 0 && w.b < a.batch && (KV ? w.kvh < a.hkv : w.h < a.hq),
+                                   ATTN_SITE_BWD_OUT, a.error_flags, a.planted))
+        store_slice(base, row_off, cc * 32, x, a.grad_f32);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK / dV: one CTA per (batch, kv head, 128-key block j); K_j and V_j stay in
+// shared memory while (Q_i, dO_i) of every query head of the group and every
+// query block i that sees block j stream through. Per step t (one (head, i)):
+//   S^T = K_j Q_i^T into buffer SB (X for even t, Y for odd), dP^T = V_j dO_i^T
+//   into the other buffer DB;
+//   phase 1 (elementwise, one key row per thread, each warpgroup 64 query
+//   columns): P^T = 2^(S^T scale log2 e - LSE log2 e), written as bf16 over
+//   the first 32 columns of its half of SB and kept in registers;
+//   dV += P^T dO_i as soon as every warp has written P^T;
+//   phase 2: dS^T = P^T (dP^T - D) over the last 32 columns of its half of SB;
+//   then S^T of step t + 1 goes into DB (free: dP^T was read), dK += dS^T Q_i,
+//   and dP^T of step t + 1 into SB (after dV and dK read it: MMAs from one
+//   thread run in issue order).
+// So the next step's S^T is computed while this step's dK accumulates, and
+// phase 1 of the next step overlaps the tensor core's dK and dP^T.
+template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Args a) {
-  using L = Layout<D>;
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const Args a) {
+  using L = KvLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* a_full = bars;
   uint64_t* ring_full = bars + 1;
   uint64_t* ring_empty = bars + 3;
-  uint64_t* sdp_full = bars + 5;  // per half: S and dP of that half are in TMEM
-  uint64_t* ps_full = bars + 7;   // per half: its warpgroup wrote P / dS into TMEM
+  uint64_t* s_full = bars + 5;   // S^T of the step is in TMEM
+  uint64_t* dp_full = bars + 6;  // dP^T of the step is in TMEM
+  uint64_t* p_full = bars + 7;   // every elementwise warp wrote P^T
+  uint64_t* ds_full = bars + 8;  // every elementwise warp wrote dS^T
   uint64_t* acc_full = bars + 9;
   uint64_t* mma_done = bars + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   const int warp = warp_id();
   const int lane = lane_id();
-  const Work w = decode_work<KV>(a);
+  const Work w = decode_work<true>(a);
 
   if (threadIdx.x == 0) {
     mbar_init(a_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_empty[s], 1);
-      mbar_init(&sdp_full[s], 1);
-      mbar_init(&ps_full[s], 4);  // one arrival per warp of the half's warpgroup
     }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, EW_WARPS);
+    mbar_init(ds_full, EW_WARPS);
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -250,11 +340,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Streamed step t: query head and block (dK/dV kernel) or key block (dQ kernel).
-  auto step_head = [&](int t) { return KV ? w.kvh * a.group + t / w.per_head : w.h; };
-  auto step_blk = [&](int t) { return KV ? w.first + t % w.per_head : t; };
+  // Streamed step t: query head and query block.
+  auto step_head = [&](int t) { return w.kvh * a.group + t / w.per_head; };
+  auto step_blk = [&](int t) { return w.first + t % w.per_head; };
   // Padded per-row vectors of query block i of head h.
   auto vec_row = [&](int h, int i) { return (((long long)w.b * a.hq + h) * a.n_qb + i) * BM; };
+  auto sb_col = [](int t) { return (uint32_t)((t & 1) * 128); };  // S^T, then P^T / dS^T, of step t
+  auto db_col = [](int t) { return (uint32_t)(128 - (t & 1) * 128); };  // dP^T of step t
 
   if (warp == TMA_WARP) {
     if (lane == 0 && w.n_steps > 0) {
@@ -266,13 +358,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(a_full, 2 * L::TILE);
       for (int c = 0; c < L::CHUNKS; ++c) {
-        if constexpr (KV) {
-          tma_load_4d(smem + L::A0_OFF + c * (BM * 128), &tm_k, a_full, c * 64, w.blk * BM, w.kvh, w.b);
-          tma_load_4d(smem + L::A1_OFF + c * (BM * 128), &tm_v, a_full, c * 64, w.blk * BM, w.kvh, w.b);
-        } else {
-          tma_load_4d(smem + L::A0_OFF + c * (BM * 128), &tm_q, a_full, c * 64, w.blk * BM, w.h, w.b);
-          tma_load_4d(smem + L::A1_OFF + c * (BM * 128), &tm_do, a_full, c * 64, w.blk * BM, w.h, w.b);
-        }
+        tma_load_4d(smem + L::K_OFF + c * (BM * 128), &tm_k, a_full, c * 64, w.blk * BM, w.kvh, w.b);
+        tma_load_4d(smem + L::V_OFF + c * (BM * 128), &tm_v, a_full, c * 64, w.blk * BM, w.kvh, w.b);
       }
       int t = 0;
       for (; t < w.n_steps; ++t) {
@@ -287,25 +374,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                 L::VEC_OFF + (2 * s + 2) * BM * 4 <= L::BAR_OFF,
                             ATTN_SITE_BWD_SMEM, a.error_flags, a.planted))
           continue;
-        if constexpr (KV) {
-          // The step's per-column LSE and D ride on the same barrier.
-          mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE + 2 * BM * 4);
-          const long long vr = vec_row(h, blk);
-          if (!ATTN_IN_BOUNDS(h >= 0 && h < a.hq && blk >= 0 && blk < a.n_qb, ATTN_SITE_BWD_OUT, a.error_flags,
-                              a.planted))
-            continue;
-          bulk_load(vec + (2 * s) * BM, a.lse2 + vr, BM * 4, &ring_full[s]);
-          bulk_load(vec + (2 * s + 1) * BM, a.delta + vr, BM * 4, &ring_full[s]);
-          for (int c = 0; c < L::CHUNKS; ++c) {
-            tma_load_4d(b0 + c * (BM * 128), &tm_q, &ring_full[s], c * 64, blk * BM, h, w.b);
-            tma_load_4d(b1 + c * (BM * 128), &tm_do, &ring_full[s], c * 64, blk * BM, h, w.b);
-          }
-        } else {
-          mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE);
-          for (int c = 0; c < L::CHUNKS; ++c) {
-            tma_load_4d(b0 + c * (BM * 128), &tm_k, &ring_full[s], c * 64, blk * BM, w.kvh, w.b);
-            tma_load_4d(b1 + c * (BM * 128), &tm_v, &ring_full[s], c * 64, blk * BM, w.kvh, w.b);
-          }
+        // The step's per-column LSE and D ride on the same barrier.
+        mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE + 2 * BM * 4);
+        const long long vr = vec_row(h, blk);
+        if (!ATTN_IN_BOUNDS(h >= 0 && h < a.hq && blk >= 0 && blk < a.n_qb, ATTN_SITE_BWD_OUT, a.error_flags,
+                            a.planted))
+          continue;
+        bulk_load(vec + (2 * s) * BM, a.lse2 + vr, BM * 4, &ring_full[s]);
+        bulk_load(vec + (2 * s + 1) * BM, a.delta + vr, BM * 4, &ring_full[s]);
+        for (int c = 0; c < L::CHUNKS; ++c) {
+          tma_load_4d(b0 + c * (BM * 128), &tm_q, &ring_full[s], c * 64, blk * BM, h, w.b);
+          tma_load_4d(b1 + c * (BM * 128), &tm_do, &ring_full[s], c * 64, blk * BM, h, w.b);
         }
       }
       // Drain: no copy may be in flight when the CTA exits. The last two
@@ -319,81 +398,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == MMA_WARP) {
     if (lane == 0 && w.n_steps > 0) {
       // ---------------------------------------------------------------- MMA issuer
-      // Per step: S-like products of half 0, then of half 1 (so half 0's
-      // elementwise work overlaps half 1's products), then the accumulating
-      // products of half 0 and of half 1 as their warpgroups finish.
-      constexpr uint32_t ID_S = instr_desc_bf16(BM, 64, 0);   // both operands K-major, N = 64
+      constexpr uint32_t ID_S = instr_desc_bf16(BM, BM, 0);   // both operands K-major, N = 128
       constexpr uint32_t ID_ACC = instr_desc_bf16(BM, D, 1);  // B MN-major
       const uint32_t hi = sw128_desc_hi(1024);
-      const uint32_t a0_lo = sw128_desc_lo(smem_addr(smem + L::A0_OFF), 16);
-      const uint32_t a1_lo = sw128_desc_lo(smem_addr(smem + L::A1_OFF), 16);
+      const uint32_t k_lo = sw128_desc_lo(smem_addr(smem + L::K_OFF), 16);
+      const uint32_t v_lo = sw128_desc_lo(smem_addr(smem + L::V_OFF), 16);
       const uint32_t ring_k = sw128_desc_lo(smem_addr(smem + L::RING_OFF), 16);        // K-major
       const uint32_t ring_mn = sw128_desc_lo(smem_addr(smem + L::RING_OFF), BM * 128);  // MN-major
       const uint32_t id_s = ID_S, id_acc = ID_ACC;
-      const uint32_t tS = tmem_base + COL_S, tDP = tmem_base + COL_DP, tA = tmem_base + COL_ACC;
-      // Stage addresses of step t's streamed tiles (K-major and MN-major views).
+      const uint32_t tDV = tmem_base + COL_ACC_KV, tDK = tDV + D;
+      // Stage addresses of step t's streamed tiles: which = 0 (Q) or 1 (dO).
       auto b_k = [&](int t, int which) { return ring_k + (uint32_t)(((2 * (t & 1) + which) * L::TILE) >> 4); };
       auto b_m = [&](int t, int which) { return ring_mn + (uint32_t)(((2 * (t & 1) + which) * L::TILE) >> 4); };
-      // S-like products of one half of step t (S^T = K Q^T, dP^T = V dO^T, or
-      // S = Q K^T, dP = dO V^T), then its barrier.
-      auto s_half = [&](int t, int half) {
-        if (half == 0) {
-          issue_s_half<D, 0>(tS, a0_lo, b_k(t, 0), hi, id_s);
-          issue_s_half<D, 0>(tDP, a1_lo, b_k(t, 1), hi, id_s);
-        } else {
-          issue_s_half<D, 1>(tS + 64, a0_lo, b_k(t, 0), hi, id_s);
-          issue_s_half<D, 1>(tDP + 64, a1_lo, b_k(t, 1), hi, id_s);
-        }
-        mma_commit(&sdp_full[half]);
+      auto issue_st = [&](int t) {  // S^T = K Q^T
+        issue_s<D>(tmem_base + sb_col(t), k_lo, b_k(t, 0), hi, id_s);
+        mma_commit(s_full);
       };
-      // Accumulating products of one half of step t, once its warpgroup has
-      // written P / dS.
-      auto acc_half = [&](int t, int half) {
-        if (half == 0) {
-          if constexpr (KV) {
-            issue_acc_half<0>(tA, tS, b_m(t, 1), hi, id_acc, t == 0);       // dV += P^T dO
-            issue_acc_half<0>(tA + D, tDP, b_m(t, 0), hi, id_acc, t == 0);  // dK += dS^T Q
-          } else {
-            issue_acc_half<0>(tA, tDP, b_m(t, 0), hi, id_acc, t == 0);  // dQ += dS K
-          }
-        } else {
-          if constexpr (KV) {
-            issue_acc_half<1>(tA, tS, b_m(t, 1), hi, id_acc, t == 0);
-            issue_acc_half<1>(tA + D, tDP, b_m(t, 0), hi, id_acc, t == 0);
-          } else {
-            issue_acc_half<1>(tA, tDP, b_m(t, 0), hi, id_acc, t == 0);
-          }
-        }
+      auto issue_dpt = [&](int t) {  // dP^T = V dO^T
+        issue_s<D>(tmem_base + db_col(t), v_lo, b_k(t, 1), hi, id_s);
+        mma_commit(dp_full);
       };
-      // Ping-pong over the two halves: half h's products of step t + 1 are
-      // issued right after its accumulating products of step t (they reuse its
-      // TMEM columns; MMAs from one thread run in issue order), so while one
-      // warpgroup works the tensor core runs the other half's products.
       bool ok = mbar_wait_bounded(a_full, 0, abort_flag, a.wait_limit);
       if (ok) ok = mbar_wait_bounded(&ring_full[0], 0, abort_flag, a.wait_limit);
       if (ok) {
         tc_fence_after();
-        s_half(0, 0);
-        s_half(0, 1);
+        issue_st(0);
+        issue_dpt(0);
       }
       for (int t = 0; t < w.n_steps && ok; ++t) {
         const bool next = t + 1 < w.n_steps;
-        ok = mbar_wait_bounded(&ps_full[0], t & 1, abort_flag, a.wait_limit);
+        ok = mbar_wait_bounded(p_full, t & 1, abort_flag, a.wait_limit);
         if (!ok) break;
         tc_fence_after();
-        acc_half(t, 0);
+        issue_acc(tDV, tmem_base + sb_col(t), b_m(t, 1), hi, id_acc, t == 0);  // dV += P^T dO
+        ok = mbar_wait_bounded(ds_full, t & 1, abort_flag, a.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
         if (next) {
           ok = mbar_wait_bounded(&ring_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag, a.wait_limit);
           if (!ok) break;
           tc_fence_after();
-          s_half(t + 1, 0);
+          issue_st(t + 1);  // into DB(t): its dP^T was read by phase 2
         }
-        ok = mbar_wait_bounded(&ps_full[1], t & 1, abort_flag, a.wait_limit);
-        if (!ok) break;
-        tc_fence_after();
-        acc_half(t, 1);
-        mma_commit(&ring_empty[t & 1]);  // step t's tiles are free once these have run
-        if (next) s_half(t + 1, 1);
+        issue_acc(tDK, tmem_base + sb_col(t) + 32, b_m(t, 0), hi, id_acc, t == 0);  // dK += dS^T Q
+        mma_commit(&ring_empty[t & 1]);  // step t's tiles and vectors are free once these have run
+        if (next) issue_dpt(t + 1);      // into SB(t), after dV and dK read it
       }
       if (ok) mma_commit(acc_full);
       // Every MMA issued must have completed before tensor memory is released
@@ -404,16 +453,318 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------------ elementwise + epilogue
     const int wq = warp & 3;
-    const int half = warp >> 2;      // this warpgroup's 64 columns
-    const int r = wq * 32 + lane;    // the resident tile's row == TMEM lane
+    const int half = warp >> 2;      // this warpgroup's 64 query columns
+    const int r = wq * 32 + lane;    // key row == TMEM lane
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
     const int off = a.seqlen_k - a.seqlen_q;
     const float sl2 = a.scale_log2;
     const float* vec = reinterpret_cast<const float*>(smem + L::VEC_OFF);
-    const int row_pos = w.blk * BM + r;  // key position (dK/dV) or query position (dQ)
+    const int row_pos = w.blk * BM + r;  // key position
+    const float2 sl2x2 = make_float2(sl2, sl2);
+    const bool cols_ok = ATTN_IN_BOUNDS(half >= 0 && half < 2 && COL_ACC_KV + 2 * D <= TMEM_COLS,
+                                        ATTN_SITE_BWD_TMEM, a.error_flags, a.planted);
+    (void)cols_ok;
+    bool ok = true;
+    for (int t = 0; t < w.n_steps && ok; ++t) {
+      const int s = t & 1;
+      const int blk = step_blk(t);
+      // Query column c (query blk BM + c, at position blk BM + c + off) sees
+      // this key when c >= c_lim.
+      const int c_lim = row_pos < a.seqlen_k ? (a.causal ? row_pos - off - blk * BM : -BM) : BM;
+      // The producer's LSE / D copies complete on the stage's full barrier.
+      ok = warp_wait(&ring_full[s], (t >> 1) & 1, abort_flag, a.wait_limit);
+      if (!ok) break;
+      const uint32_t lse_a = smem_addr(vec + (2 * s) * BM) + (uint32_t)(half * 64 * 4);
+      const uint32_t delta_a = smem_addr(vec + (2 * s + 1) * BM) + (uint32_t)(half * 64 * 4);
+      const uint32_t tS = lane_base + sb_col(t) + half * 64, tD = lane_base + db_col(t) + half * 64;
+      // The whole half is visible on all but the diagonal and ragged tiles.
+      const bool all_vis = c_lim <= half * 64;
+      // ---- phase 1: P^T
+      ok = warp_wait(s_full, t & 1, abort_flag, a.wait_limit);
+      if (!ok) break;
+      tc_fence_after();
+      float p[64];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sv[32];
+        if (cols_ok) tmem_ld32(tS + cc * 32, sv);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {  // 16 columns at a time: their -LSE log2 e loaded first
+          float4 lv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) lv[q] = lds_f4(lse_a + (uint32_t)(cc * 32 + g * 16 + 4 * q) * 4u);
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const int jj = g * 16 + j;
+            const float4 l4 = lv[j >> 2];
+            const float2 nl = (j & 2) ? make_float2(l4.z, l4.w) : make_float2(l4.x, l4.y);
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[jj]), __uint_as_float(sv[jj + 1])), sl2x2, nl);
+            float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (!all_vis) {
+              const int c = half * 64 + cc * 32 + jj;
+              pp.x = c >= c_lim ? pp.x : 0.f;
+              pp.y = c + 1 >= c_lim ? pp.y : 0.f;
+            }
+            p[cc * 32 + jj] = pp.x;
+            p[cc * 32 + jj + 1] = pp.y;
+            pk[jj / 2] = pack_bf16x2(pp.x, pp.y);
+          }
+        }
+        // bf16 pairs over the first 32 columns of this half, read already.
+        if (cols_ok) tmem_st16(tS + cc * 16, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      // ---- phase 2: dS^T
+      ok = warp_wait(dp_full, t & 1, abort_flag, a.wait_limit);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t dv[32];
+        if (cols_ok) tmem_ld32(tD + cc * 32, dv);
+        tmem_ld_wait();
+        uint32_t dk[16];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          float4 nd4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) nd4[q] = lds_f4(delta_a + (uint32_t)(cc * 32 + g * 16 + 4 * q) * 4u);
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const int jj = g * 16 + j;
+            const float4 d4 = nd4[j >> 2];
+            const float2 nd = (j & 2) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+            const float2 ds = __fmul2_rn(make_float2(p[cc * 32 + jj], p[cc * 32 + jj + 1]),
+                                         __fadd2_rn(make_float2(__uint_as_float(dv[jj]), __uint_as_float(dv[jj + 1])), nd));
+            dk[jj / 2] = pack_bf16x2(ds.x, ds.y);
+          }
+        }
+        // bf16 pairs over the last 32 columns of this half of SB (its S^T was
+        // read in phase 1).
+        if (cols_ok) tmem_st16(tS + 32 + cc * 16, dk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
+    }
+    // ---- epilogue: each warpgroup stores half of the columns of its rows
+    if (ok && w.n_steps > 0) ok = warp_wait(acc_full, 0, abort_flag, a.wait_limit);
+    if (ok) {
+      tc_fence_after();
+      store_grads<D, true>(a, w, lane_base, COL_ACC_KV, half, row_pos, w.n_steps > 0 && cols_ok);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag && a.error_flags) atomicOr(a.error_flags, ATTN_FAULT_TIMEOUT);
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ: one CTA per (batch, query head, 128-query block i); Q_i and dO_i stay in
+// shared memory while K_j, V_j stream. Per step t (key block j = t):
+//   S_t = Q_i K_j^T (product 2t) and dP_t = dO_i V_j^T (product 2t + 1), product
+//   p into TMEM buffer p mod 3; the elementwise warps (one query row per
+//   thread, each warpgroup 64 key columns) write dS_t = P_t (dP_t - D) as
+//   bf16 over the dP buffer; dQ += dS_t K_j.
+// Issue order after step t's elementwise work: dP_{t+1} (into S_t's buffer,
+// read already), dQ += dS_t K_j, S_{t+2} (into dP_t's buffer, after the
+// accumulation read it). S is two steps ahead and dP one, so the tensor core
+// runs dQ and S while the elementwise warps work on the next step.
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Args a) {
+  using L = QLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* a_full = bars;
+  uint64_t* k_full = bars + 1;                  // [K_SLOTS]
+  uint64_t* k_empty = k_full + L::K_SLOTS;      // [K_SLOTS]
+  uint64_t* v_full = k_empty + L::K_SLOTS;      // [V_SLOTS]
+  uint64_t* v_empty = v_full + L::V_SLOTS;      // [V_SLOTS]
+  uint64_t* sdp_full = v_empty + L::V_SLOTS;    // S and dP of the step are in TMEM
+  uint64_t* ps_full = sdp_full + 1;             // every elementwise warp wrote dS
+  uint64_t* acc_full = ps_full + 1;
+  uint64_t* mma_done = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const Work w = decode_work<false>(a);
+  const int n = w.n_steps;
+
+  if (threadIdx.x == 0) {
+    mbar_init(a_full, 1);
+    for (int s = 0; s < L::K_SLOTS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < L::V_SLOTS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(sdp_full, 1);
+    mbar_init(ps_full, EW_WARPS);
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  auto buf_col = [](int p) { return (uint32_t)((p % 3) * 128); };  // TMEM buffer of product p
+
+  if (warp == TMA_WARP) {
+    if (lane == 0 && n > 0) {
+      // ---------------------------------------------------------------- producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(a_full, 2 * L::TILE);
+      for (int c = 0; c < L::CHUNKS; ++c) {
+        tma_load_4d(smem + L::Q_OFF + c * (BM * 128), &tm_q, a_full, c * 64, w.blk * BM, w.h, w.b);
+        tma_load_4d(smem + L::DO_OFF + c * (BM * 128), &tm_do, a_full, c * 64, w.blk * BM, w.h, w.b);
+      }
+      // K_u then V_u for u = 0, 1, ...; each waits for the block a whole ring
+      // back to be released.
+      int nk = 0, nv = 0;
+      bool ok = true;
+      for (int u = 0; u < n && ok; ++u) {
+        const int ks = u % L::K_SLOTS, vs = u % L::V_SLOTS;
+        if (u >= L::K_SLOTS &&
+            !mbar_wait_bounded(&k_empty[ks], ((u / L::K_SLOTS) - 1) & 1, abort_flag, a.wait_limit)) {
+          ok = false;
+          break;
+        }
+        if (ATTN_IN_BOUNDS(ks >= 0 && ks < L::K_SLOTS && L::K_OFF + (ks + 1) * L::TILE <= L::V_OFF,
+                           ATTN_SITE_BWD_SMEM, a.error_flags, a.planted)) {
+          mbar_arrive_expect_tx(&k_full[ks], L::TILE);
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_4d(smem + L::K_OFF + ks * L::TILE + c * (BM * 128), &tm_k, &k_full[ks], c * 64, u * BM, w.kvh,
+                        w.b);
+        }
+        ++nk;
+        if (u >= L::V_SLOTS &&
+            !mbar_wait_bounded(&v_empty[vs], ((u / L::V_SLOTS) - 1) & 1, abort_flag, a.wait_limit)) {
+          ok = false;
+          break;
+        }
+        if (ATTN_IN_BOUNDS(vs >= 0 && vs < L::V_SLOTS && L::V_OFF + (vs + 1) * L::TILE <= L::BAR_OFF,
+                           ATTN_SITE_BWD_SMEM, a.error_flags, a.planted)) {
+          mbar_arrive_expect_tx(&v_full[vs], L::TILE);
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_4d(smem + L::V_OFF + vs * L::TILE + c * (BM * 128), &tm_v, &v_full[vs], c * 64, u * BM, w.kvh,
+                        w.b);
+        }
+        ++nv;
+      }
+      // Drain: the last copy into each slot (earlier ones completed before
+      // their slot was released); the waits ignore the abort flag.
+      mbar_wait_drain(a_full, 0);
+      for (int u = nk - L::K_SLOTS > 0 ? nk - L::K_SLOTS : 0; u < nk; ++u)
+        mbar_wait_drain(&k_full[u % L::K_SLOTS], (u / L::K_SLOTS) & 1);
+      for (int u = nv - L::V_SLOTS > 0 ? nv - L::V_SLOTS : 0; u < nv; ++u)
+        mbar_wait_drain(&v_full[u % L::V_SLOTS], (u / L::V_SLOTS) & 1);
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0 && n > 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      constexpr uint32_t ID_S = instr_desc_bf16(BM, BM, 0);
+      constexpr uint32_t ID_ACC = instr_desc_bf16(BM, D, 1);
+      const uint32_t hi = sw128_desc_hi(1024);
+      const uint32_t q_lo = sw128_desc_lo(smem_addr(smem + L::Q_OFF), 16);
+      const uint32_t do_lo = sw128_desc_lo(smem_addr(smem + L::DO_OFF), 16);
+      const uint32_t k_k = sw128_desc_lo(smem_addr(smem + L::K_OFF), 16);          // K-major
+      const uint32_t k_mn = sw128_desc_lo(smem_addr(smem + L::K_OFF), BM * 128);   // MN-major
+      const uint32_t v_k = sw128_desc_lo(smem_addr(smem + L::V_OFF), 16);
+      const uint32_t id_s = ID_S, id_acc = ID_ACC;
+      const uint32_t tDQ = tmem_base + COL_ACC_Q;
+      auto kslot = [&](int u) { return (uint32_t)(((u % L::K_SLOTS) * L::TILE) >> 4); };
+      auto vslot = [&](int u) { return (uint32_t)(((u % L::V_SLOTS) * L::TILE) >> 4); };
+      auto wait_k = [&](int u) {
+        return mbar_wait_bounded(&k_full[u % L::K_SLOTS], (u / L::K_SLOTS) & 1, abort_flag, a.wait_limit);
+      };
+      auto wait_v = [&](int u) {
+        return mbar_wait_bounded(&v_full[u % L::V_SLOTS], (u / L::V_SLOTS) & 1, abort_flag, a.wait_limit);
+      };
+      auto issue_sq = [&](int u) { issue_s<D>(tmem_base + buf_col(2 * u), q_lo, k_k + kslot(u), hi, id_s); };
+      auto issue_dp = [&](int u) {  // then the step's S and dP are complete once this has run
+        issue_s<D>(tmem_base + buf_col(2 * u + 1), do_lo, v_k + vslot(u), hi, id_s);
+        mma_commit(sdp_full);
+        mma_commit(&v_empty[u % L::V_SLOTS]);
+      };
+      bool ok = mbar_wait_bounded(a_full, 0, abort_flag, a.wait_limit);
+      if (ok) ok = wait_k(0);
+      if (ok) {
+        tc_fence_after();
+        issue_sq(0);
+        ok = wait_v(0);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_dp(0);
+        if (n > 1) {
+          ok = wait_k(1);
+          if (ok) {
+            tc_fence_after();
+            issue_sq(1);
+          }
+        }
+      }
+      for (int t = 0; t < n && ok; ++t) {
+        ok = mbar_wait_bounded(ps_full, t & 1, abort_flag, a.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
+        if (t + 1 < n) {
+          ok = wait_v(t + 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dp(t + 1);  // into S_t's buffer, read by step t's elementwise work
+        }
+        issue_acc(tDQ, tmem_base + buf_col(2 * t + 1), k_mn + kslot(t), hi, id_acc, t == 0);  // dQ += dS K
+        mma_commit(&k_empty[t % L::K_SLOTS]);  // K_t's last reader
+        if (t + 2 < n) {
+          ok = wait_k(t + 2);
+          if (!ok) break;
+          tc_fence_after();
+          issue_sq(t + 2);  // into dP_t's buffer, after the accumulation read dS_t
+        }
+      }
+      if (ok) mma_commit(acc_full);
+      mma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise + epilogue
+    const int wq = warp & 3;
+    const int half = warp >> 2;      // this warpgroup's 64 key columns
+    const int r = wq * 32 + lane;    // query row == TMEM lane
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
+    const int off = a.seqlen_k - a.seqlen_q;
+    const float sl2 = a.scale_log2;
+    const int row_pos = w.blk * BM + r;  // query position
     float nlse_r = -INFINITY, ndelta_r = 0.f;
-    if constexpr (!KV) {
-      const long long vr = vec_row(w.h, w.blk) + r;  // padded: -inf / 0 past Sq
+    {
+      const long long vr = (((long long)w.b * a.hq + w.h) * a.n_qb + w.blk) * BM + r;  // padded: -inf / 0 past Sq
       if (ATTN_IN_BOUNDS(w.h >= 0 && w.h < a.hq && w.blk >= 0 && w.blk < a.n_qb && r >= 0 && r < BM,
                          ATTN_SITE_BWD_OUT, a.error_flags, a.planted)) {
         nlse_r = a.lse2[vr];
@@ -421,127 +772,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
     const float2 sl2x2 = make_float2(sl2, sl2);
-    // This warpgroup's S / dP columns and the accumulators stay inside the
-    // allocation.
-    const bool cols_ok = ATTN_IN_BOUNDS(half >= 0 && half < 2 && COL_DP + half * 64 + 64 <= COL_ACC &&
-                                            COL_ACC + (KV ? 2 : 1) * D <= TMEM_COLS,
-                                        ATTN_SITE_BWD_TMEM, a.error_flags, a.planted);
+    const float2 nl = make_float2(nlse_r, nlse_r), nd = make_float2(ndelta_r, ndelta_r);
+    const bool cols_ok = ATTN_IN_BOUNDS(half >= 0 && half < 2 && COL_ACC_Q + D <= TMEM_COLS, ATTN_SITE_BWD_TMEM,
+                                        a.error_flags, a.planted);
     (void)cols_ok;
     bool ok = true;
-    for (int t = 0; t < w.n_steps && ok; ++t) {
-      const int s = t & 1;
-      const int blk = step_blk(t);
-      // KV: columns c >= c_lim are visible (query blk BM + c sits at position
-      // blk BM + c + off and sees this key when row_pos <= that). Q: columns
-      // c < c_lim are visible (key blk BM + c, below Sk and, causal, at most
-      // row_pos + off).
-      int c_lim;
-      if constexpr (KV) {
-        c_lim = row_pos < a.seqlen_k ? (a.causal ? row_pos - off - blk * BM : -BM) : BM;
-        // The producer's LSE / D copies complete on the stage's full barrier.
-        ok = warp_wait(&ring_full[s], (t >> 1) & 1, abort_flag, a.wait_limit);
-        if (!ok) break;
-      } else {
-        int lim = a.seqlen_k - blk * BM;
-        if (a.causal) {
-          const int cl = row_pos + off - blk * BM + 1;
-          lim = cl < lim ? cl : lim;
-        }
-        c_lim = lim;
+    for (int t = 0; t < n && ok; ++t) {
+      // Key column c (key t BM + c) is visible when c < c_lim: below Sk and,
+      // causal, at most row_pos + off.
+      int c_lim = a.seqlen_k - t * BM;
+      if (a.causal) {
+        const int cl = row_pos + off - t * BM + 1;
+        c_lim = cl < c_lim ? cl : c_lim;
       }
-      const float* lse_c = vec + (2 * s) * BM;
-      const float* delta_c = vec + (2 * s + 1) * BM;
-      ok = warp_wait(&sdp_full[half], t & 1, abort_flag, a.wait_limit);
+      const bool all_vis = c_lim >= half * 64 + 64;
+      const uint32_t tS = lane_base + buf_col(2 * t) + half * 64, tD = lane_base + buf_col(2 * t + 1) + half * 64;
+      ok = warp_wait(sdp_full, t & 1, abort_flag, a.wait_limit);
       if (!ok) break;
       tc_fence_after();
-      // The whole half is visible on all but the diagonal and ragged tiles:
-      // no per-element mask there.
-      const bool all_vis = KV ? (c_lim <= half * 64) : (c_lim >= half * 64 + 64);
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        const int col = half * 64 + cc * 32;
         uint32_t sv[32], dv[32];
         if (cols_ok) {
-          tmem_ld32(lane_base + COL_S + col, sv);
-          tmem_ld32(lane_base + COL_DP + col, dv);
+          tmem_ld32(tS + cc * 32, sv);
+          tmem_ld32(tD + cc * 32, dv);
         }
         tmem_ld_wait();
-        uint32_t pk[16], dk[16];
+        uint32_t dk[16];
 #pragma unroll
-        for (int j4 = 0; j4 < 32; j4 += 4) {
-          float2 nl[2], nd[2];
-          if constexpr (KV) {
-            const float4 lv = *reinterpret_cast<const float4*>(lse_c + col + j4);
-            const float4 dv4 = *reinterpret_cast<const float4*>(delta_c + col + j4);
-            nl[0] = make_float2(lv.x, lv.y), nl[1] = make_float2(lv.z, lv.w);
-            nd[0] = make_float2(dv4.x, dv4.y), nd[1] = make_float2(dv4.z, dv4.w);
-          } else {
-            nl[0] = nl[1] = make_float2(nlse_r, nlse_r);
-            nd[0] = nd[1] = make_float2(ndelta_r, ndelta_r);
+        for (int j = 0; j < 32; j += 2) {
+          // P = 2^(S scale log2 e - LSE log2 e); dS = P (dP - D).
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nl);
+          float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          if (!all_vis) {
+            const int c = half * 64 + cc * 32 + j;
+            pp.x = c < c_lim ? pp.x : 0.f;
+            pp.y = c + 1 < c_lim ? pp.y : 0.f;
           }
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int j = j4 + 2 * u;
-            // P = 2^(S scale log2 e - LSE log2 e); dS = P (dP - D).
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nl[u]);
-            float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            if (!all_vis) {
-              const int c = col + j;
-              const bool v0 = KV ? (c >= c_lim) : (c < c_lim);
-              const bool v1 = KV ? (c + 1 >= c_lim) : (c + 1 < c_lim);
-              p.x = v0 ? p.x : 0.f;
-              p.y = v1 ? p.y : 0.f;
-            }
-            const float2 ds =
-                __fmul2_rn(p, __fadd2_rn(make_float2(__uint_as_float(dv[j]), __uint_as_float(dv[j + 1])), nd[u]));
-            pk[j / 2] = pack_bf16x2(p.x, p.y);
-            dk[j / 2] = pack_bf16x2(ds.x, ds.y);
-          }
+          const float2 ds = __fmul2_rn(pp, __fadd2_rn(make_float2(__uint_as_float(dv[j]), __uint_as_float(dv[j + 1])), nd));
+          dk[j / 2] = pack_bf16x2(ds.x, ds.y);
         }
-        // bf16 pairs over this half's first 32 columns, all read already.
-        if (cols_ok) {
-          if constexpr (KV) tmem_st16(lane_base + COL_S + half * 64 + cc * 16, pk);
-          tmem_st16(lane_base + COL_DP + half * 64 + cc * 16, dk);
-        }
+        // bf16 pairs over this half's first 32 columns of the dP buffer, read already.
+        if (cols_ok) tmem_st16(tD + cc * 16, dk);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ps_full[half]);
+      if (lane == 0) mbar_arrive(ps_full);
     }
-    // ---- epilogue: each warpgroup stores half of the columns of its rows
-    const bool row_ok = row_pos < (KV ? a.seqlen_k : a.seqlen_q);
-    if (ok && w.n_steps > 0) ok = warp_wait(acc_full, 0, abort_flag, a.wait_limit);
+    if (ok && n > 0) ok = warp_wait(acc_full, 0, abort_flag, a.wait_limit);
     if (ok) {
       tc_fence_after();
-      const int n_out = KV ? 2 : 1;
-      for (int o = 0; o < n_out; ++o) {
-        // dK/dV kernel: o = 0 -> dV (unscaled), o = 1 -> dK (scale); dQ kernel: dQ (scale).
-        const bool is_dv = KV && o == 0;
-        void* base = KV ? (is_dv ? a.dv : a.dk) : a.dq;
-        const long long row_off =
-            KV ? (is_dv ? (long long)w.b * a.dv_bs + (long long)w.kvh * a.dv_hs + (long long)row_pos * a.dv_rs
-                        : (long long)w.b * a.dk_bs + (long long)w.kvh * a.dk_hs + (long long)row_pos * a.dk_rs)
-               : (long long)w.b * a.dq_bs + (long long)w.h * a.dq_hs + (long long)row_pos * a.dq_rs;
-        const float mul = is_dv ? 1.f : a.scale;
-#pragma unroll 1
-        for (int cc = half * (D / 64); cc < (half + 1) * (D / 64); ++cc) {
-          float x[32];
-          if (w.n_steps > 0 && cols_ok) {
-            uint32_t v[32];
-            tmem_ld32(lane_base + COL_ACC + o * D + cc * 32, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(v[k]) * mul;
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) x[k] = 0.f;  // no visible pair: the gradient is 0
-          }
-          if (row_ok && ATTN_IN_BOUNDS(w.b >= 0 && w.b < a.batch && (KV ? w.kvh < a.hkv : w.h < a.hq),
-                                       ATTN_SITE_BWD_OUT, a.error_flags, a.planted))
-            store_slice(base, row_off, cc * 32, x, a.grad_f32);
-        }
-      }
+      store_grads<D, false>(a, w, lane_base, COL_ACC_Q, half, row_pos, n > 0 && cols_ok);
     }
   }
 
@@ -672,12 +954,12 @@ size_t backward_workspace_bytes(const attn_backward_params& p) {
 template <int D, bool KV>
 static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const bwd::Args& a, long long grid, cudaStream_t stream) {
-  using L = bwd::Layout<D>;
-  static_assert(L::SMEM_BYTES <= 232448, "shared memory budget");
-  auto kern = bwd::bwd_kernel<D, KV>;
+  constexpr int SMEM = KV ? bwd::KvLayout<D>::SMEM_BYTES : bwd::QLayout<D>::SMEM_BYTES;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  auto kern = KV ? bwd::bwd_dkdv_kernel<D> : bwd::bwd_dq_kernel<D>;
   static DeviceOnce setup;  // the shared-memory attribute, once per device
   const attn_status_t st = setup.run([&]() -> attn_status_t {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES) != cudaSuccess) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
       cudaGetLastError();
       return ATTN_ERR_CUDA;
     }
@@ -686,7 +968,7 @@ static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   if (st != ATTN_OK) return st;
   if (grid <= 0) return ATTN_OK;
   if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-  kern<<<(unsigned)grid, bwd::NUM_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<(unsigned)grid, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -60,11 +60,16 @@ DECODE_CFG = wl.PAGED_DECODE
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
     "prefill": ["attention_tiled_exact_b200/csrc/prefill_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh",
-                "attention_tiled_exact_b200/csrc/exp2_poly.cuh"],
+                "attention_tiled_exact_b200/csrc/exp2_poly.cuh", "attention_tiled_exact_b200/csrc/bounds_check.cuh"],
     "prefill_16k": ["attention_tiled_exact_b200/csrc/prefill_sm100.cu",
-                    "attention_tiled_exact_b200/csrc/sm100_ptx.cuh", "attention_tiled_exact_b200/csrc/exp2_poly.cuh"],
-    "decode": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
-    "decode_fp8": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh"],
+                    "attention_tiled_exact_b200/csrc/sm100_ptx.cuh", "attention_tiled_exact_b200/csrc/exp2_poly.cuh",
+                    "attention_tiled_exact_b200/csrc/bounds_check.cuh"],
+    "decode": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh",
+               "attention_tiled_exact_b200/csrc/bounds_check.cuh"],
+    "decode_fp8": ["attention_tiled_exact_b200/csrc/decode_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh",
+                   "attention_tiled_exact_b200/csrc/bounds_check.cuh"],
+    "backward": ["attention_tiled_exact_b200/csrc/backward_sm100.cu", "attention_tiled_exact_b200/csrc/sm100_ptx.cuh",
+                 "attention_tiled_exact_b200/csrc/bounds_check.cuh"],
 }
 LEGS = ("tiny", "prefill", "prefill16k", "decode", "decodefp8", "mixed", "sharedprefix", "backward", "decodesteps")
 
@@ -724,7 +729,7 @@ def bench_backward(c: Ctx):
            "roofline": {"bound": "tensor", "kernel": "whole call (prep + dK/dV + dQ)", "achieved": round(tf, 2),
                         "peak": peak_t, "unit": "TFLOP/s", "frac": round(tf / peak_t, 4),
                         "peak_source": f"{c.peak_src} bf16 GEMM", "algorithmic_flops_per_launch": flops,
-                        "executed_flops_per_launch": 3.5 * fwd_flops},
+                        "executed_flops_per_launch": 3.5 * fwd_flops, "traffic": profiled_traffic("backward")},
            "gpu_launches_per_step": 3, "clocks": clk.summary()}
     if c.with_oracle:
         from oracle import attention_ref as ref

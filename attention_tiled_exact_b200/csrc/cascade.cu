@@ -24,7 +24,9 @@
 //   2. suffix: the split-KV decode over each sequence's own tokens past the
 //      prefix (block table entries from prefix_len / 16 on, lengths
 //      seq_lens[b] - prefix_len), giving one more partial per row;
-//   3. merge: one warp per (sequence, head) row combines the S + 1 partials.
+//   3. merge: one warp per (sequence, head) row combines the S prefix
+//      partials with the suffix decode's split partials (the decode's own
+//      combine is not run).
 // A small kernel before step 1 writes the suffix lengths (flagging sequences
 // shorter than the prefix), the per-range prefix lengths and the q copies,
 // and flags table rows whose prefix entries differ from row 0's.
@@ -84,14 +86,22 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// One warp per row r = b * hq + h. Prefix range s: O at pre_o[(s * rows + h *
-// n_seq + b) * HD] and LSE at pre_lse[s * rows + h * n_seq + b] (the prefill's
-// [range][kv head][g * N + n] row order); suffix: O at suf_o[r * HD], LSE at
-// suf_lse[r] (absent when no sequence can have a suffix).
+// One warp per row r = b * hq + h, over all partials of the row:
+//  - prefix range s < ranges: O at pre_o[(s * rows + h * n_seq + b) * HD],
+//    LSE at pre_lse[s * rows + h * n_seq + b] (the prefill's [range][kv head]
+//    [g * N + n] row order);
+//  - the suffix (when suf_o is not NULL), of n = max(1, ceil(L / T)) splits
+//    for suffix length L = suffix_lens[b] (at most max_splits): with n == 1
+//    the decode wrote it to suf_o[r * HD] / suf_lse[r], else its split i is
+//    at part_o[(i * rows + r) * HD] / part_lse[i * rows + r] (the decode's own
+//    combine is not run: this kernel merges its splits with the prefix).
+// A partial with LSE -inf has weight 0 and is not read.
 template <int HD>
 __global__ void __launch_bounds__(256)
     merge_kernel(const float* __restrict__ pre_o, const float* __restrict__ pre_lse, int ranges, int n_seq, int hq,
-                 const float* __restrict__ suf_o, const float* __restrict__ suf_lse, void* out_o, int out_f32,
+                 const float* __restrict__ suf_o, const float* __restrict__ suf_lse,
+                 const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                 const int32_t* __restrict__ suffix_lens, int split_tokens, int max_splits, void* out_o, int out_f32,
                  float* __restrict__ out_lse) {
   constexpr int PER = HD / 32;
   constexpr float LOG2E = 1.4426950408889634f;
@@ -100,36 +110,54 @@ __global__ void __launch_bounds__(256)
   const int lane = lane_id();
   if (r >= rows) return;
   const int b = r / hq, h = r - b * hq;
-  float ls[MAX_RANGES + 1];
-  float M = -INFINITY;
-#pragma unroll
-  for (int s = 0; s < MAX_RANGES; ++s) {
-    ls[s] = s < ranges ? pre_lse[(long long)s * rows + (long long)h * n_seq + b] : -INFINITY;
-    M = fmaxf(M, ls[s]);
+  int ns = 0;  // suffix partials of this row
+  if (suf_o) {
+    const int L = suffix_lens[b];
+    ns = L > 0 ? (L + split_tokens - 1) / split_tokens : 1;
+    ns = ns < 1 ? 1 : (ns > max_splits ? max_splits : ns);
+    if (ns > 1 && !part_o) ns = 1;
   }
-  ls[MAX_RANGES] = suf_lse ? suf_lse[r] : -INFINITY;
-  M = fmaxf(M, ls[MAX_RANGES]);
+  const int total = ranges + ns;
+  auto lse_of = [&](int s) -> float {
+    if (s < ranges) return pre_lse[(long long)s * rows + (long long)h * n_seq + b];
+    return ns == 1 ? suf_lse[r] : part_lse[(long long)(s - ranges) * rows + r];
+  };
+  auto o_of = [&](int s) -> const float* {
+    if (s < ranges) return pre_o + ((long long)s * rows + (long long)h * n_seq + b) * HD;
+    return ns == 1 ? suf_o + (long long)r * HD : part_o + ((long long)(s - ranges) * rows + r) * HD;
+  };
+  // The partials' LSEs, lanes strided over them (32 at a time): max, then
+  // the sum of exp(lse - max).
+  float M = -INFINITY;
+  for (int s = lane; s < total; s += 32) M = fmaxf(M, lse_of(s));
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float out[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) out[i] = 0.f;
   float lse = -INFINITY;
   if (M != -INFINITY) {
     float sum = 0.f;
+    for (int s = lane; s < total; s += 32) sum += ex2_approx((lse_of(s) - M) * LOG2E);  // exp(-inf) = 0
 #pragma unroll
-    for (int s = 0; s <= MAX_RANGES; ++s) sum += ex2_approx((ls[s] - M) * LOG2E);  // exp(-inf) = 0
+    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     lse = M + logf(sum);
+    for (int s0 = 0; s0 < total; s0 += 32) {
+      // Lane j holds partial s0 + j's weight; every lane reads its slice of
+      // each partial's O (weight 0: not read).
+      const float ls = s0 + lane < total ? lse_of(s0 + lane) : -INFINITY;
+      const float wl = ls == -INFINITY ? 0.f : ex2_approx((ls - lse) * LOG2E);
+      const int n = total - s0 < 32 ? total - s0 : 32;
+      for (int j = 0; j < n; ++j) {
+        const float wgt = __shfl_sync(0xffffffffu, wl, j);
+        if (wgt == 0.f) continue;  // warp-uniform
+        const float* src = o_of(s0 + j) + lane * PER;
 #pragma unroll
-    for (int s = 0; s <= MAX_RANGES; ++s) {
-      if (ls[s] == -INFINITY) continue;  // weight 0: the partial is not read
-      const float wgt = ex2_approx((ls[s] - lse) * LOG2E);
-      const float* src = (s < MAX_RANGES ? pre_o + ((long long)s * rows + (long long)h * n_seq + b) * HD
-                                         : suf_o + (long long)r * HD) +
-                         lane * PER;
-#pragma unroll
-      for (int i = 0; i < PER; i += 2) {
-        const float2 x = *reinterpret_cast<const float2*>(src + i);
-        out[i] = fmaf(wgt, x.x, out[i]);
-        out[i + 1] = fmaf(wgt, x.y, out[i + 1]);
+        for (int i = 0; i < PER; i += 2) {
+          const float2 x = *reinterpret_cast<const float2*>(src + i);
+          out[i] = fmaf(wgt, x.x, out[i]);
+          out[i + 1] = fmaf(wgt, x.y, out[i + 1]);
+        }
       }
     }
   }
@@ -272,22 +300,32 @@ attn_status_t launch_cascade(const attn_decode_params& p, const CascadePlan& c, 
   if (st != ATTN_OK) return st;
 
   // 2. suffix decode (skipped when the prefix fills every table row).
+  // Its splits stay in the decode workspace: the merge below combines them
+  // with the prefix ranges in one pass.
   const bool has_suffix = c.suffix_cap > 0;
+  const float* part_o = nullptr;
+  const float* part_lse = nullptr;
   if (has_suffix) {
     attn_decode_params ps = c.suffix;
     ps.seq_lens = suffix_lens;
     ps.o = suf_o;
     ps.lse = suf_lse;
-    st = launch_decode(ps, c.suffix_plan, ws + c.off_decode, stream);
+    st = launch_decode(ps, c.suffix_plan, ws + c.off_decode, stream, /*combine=*/false);
     if (st != ATTN_OK) return st;
+    if (c.suffix_plan.max_splits > 1) {
+      const size_t po = (size_t)c.suffix_plan.max_splits * rows * D * sizeof(float);
+      part_o = reinterpret_cast<const float*>(ws + c.off_decode);
+      part_lse = reinterpret_cast<const float*>(ws + c.off_decode + align256(po));
+    }
   }
 
-  // 3. merge.
+  // 3. merge: prefix ranges and suffix splits of every row.
   const int warps = 8;
   const int grid = (int)((rows + warps - 1) / warps);
-  merge_kernel<128><<<grid, warps * 32, 0, stream>>>(pre_o, pre_lse, c.ranges, p.batch, p.num_q_heads,
-                                                    has_suffix ? suf_o : nullptr, has_suffix ? suf_lse : nullptr,
-                                                    p.o, p.o_dtype == ATTN_DTYPE_F32, p.lse);
+  merge_kernel<128><<<grid, warps * 32, 0, stream>>>(
+      pre_o, pre_lse, c.ranges, p.batch, p.num_q_heads, has_suffix ? suf_o : nullptr,
+      has_suffix ? suf_lse : nullptr, part_o, part_lse, suffix_lens, c.suffix_plan.split_tokens,
+      c.suffix_plan.max_splits, p.o, p.o_dtype == ATTN_DTYPE_F32, p.lse);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

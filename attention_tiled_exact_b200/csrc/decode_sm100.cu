@@ -764,7 +764,7 @@ static attn_status_t launch_decode_g(const decode::Args& a, const DecodePlan& pl
 }
 
 attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan, void* workspace,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, bool combine) {
   if (p.batch == 0) return ATTN_OK;
   decode::Args a;
   a.q = reinterpret_cast<const __nv_bfloat16*>(p.q);
@@ -801,7 +801,7 @@ attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan,
     case 8: st = fp8 ? launch_decode_g<8, true>(a, plan, stream) : launch_decode_g<8, false>(a, plan, stream); break;
     default: return ATTN_ERR_UNSUPPORTED;
   }
-  if (st != ATTN_OK || plan.max_splits <= 1) return st;
+  if (st != ATTN_OK || plan.max_splits <= 1 || !combine) return st;
   return launch_combine(a.part_o, a.part_lse, plan.max_splits, (int)rows, p.head_dim, nullptr, p.seq_lens,
                         plan.split_tokens, p.num_q_heads, p.o, p.o_dtype, p.lse, stream, p.error_flags);
 }

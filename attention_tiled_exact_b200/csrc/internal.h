@@ -72,8 +72,11 @@ struct DecodePlan {
 };
 DecodePlan plan_decode(const attn_decode_params& p);
 
+// combine = false: rows of more than one split keep their partials in the
+// workspace (O at its start, LSE 256-byte aligned after it) for the caller to
+// merge; rows of one split are written to p.o / p.lse as usual.
 attn_status_t launch_decode(const attn_decode_params& p, const DecodePlan& plan, void* workspace,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool combine = true);
 
 // The decode kernels' one-time set-up for these parameters (kernel
 // attributes), without launching anything: to be done before a stream capture.

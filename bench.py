@@ -684,7 +684,6 @@ def bench_shared_prefix(c: Ctx):
     prefix_flops = 4.0 * cfg.batch * cfg.q_heads * cfg.prefix_len * cfg.head_dim
     peak_h = c.peak("hbm_gbs")
     gbs = ubytes / (ms * 1e-3) / 1e9
-    max_splits = -(-(max_len - cfg.prefix_len) // 512)
     res = {"workload": cfg.name, "value": round(logical * world / (ms * 1e-3), 1), "unit": "kv_tokens/s",
            "ms_per_step": round(ms, 4), "steps": steps, "kv_tokens": logical, "unique_kv_tokens": unique,
            "plain_decode_ms_per_step": round(ms_plain, 4), "speedup_vs_plain_decode": round(ms_plain / ms, 3),
@@ -692,7 +691,7 @@ def bench_shared_prefix(c: Ctx):
                         "achieved": round(gbs, 1), "peak": peak_h, "unit": "GB/s", "frac": round(gbs / peak_h, 4),
                         "peak_source": f"{c.peak_src} copy bandwidth", "traffic": None,
                         "algorithmic_bytes_per_launch": ubytes, "prefix_tensor_flops": prefix_flops},
-           "gpu_launches_per_step": 4 + (1 if max_splits > 1 else 0), "clocks": clk.summary()}
+           "gpu_launches_per_step": 4, "clocks": clk.summary()}
     if c.with_oracle:
         cpu, par = oracle_decode_sequences(d, _bf16_to_f64(out), lse.cpu().numpy(), args.cpu_seconds, seed=14,
                                            unit="kv_tokens/s")

@@ -31,6 +31,22 @@ int planted_bounds_site() { return g_planted_site.load(std::memory_order_relaxed
 
 static bool mult8(int64_t s) { return (s % 8) == 0; }
 
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    streams[dev] = nullptr;
+  }
+  return streams[dev];
+}
+
 int device_sm_count() {
   static std::mutex mu;
   static int cache[kMaxDevices] = {0};

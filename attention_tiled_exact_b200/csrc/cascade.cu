@@ -296,13 +296,38 @@ attn_status_t launch_cascade(const attn_decode_params& p, const CascadePlan& c, 
   pp.num_blocks = p.num_blocks;
   pp.block_size = 16;
   pp.error_flags = p.error_flags;
-  attn_status_t st = launch_prefill(pp, stream);
-  if (st != ATTN_OK) return st;
+  // The prefix prefill (short, latency-bound items on up to one CTA per SM)
+  // and the suffix decode (memory-bound) are independent: the prefill runs on
+  // a side stream, launched first, and the decode's CTAs take the SMs it
+  // leaves and those it frees; the merge waits for both. (Capping the
+  // prefill to a third or fewer of the SMs was slower, measured.) Without a
+  // side stream or events they run one after the other on `stream`.
+  const bool has_suffix = c.suffix_cap > 0;
+  cudaStream_t side = has_suffix ? side_stream() : nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (side && (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+               cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess ||
+               cudaEventRecord(fork, stream) != cudaSuccess || cudaStreamWaitEvent(side, fork, 0) != cudaSuccess)) {
+    cudaGetLastError();
+    side = nullptr;
+  }
+  auto release = [&]() {
+    if (fork) cudaEventDestroy(fork);
+    if (join) cudaEventDestroy(join);
+  };
+  attn_status_t st = launch_prefill(pp, side ? side : stream);
+  if (st == ATTN_OK && side && (cudaEventRecord(join, side) != cudaSuccess)) {
+    cudaGetLastError();
+    st = ATTN_ERR_CUDA;
+  }
+  if (st != ATTN_OK) {
+    release();
+    return st;
+  }
 
   // 2. suffix decode (skipped when the prefix fills every table row).
   // Its splits stay in the decode workspace: the merge below combines them
   // with the prefix ranges in one pass.
-  const bool has_suffix = c.suffix_cap > 0;
   const float* part_o = nullptr;
   const float* part_lse = nullptr;
   if (has_suffix) {
@@ -311,11 +336,24 @@ attn_status_t launch_cascade(const attn_decode_params& p, const CascadePlan& c, 
     ps.o = suf_o;
     ps.lse = suf_lse;
     st = launch_decode(ps, c.suffix_plan, ws + c.off_decode, stream, /*combine=*/false);
-    if (st != ATTN_OK) return st;
+    if (st != ATTN_OK) {
+      if (side) cudaStreamWaitEvent(stream, join, 0);
+      release();
+      return st;
+    }
     if (c.suffix_plan.max_splits > 1) {
       const size_t po = (size_t)c.suffix_plan.max_splits * rows * D * sizeof(float);
       part_o = reinterpret_cast<const float*>(ws + c.off_decode);
       part_lse = reinterpret_cast<const float*>(ws + c.off_decode + align256(po));
+    }
+  }
+
+  if (side) {
+    const bool joined = cudaStreamWaitEvent(stream, join, 0) == cudaSuccess;
+    release();
+    if (!joined) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
     }
   }
 

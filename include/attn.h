@@ -19,7 +19,8 @@
  *    LSE is fp32, natural log; O is bf16 or fp32 (attn_dtype_t).
  *  - Every pointer is DEVICE memory owned by the caller. The library allocates
  *    no device memory and keeps no state besides a per-device cache of the SM
- *    count and of kernel attributes. Host pointers are used only where a
+ *    count and of kernel attributes, and one non-blocking stream per device
+ *    for attn_decode_paged_shared_prefix. Host pointers are used only where a
  *    parameter says "host".
  *  - Calls are asynchronous and stream-ordered: they validate arguments on the
  *    host, enqueue kernels on `stream` and return. Nothing synchronises.
@@ -348,7 +349,11 @@ ATTN_API attn_status_t attn_prefill_backward(const attn_backward_params* p, void
  * over the prefix (cut into up to 16 key ranges when the batch is small),
  * the split-KV decode covers each sequence's suffix, and one kernel merges
  * the partials ("GPU Kernel 调度:大模型推理的拐点 2026", Flash Decoding
- * section: partials merged by their log-sum-exp).
+ * section: partials merged by their log-sum-exp). The prefix prefill and the
+ * suffix decode are independent, so the prefill runs on the library's second
+ * stream of the device (forked from `stream` and joined back with events;
+ * stream capture follows the fork, so the call can be captured into a CUDA
+ * graph). Calls from several threads share that second stream.
  *
  * Parameters as attn_decode_paged, plus prefix_len (host): a multiple of 16
  * with 0 <= prefix_len <= max_blocks_per_seq * 16, else

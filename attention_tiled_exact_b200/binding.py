@@ -76,6 +76,12 @@ class PrefillParams(ctypes.Structure):
     ]
 
 
+class PrefillHostIO(ctypes.Structure):
+    """Mirror of ``attn_prefill_host_io`` (host pointers)."""
+
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp), ("kv_heads_per_chunk", _i32)]
+
+
 class BackwardParams(ctypes.Structure):
     """Mirror of ``attn_backward_params``."""
 
@@ -118,6 +124,8 @@ def _load():
     lib = ctypes.CDLL(_LIB_FILE)
     lib.attn_prefill.argtypes = [ctypes.POINTER(PrefillParams), _vp]
     lib.attn_prefill.restype = ctypes.c_int
+    lib.attn_prefill_from_host.argtypes = [ctypes.POINTER(PrefillParams), ctypes.POINTER(PrefillHostIO), _vp]
+    lib.attn_prefill_from_host.restype = ctypes.c_int
     lib.attn_decode_paged.argtypes = [ctypes.POINTER(DecodeParams), _vp, ctypes.c_size_t,
                                       ctypes.POINTER(ctypes.c_size_t), _vp]
     lib.attn_decode_paged.restype = ctypes.c_int
@@ -338,6 +346,49 @@ def prefill(q, k, v, scale: float | None = None, causal: bool = False, out=None,
     p.seqlens_q, p.seqlens_k = _ptr(seqlens_q), _ptr(seqlens_k)
     _check(LIB.attn_prefill(ctypes.byref(p), _stream(q.device)), "attn_prefill")
     return out, lse
+
+
+def prefill_from_host(q_host, k_host, v_host, q, k, v, o, o_host, lse=None, lse_host=None,
+                      scale: float | None = None, causal: bool = False, kv_heads_per_chunk: int = 0,
+                      error_flags=None):
+    """Dense prefill from and to host memory, copies overlapped with compute.
+
+    q_host / k_host / v_host (CPU bf16, pinned, contiguous [B,H,S,D]) are
+    copied into the device staging tensors q / k / v (contiguous, same
+    shapes); O (and the LSE, when ``lse`` is given) are computed into ``o`` /
+    ``lse`` and copied back into ``o_host`` / ``lse_host``, chunk by chunk
+    (one batch entry and ``kv_heads_per_chunk`` kv heads per chunk; 0 = all).
+    Asynchronous on the current stream; the host tensors are ready after it
+    synchronises. Returns ``(o_host, lse_host)``.
+    """
+    for t in (q_host, k_host, v_host, o_host) + ((lse_host,) if lse is not None else ()):
+        _need(t is not None and not t.is_cuda and t.is_contiguous(), "host tensors: CPU, contiguous")
+    for t in (q, k, v, o) + ((lse,) if lse is not None else ()):
+        _need(t.is_cuda and t.is_contiguous(), "device tensors: CUDA, contiguous")
+    _need(tuple(q_host.shape) == tuple(q.shape) and tuple(k_host.shape) == tuple(k.shape) and
+          tuple(v_host.shape) == tuple(v.shape) and tuple(o_host.shape) == tuple(o.shape), "host/device shapes")
+    _need(q.dtype == k.dtype == v.dtype == q_host.dtype == k_host.dtype == v_host.dtype == torch.bfloat16,
+          "bf16 inputs")
+    _need(o.dtype == o_host.dtype and o.dtype in (torch.bfloat16, torch.float32), "o: bf16 or fp32 on both sides")
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    p = PrefillParams()
+    p.q, p.k, p.v, p.o = _ptr(q), _ptr(k), _ptr(v), _ptr(o)
+    p.lse = _ptr(lse)
+    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.seqlen_q, p.seqlen_k = B, Hq, Hkv, D, Sq, Sk
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        setattr(p, f"{name}_batch_stride", t.stride(0))
+        setattr(p, f"{name}_head_stride", t.stride(1))
+        setattr(p, f"{name}_row_stride", t.stride(2))
+    p.scale = float(scale if scale is not None else 1.0 / math.sqrt(D))
+    p.causal, p.o_dtype = int(bool(causal)), _out_code(o.dtype)
+    p.error_flags = _ptr(error_flags)
+    io = PrefillHostIO()
+    io.q, io.k, io.v, io.o = (ctypes.c_void_p(t.data_ptr()) for t in (q_host, k_host, v_host, o_host))
+    io.lse = ctypes.c_void_p(lse_host.data_ptr()) if lse is not None else None
+    io.kv_heads_per_chunk = int(kv_heads_per_chunk)
+    _check(LIB.attn_prefill_from_host(ctypes.byref(p), ctypes.byref(io), _stream(q.device)), "attn_prefill_from_host")
+    return o_host, lse_host
 
 
 def _backward_params(q, k, v, o, lse, dout, dq, dk, dv, scale, causal, error_flags):

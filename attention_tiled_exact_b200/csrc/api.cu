@@ -31,20 +31,22 @@ int planted_bounds_site() { return g_planted_site.load(std::memory_order_relaxed
 
 static bool mult8(int64_t s) { return (s % 8) == 0; }
 
-cudaStream_t side_stream() {
+cudaStream_t side_stream(int which) {
   static std::mutex mu;
-  static cudaStream_t streams[kMaxDevices] = {};
+  static cudaStream_t streams[2][kMaxDevices] = {};
   int dev = 0;
+  if (which < 0 || which > 1) return nullptr;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
+  cudaStream_t& s = streams[which][dev];
+  if (!s && cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) {
     cudaGetLastError();
-    streams[dev] = nullptr;
+    s = nullptr;
   }
-  return streams[dev];
+  return s;
 }
 
 int device_sm_count() {
@@ -76,7 +78,7 @@ attn_status_t check_device() {
   return (major == 10 && minor == 0) ? ATTN_OK : ATTN_ERR_NO_DEVICE;
 }
 
-static attn_status_t validate_prefill(const attn_prefill_params* p) {
+attn_status_t validate_prefill(const attn_prefill_params* p) {
   if (!p) return ATTN_ERR_INVALID_ARG;
   if (p->batch < 0 || p->num_q_heads < 0 || p->num_kv_heads < 0 || p->seqlen_q < 0 || p->seqlen_k < 0)
     return ATTN_ERR_INVALID_ARG;

@@ -63,9 +63,13 @@ attn_status_t validate_decode(const attn_decode_params* p);
 // Prefill launcher. Arguments were validated by the caller.
 attn_status_t launch_prefill(const attn_prefill_params& p, cudaStream_t stream);
 
-// A non-blocking stream of the current device, created once and kept for the
-// process: the second stream of calls that run two kernels side by side.
-cudaStream_t side_stream();
+// Non-blocking streams of the current device (which = 0 or 1), created once
+// and kept for the process: the extra streams of calls that overlap kernels
+// or copies with their main stream.
+cudaStream_t side_stream(int which = 0);
+
+// Host-side argument checks of attn_prefill (ATTN_OK when valid).
+attn_status_t validate_prefill(const attn_prefill_params* p);
 
 // Decode plan: tokens per split (multiple of 16) and the maximum number of
 // splits a sequence can have.

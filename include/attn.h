@@ -19,9 +19,9 @@
  *    LSE is fp32, natural log; O is bf16 or fp32 (attn_dtype_t).
  *  - Every pointer is DEVICE memory owned by the caller. The library allocates
  *    no device memory and keeps no state besides a per-device cache of the SM
- *    count and of kernel attributes, and one non-blocking stream per device
- *    for attn_decode_paged_shared_prefix. Host pointers are used only where a
- *    parameter says "host".
+ *    count and of kernel attributes, and two non-blocking streams per device
+ *    (attn_decode_paged_shared_prefix, attn_prefill_from_host). Host pointers
+ *    are used only where a parameter says "host".
  *  - Calls are asynchronous and stream-ordered: they validate arguments on the
  *    host, enqueue kernels on `stream` and return. Nothing synchronises.
  *  - Errors: a call returns ATTN_OK or an attn_status_t; it never aborts,
@@ -194,6 +194,44 @@ typedef struct {
 } attn_prefill_params;
 
 ATTN_API attn_status_t attn_prefill(const attn_prefill_params* p, attn_stream_t stream);
+
+/*
+ * attn_prefill with the inputs taken from, and the outputs returned to, HOST
+ * memory, the copies overlapped with the computation: the call a serving
+ * process makes when Q/K/V arrive in host memory (the inputs and outputs of
+ * "推理加速" FlashAttention's flow, moved over PCIe).
+ *
+ * p describes a dense prefill (no paged keys, no variable or packed lengths)
+ * whose DEVICE tensors q, k, v, o (and lse, nullable) are contiguous in the
+ * [batch, heads, seqlen, head_dim] layout (row stride head_dim, head stride
+ * seqlen * head_dim, batch stride heads * seqlen * head_dim); they are the
+ * caller's staging buffers. io gives the HOST tensors in the same layouts:
+ * q, k, v (read), o (and lse when p->lse is set; written); they should be
+ * pinned (page-locked) for the copies to overlap. The work is cut into chunks
+ * of one batch entry and kv_heads_per_chunk key/value heads (with their query
+ * heads; 0 = all heads of a batch entry); kv_heads_per_chunk must divide
+ * num_kv_heads. Per chunk: the inputs are copied host -> device on one of the
+ * library's side streams, the prefill of that chunk runs on `stream`, and its
+ * O and LSE go device -> host on a second side stream, so that chunk c + 1's
+ * inputs travel while chunk c computes and chunk c - 1's outputs travel back.
+ * Work enqueued on `stream` after the call starts after every copy of the
+ * call has completed. Host and device buffers must not be touched until then.
+ * Errors: as attn_prefill, plus ATTN_ERR_INVALID_ARG for a null or
+ * non-dividing io field, ATTN_ERR_UNSUPPORTED for non-contiguous device
+ * tensors, paged / variable-length parameters or an O in another dtype than
+ * io's layout implies (o_dtype decides the host O element size).
+ */
+typedef struct {
+  const void* q;   /* host [batch, num_q_heads, seqlen_q, head_dim] bf16 */
+  const void* k;   /* host [batch, num_kv_heads, seqlen_k, head_dim] bf16 */
+  const void* v;   /* host, as k */
+  void* o;         /* host [batch, num_q_heads, seqlen_q, head_dim], o_dtype */
+  float* lse;      /* host [batch, num_q_heads, seqlen_q] fp32; required when p->lse is set */
+  int kv_heads_per_chunk;
+} attn_prefill_host_io;
+
+ATTN_API attn_status_t attn_prefill_from_host(const attn_prefill_params* p, const attn_prefill_host_io* io,
+                                              attn_stream_t stream);
 
 /*
  * Paged decode (Flash-Decoding): one query token per sequence against its

@@ -49,6 +49,9 @@ def test_struct_layouts_match_the_header(lib):
     body.append('printf("D %zu\\n", sizeof(attn_decode_params));')
     body.append('printf("B %zu\\n", sizeof(attn_backward_params));')
     body.append('printf("C %zu\\n", sizeof(attn_persistent_cmd));')
+    body.append('printf("H %zu\\n", sizeof(attn_prefill_host_io));')
+    for f, _ in lib.PrefillHostIO._fields_:
+        body.append(f'printf("h.{f} %zu\\n", offsetof(attn_prefill_host_io, {f}));')
     for f, _ in lib.PersistentCmd._fields_:
         body.append(f'printf("c.{f} %zu\\n", offsetof(attn_persistent_cmd, {f}));')
     for f in fields_p:
@@ -73,6 +76,9 @@ def test_struct_layouts_match_the_header(lib):
     assert int(got["C"]) == ctypes.sizeof(lib.PersistentCmd)
     for f, _ in lib.PersistentCmd._fields_:
         assert int(got[f"c.{f}"]) == getattr(lib.PersistentCmd, f).offset, f
+    assert int(got["H"]) == ctypes.sizeof(lib.PrefillHostIO)
+    for f, _ in lib.PrefillHostIO._fields_:
+        assert int(got[f"h.{f}"]) == getattr(lib.PrefillHostIO, f).offset, f
     assert int(got["B"]) == ctypes.sizeof(lib.BackwardParams)
     for f in fields_b:
         assert int(got[f"b.{f}"]) == getattr(lib.BackwardParams, f).offset, f
@@ -267,3 +273,25 @@ def test_product_path_has_no_cpu_fallback():
             assert "import oracle" not in src and "from oracle" not in src, fn
     binding = open(os.path.join(pkg, "binding.py")).read()
     assert "raise ImportError" in binding
+
+
+def test_prefill_from_host_argument_checks(lib):
+    import ctypes
+    p = lib.PrefillParams()
+    p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.seqlen_q, p.seqlen_k = 1, 4, 2, 128, 16, 16
+    p.q, p.k, p.v, p.o = (ctypes.c_void_p(4096 * (i + 1)) for i in range(4))
+    for nm in ("q", "o"):
+        setattr(p, f"{nm}_row_stride", 128), setattr(p, f"{nm}_head_stride", 16 * 128)
+        setattr(p, f"{nm}_batch_stride", 4 * 16 * 128)
+    for nm in ("k", "v"):
+        setattr(p, f"{nm}_row_stride", 128), setattr(p, f"{nm}_head_stride", 16 * 128)
+        setattr(p, f"{nm}_batch_stride", 2 * 16 * 128)
+    p.scale = 0.1
+    io = lib.PrefillHostIO()
+    assert lib.LIB.attn_prefill_from_host(ctypes.byref(p), ctypes.byref(io), None) == lib.ATTN_ERR_INVALID_ARG
+    io.q, io.k, io.v, io.o = (ctypes.c_void_p(8192 * (i + 1)) for i in range(4))
+    io.kv_heads_per_chunk = 3  # does not divide 2
+    assert lib.LIB.attn_prefill_from_host(ctypes.byref(p), ctypes.byref(io), None) == lib.ATTN_ERR_INVALID_ARG
+    io.kv_heads_per_chunk = 1
+    p.q_head_stride = 32 * 128  # not contiguous
+    assert lib.LIB.attn_prefill_from_host(ctypes.byref(p), ctypes.byref(io), None) == lib.ATTN_ERR_UNSUPPORTED

@@ -164,3 +164,39 @@ def test_full_size_every_row(lib, cfg):
     o32, lse32 = _run(lib, d, out_dtype=torch.float32)
     assert_o_close(o32, O_ref, False, f"{cfg.name} fp32 out")
     assert np.array_equal(lse32, lse16)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,Hq,Hkv,S,Sk,D,causal,hpc,f32,with_lse", [
+    (2, 8, 2, 300, 300, 128, True, 1, False, True),
+    (3, 6, 3, 200, 450, 64, False, 0, True, True),
+    (1, 4, 4, 129, 129, 128, True, 2, False, False),
+    (2, 4, 2, 64, 0, 128, False, 1, True, True),
+])
+def test_prefill_from_host_matches_the_device_call(lib, B, Hq, Hkv, S, Sk, D, causal, hpc, f32, with_lse):
+    """Chunked host<->device pipeline: the same bits as one device call (each
+    chunk's items compute exactly what they compute in the whole call), and
+    the oracle's values."""
+    import torch
+    d = wl.make_prefill(wl.PrefillConfig("from_host", B, Hq, Hkv, S, max(Sk, 1), D, causal, 81 + D))
+    k_bits, v_bits = d["k"][:, :, :Sk], d["v"][:, :, :Sk]
+    host = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hq, hk, hv = host(d["q"]), host(k_bits), host(v_bits)
+    odt = torch.float32 if f32 else torch.bfloat16
+    q, k, v = torch.empty_like(hq, device="cuda"), torch.empty_like(hk, device="cuda"), torch.empty_like(hv, device="cuda")
+    o = torch.empty((B, Hq, S, D), dtype=odt, device="cuda")
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device="cuda") if with_lse else None
+    ho = torch.full((B, Hq, S, D), 7.0, dtype=odt).pin_memory()
+    hl = torch.full((B, Hq, S), 7.0, dtype=torch.float32).pin_memory() if with_lse else None
+    lib.prefill_from_host(hq, hk, hv, q, k, v, o, ho, lse, hl, d["scale"], causal, kv_heads_per_chunk=hpc)
+    torch.cuda.synchronize()
+    o_ref, l_ref = lib.prefill(hq.cuda(), hk.cuda(), hv.cuda(), d["scale"], causal, out_dtype=odt)
+    torch.cuda.synchronize()
+    assert torch.equal(ho, o_ref.cpu())
+    if with_lse:
+        assert torch.equal(hl, l_ref.cpu())
+    O, L = ref.ref_attention(d["q"], k_bits, v_bits, d["scale"], causal)
+    assert_o_close(ho.double().numpy(), O, not f32, "from host")
+    if with_lse:
+        assert_lse_close(hl.double().numpy(), L, "from host")
+

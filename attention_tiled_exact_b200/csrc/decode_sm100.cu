@@ -53,7 +53,12 @@ namespace decode {
 constexpr int D = 128;
 constexpr int BS = 16;          // tokens per cache block
 constexpr int WARPS = 4;
-constexpr int NST = 3;          // per-warp pipeline stages
+// Per-warp pipeline stages: an FP8 block is half the bytes of a bf16 one, so
+// its kernel keeps one more stage in flight per warp.
+template <bool FP8>
+constexpr int stages() {
+  return FP8 ? 4 : 3;
+}
 constexpr int BLOCK_BYTES = BS * D * 2;  // 4 KB
 constexpr float RESCALE_THRESHOLD = 8.0f;
 constexpr float LN2 = 0.69314718055994530942f;
@@ -78,7 +83,7 @@ struct Args {
 
 template <int G, bool FP8 = false>
 struct Smem {
-  uint8_t kv[WARPS][NST][2][FP8 ? BLOCK_BYTES / 2 : BLOCK_BYTES];  // 96 KB (bf16) / 48 KB (FP8)
+  uint8_t kv[WARPS][stages<FP8>()][2][FP8 ? BLOCK_BYTES / 2 : BLOCK_BYTES];  // 96 KB (bf16) / 64 KB (FP8)
   float p[WARPS][2][BS / 2][G];  // bf16 caches: probabilities, [token parity][token / 2][head]
   float alpha[WARPS][G];
 };
@@ -212,6 +217,7 @@ __device__ __forceinline__ void split_task(const Args& a, int split, int kvh, in
   constexpr int ROW = D * ELEM;                  // bytes per cached token row
   constexpr int CHUNKS16 = BS * ROW / (16 * 32);  // 16-byte copies per lane per block
   Smem<G, FP8>& sm = *reinterpret_cast<Smem<G, FP8>*>(smem_raw);
+  constexpr int NST = stages<FP8>();
 
   const int warp = warp_id(), lane = lane_id();
   const int hw = lane >> 4, c = lane & 15;  // half-warp, 16-byte chunk of head_dim

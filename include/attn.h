@@ -216,6 +216,9 @@ ATTN_API attn_status_t attn_prefill(const attn_prefill_params* p, attn_stream_t 
  * inputs travel while chunk c computes and chunk c - 1's outputs travel back.
  * Work enqueued on `stream` after the call starts after every copy of the
  * call has completed. Host and device buffers must not be touched until then.
+ * The two side streams are the library's, shared by all threads (calls from
+ * several threads are ordered on them, which is correct but serialises their
+ * copies).
  * Errors: as attn_prefill, plus ATTN_ERR_INVALID_ARG for a null or
  * non-dividing io field, ATTN_ERR_UNSUPPORTED for non-contiguous device
  * tensors, paged / variable-length parameters or an O in another dtype than
@@ -391,7 +394,9 @@ ATTN_API attn_status_t attn_prefill_backward(const attn_backward_params* p, void
  * suffix decode are independent, so the prefill runs on the library's second
  * stream of the device (forked from `stream` and joined back with events;
  * stream capture follows the fork, so the call can be captured into a CUDA
- * graph). Calls from several threads share that second stream.
+ * graph). Calls from several threads share that second stream: one of them
+ * being captured while another runs eagerly makes the eager one fail with
+ * ATTN_ERR_CUDA (a stream in capture takes no eager work).
  *
  * Parameters as attn_decode_paged, plus prefix_len (host): a multiple of 16
  * with 0 <= prefix_len <= max_blocks_per_seq * 16, else

@@ -111,8 +111,8 @@ struct QLayout {
   static constexpr int K_OFF = 2 * TILE;
   static constexpr int V_OFF = K_OFF + K_SLOTS * TILE;
   static constexpr int BAR_OFF = V_OFF + V_SLOTS * TILE;
-  // a_full, k_full[3], k_empty[3], v_full[2], v_empty[2], sdp_full, ps_full, acc_full, mma_done
-  static constexpr int NUM_BARS = 1 + 2 * K_SLOTS + 2 * V_SLOTS + 4;
+  // a_full, a_empty, k_full[3], k_empty[3], v_full[2], v_empty[2], sdp_full, ps_full, acc_full, mma_done
+  static constexpr int NUM_BARS = 2 + 2 * K_SLOTS + 2 * V_SLOTS + 4;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
 };
@@ -199,10 +199,9 @@ struct Work {
 };
 
 template <bool KV>
-__device__ __forceinline__ Work decode_work(const Args& a) {
+__device__ __forceinline__ Work decode_work(const Args& a, int item) {
   Work w;
   const int off = a.seqlen_k - a.seqlen_q;  // bottom-right causal alignment
-  const int item = blockIdx.x;
   if constexpr (KV) {
     // Key block 0 first: under the causal mask it has the most query blocks.
     const int bh = item % (a.batch * a.hkv);
@@ -314,7 +313,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   const int warp = warp_id();
   const int lane = lane_id();
-  const Work w = decode_work<true>(a);
+  const Work w = decode_work<true>(a, blockIdx.x);
 
   if (threadIdx.x == 0) {
     mbar_init(a_full, 1);
@@ -571,8 +570,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// dQ: one CTA per (batch, query head, 128-query block i); Q_i and dO_i stay in
-// shared memory while K_j, V_j stream. Per step t (key block j = t):
+// dQ: persistent, one CTA per SM; CTA c takes the items (batch, query head,
+// 128-query block i) c, 2G-1-c, 2G+c, ... of the heaviest-first numbering
+// (G CTAs), so heavy and light causal blocks pair up on every CTA. Q_i and
+// dO_i stay in shared memory for the item while K_j, V_j stream; the rings,
+// the TMEM allocation and the barrier phases continue across items, so an
+// item's first K/V blocks are already under way while the previous item ends,
+// and its Q_i / dO_i load starts as soon as the previous item's last S and dP
+// have read theirs. Per step t (key block j = t):
 //   S_t = Q_i K_j^T (product 2t) and dP_t = dO_i V_j^T (product 2t + 1), product
 //   p into TMEM buffer p mod 3; the elementwise warps (one query row per
 //   thread, each warpgroup 64 key columns) write dS_t = P_t (dP_t - D) as
@@ -580,33 +585,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // Issue order after step t's elementwise work: dP_{t+1} (into S_t's buffer,
 // read already), dQ += dS_t K_j, S_{t+2} (into dP_t's buffer, after the
 // accumulation read it). S is two steps ahead and dP one, so the tensor core
-// runs dQ and S while the elementwise warps work on the next step.
+// runs dQ and S while the elementwise warps work on the next step. The next
+// item's first dQ product overwrites the accumulator only after the
+// elementwise warps (which also store it) have finished the previous item.
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Args a) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Args a,
+                  int n_items) {
   using L = QLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-  uint64_t* a_full = bars;
-  uint64_t* k_full = bars + 1;                  // [K_SLOTS]
+  uint64_t* a_full = bars;                      // the item's Q_i, dO_i
+  uint64_t* a_empty = bars + 1;                 // the item's last S and dP have read them
+  uint64_t* k_full = bars + 2;                  // [K_SLOTS]
   uint64_t* k_empty = k_full + L::K_SLOTS;      // [K_SLOTS]
   uint64_t* v_full = k_empty + L::K_SLOTS;      // [V_SLOTS]
   uint64_t* v_empty = v_full + L::V_SLOTS;      // [V_SLOTS]
   uint64_t* sdp_full = v_empty + L::V_SLOTS;    // S and dP of the step are in TMEM
   uint64_t* ps_full = sdp_full + 1;             // every elementwise warp wrote dS
-  uint64_t* acc_full = ps_full + 1;
+  uint64_t* acc_full = ps_full + 1;             // the item's dQ is complete
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   const int warp = warp_id();
   const int lane = lane_id();
-  const Work w = decode_work<false>(a);
-  const int n = w.n_steps;
+  // The k-th item of this CTA (-1 past its last).
+  auto cta_item = [&](int k) -> int {
+    const int G = gridDim.x, c = blockIdx.x;
+    const long long it = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
+    return it < n_items ? (int)it : -1;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(a_full, 1);
+    mbar_init(a_empty, 1);
     for (int s = 0; s < L::K_SLOTS; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -630,63 +644,71 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  auto buf_col = [](int p) { return (uint32_t)((p % 3) * 128); };  // TMEM buffer of product p
+  auto buf_col = [](int p) { return (uint32_t)((p % 3) * 128); };  // TMEM buffer of product p of an item
 
   if (warp == TMA_WARP) {
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       // ---------------------------------------------------------------- producer
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(a_full, 2 * L::TILE);
-      for (int c = 0; c < L::CHUNKS; ++c) {
-        tma_load_4d(smem + L::Q_OFF + c * (BM * 128), &tm_q, a_full, c * 64, w.blk * BM, w.h, w.b);
-        tma_load_4d(smem + L::DO_OFF + c * (BM * 128), &tm_do, a_full, c * 64, w.blk * BM, w.h, w.b);
-      }
-      // K_u then V_u for u = 0, 1, ...; each waits for the block a whole ring
-      // back to be released.
-      int nk = 0, nv = 0;
+      // K_u then V_u for every item's blocks u = 0, 1, ... in ring order;
+      // each load waits for the block a whole ring back to be released, and
+      // an item's Q_i, dO_i wait for the previous item's last S and dP.
+      int nk = 0, nv = 0, na = 0;  // K, V and Q/dO loads issued so far (all items)
       bool ok = true;
-      for (int u = 0; u < n && ok; ++u) {
-        const int ks = u % L::K_SLOTS, vs = u % L::V_SLOTS;
-        if (u >= L::K_SLOTS &&
-            !mbar_wait_bounded(&k_empty[ks], ((u / L::K_SLOTS) - 1) & 1, abort_flag, a.wait_limit)) {
-          ok = false;
-          break;
+      for (int kk = 0, item; ok && (item = cta_item(kk)) >= 0; ++kk) {
+        const Work w = decode_work<false>(a, item);
+        if (w.n_steps == 0) continue;
+        if (na > 0 && !mbar_wait_bounded(a_empty, (na - 1) & 1, abort_flag, a.wait_limit)) break;
+        mbar_arrive_expect_tx(a_full, 2 * L::TILE);
+        for (int c = 0; c < L::CHUNKS; ++c) {
+          tma_load_4d(smem + L::Q_OFF + c * (BM * 128), &tm_q, a_full, c * 64, w.blk * BM, w.h, w.b);
+          tma_load_4d(smem + L::DO_OFF + c * (BM * 128), &tm_do, a_full, c * 64, w.blk * BM, w.h, w.b);
         }
-        if (ATTN_IN_BOUNDS(ks >= 0 && ks < L::K_SLOTS && L::K_OFF + (ks + 1) * L::TILE <= L::V_OFF,
-                           ATTN_SITE_BWD_SMEM, a.error_flags, a.planted)) {
-          mbar_arrive_expect_tx(&k_full[ks], L::TILE);
-          for (int c = 0; c < L::CHUNKS; ++c)
-            tma_load_4d(smem + L::K_OFF + ks * L::TILE + c * (BM * 128), &tm_k, &k_full[ks], c * 64, u * BM, w.kvh,
-                        w.b);
+        ++na;
+        for (int u = 0; u < w.n_steps; ++u) {
+          const int ks = nk % L::K_SLOTS, vs = nv % L::V_SLOTS;
+          if (nk >= L::K_SLOTS &&
+              !mbar_wait_bounded(&k_empty[ks], ((nk / L::K_SLOTS) - 1) & 1, abort_flag, a.wait_limit)) {
+            ok = false;
+            break;
+          }
+          if (ATTN_IN_BOUNDS(ks >= 0 && ks < L::K_SLOTS && L::K_OFF + (ks + 1) * L::TILE <= L::V_OFF,
+                             ATTN_SITE_BWD_SMEM, a.error_flags, a.planted)) {
+            mbar_arrive_expect_tx(&k_full[ks], L::TILE);
+            for (int c = 0; c < L::CHUNKS; ++c)
+              tma_load_4d(smem + L::K_OFF + ks * L::TILE + c * (BM * 128), &tm_k, &k_full[ks], c * 64, u * BM,
+                          w.kvh, w.b);
+          }
+          ++nk;
+          if (nv >= L::V_SLOTS &&
+              !mbar_wait_bounded(&v_empty[vs], ((nv / L::V_SLOTS) - 1) & 1, abort_flag, a.wait_limit)) {
+            ok = false;
+            break;
+          }
+          if (ATTN_IN_BOUNDS(vs >= 0 && vs < L::V_SLOTS && L::V_OFF + (vs + 1) * L::TILE <= L::BAR_OFF,
+                             ATTN_SITE_BWD_SMEM, a.error_flags, a.planted)) {
+            mbar_arrive_expect_tx(&v_full[vs], L::TILE);
+            for (int c = 0; c < L::CHUNKS; ++c)
+              tma_load_4d(smem + L::V_OFF + vs * L::TILE + c * (BM * 128), &tm_v, &v_full[vs], c * 64, u * BM,
+                          w.kvh, w.b);
+          }
+          ++nv;
         }
-        ++nk;
-        if (u >= L::V_SLOTS &&
-            !mbar_wait_bounded(&v_empty[vs], ((u / L::V_SLOTS) - 1) & 1, abort_flag, a.wait_limit)) {
-          ok = false;
-          break;
-        }
-        if (ATTN_IN_BOUNDS(vs >= 0 && vs < L::V_SLOTS && L::V_OFF + (vs + 1) * L::TILE <= L::BAR_OFF,
-                           ATTN_SITE_BWD_SMEM, a.error_flags, a.planted)) {
-          mbar_arrive_expect_tx(&v_full[vs], L::TILE);
-          for (int c = 0; c < L::CHUNKS; ++c)
-            tma_load_4d(smem + L::V_OFF + vs * L::TILE + c * (BM * 128), &tm_v, &v_full[vs], c * 64, u * BM, w.kvh,
-                        w.b);
-        }
-        ++nv;
       }
-      // Drain: the last copy into each slot (earlier ones completed before
-      // their slot was released); the waits ignore the abort flag.
-      mbar_wait_drain(a_full, 0);
+      // Drain: the last copy into each slot and of Q/dO (earlier ones
+      // completed before their slot was released); the waits ignore the
+      // abort flag.
+      if (na > 0) mbar_wait_drain(a_full, (na - 1) & 1);
       for (int u = nk - L::K_SLOTS > 0 ? nk - L::K_SLOTS : 0; u < nk; ++u)
         mbar_wait_drain(&k_full[u % L::K_SLOTS], (u / L::K_SLOTS) & 1);
       for (int u = nv - L::V_SLOTS > 0 ? nv - L::V_SLOTS : 0; u < nv; ++u)
         mbar_wait_drain(&v_full[u % L::V_SLOTS], (u / L::V_SLOTS) & 1);
     }
   } else if (warp == MMA_WARP) {
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
       constexpr uint32_t ID_S = instr_desc_bf16(BM, BM, 0);
       constexpr uint32_t ID_ACC = instr_desc_bf16(BM, D, 1);
@@ -698,58 +720,75 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t v_k = sw128_desc_lo(smem_addr(smem + L::V_OFF), 16);
       const uint32_t id_s = ID_S, id_acc = ID_ACC;
       const uint32_t tDQ = tmem_base + COL_ACC_Q;
-      auto kslot = [&](int u) { return (uint32_t)(((u % L::K_SLOTS) * L::TILE) >> 4); };
-      auto vslot = [&](int u) { return (uint32_t)(((u % L::V_SLOTS) * L::TILE) >> 4); };
-      auto wait_k = [&](int u) {
-        return mbar_wait_bounded(&k_full[u % L::K_SLOTS], (u / L::K_SLOTS) & 1, abort_flag, a.wait_limit);
-      };
-      auto wait_v = [&](int u) {
-        return mbar_wait_bounded(&v_full[u % L::V_SLOTS], (u / L::V_SLOTS) & 1, abort_flag, a.wait_limit);
-      };
-      auto issue_sq = [&](int u) { issue_s<D>(tmem_base + buf_col(2 * u), q_lo, k_k + kslot(u), hi, id_s); };
-      auto issue_dp = [&](int u) {  // then the step's S and dP are complete once this has run
-        issue_s<D>(tmem_base + buf_col(2 * u + 1), do_lo, v_k + vslot(u), hi, id_s);
-        mma_commit(sdp_full);
-        mma_commit(&v_empty[u % L::V_SLOTS]);
-      };
-      bool ok = mbar_wait_bounded(a_full, 0, abort_flag, a.wait_limit);
-      if (ok) ok = wait_k(0);
-      if (ok) {
-        tc_fence_after();
-        issue_sq(0);
-        ok = wait_v(0);
-      }
-      if (ok) {
-        tc_fence_after();
-        issue_dp(0);
-        if (n > 1) {
-          ok = wait_k(1);
-          if (ok) {
-            tc_fence_after();
-            issue_sq(1);
+      int kb = 0;  // K / V blocks of the CTA's earlier items (ring positions)
+      int gt = 0;  // steps of the CTA's earlier items (sdp / ps phases)
+      int na = 0;  // items with work so far (a_full / acc_full phases)
+      bool ok = true;
+      for (int kk = 0, item; ok && (item = cta_item(kk)) >= 0; ++kk) {
+        const Work w = decode_work<false>(a, item);
+        const int n = w.n_steps;
+        if (n == 0) continue;
+        // Ring position u of this item's block u is kb + u.
+        auto kslot = [&](int u) { return (uint32_t)((((kb + u) % L::K_SLOTS) * L::TILE) >> 4); };
+        auto vslot = [&](int u) { return (uint32_t)((((kb + u) % L::V_SLOTS) * L::TILE) >> 4); };
+        auto wait_k = [&](int u) {
+          const int g = kb + u;
+          return mbar_wait_bounded(&k_full[g % L::K_SLOTS], (g / L::K_SLOTS) & 1, abort_flag, a.wait_limit);
+        };
+        auto wait_v = [&](int u) {
+          const int g = kb + u;
+          return mbar_wait_bounded(&v_full[g % L::V_SLOTS], (g / L::V_SLOTS) & 1, abort_flag, a.wait_limit);
+        };
+        auto issue_sq = [&](int u) { issue_s<D>(tmem_base + buf_col(2 * u), q_lo, k_k + kslot(u), hi, id_s); };
+        auto issue_dp = [&](int u) {  // then the step's S and dP are complete once this has run
+          issue_s<D>(tmem_base + buf_col(2 * u + 1), do_lo, v_k + vslot(u), hi, id_s);
+          mma_commit(sdp_full);
+          mma_commit(&v_empty[(kb + u) % L::V_SLOTS]);
+          if (u == n - 1) mma_commit(a_empty);  // the item's last S and dP: Q_i, dO_i are free
+        };
+        ok = mbar_wait_bounded(a_full, na & 1, abort_flag, a.wait_limit);
+        if (ok) ok = wait_k(0);
+        if (ok) {
+          tc_fence_after();
+          issue_sq(0);
+          ok = wait_v(0);
+        }
+        if (ok) {
+          tc_fence_after();
+          issue_dp(0);
+          if (n > 1) {
+            ok = wait_k(1);
+            if (ok) {
+              tc_fence_after();
+              issue_sq(1);
+            }
           }
         }
-      }
-      for (int t = 0; t < n && ok; ++t) {
-        ok = mbar_wait_bounded(ps_full, t & 1, abort_flag, a.wait_limit);
+        for (int t = 0; t < n && ok; ++t) {
+          ok = mbar_wait_bounded(ps_full, (gt + t) & 1, abort_flag, a.wait_limit);
+          if (!ok) break;
+          tc_fence_after();
+          if (t + 1 < n) {
+            ok = wait_v(t + 1);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dp(t + 1);  // into S_t's buffer, read by step t's elementwise work
+          }
+          issue_acc(tDQ, tmem_base + buf_col(2 * t + 1), k_mn + kslot(t), hi, id_acc, t == 0);  // dQ += dS K
+          mma_commit(&k_empty[(kb + t) % L::K_SLOTS]);  // K_t's last reader
+          if (t + 2 < n) {
+            ok = wait_k(t + 2);
+            if (!ok) break;
+            tc_fence_after();
+            issue_sq(t + 2);  // into dP_t's buffer, after the accumulation read dS_t
+          }
+        }
         if (!ok) break;
-        tc_fence_after();
-        if (t + 1 < n) {
-          ok = wait_v(t + 1);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dp(t + 1);  // into S_t's buffer, read by step t's elementwise work
-        }
-        issue_acc(tDQ, tmem_base + buf_col(2 * t + 1), k_mn + kslot(t), hi, id_acc, t == 0);  // dQ += dS K
-        mma_commit(&k_empty[t % L::K_SLOTS]);  // K_t's last reader
-        if (t + 2 < n) {
-          ok = wait_k(t + 2);
-          if (!ok) break;
-          tc_fence_after();
-          issue_sq(t + 2);  // into dP_t's buffer, after the accumulation read dS_t
-        }
+        mma_commit(acc_full);
+        kb += n;
+        gt += n;
+        ++na;
       }
-      if (ok) mma_commit(acc_full);
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0);
     }
@@ -761,69 +800,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
     const int off = a.seqlen_k - a.seqlen_q;
     const float sl2 = a.scale_log2;
-    const int row_pos = w.blk * BM + r;  // query position
-    float nlse_r = -INFINITY, ndelta_r = 0.f;
-    {
-      const long long vr = (((long long)w.b * a.hq + w.h) * a.n_qb + w.blk) * BM + r;  // padded: -inf / 0 past Sq
-      if (ATTN_IN_BOUNDS(w.h >= 0 && w.h < a.hq && w.blk >= 0 && w.blk < a.n_qb && r >= 0 && r < BM,
-                         ATTN_SITE_BWD_OUT, a.error_flags, a.planted)) {
-        nlse_r = a.lse2[vr];
-        ndelta_r = a.delta[vr];
-      }
-    }
     const float2 sl2x2 = make_float2(sl2, sl2);
-    const float2 nl = make_float2(nlse_r, nlse_r), nd = make_float2(ndelta_r, ndelta_r);
     const bool cols_ok = ATTN_IN_BOUNDS(half >= 0 && half < 2 && COL_ACC_Q + D <= TMEM_COLS, ATTN_SITE_BWD_TMEM,
                                         a.error_flags, a.planted);
     (void)cols_ok;
+    int gt = 0;  // steps of earlier items (sdp / ps phases)
+    int na = 0;  // items with work so far (acc_full phases)
     bool ok = true;
-    for (int t = 0; t < n && ok; ++t) {
-      // Key column c (key t BM + c) is visible when c < c_lim: below Sk and,
-      // causal, at most row_pos + off.
-      int c_lim = a.seqlen_k - t * BM;
-      if (a.causal) {
-        const int cl = row_pos + off - t * BM + 1;
-        c_lim = cl < c_lim ? cl : c_lim;
-      }
-      const bool all_vis = c_lim >= half * 64 + 64;
-      const uint32_t tS = lane_base + buf_col(2 * t) + half * 64, tD = lane_base + buf_col(2 * t + 1) + half * 64;
-      ok = warp_wait(sdp_full, t & 1, abort_flag, a.wait_limit);
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sv[32], dv[32];
-        if (cols_ok) {
-          tmem_ld32(tS + cc * 32, sv);
-          tmem_ld32(tD + cc * 32, dv);
+    for (int kk = 0, item; ok && (item = cta_item(kk)) >= 0; ++kk) {
+      const Work w = decode_work<false>(a, item);
+      const int n = w.n_steps;
+      const int row_pos = w.blk * BM + r;  // query position
+      float nlse_r = -INFINITY, ndelta_r = 0.f;
+      {
+        const long long vr = (((long long)w.b * a.hq + w.h) * a.n_qb + w.blk) * BM + r;  // padded: -inf / 0 past Sq
+        if (ATTN_IN_BOUNDS(w.h >= 0 && w.h < a.hq && w.blk >= 0 && w.blk < a.n_qb && r >= 0 && r < BM,
+                           ATTN_SITE_BWD_OUT, a.error_flags, a.planted)) {
+          nlse_r = a.lse2[vr];
+          ndelta_r = a.delta[vr];
         }
-        tmem_ld_wait();
-        uint32_t dk[16];
+      }
+      const float2 nl = make_float2(nlse_r, nlse_r), nd = make_float2(ndelta_r, ndelta_r);
+      for (int t = 0; t < n && ok; ++t) {
+        // Key column c (key t BM + c) is visible when c < c_lim: below Sk and,
+        // causal, at most row_pos + off.
+        int c_lim = a.seqlen_k - t * BM;
+        if (a.causal) {
+          const int cl = row_pos + off - t * BM + 1;
+          c_lim = cl < c_lim ? cl : c_lim;
+        }
+        const bool all_vis = c_lim >= half * 64 + 64;
+        const uint32_t tS = lane_base + buf_col(2 * t) + half * 64, tD = lane_base + buf_col(2 * t + 1) + half * 64;
+        ok = warp_wait(sdp_full, (gt + t) & 1, abort_flag, a.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          // P = 2^(S scale log2 e - LSE log2 e); dS = P (dP - D).
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nl);
-          float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          if (!all_vis) {
-            const int c = half * 64 + cc * 32 + j;
-            pp.x = c < c_lim ? pp.x : 0.f;
-            pp.y = c + 1 < c_lim ? pp.y : 0.f;
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sv[32], dv[32];
+          if (cols_ok) {
+            tmem_ld32(tS + cc * 32, sv);
+            tmem_ld32(tD + cc * 32, dv);
           }
-          const float2 ds = __fmul2_rn(pp, __fadd2_rn(make_float2(__uint_as_float(dv[j]), __uint_as_float(dv[j + 1])), nd));
-          dk[j / 2] = pack_bf16x2(ds.x, ds.y);
+          tmem_ld_wait();
+          uint32_t dk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            // P = 2^(S scale log2 e - LSE log2 e); dS = P (dP - D).
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nl);
+            float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (!all_vis) {
+              const int c = half * 64 + cc * 32 + j;
+              pp.x = c < c_lim ? pp.x : 0.f;
+              pp.y = c + 1 < c_lim ? pp.y : 0.f;
+            }
+            const float2 ds =
+                __fmul2_rn(pp, __fadd2_rn(make_float2(__uint_as_float(dv[j]), __uint_as_float(dv[j + 1])), nd));
+            dk[j / 2] = pack_bf16x2(ds.x, ds.y);
+          }
+          // bf16 pairs over this half's first 32 columns of the dP buffer, read already.
+          if (cols_ok) tmem_st16(tD + cc * 16, dk);
         }
-        // bf16 pairs over this half's first 32 columns of the dP buffer, read already.
-        if (cols_ok) tmem_st16(tD + cc * 16, dk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ps_full);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ps_full);
-    }
-    if (ok && n > 0) ok = warp_wait(acc_full, 0, abort_flag, a.wait_limit);
-    if (ok) {
-      tc_fence_after();
+      if (!ok) break;
+      if (n > 0) {
+        ok = warp_wait(acc_full, na & 1, abort_flag, a.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      // The next item's first dQ product overwrites the accumulator after
+      // this warp's next ps_full arrival, which follows these loads.
       store_grads<D, false>(a, w, lane_base, COL_ACC_Q, half, row_pos, n > 0 && cols_ok);
+      gt += n;
+      na += n > 0 ? 1 : 0;
     }
   }
 
@@ -956,7 +1008,10 @@ static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, co
                                 const CUtensorMap& tdo, const bwd::Args& a, long long grid, cudaStream_t stream) {
   constexpr int SMEM = KV ? bwd::KvLayout<D>::SMEM_BYTES : bwd::QLayout<D>::SMEM_BYTES;
   static_assert(SMEM <= 232448, "shared memory budget");
-  auto kern = KV ? bwd::bwd_dkdv_kernel<D> : bwd::bwd_dq_kernel<D>;
+  auto kern = [] {
+    if constexpr (KV) return bwd::bwd_dkdv_kernel<D>;
+    else return bwd::bwd_dq_kernel<D>;
+  }();
   static DeviceOnce setup;  // the shared-memory attribute, once per device
   const attn_status_t st = setup.run([&]() -> attn_status_t {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
@@ -968,7 +1023,13 @@ static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   if (st != ATTN_OK) return st;
   if (grid <= 0) return ATTN_OK;
   if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-  kern<<<(unsigned)grid, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a);
+  if constexpr (KV) {
+    kern<<<(unsigned)grid, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a);
+  } else {
+    // Persistent: at most one CTA per SM over all items (grid = the item count).
+    const long long ctas = grid < device_sm_count() ? grid : device_sm_count();
+    kern<<<(unsigned)ctas, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a, (int)grid);
+  }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

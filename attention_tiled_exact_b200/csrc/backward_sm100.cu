@@ -91,8 +91,8 @@ struct KvLayout {
   static constexpr int RING_OFF = 2 * TILE;            // stage s: Q at + 2 s TILE, dO at + (2 s + 1) TILE
   static constexpr int VEC_OFF = RING_OFF + 4 * TILE;  // [stage][lse2, delta][BM] floats
   static constexpr int BAR_OFF = VEC_OFF + 2 * 2 * BM * 4;
-  // a_full, ring_full[2], ring_empty[2], s_full, dp_full, p_full, ds_full, acc_full, mma_done
-  static constexpr int NUM_BARS = 11;
+  // a_full, a_empty, ring_full[2], ring_empty[2], s_full, dp_full, p_full, ds_full, acc_full, mma_done
+  static constexpr int NUM_BARS = 12;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // tmem address, abort flag
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024-byte alignment
 };
@@ -276,9 +276,14 @@ __device__ __forceinline__ void store_grads(const Args& a, const Work& w, uint32
 }
 
 // ---------------------------------------------------------------------------
-// dK / dV: one CTA per (batch, kv head, 128-key block j); K_j and V_j stay in
-// shared memory while (Q_i, dO_i) of every query head of the group and every
-// query block i that sees block j stream through. Per step t (one (head, i)):
+// dK / dV: persistent, one CTA per SM over the (batch, kv head, 128-key
+// block j) items in a heaviest-first snake (as the dQ kernel). K_j and V_j
+// stay in shared memory for the item while (Q_i, dO_i) of every query head of
+// the group and every query block i that sees block j stream through; the
+// ring, TMEM and barrier phases continue across items, so the next item's
+// K_j / V_j load starts once the current item's last S^T and dP^T have read
+// theirs and the finished item's dK / dV store overlaps the next item's first
+// products. Per step t (one (head, i)):
 //   S^T = K_j Q_i^T into buffer SB (X for even t, Y for odd), dP^T = V_j dO_i^T
 //   into the other buffer DB;
 //   phase 1 (elementwise, one key row per thread, each warpgroup 64 query
@@ -295,28 +300,35 @@ template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const Args a) {
+                    const Args a, int n_items) {
   using L = KvLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-  uint64_t* a_full = bars;
-  uint64_t* ring_full = bars + 1;
-  uint64_t* ring_empty = bars + 3;
-  uint64_t* s_full = bars + 5;   // S^T of the step is in TMEM
-  uint64_t* dp_full = bars + 6;  // dP^T of the step is in TMEM
-  uint64_t* p_full = bars + 7;   // every elementwise warp wrote P^T
-  uint64_t* ds_full = bars + 8;  // every elementwise warp wrote dS^T
-  uint64_t* acc_full = bars + 9;
-  uint64_t* mma_done = bars + 10;
+  uint64_t* a_full = bars;        // the item's K_j, V_j
+  uint64_t* a_empty = bars + 1;   // the item's last S^T and dP^T have read them
+  uint64_t* ring_full = bars + 2;
+  uint64_t* ring_empty = bars + 4;
+  uint64_t* s_full = bars + 6;    // S^T of the step is in TMEM
+  uint64_t* dp_full = bars + 7;   // dP^T of the step is in TMEM
+  uint64_t* p_full = bars + 8;    // every elementwise warp wrote P^T
+  uint64_t* ds_full = bars + 9;   // every elementwise warp wrote dS^T
+  uint64_t* acc_full = bars + 10; // the item's dK and dV are complete
+  uint64_t* mma_done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   const int warp = warp_id();
   const int lane = lane_id();
-  const Work w = decode_work<true>(a, blockIdx.x);
+  // The k-th item of this CTA (-1 past its last).
+  auto cta_item = [&](int k) -> int {
+    const int G = gridDim.x, c = blockIdx.x;
+    const long long it = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
+    return it < n_items ? (int)it : -1;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(a_full, 1);
+    mbar_init(a_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_empty[s], 1);
@@ -339,63 +351,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Streamed step t: query head and query block.
-  auto step_head = [&](int t) { return w.kvh * a.group + t / w.per_head; };
-  auto step_blk = [&](int t) { return w.first + t % w.per_head; };
-  // Padded per-row vectors of query block i of head h.
-  auto vec_row = [&](int h, int i) { return (((long long)w.b * a.hq + h) * a.n_qb + i) * BM; };
-  auto sb_col = [](int t) { return (uint32_t)((t & 1) * 128); };  // S^T, then P^T / dS^T, of step t
-  auto db_col = [](int t) { return (uint32_t)(128 - (t & 1) * 128); };  // dP^T of step t
+  // Padded per-row vectors of query block i of head h of batch b.
+  auto vec_row = [&](int b, int h, int i) { return (((long long)b * a.hq + h) * a.n_qb + i) * BM; };
+  auto sb_col = [](int t) { return (uint32_t)((t & 1) * 128); };        // S^T, then P^T / dS^T, of item step t
+  auto db_col = [](int t) { return (uint32_t)(128 - (t & 1) * 128); };  // dP^T of item step t
 
   if (warp == TMA_WARP) {
-    if (lane == 0 && w.n_steps > 0) {
+    if (lane == 0) {
       // ---------------------------------------------------------------- producer
       float* vec = reinterpret_cast<float*>(smem + L::VEC_OFF);
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(a_full, 2 * L::TILE);
-      for (int c = 0; c < L::CHUNKS; ++c) {
-        tma_load_4d(smem + L::K_OFF + c * (BM * 128), &tm_k, a_full, c * 64, w.blk * BM, w.kvh, w.b);
-        tma_load_4d(smem + L::V_OFF + c * (BM * 128), &tm_v, a_full, c * 64, w.blk * BM, w.kvh, w.b);
-      }
-      int t = 0;
-      for (; t < w.n_steps; ++t) {
-        const int s = t & 1;
-        if (t >= 2 && !mbar_wait_bounded(&ring_empty[s], ((t >> 1) - 1) & 1, abort_flag, a.wait_limit)) break;
-        const int h = step_head(t), blk = step_blk(t);
-        uint8_t* b0 = smem + L::RING_OFF + (2 * s) * L::TILE;
-        uint8_t* b1 = b0 + L::TILE;
-        // The stage's two tiles and its per-row vectors stay inside the ring
-        // and the vector area.
-        if (!ATTN_IN_BOUNDS(s >= 0 && s < 2 && L::RING_OFF + (2 * s + 2) * L::TILE <= L::VEC_OFF &&
-                                L::VEC_OFF + (2 * s + 2) * BM * 4 <= L::BAR_OFF,
-                            ATTN_SITE_BWD_SMEM, a.error_flags, a.planted))
-          continue;
-        // The step's per-column LSE and D ride on the same barrier.
-        mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE + 2 * BM * 4);
-        const long long vr = vec_row(h, blk);
-        if (!ATTN_IN_BOUNDS(h >= 0 && h < a.hq && blk >= 0 && blk < a.n_qb, ATTN_SITE_BWD_OUT, a.error_flags,
-                            a.planted))
-          continue;
-        bulk_load(vec + (2 * s) * BM, a.lse2 + vr, BM * 4, &ring_full[s]);
-        bulk_load(vec + (2 * s + 1) * BM, a.delta + vr, BM * 4, &ring_full[s]);
+      int g = 0, na = 0;  // ring steps and K/V loads issued so far (all items)
+      bool ok = true;
+      for (int kk = 0, item; ok && (item = cta_item(kk)) >= 0; ++kk) {
+        const Work w = decode_work<true>(a, item);
+        if (w.n_steps == 0) continue;
+        if (na > 0 && !mbar_wait_bounded(a_empty, (na - 1) & 1, abort_flag, a.wait_limit)) break;
+        mbar_arrive_expect_tx(a_full, 2 * L::TILE);
         for (int c = 0; c < L::CHUNKS; ++c) {
-          tma_load_4d(b0 + c * (BM * 128), &tm_q, &ring_full[s], c * 64, blk * BM, h, w.b);
-          tma_load_4d(b1 + c * (BM * 128), &tm_do, &ring_full[s], c * 64, blk * BM, h, w.b);
+          tma_load_4d(smem + L::K_OFF + c * (BM * 128), &tm_k, a_full, c * 64, w.blk * BM, w.kvh, w.b);
+          tma_load_4d(smem + L::V_OFF + c * (BM * 128), &tm_v, a_full, c * 64, w.blk * BM, w.kvh, w.b);
+        }
+        ++na;
+        for (int t = 0; t < w.n_steps; ++t, ++g) {
+          const int s = g & 1;
+          if (g >= 2 && !mbar_wait_bounded(&ring_empty[s], ((g >> 1) - 1) & 1, abort_flag, a.wait_limit)) {
+            ok = false;
+            break;
+          }
+          const int h = w.kvh * a.group + t / w.per_head, blk = w.first + t % w.per_head;
+          uint8_t* b0 = smem + L::RING_OFF + (2 * s) * L::TILE;
+          uint8_t* b1 = b0 + L::TILE;
+          // The stage's two tiles and its per-row vectors stay inside the ring
+          // and the vector area.
+          if (!ATTN_IN_BOUNDS(s >= 0 && s < 2 && L::RING_OFF + (2 * s + 2) * L::TILE <= L::VEC_OFF &&
+                                  L::VEC_OFF + (2 * s + 2) * BM * 4 <= L::BAR_OFF,
+                              ATTN_SITE_BWD_SMEM, a.error_flags, a.planted))
+            continue;
+          // The step's per-column LSE and D ride on the same barrier.
+          mbar_arrive_expect_tx(&ring_full[s], 2 * L::TILE + 2 * BM * 4);
+          const long long vr = vec_row(w.b, h, blk);
+          if (!ATTN_IN_BOUNDS(h >= 0 && h < a.hq && blk >= 0 && blk < a.n_qb, ATTN_SITE_BWD_OUT, a.error_flags,
+                              a.planted))
+            continue;
+          bulk_load(vec + (2 * s) * BM, a.lse2 + vr, BM * 4, &ring_full[s]);
+          bulk_load(vec + (2 * s + 1) * BM, a.delta + vr, BM * 4, &ring_full[s]);
+          for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_4d(b0 + c * (BM * 128), &tm_q, &ring_full[s], c * 64, blk * BM, h, w.b);
+            tma_load_4d(b1 + c * (BM * 128), &tm_do, &ring_full[s], c * 64, blk * BM, h, w.b);
+          }
         }
       }
-      // Drain: no copy may be in flight when the CTA exits. The last two
-      // steps' copies are the only ones that can still run (a stage's earlier
-      // copy completed before its empty barrier let the next one start); on
-      // the abort path they still land by themselves, so these waits ignore
-      // the abort flag.
-      mbar_wait_drain(a_full, 0);
-      for (int u = t - 2 > 0 ? t - 2 : 0; u < t; ++u) mbar_wait_drain(&ring_full[u & 1], (u >> 1) & 1);
+      // Drain: no copy may be in flight when the CTA exits: the last K/V load
+      // and the last two ring steps (earlier copies completed before their
+      // slot was released); on the abort path they still land by themselves,
+      // so these waits ignore the abort flag.
+      if (na > 0) mbar_wait_drain(a_full, (na - 1) & 1);
+      for (int u = g - 2 > 0 ? g - 2 : 0; u < g; ++u) mbar_wait_drain(&ring_full[u & 1], (u >> 1) & 1);
     }
   } else if (warp == MMA_WARP) {
-    if (lane == 0 && w.n_steps > 0) {
+    if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
       constexpr uint32_t ID_S = instr_desc_bf16(BM, BM, 0);   // both operands K-major, N = 128
       constexpr uint32_t ID_ACC = instr_desc_bf16(BM, D, 1);  // B MN-major
@@ -406,44 +424,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t ring_mn = sw128_desc_lo(smem_addr(smem + L::RING_OFF), BM * 128);  // MN-major
       const uint32_t id_s = ID_S, id_acc = ID_ACC;
       const uint32_t tDV = tmem_base + COL_ACC_KV, tDK = tDV + D;
-      // Stage addresses of step t's streamed tiles: which = 0 (Q) or 1 (dO).
-      auto b_k = [&](int t, int which) { return ring_k + (uint32_t)(((2 * (t & 1) + which) * L::TILE) >> 4); };
-      auto b_m = [&](int t, int which) { return ring_mn + (uint32_t)(((2 * (t & 1) + which) * L::TILE) >> 4); };
-      auto issue_st = [&](int t) {  // S^T = K Q^T
-        issue_s<D>(tmem_base + sb_col(t), k_lo, b_k(t, 0), hi, id_s);
-        mma_commit(s_full);
-      };
-      auto issue_dpt = [&](int t) {  // dP^T = V dO^T
-        issue_s<D>(tmem_base + db_col(t), v_lo, b_k(t, 1), hi, id_s);
-        mma_commit(dp_full);
-      };
-      bool ok = mbar_wait_bounded(a_full, 0, abort_flag, a.wait_limit);
-      if (ok) ok = mbar_wait_bounded(&ring_full[0], 0, abort_flag, a.wait_limit);
-      if (ok) {
-        tc_fence_after();
-        issue_st(0);
-        issue_dpt(0);
-      }
-      for (int t = 0; t < w.n_steps && ok; ++t) {
-        const bool next = t + 1 < w.n_steps;
-        ok = mbar_wait_bounded(p_full, t & 1, abort_flag, a.wait_limit);
-        if (!ok) break;
-        tc_fence_after();
-        issue_acc(tDV, tmem_base + sb_col(t), b_m(t, 1), hi, id_acc, t == 0);  // dV += P^T dO
-        ok = mbar_wait_bounded(ds_full, t & 1, abort_flag, a.wait_limit);
-        if (!ok) break;
-        tc_fence_after();
-        if (next) {
-          ok = mbar_wait_bounded(&ring_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag, a.wait_limit);
+      int gt = 0, na = 0;  // steps and items with work so far (all phases)
+      bool ok = true;
+      for (int kk = 0, item; ok && (item = cta_item(kk)) >= 0; ++kk) {
+        const Work w = decode_work<true>(a, item);
+        const int n = w.n_steps;
+        if (n == 0) continue;
+        // Ring stage addresses of item step t's streamed tiles: which = 0 (Q) or 1 (dO).
+        auto b_k = [&](int t, int which) {
+          return ring_k + (uint32_t)(((2 * ((gt + t) & 1) + which) * L::TILE) >> 4);
+        };
+        auto b_m = [&](int t, int which) {
+          return ring_mn + (uint32_t)(((2 * ((gt + t) & 1) + which) * L::TILE) >> 4);
+        };
+        auto wait_ring = [&](int t) {
+          const int g = gt + t;
+          return mbar_wait_bounded(&ring_full[g & 1], (g >> 1) & 1, abort_flag, a.wait_limit);
+        };
+        auto issue_st = [&](int t) {  // S^T = K Q^T
+          issue_s<D>(tmem_base + sb_col(t), k_lo, b_k(t, 0), hi, id_s);
+          mma_commit(s_full);
+        };
+        auto issue_dpt = [&](int t) {  // dP^T = V dO^T
+          issue_s<D>(tmem_base + db_col(t), v_lo, b_k(t, 1), hi, id_s);
+          mma_commit(dp_full);
+          if (t == n - 1) mma_commit(a_empty);  // the item's last S^T and dP^T: K_j, V_j are free
+        };
+        ok = mbar_wait_bounded(a_full, na & 1, abort_flag, a.wait_limit);
+        if (ok) ok = wait_ring(0);
+        if (ok) {
+          tc_fence_after();
+          issue_st(0);
+          issue_dpt(0);
+        }
+        for (int t = 0; t < n && ok; ++t) {
+          const bool next = t + 1 < n;
+          ok = mbar_wait_bounded(p_full, (gt + t) & 1, abort_flag, a.wait_limit);
           if (!ok) break;
           tc_fence_after();
-          issue_st(t + 1);  // into DB(t): its dP^T was read by phase 2
+          issue_acc(tDV, tmem_base + sb_col(t), b_m(t, 1), hi, id_acc, t == 0);  // dV += P^T dO
+          ok = mbar_wait_bounded(ds_full, (gt + t) & 1, abort_flag, a.wait_limit);
+          if (!ok) break;
+          tc_fence_after();
+          if (next) {
+            ok = wait_ring(t + 1);
+            if (!ok) break;
+            tc_fence_after();
+            issue_st(t + 1);  // into DB(t): its dP^T was read by phase 2
+          }
+          issue_acc(tDK, tmem_base + sb_col(t) + 32, b_m(t, 0), hi, id_acc, t == 0);  // dK += dS^T Q
+          mma_commit(&ring_empty[(gt + t) & 1]);  // step t's tiles and vectors are free once these have run
+          if (next) issue_dpt(t + 1);              // into SB(t), after dV and dK read it
         }
-        issue_acc(tDK, tmem_base + sb_col(t) + 32, b_m(t, 0), hi, id_acc, t == 0);  // dK += dS^T Q
-        mma_commit(&ring_empty[t & 1]);  // step t's tiles and vectors are free once these have run
-        if (next) issue_dpt(t + 1);      // into SB(t), after dV and dK read it
+        if (!ok) break;
+        mma_commit(acc_full);
+        gt += n;
+        ++na;
       }
-      if (ok) mma_commit(acc_full);
       // Every MMA issued must have completed before tensor memory is released
       // (on the abort path too: they finish by themselves).
       mma_commit(mma_done);
@@ -458,105 +495,118 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int off = a.seqlen_k - a.seqlen_q;
     const float sl2 = a.scale_log2;
     const float* vec = reinterpret_cast<const float*>(smem + L::VEC_OFF);
-    const int row_pos = w.blk * BM + r;  // key position
     const float2 sl2x2 = make_float2(sl2, sl2);
     const bool cols_ok = ATTN_IN_BOUNDS(half >= 0 && half < 2 && COL_ACC_KV + 2 * D <= TMEM_COLS,
                                         ATTN_SITE_BWD_TMEM, a.error_flags, a.planted);
     (void)cols_ok;
+    int gt = 0, na = 0;  // steps and items with work so far (all phases)
     bool ok = true;
-    for (int t = 0; t < w.n_steps && ok; ++t) {
-      const int s = t & 1;
-      const int blk = step_blk(t);
-      // Query column c (query blk BM + c, at position blk BM + c + off) sees
-      // this key when c >= c_lim.
-      const int c_lim = row_pos < a.seqlen_k ? (a.causal ? row_pos - off - blk * BM : -BM) : BM;
-      // The producer's LSE / D copies complete on the stage's full barrier.
-      ok = warp_wait(&ring_full[s], (t >> 1) & 1, abort_flag, a.wait_limit);
-      if (!ok) break;
-      const uint32_t lse_a = smem_addr(vec + (2 * s) * BM) + (uint32_t)(half * 64 * 4);
-      const uint32_t delta_a = smem_addr(vec + (2 * s + 1) * BM) + (uint32_t)(half * 64 * 4);
-      const uint32_t tS = lane_base + sb_col(t) + half * 64, tD = lane_base + db_col(t) + half * 64;
-      // The whole half is visible on all but the diagonal and ragged tiles.
-      const bool all_vis = c_lim <= half * 64;
-      // ---- phase 1: P^T
-      ok = warp_wait(s_full, t & 1, abort_flag, a.wait_limit);
-      if (!ok) break;
-      tc_fence_after();
-      float p[64];
+    for (int kk = 0, item; ok && (item = cta_item(kk)) >= 0; ++kk) {
+      const Work w = decode_work<true>(a, item);
+      const int n = w.n_steps;
+      const int row_pos = w.blk * BM + r;  // key position
+      for (int t = 0; t < n && ok; ++t) {
+        const int g = gt + t;
+        const int s = g & 1;
+        const int blk = w.first + t % w.per_head;
+        // Query column c (query blk BM + c, at position blk BM + c + off) sees
+        // this key when c >= c_lim.
+        const int c_lim = row_pos < a.seqlen_k ? (a.causal ? row_pos - off - blk * BM : -BM) : BM;
+        // The producer's LSE / D copies complete on the stage's full barrier.
+        ok = warp_wait(&ring_full[s], (g >> 1) & 1, abort_flag, a.wait_limit);
+        if (!ok) break;
+        const uint32_t lse_a = smem_addr(vec + (2 * s) * BM) + (uint32_t)(half * 64 * 4);
+        const uint32_t delta_a = smem_addr(vec + (2 * s + 1) * BM) + (uint32_t)(half * 64 * 4);
+        const uint32_t tS = lane_base + sb_col(t) + half * 64, tD = lane_base + db_col(t) + half * 64;
+        // The whole half is visible on all but the diagonal and ragged tiles.
+        const bool all_vis = c_lim <= half * 64;
+        // ---- phase 1: P^T
+        ok = warp_wait(s_full, g & 1, abort_flag, a.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
+        float p[64];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sv[32];
-        if (cols_ok) tmem_ld32(tS + cc * 32, sv);
-        tmem_ld_wait();
-        uint32_t pk[16];
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sv[32];
+          if (cols_ok) tmem_ld32(tS + cc * 32, sv);
+          tmem_ld_wait();
+          uint32_t pk[16];
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {  // 16 columns at a time: their -LSE log2 e loaded first
-          float4 lv[4];
+          for (int gg = 0; gg < 2; ++gg) {  // 16 columns at a time: their -LSE log2 e loaded first
+            float4 lv[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) lv[q] = lds_f4(lse_a + (uint32_t)(cc * 32 + g * 16 + 4 * q) * 4u);
+            for (int q = 0; q < 4; ++q) lv[q] = lds_f4(lse_a + (uint32_t)(cc * 32 + gg * 16 + 4 * q) * 4u);
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const int jj = g * 16 + j;
-            const float4 l4 = lv[j >> 2];
-            const float2 nl = (j & 2) ? make_float2(l4.z, l4.w) : make_float2(l4.x, l4.y);
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[jj]), __uint_as_float(sv[jj + 1])), sl2x2, nl);
-            float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            if (!all_vis) {
-              const int c = half * 64 + cc * 32 + jj;
-              pp.x = c >= c_lim ? pp.x : 0.f;
-              pp.y = c + 1 >= c_lim ? pp.y : 0.f;
+            for (int j = 0; j < 16; j += 2) {
+              const int jj = gg * 16 + j;
+              const float4 l4 = lv[j >> 2];
+              const float2 nl = (j & 2) ? make_float2(l4.z, l4.w) : make_float2(l4.x, l4.y);
+              const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[jj]), __uint_as_float(sv[jj + 1])), sl2x2, nl);
+              float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              if (!all_vis) {
+                const int c = half * 64 + cc * 32 + jj;
+                pp.x = c >= c_lim ? pp.x : 0.f;
+                pp.y = c + 1 >= c_lim ? pp.y : 0.f;
+              }
+              p[cc * 32 + jj] = pp.x;
+              p[cc * 32 + jj + 1] = pp.y;
+              pk[jj / 2] = pack_bf16x2(pp.x, pp.y);
             }
-            p[cc * 32 + jj] = pp.x;
-            p[cc * 32 + jj + 1] = pp.y;
-            pk[jj / 2] = pack_bf16x2(pp.x, pp.y);
           }
+          // bf16 pairs over the first 32 columns of this half, read already.
+          if (cols_ok) tmem_st16(tS + cc * 16, pk);
         }
-        // bf16 pairs over the first 32 columns of this half, read already.
-        if (cols_ok) tmem_st16(tS + cc * 16, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+        // ---- phase 2: dS^T
+        ok = warp_wait(dp_full, g & 1, abort_flag, a.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t dv[32];
+          if (cols_ok) tmem_ld32(tD + cc * 32, dv);
+          tmem_ld_wait();
+          uint32_t dk[16];
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg) {
+            float4 nd4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) nd4[q] = lds_f4(delta_a + (uint32_t)(cc * 32 + gg * 16 + 4 * q) * 4u);
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+              const int jj = gg * 16 + j;
+              const float4 d4 = nd4[j >> 2];
+              const float2 nd = (j & 2) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+              const float2 ds = __fmul2_rn(make_float2(p[cc * 32 + jj], p[cc * 32 + jj + 1]),
+                                           __fadd2_rn(make_float2(__uint_as_float(dv[jj]), __uint_as_float(dv[jj + 1])), nd));
+              dk[jj / 2] = pack_bf16x2(ds.x, ds.y);
+            }
+          }
+          // bf16 pairs over the last 32 columns of this half of SB (its S^T was
+          // read in phase 1).
+          if (cols_ok) tmem_st16(tS + 32 + cc * 16, dk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-      // ---- phase 2: dS^T
-      ok = warp_wait(dp_full, t & 1, abort_flag, a.wait_limit);
       if (!ok) break;
-      tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t dv[32];
-        if (cols_ok) tmem_ld32(tD + cc * 32, dv);
-        tmem_ld_wait();
-        uint32_t dk[16];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          float4 nd4[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) nd4[q] = lds_f4(delta_a + (uint32_t)(cc * 32 + g * 16 + 4 * q) * 4u);
-#pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const int jj = g * 16 + j;
-            const float4 d4 = nd4[j >> 2];
-            const float2 nd = (j & 2) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
-            const float2 ds = __fmul2_rn(make_float2(p[cc * 32 + jj], p[cc * 32 + jj + 1]),
-                                         __fadd2_rn(make_float2(__uint_as_float(dv[jj]), __uint_as_float(dv[jj + 1])), nd));
-            dk[jj / 2] = pack_bf16x2(ds.x, ds.y);
-          }
-        }
-        // bf16 pairs over the last 32 columns of this half of SB (its S^T was
-        // read in phase 1).
-        if (cols_ok) tmem_st16(tS + 32 + cc * 16, dk);
+      // ---- epilogue: each warpgroup stores half of the columns of its rows
+      if (n > 0) {
+        ok = warp_wait(acc_full, na & 1, abort_flag, a.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
-    }
-    // ---- epilogue: each warpgroup stores half of the columns of its rows
-    if (ok && w.n_steps > 0) ok = warp_wait(acc_full, 0, abort_flag, a.wait_limit);
-    if (ok) {
-      tc_fence_after();
-      store_grads<D, true>(a, w, lane_base, COL_ACC_KV, half, row_pos, w.n_steps > 0 && cols_ok);
+      // The next item's first dV / dK products overwrite the accumulators
+      // after this warp's next p_full / ds_full arrivals, which follow these
+      // loads.
+      store_grads<D, true>(a, w, lane_base, COL_ACC_KV, half, row_pos, n > 0 && cols_ok);
+      gt += n;
+      na += n > 0 ? 1 : 0;
     }
   }
 
@@ -1023,13 +1073,9 @@ static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   if (st != ATTN_OK) return st;
   if (grid <= 0) return ATTN_OK;
   if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-  if constexpr (KV) {
-    kern<<<(unsigned)grid, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a);
-  } else {
-    // Persistent: at most one CTA per SM over all items (grid = the item count).
-    const long long ctas = grid < device_sm_count() ? grid : device_sm_count();
-    kern<<<(unsigned)ctas, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a, (int)grid);
-  }
+  // Persistent: at most one CTA per SM over all items (grid = the item count).
+  const long long ctas = grid < device_sm_count() ? grid : device_sm_count();
+  kern<<<(unsigned)ctas, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a, (int)grid);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -350,6 +350,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The dQ kernel, launched as a programmatic dependent, may now be scheduled:
+  // its CTAs take the SMs this grid's CTAs leave when they finish.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // Padded per-row vectors of query block i of head h of batch b.
   auto vec_row = [&](int b, int h, int i) { return (((long long)b * a.hq + h) * a.n_qb + i) * BM; };
@@ -936,73 +939,93 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
+  // This grid may have started before the dK/dV grid ended; it ends only
+  // after that grid, so that work after the call on the stream follows both.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Per query row, padded to whole 128-row blocks: -D = -rowsum(dO * O) and
 // -LSE * log2(e) (-inf for rows that see no key and for padding rows, whose D
-// is 0). One warp per row, vector loads.
-template <int D>
+// is 0). One CTA per (batch, head, 128-row block); D / 8 threads share a row,
+// each with 16-byte loads of 8 elements, and every thread issues the loads of
+// UNR rows (and their LSE) before it reduces any of them, so that enough bytes
+// are in flight to keep HBM busy.
+template <int D, bool OF32>
 __global__ void __launch_bounds__(256)
-    bwd_prep_kernel(const void* o, int o_f32, long long o_bs, long long o_hs, long long o_rs,
-                    const __nv_bfloat16* dout, long long do_bs, long long do_hs, long long do_rs, const float* lse,
-                    int batch, int hq, int seqlen_q, int n_qb, float* lse2, float* delta) {
-  constexpr int PER = D / 32;  // 4 (head_dim 128) or 2 (64)
-  const long long padded = (long long)n_qb * 128;
-  const long long row = (long long)blockIdx.x * 8 + warp_id();
-  const int lane = lane_id();
-  if (row >= (long long)batch * hq * padded) return;
-  const int q = (int)(row % padded);
-  const long long bh = row / padded;
-  if (q >= seqlen_q) {
-    if (lane == 0) {
-      lse2[row] = -INFINITY;
-      delta[row] = 0.f;
-    }
-    return;
-  }
-  const int h = (int)(bh % hq), b = (int)(bh / hq);
-  const __nv_bfloat16* dr = dout + b * do_bs + h * do_hs + q * do_rs + lane * PER;
-  float dov[PER], ov[PER];
-  if constexpr (PER == 4) {
-    const uint2 x = *reinterpret_cast<const uint2*>(dr);
-    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
-    const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
-    dov[0] = a0.x, dov[1] = a0.y, dov[2] = a1.x, dov[3] = a1.y;
-  } else {
-    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dr));
-    dov[0] = a0.x, dov[1] = a0.y;
-  }
-  if (o_f32) {
-    const float* orow = reinterpret_cast<const float*>(o) + b * o_bs + h * o_hs + q * o_rs + lane * PER;
-    if constexpr (PER == 4) {
-      const float4 x = *reinterpret_cast<const float4*>(orow);
-      ov[0] = x.x, ov[1] = x.y, ov[2] = x.z, ov[3] = x.w;
-    } else {
-      const float2 x = *reinterpret_cast<const float2*>(orow);
-      ov[0] = x.x, ov[1] = x.y;
-    }
-  } else {
-    const __nv_bfloat16* orow =
-        reinterpret_cast<const __nv_bfloat16*>(o) + b * o_bs + h * o_hs + q * o_rs + lane * PER;
-    if constexpr (PER == 4) {
-      const uint2 x = *reinterpret_cast<const uint2*>(orow);
-      const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
-      const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
-      ov[0] = a0.x, ov[1] = a0.y, ov[2] = a1.x, ov[3] = a1.y;
-    } else {
-      const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(orow));
-      ov[0] = a0.x, ov[1] = a0.y;
-    }
-  }
-  float acc = 0.f;
+    bwd_prep_kernel(const void* o, long long o_bs, long long o_hs, long long o_rs, const __nv_bfloat16* dout,
+                    long long do_bs, long long do_hs, long long do_rs, const float* lse, int hq, int seqlen_q,
+                    int n_qb, float* lse2, float* delta) {
+  constexpr int TPR = D / 8;         // threads per row: 16 (head_dim 128) or 8 (64)
+  constexpr int RPP = 256 / TPR;     // rows per pass: 16 or 32
+  constexpr int PASSES = BM / RPP;   // 8 or 4
+  constexpr int UNR = 4;
+  static_assert(PASSES % UNR == 0, "whole unrolled groups");
+  const int qb = (int)(blockIdx.x % (unsigned)n_qb);
+  const int bh = (int)(blockIdx.x / (unsigned)n_qb);
+  const int h = bh % hq, b = bh / hq;
+  const int sub = threadIdx.x % TPR, r0 = threadIdx.x / TPR;
+  // Padded row (bh n_qb + qb) BM + r == blockIdx.x BM + r.
+  float* lse2_blk = lse2 + (long long)blockIdx.x * BM;
+  float* delta_blk = delta + (long long)blockIdx.x * BM;
+  const __nv_bfloat16* drow = dout + b * do_bs + h * do_hs + sub * 8;
+  const float* lrow = lse + (long long)bh * seqlen_q;
 #pragma unroll
-  for (int k = 0; k < PER; ++k) acc = fmaf(dov[k], ov[k], acc);
+  for (int p0 = 0; p0 < PASSES; p0 += UNR) {
+    uint4 dv[UNR], ov[UNR], ov2[UNR];
+    float lv[UNR];
 #pragma unroll
-  for (int sh = 16; sh >= 1; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
-  if (lane == 0) {
-    const float l = lse[bh * seqlen_q + q];
-    lse2[row] = l == -INFINITY ? -INFINITY : -l * LOG2E;
-    delta[row] = -acc;
+    for (int u = 0; u < UNR; ++u) {
+      const int q = qb * BM + (p0 + u) * RPP + r0;
+      dv[u] = ov[u] = ov2[u] = make_uint4(0u, 0u, 0u, 0u);
+      lv[u] = 0.f;
+      if (q < seqlen_q) {
+        dv[u] = __ldg(reinterpret_cast<const uint4*>(drow + q * do_rs));
+        if constexpr (OF32) {
+          const float* orow = reinterpret_cast<const float*>(o) + b * o_bs + h * o_hs + q * o_rs + sub * 8;
+          ov[u] = __ldcs(reinterpret_cast<const uint4*>(orow));
+          ov2[u] = __ldcs(reinterpret_cast<const uint4*>(orow + 4));
+        } else {
+          const __nv_bfloat16* orow =
+              reinterpret_cast<const __nv_bfloat16*>(o) + b * o_bs + h * o_hs + q * o_rs + sub * 8;
+          ov[u] = __ldcs(reinterpret_cast<const uint4*>(orow));
+        }
+        if (sub == 0) lv[u] = __ldg(lrow + q);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const uint32_t dw[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
+      float of[8];
+      if constexpr (OF32) {
+        of[0] = __uint_as_float(ov[u].x), of[1] = __uint_as_float(ov[u].y);
+        of[2] = __uint_as_float(ov[u].z), of[3] = __uint_as_float(ov[u].w);
+        of[4] = __uint_as_float(ov2[u].x), of[5] = __uint_as_float(ov2[u].y);
+        of[6] = __uint_as_float(ov2[u].z), of[7] = __uint_as_float(ov2[u].w);
+      } else {
+        const uint32_t ow[4] = {ov[u].x, ov[u].y, ov[u].z, ov[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[e]));
+          of[2 * e] = f.x, of[2 * e + 1] = f.y;
+        }
+      }
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dw[e]));
+        acc = fmaf(f.x, of[2 * e], acc);
+        acc = fmaf(f.y, of[2 * e + 1], acc);
+      }
+#pragma unroll
+      for (int sh = TPR / 2; sh >= 1; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+      const int r = (p0 + u) * RPP + r0;
+      if (sub == 0) {
+        const bool live = qb * BM + r < seqlen_q;
+        const float l = lv[u];
+        lse2_blk[r] = live && l != -INFINITY ? -l * LOG2E : -INFINITY;
+        delta_blk[r] = live ? -acc : 0.f;
+      }
+    }
   }
 }
 
@@ -1075,7 +1098,24 @@ static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   // Persistent: at most one CTA per SM over all items (grid = the item count).
   const long long ctas = grid < device_sm_count() ? grid : device_sm_count();
-  kern<<<(unsigned)ctas, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a, (int)grid);
+  if constexpr (KV) {
+    kern<<<(unsigned)ctas, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a, (int)grid);
+  } else {
+    // The dQ kernel reads nothing the dK/dV kernel writes: as a programmatic
+    // dependent its CTAs start on the SMs the dK/dV kernel's last items leave
+    // idle instead of after the whole grid.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(bwd::NUM_THREADS);
+    cfg.dynamicSmemBytes = SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tdo, a, (int)grid) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -1088,18 +1128,19 @@ attn_status_t launch_backward(const attn_backward_params& p, void* workspace, cu
   float* delta = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + (n * 4 + 255) / 256 * 256);
   const bool o_f32 = p.o_dtype == ATTN_DTYPE_F32;
   if (n > 0) {
-    const long long blocks = (long long)((n + 7) / 8);
+    // One CTA per (batch, head, 128-row block): n / 128 of them.
+    const long long blocks = (long long)(n / bwd::BM);
     if (blocks > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    auto prep = [&](auto kern) {
+      kern<<<(unsigned)blocks, 256, 0, stream>>>(p.o, p.o_batch_stride, p.o_head_stride, p.o_row_stride,
+                                                  reinterpret_cast<const __nv_bfloat16*>(p.dout), p.do_batch_stride,
+                                                  p.do_head_stride, p.do_row_stride, p.lse, p.num_q_heads,
+                                                  p.seqlen_q, n_qb, lse2, delta);
+    };
     if (D == 128)
-      bwd::bwd_prep_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
-          p.o, o_f32, p.o_batch_stride, p.o_head_stride, p.o_row_stride,
-          reinterpret_cast<const __nv_bfloat16*>(p.dout), p.do_batch_stride, p.do_head_stride, p.do_row_stride, p.lse,
-          p.batch, p.num_q_heads, p.seqlen_q, n_qb, lse2, delta);
+      o_f32 ? prep(bwd::bwd_prep_kernel<128, true>) : prep(bwd::bwd_prep_kernel<128, false>);
     else
-      bwd::bwd_prep_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
-          p.o, o_f32, p.o_batch_stride, p.o_head_stride, p.o_row_stride,
-          reinterpret_cast<const __nv_bfloat16*>(p.dout), p.do_batch_stride, p.do_head_stride, p.do_row_stride, p.lse,
-          p.batch, p.num_q_heads, p.seqlen_q, n_qb, lse2, delta);
+      o_f32 ? prep(bwd::bwd_prep_kernel<64, true>) : prep(bwd::bwd_prep_kernel<64, false>);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   // Tensor maps need at least one row; an empty side is never loaded.

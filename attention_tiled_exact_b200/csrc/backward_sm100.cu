@@ -1078,7 +1078,8 @@ size_t backward_workspace_bytes(const attn_backward_params& p) {
 
 template <int D, bool KV>
 static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                const CUtensorMap& tdo, const bwd::Args& a, long long grid, cudaStream_t stream) {
+                                const CUtensorMap& tdo, const bwd::Args& a, long long grid, bool dependent,
+                                cudaStream_t stream) {
   constexpr int SMEM = KV ? bwd::KvLayout<D>::SMEM_BYTES : bwd::QLayout<D>::SMEM_BYTES;
   static_assert(SMEM <= 232448, "shared memory budget");
   auto kern = [] {
@@ -1098,12 +1099,12 @@ static attn_status_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, co
   if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
   // Persistent: at most one CTA per SM over all items (grid = the item count).
   const long long ctas = grid < device_sm_count() ? grid : device_sm_count();
-  if constexpr (KV) {
+  if (!dependent) {
     kern<<<(unsigned)ctas, bwd::NUM_THREADS, SMEM, stream>>>(tq, tk, tv, tdo, a, (int)grid);
   } else {
     // The dQ kernel reads nothing the dK/dV kernel writes: as a programmatic
-    // dependent its CTAs start on the SMs the dK/dV kernel's last items leave
-    // idle instead of after the whole grid.
+    // dependent of the dK/dV launch right before it, its CTAs start on the
+    // SMs the dK/dV kernel's last items leave idle instead of after the grid.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ctas);
     cfg.blockDim = dim3(bwd::NUM_THREADS);
@@ -1187,12 +1188,15 @@ attn_status_t launch_backward(const attn_backward_params& p, void* workspace, cu
   const long long q_items = (long long)a.n_qb * p.batch * p.num_q_heads;
   attn_status_t st;
   if (D == 128) {
-    st = launch_bwd<128, true>(tq, tk, tv, tdo, a, kv_items, stream);
-    if (st == ATTN_OK) st = launch_bwd<128, false>(tq, tk, tv, tdo, a, q_items, stream);
+    st = launch_bwd<128, true>(tq, tk, tv, tdo, a, kv_items, false, stream);
+    if (st == ATTN_OK) st = launch_bwd<128, false>(tq, tk, tv, tdo, a, q_items, kv_items > 0, stream);
   } else {
-    st = launch_bwd<64, true>(tq, tk, tv, tdo, a, kv_items, stream);
-    if (st == ATTN_OK) st = launch_bwd<64, false>(tq, tk, tv, tdo, a, q_items, stream);
+    st = launch_bwd<64, true>(tq, tk, tv, tdo, a, kv_items, false, stream);
+    if (st == ATTN_OK) st = launch_bwd<64, false>(tq, tk, tv, tdo, a, q_items, kv_items > 0, stream);
   }
+  // The dQ kernel is a dependent only of this call's dK/dV launch (a kernel
+  // before the call may trigger its dependents early, and the prep kernel's
+  // results must be complete before the dQ kernel reads them).
   return st;
 }
 

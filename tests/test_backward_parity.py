@@ -58,6 +58,7 @@ def _backward(lib, q, k, v, do, o, lse, scale, causal, grad_dtype=None, **kw):
     (2, 4, 4, 1, 777, 128, False),     # one query row
     (1, 8, 2, 513, 513, 64, True),     # G = 4, head_dim 64
     (1, 2, 1, 130, 70, 128, False),    # fewer keys than one tile
+    (1, 8, 1, 2048, 128, 128, False),  # one dK/dV item, 128 dQ items: dQ CTAs on idle SMs from the start
 ])
 def test_backward_matches_oracle(lib, B, Hq, Hkv, Sq, Sk, D, causal):
     seed = 7 * Sq + Sk + D + Hq

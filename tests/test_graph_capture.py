@@ -1,6 +1,8 @@
 """CUDA-graph capture of the hot path: a decode step (split kernel + combine,
-caller-owned workspace) and a prefill call are captured once on static
-buffers and replayed with new inputs written into those buffers.
+caller-owned workspace), a prefill call and a backward call (three launches,
+the second and third as programmatic dependents of the one before) are
+captured once on static buffers and replayed with new inputs written into
+those buffers.
 
 The split plan is fixed at capture from the host-side length bound, and the
 kernels read lengths and block tables from device memory on every replay, so
@@ -122,3 +124,56 @@ def test_prefill_graph_replay(lib):
         call()
         torch.cuda.synchronize()
         assert np.array_equal(to_f64(o_s), o_graph) and np.array_equal(to_f64(l_s), l_graph)
+
+
+def test_backward_graph_replay(lib):
+    import torch
+    B_, HQ_, HKV_, S, D_ = 2, 8, 2, 300, 128
+    q_s = torch.empty((B_, HQ_, S, D_), dtype=torch.bfloat16, device="cuda")
+    k_s = torch.empty((B_, HKV_, S, D_), dtype=torch.bfloat16, device="cuda")
+    v_s = torch.empty_like(k_s)
+    do_s = torch.empty_like(q_s)
+    o_s = torch.empty((B_, HQ_, S, D_), dtype=torch.float32, device="cuda")
+    l_s = torch.empty((B_, HQ_, S), dtype=torch.float32, device="cuda")
+    grads = [torch.empty(t.shape, dtype=torch.float32, device="cuda") for t in (q_s, k_s, v_s)]
+    scale = 1.0 / np.sqrt(D_)
+
+    def load(seed):
+        q = wl.normal_bf16(seed, q_s.shape, 40)
+        k = wl.normal_bf16(seed, k_s.shape, 41)
+        v = wl.normal_bf16(seed, v_s.shape, 42)
+        do = wl.normal_bf16(seed, do_s.shape, 43)
+        r = ref.ref_attention_backward(q, k, v, do, scale, True)
+        for dst, src in ((q_s, q), (k_s, k), (v_s, v), (do_s, do)):
+            dst.copy_(to_dev_bf16(src))
+        o_s.copy_(torch.tensor(np.asarray(r["o"], dtype=np.float32)))
+        l_s.copy_(torch.tensor(np.asarray(r["lse"], dtype=np.float32)))
+        return r
+
+    load(800)
+    ws = torch.empty(64 << 20, dtype=torch.uint8, device="cuda")
+
+    def call():
+        lib.prefill_backward(q_s, k_s, v_s, o_s, l_s, do_s, scale, True, dq=grads[0], dk=grads[1], dv=grads[2],
+                             workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for seed in (801, 802):
+        r = load(seed)
+        g.replay()
+        torch.cuda.synchronize()
+        got = [to_f64(t) for t in grads]
+        for x, name in zip(got, ("dq", "dk", "dv")):
+            peak = float(np.abs(r[name]).max())
+            assert float(np.abs(x - r[name]).max()) <= 1e-2 * peak, (seed, name)
+        call()
+        torch.cuda.synchronize()
+        assert all(np.array_equal(to_f64(t), x) for t, x in zip(grads, got))

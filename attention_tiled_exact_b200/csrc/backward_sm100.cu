@@ -12,22 +12,28 @@
 // forward's LSE, exactly as the forward builds S tile by tile.
 //
 // Three launches:
-//   * prep (one warp per query row): -D = -rowsum(dO * O) and -LSE log2(e)
+//   * prep (one CTA per (batch, head, 128-row block), 16-byte loads, four
+//     rows of a thread in flight): -D = -rowsum(dO * O) and -LSE log2(e)
 //     (-inf for rows that see no key, so that their P is exactly 0), padded
 //     to whole 128-row blocks;
-//   * dK/dV kernel, one CTA per (batch, kv head, 128-key block j): K_j and V_j
-//     stay in shared memory; for every query head of the group and every
-//     query block i that sees block j, TMA streams Q_i and dO_i through a
-//     two-stage ring and one thread issues
+//   * dK/dV kernel, persistent (one CTA per SM over the (batch, kv head,
+//     128-key block j) items, heaviest first): K_j and V_j stay in shared
+//     memory for the item; for every query head of the group and every query
+//     block i that sees block j, TMA streams Q_i and dO_i through a two-stage
+//     ring and one thread issues
 //         S^T = K_j Q_i^T, dP^T = V_j dO_i^T          (tcgen05, fp32 in TMEM)
-//     four warps (one key row per thread, the TMEM lane) turn them into
-//     P^T = exp2(S^T scale log2 e - LSE log2 e) and dS^T = P^T (dP^T - D),
-//     written back into TMEM as bf16 over S^T and dP^T, and the thread issues
+//     two warpgroups (one key row per thread, the TMEM lane; 64 query columns
+//     each) turn them into P^T = exp2(S^T scale log2 e - LSE log2 e) and
+//     dS^T = P^T (dP^T - D), written back into TMEM as bf16, and the thread
+//     issues
 //         dV += P^T dO_i, dK += dS^T Q_i              (A from TMEM)
-//     into two accumulators that stay in TMEM for the whole CTA;
-//   * dQ kernel, one CTA per (batch, query head, 128-query block i): Q_i and
-//     dO_i stay in shared memory, K_j and V_j stream, S and dP are recomputed
-//     the same way and dQ += dS K_j accumulates in TMEM.
+//     into two accumulators that stay in TMEM for the item;
+//   * dQ kernel, persistent over the (batch, query head, 128-query block i)
+//     items: Q_i and dO_i stay in shared memory for the item, K_j and V_j
+//     stream, S and dP are recomputed the same way and dQ += dS K_j
+//     accumulates in TMEM. It is launched as a programmatic dependent of the
+//     dK/dV kernel, whose results it does not read, so that its CTAs start on
+//     the SMs the dK/dV kernel's last items leave.
 // dQ is recomputed rather than accumulated with atomics from the dK/dV
 // kernel (7 products per tile pair instead of 5): the result is
 // deterministic, and TMEM has no room for a fifth 128-column accumulator

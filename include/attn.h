@@ -332,7 +332,10 @@ ATTN_API attn_status_t attn_decode_paged(const attn_decode_params* p, void* work
  * aligned (two fp32 values per query row, rows padded to a multiple of 128
  * per head). workspace = NULL only queries the
  * size (returns ATTN_OK, enqueues nothing); a smaller workspace returns
- * ATTN_ERR_WORKSPACE and enqueues nothing. Asynchronous on `stream`.
+ * ATTN_ERR_WORKSPACE and enqueues nothing. Asynchronous on `stream`: up to
+ * three kernels, the last a programmatic dependent of the one before it
+ * (capturable in a CUDA graph); work enqueued on `stream` after the call
+ * starts after all of them.
  */
 typedef struct {
   const void* q;
